@@ -1,0 +1,265 @@
+"""Plain, slow, obviously correct CPU oracle (test infrastructure only).
+
+Scalar quantizers come from qat_oracle.c through ctypes; the dense algebra is
+numpy float64 on the exact values of the bf16 operands.  Nothing here is
+blocked, fused or reordered beyond the definitions it restates.
+
+Page references (title, section):
+  P5 = "parameter-golf 16MB 极限压缩实战：11L MLP3x + Int6 QAT + zstd-22 记录详解"
+  P1 = "Depth Recurrence + Mixed-Precision Quant" write-up (PR #363)
+"""
+import ctypes
+import re
+
+import numpy as np
+
+from .build import build_oracle
+
+# P5 "后训练量化导出": per-row clip at the 99.99984th percentile.
+EXPORT_CLIP_Q = 0.9999984
+# P5 "后训练量化导出": INT8_KEEP_FLOAT_MAX_NUMEL = 65_536 (reading: <= passes through).
+KEEP_FLOAT_MAX_NUMEL = 65536
+
+_lib = None
+
+
+def _c():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build_oracle())
+        P = ctypes.c_void_p
+        I64 = ctypes.c_int64
+        lib.oracle_qat_scales.argtypes = [P, I64, I64, P]
+        lib.oracle_qat_codes.argtypes = [P, I64, I64, P, ctypes.c_int, P]
+        lib.oracle_qat_codes.restype = ctypes.c_int
+        lib.oracle_dequant_f32.argtypes = [P, P, I64, I64, P]
+        lib.oracle_operand_bf16.argtypes = [P, P, I64, I64, P]
+        lib.oracle_row_quantile_abs.argtypes = [P, I64, ctypes.c_double]
+        lib.oracle_row_quantile_abs.restype = ctypes.c_float
+        lib.oracle_export_rows.argtypes = [P, I64, I64, ctypes.c_int, ctypes.c_double, P, P, P]
+        lib.oracle_export_rows.restype = ctypes.c_int
+        lib.oracle_dequant_export.argtypes = [P, P, I64, I64, P]
+        lib.oracle_fp16_array.argtypes = [P, I64, P]
+        lib.oracle_bf16_array.argtypes = [P, I64, P]
+        _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _f32(a):
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+# ---------------------------------------------------------------- conversions
+
+def bf16_bits(x):
+    """bf16 round-to-nearest-even of fp32 values, as uint16 bit patterns."""
+    x = _f32(x)
+    out = np.empty(x.shape, np.uint16)
+    _c().oracle_bf16_array(_ptr(x), x.size, _ptr(out))
+    return out
+
+
+def bf16_bits_to_f32(b):
+    return (np.asarray(b, np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def bf16_round(x):
+    """Values of bf16_rne(x) as fp32."""
+    return bf16_bits_to_f32(bf16_bits(x))
+
+
+def fp16_bits(x):
+    """binary16 round-to-nearest-even of fp32 values, as uint16 bit patterns."""
+    x = _f32(x)
+    out = np.empty(x.shape, np.uint16)
+    _c().oracle_fp16_array(_ptr(x), x.size, _ptr(out))
+    return out
+
+
+# ------------------------------------------------- QAT fake quantization (P5)
+
+def qat_scales(W):
+    """P5 "训练时的模拟量化": s_i = max(max_j |W_ij|, 1e-12) / 127 (fp32)."""
+    W = _f32(W)
+    N, K = W.shape
+    s = np.empty(N, np.float32)
+    _c().oracle_qat_scales(_ptr(W), N, K, _ptr(s))
+    return s
+
+
+def qat_codes(W, scales, bits):
+    """P5 "训练时的模拟量化": int6 c = clamp(4*rne(rne(w/s)/4), -128, 124);
+    int8 c = clamp(rne(w/s), -127, 127)."""
+    W = _f32(W)
+    s = _f32(scales)
+    N, K = W.shape
+    c = np.empty((N, K), np.int8)
+    rc = _c().oracle_qat_codes(_ptr(W), N, K, _ptr(s), int(bits), _ptr(c))
+    if rc != 0:
+        raise ValueError("bits must be 6 or 8")
+    return c
+
+
+def dequant(codes, scales):
+    """STE forward value Wq = fl32(c * s)."""
+    c = np.ascontiguousarray(codes, np.int8)
+    s = _f32(scales)
+    N, K = c.shape
+    out = np.empty((N, K), np.float32)
+    _c().oracle_dequant_f32(_ptr(c), _ptr(s), N, K, _ptr(out))
+    return out
+
+
+def operand_bf16_bits(codes, scales):
+    """GEMM operand bf16_rne(fl32(c * s)) as uint16 bits (P5: CastedLinear
+    casts the quantized weight to the activation dtype)."""
+    c = np.ascontiguousarray(codes, np.int8)
+    s = _f32(scales)
+    N, K = c.shape
+    out = np.empty((N, K), np.uint16)
+    _c().oracle_operand_bf16(_ptr(c), _ptr(s), N, K, _ptr(out))
+    return out
+
+
+def quantize_weight(W, bits):
+    """Quantize once (also the recurrence cache: P1 "税 1", shared weights are
+    stored once and quantized once).  Returns codes, scales, the fp32 STE
+    value and the bf16 operand (as float64 for the algebra)."""
+    s = qat_scales(W)
+    c = qat_codes(W, s, bits)
+    op = bf16_bits_to_f32(operand_bf16_bits(c, s)).astype(np.float64)
+    return {"codes": c, "scales": s, "wq": dequant(c, s), "operand": op}
+
+
+# -------------------------------------------------------- dense algebra (fp64)
+
+def _f64(x):
+    return np.asarray(x, dtype=np.float64)
+
+
+def linear_fwd(Wop, X):
+    """P5 CastedLinear forward: Y = X . Wq^T (Wq the bf16 operand)."""
+    return _f64(X) @ _f64(Wop).T
+
+
+def linear_bwd(Wop, X, dY):
+    """STE backward (P5 "训练时的模拟量化": the gradient w.r.t. the fp32 weight
+    is the gradient w.r.t. the quantized weight): dX = dY . Wq, dW = dY^T . X."""
+    dY = _f64(dY)
+    return dY @ _f64(Wop), dY.T @ _f64(X)
+
+
+def relu2(x):
+    x = _f64(x)
+    r = np.maximum(x, 0.0)
+    return r * r
+
+
+def mlp_fwd(Wfc_op, Wproj_op, X):
+    """P5 "架构": MLP(x) = proj(relu(fc(x))^2).  Returns pre, h, Y."""
+    pre = _f64(X) @ _f64(Wfc_op).T
+    h = relu2(pre)
+    return pre, h, h @ _f64(Wproj_op).T
+
+
+def mlp_bwd(Wfc_op, Wproj_op, X, pre, h, dY):
+    """Chain rule through proj, relu^2 (derivative 2*relu(pre)) and fc, with the
+    STE making the quantized weights' gradients the weights' gradients."""
+    dY = _f64(dY)
+    dh = dY @ _f64(Wproj_op)
+    dpre = dh * 2.0 * np.maximum(_f64(pre), 0.0)
+    dWproj = dY.T @ _f64(h)
+    dWfc = dpre.T @ _f64(X)
+    dX = dpre @ _f64(Wfc_op)
+    return dX, dWfc, dWproj
+
+
+def recurrent_core_fwd(q_qkv, q_o, q_fc, q_proj, X, R, d):
+    """Depth-recurrent core (P1 "Stem / Core / Tail", "税 1"): the block's
+    linears, quantized once, applied R times.  Attention is left out, so the
+    O projection reads the query slice of QKV (reading stated in the design
+    notes).  Per application, in fp64:
+        qkv = x Wqkv^T ; x1 = x + q Wo^T ; x2 = x1 + proj(relu(fc(x1))^2)
+    and x is rounded to bf16 between applications (activations are bf16)."""
+    x = _f64(X)
+    for _ in range(R):
+        qkv = x @ q_qkv["operand"].T
+        x1 = x + qkv[:, :d] @ q_o["operand"].T
+        _, _, m = mlp_fwd(q_fc["operand"], q_proj["operand"], x1)
+        x = bf16_round((x1 + m).astype(np.float32)).astype(np.float64)
+    return x
+
+
+def head_mlp_step(q_emb, q_fc, q_proj, X, dLogits):
+    """Tied-head throughput step: Z = MLP(X), logits = Z Wemb^T, then the STE
+    backward of both from the upstream gradient dLogits."""
+    pre, h, Z = mlp_fwd(q_fc["operand"], q_proj["operand"], X)
+    logits = Z @ q_emb["operand"].T
+    dZ, dWemb = linear_bwd(q_emb["operand"], Z, dLogits)
+    dX, dWfc, dWproj = mlp_bwd(q_fc["operand"], q_proj["operand"], X, pre, h, dZ)
+    return {"pre": pre, "h": h, "Z": Z, "logits": logits, "dZ": dZ, "dWemb": dWemb,
+            "dX": dX, "dWfc": dWfc, "dWproj": dWproj}
+
+
+# ---------------------------------------------------------- export quantizer
+
+def row_quantile_abs(row, q=EXPORT_CLIP_Q):
+    """Linear-interpolated quantile of |row| (P5 "后训练量化导出")."""
+    r = _f32(row)
+    return float(_c().oracle_row_quantile_abs(_ptr(r), r.size, float(q)))
+
+
+def export_rows(W, bits, q=EXPORT_CLIP_Q):
+    """P5 "后训练量化导出": per-row clip, int6/int8 codes, fp16 scales.
+    Returns codes (int8), fp16 scale bits (uint16), fp32 scales."""
+    W = _f32(W)
+    rows, cols = W.shape
+    c = np.empty((rows, cols), np.int8)
+    s16 = np.empty(rows, np.uint16)
+    s32 = np.empty(rows, np.float32)
+    rc = _c().oracle_export_rows(_ptr(W), rows, cols, int(bits), float(q), _ptr(c),
+                                 _ptr(s16), _ptr(s32))
+    if rc != 0:
+        raise ValueError("bits must be 6 or 8")
+    return c, s16, s32
+
+
+def dequant_export(codes, scale16_bits):
+    """Roundtrip dequantize: fl32(c * fp32(fp16 scale))."""
+    c = np.ascontiguousarray(codes, np.int8)
+    s = np.ascontiguousarray(scale16_bits, np.uint16)
+    rows, cols = c.shape
+    out = np.empty((rows, cols), np.float32)
+    _c().oracle_dequant_export(_ptr(c), _ptr(s), rows, cols, _ptr(out))
+    return out
+
+
+_BLOCK_RE = re.compile(r"^blocks\.(\d+)\.")
+
+
+def export_state_dict(sd, int6_start=0, int6_end=10, fp16_embed_name="tok_emb.weight",
+                      keep_float_max=KEEP_FLOAT_MAX_NUMEL):
+    """P5 "后训练量化导出" rules, tensor by tensor:
+    non-2D or numel <= keep_float_max -> fp16 passthrough; the tied embedding
+    -> fp16 passthrough; other 2D tensors -> per-row codes, int6 when the
+    tensor belongs to block i with int6_start <= i <= int6_end (inclusive,
+    -1 switches int6 off), else int8."""
+    out = {}
+    for name, t in sd.items():
+        t = _f32(t)
+        if t.ndim != 2 or t.size <= keep_float_max or name == fp16_embed_name:
+            out[name] = {"kind": "fp16", "bits16": fp16_bits(t)}
+            continue
+        m = _BLOCK_RE.match(name)
+        bits = 8
+        if m and int6_start >= 0 and int6_end >= 0:
+            i = int(m.group(1))
+            if int6_start <= i <= int6_end:
+                bits = 6
+        c, s16, _ = export_rows(t, bits)
+        out[name] = {"kind": "int%d" % bits, "codes": c, "scale16": s16}
+    return out
