@@ -1,0 +1,449 @@
+#!/usr/bin/env python
+"""Benchmark of the int6 QAT training hot path on B200.
+
+One step = one QAT training step of the tied int8 head (8192 x 512) over the
+int6 ReLU^2 MLP 512 -> 2048 -> 512 at 65,536 tokens per GPU: per-row weight
+quantization of all three weights, MLP forward (relu^2 fused), logits GEMM,
+the STE backward of both (dX and fp32 dW GEMMs, fused 2*relu(pre)), and with
+N > 1 GPUs the data-parallel all-reduce of the weight gradients over NCCL.
+
+Prints ONE JSON line (rank 0).  Also measured in the same run and reported as
+sub-objects: the export quantizer over the 11-layer d=512 state dict (one
+grouped launch) and the 3x3 recurrent core at d=640, 16x1024 tokens, R=3.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "QAT linear/MLP TFLOP/s (% B200 bf16 peak); export quantizer GB/s (% HBM)"
+T_TOKENS = 65536
+VOCAB, D, H = 8192, 512, 2048
+
+# DRAM bytes per launch of the logits GEMM from an ncu capture, with the hash
+# of the GEMM sources it was taken on (reported only while they still match).
+NCU_TRAFFIC = {"kernel_hash": None, "bytes_per_launch": None}
+
+
+def gemm_source_hash():
+    h = hashlib.sha256()
+    for f in ("gemm_sm100.cu", "gemm_sm100.cuh", "sm100_ptx.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "quantization_aware_tiny_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"],
+                "bf16_tflops_sustained": j.get("bf16_tflops_sustained", j["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index, self.proc = index, None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        if self.proc is None:
+            return None
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in self.out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(mx),
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    return int(os.environ.get("RANK", "0")), ws, int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def make_inputs(seed, device):
+    """Synthetic step inputs of one rank, generated on the host and copied in."""
+    from quantization_aware_tiny_b200 import synthetic as sy
+    c = sy.head_mlp_case(T=T_TOKENS, vocab=VOCAB, d=D, H=H, seed=seed)
+    return {k: (torch.from_numpy(v) if isinstance(v, np.ndarray) else v) for k, v in c.items()}
+
+
+def timed_calls(step, X, dL, ev_pairs, stream):
+    """One step with CUDA events around each single-kernel head GEMM call."""
+    from quantization_aware_tiny_b200 import qat
+    qe, qf, qp = step.q
+    step.quantize(stream)
+    qat.qat_mlp_fwd(X, step.Z, 6, D, H, qfc=qf, qproj=qp, pre_save=step.pre, h_save=step.h,
+                    stream=stream)
+    ev_pairs["logits_fwd"][0].record(stream)
+    qat.qat_linear_fwd(step.Z, step.logits, 8, qw=qe, stream=stream)
+    ev_pairs["logits_fwd"][1].record(stream)
+    ev_pairs["head_dX"][0].record(stream)
+    qat.qat_linear_bwd(step.Z, dL, 8, qw=qe, dX=step.dZ, stream=stream)
+    ev_pairs["head_dX"][1].record(stream)
+    ev_pairs["head_dW"][0].record(stream)
+    qat.qat_linear_bwd(step.Z, dL, 8, dW=step.dWemb, N=VOCAB, K=D, stream=stream)
+    ev_pairs["head_dW"][1].record(stream)
+    qat.qat_mlp_bwd(X, step.pre, step.h, step.dZ, 6, D, H, qfc=qf, qproj=qp, dX=step.dX,
+                    dWfc=step.dWfc, dWproj=step.dWproj, workspace=step.ws, stream=stream)
+
+
+def run_ours(args):
+    from quantization_aware_tiny_b200 import qat, steps
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+    stream = torch.cuda.current_stream()
+    inp = make_inputs(seed=rank, device=dev)
+    W = {k: inp[k].to(dev) for k in ("Wemb", "Wfc", "Wproj")}
+    X, dL = inp["X"].to(dev), inp["dLogits"].to(dev)
+    step = steps.HeadMlpStep(W["Wemb"], W["Wfc"], W["Wproj"], T_TOKENS)
+    flops_step = step.flops_per_token() * T_TOKENS
+    names = ("logits_fwd", "head_dX", "head_dW")
+    per_step_events = []
+
+    def one(i, timed):
+        if timed:
+            ev = {n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for n in names}
+            per_step_events.append(ev)
+            timed_calls(step, X, dL, ev, stream)
+        else:
+            step.step(X, dL, stream)
+        if pg is not None:
+            for g in step.grads():
+                pg.all_reduce(g)
+
+    for i in range(args.warmup):
+        one(i, False)
+    if pg is not None:
+        pg.barrier()
+    torch.cuda.synchronize()
+    n0 = qat.launch_count()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            one(i, True)
+        end.record(stream)
+        torch.cuda.synchronize()
+    if pg is not None:
+        pg.barrier()
+    launches = qat.launch_count() - n0
+    ms = start.elapsed_time(end)
+    if pg is not None:
+        t = torch.tensor([ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms = float(t.item())
+    err = qat.device_error()
+    value = flops_step * world * args.steps / (ms * 1e-3) / 1e12
+
+    # per-kernel durations of the head GEMMs (same stream, inside the timed region)
+    kt = {n: statistics.mean(e[n][0].elapsed_time(e[n][1]) for e in per_step_events) for n in names}
+    dom = max(kt, key=kt.get)
+    kflops = {"logits_fwd": 2.0 * T_TOKENS * VOCAB * D, "head_dX": 2.0 * T_TOKENS * VOCAB * D,
+              "head_dW": 2.0 * T_TOKENS * VOCAB * D}
+    pk = peaks()
+    achieved = kflops[dom] / (kt[dom] * 1e-3) / 1e12
+    traffic = (NCU_TRAFFIC["bytes_per_launch"]
+               if NCU_TRAFFIC["kernel_hash"] == gemm_source_hash() else None)
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1),
+                "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                "frac": round(achieved / pk["bf16_tflops_sustained"], 4), "traffic": traffic,
+                "peak_kind": "sustained bf16 (%s)" % pk["source"],
+                "kernel_ms": {k: round(v, 4) for k, v in kt.items()}}
+
+    out = None
+    if rank == 0:
+        out = {"metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+               "steps": args.steps, "warmup": args.warmup,
+               "ms_per_step": round(ms / args.steps, 4), "higher_is_better": True,
+               "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+               "data": "synthetic (seeded N(0,0.02) weights, N(0,1) bf16 activations, "
+                       "N(0,0.01) bf16 upstream grads)",
+               "config": {"workload": "tied int8 head 8192x512 + int6 ReLU^2 MLP 512-2048-512, "
+                                      "fwd + STE bwd, 65536 tokens per GPU",
+                          "tokens_per_gpu": T_TOKENS, "vocab": VOCAB, "d": D, "mlp_hidden": H,
+                          "head_bits": 8, "mlp_bits": 6, "global_batch_tokens": T_TOKENS * world,
+                          "parallelism": "dp%d" % world,
+                          "l2": "inputs larger than L2 (dLogits 1 GiB per step)"},
+               "frac_of_peak": round(value / pk["bf16_tflops_sustained"], 4),
+               "roofline": roofline, "gpu_launches": launches, "device_error": err}
+        out["clocks"] = clk.summary()
+    # end-to-end through the C ABI with host buffers (all ranks take the same steps)
+    e2e = measure_e2e(step, inp, dev, stream, args, pg, flops_step, world)
+    if rank == 0:
+        out["e2e"] = e2e
+        if world == 1:
+            out["export"] = measure_export(dev, stream, pk)
+            out["recurrent_core"] = measure_core(dev, stream, pk)
+            out["cpu_baseline"] = cpu_baseline()
+        print(json.dumps(out), flush=True)
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+def measure_e2e(step, inp, dev, stream, args, pg, flops_step, world):
+    """Same step with the inputs copied from pinned host memory and the weight
+    gradients read back every step, inside the timed region."""
+    hX = inp["X"].pin_memory()
+    hdL = inp["dLogits"].pin_memory()
+    X = torch.empty_like(hX, device=dev)
+    dL = torch.empty_like(hdL, device=dev)
+    hg = [torch.empty(g.shape, dtype=g.dtype, pin_memory=True) for g in step.grads()]
+    steps_e2e = max(3, min(args.steps, 10))
+
+    def one():
+        X.copy_(hX, non_blocking=True)
+        dL.copy_(hdL, non_blocking=True)
+        step.step(X, dL, stream)
+        if pg is not None:
+            for g in step.grads():
+                pg.all_reduce(g)
+        for h, g in zip(hg, step.grads()):
+            h.copy_(g, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    if pg is not None:
+        pg.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps_e2e):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    if pg is not None:
+        t = torch.tensor([ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms = float(t.item())
+    h2d = hX.numel() * 2 + hdL.numel() * 2
+    d2h = sum(g.numel() * 4 for g in hg)
+    return {"value": round(flops_step * world * steps_e2e / (ms * 1e-3) / 1e12, 2),
+            "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "steps": steps_e2e, "ms_per_step": round(ms / steps_e2e, 3)}
+
+
+def flush_l2(buf):
+    buf.add_(1)
+
+
+def measure_export(dev, stream, pk):
+    """Export quantizer over the 11-layer d=512 state dict: one grouped launch,
+    L2 flushed (256 MB write) before every timed launch."""
+    from quantization_aware_tiny_b200 import export as qexport
+    from quantization_aware_tiny_b200 import qat
+    from quantization_aware_tiny_b200 import synthetic as sy
+    sd = {k: torch.from_numpy(v).to(dev) for k, v in sy.state_dict_case().items()}
+    out = qexport.export_state_dict(sd)  # allocates outputs once
+    descs = []
+    algo = 0
+    for name, mode in qexport.plan(sd):
+        t = sd[name]
+        o = out[name]
+        if mode == qat.QAT_EXPORT_FP16:
+            descs.append((t.reshape(-1), mode, o["values"], None))
+            algo += t.numel() * (4 + 2)
+        else:
+            descs.append((t, mode, o["codes"], o["scale16"]))
+            algo += t.numel() * (4 + 1) + t.shape[0] * 2
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+    times = []
+    for i in range(25):
+        flush_l2(flush)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        qat.quantize_export_batch(descs, stream=stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i >= 5:
+            times.append(a.elapsed_time(b))
+    ms = statistics.median(times)
+    gbs = algo / (ms * 1e-3) / 1e9
+    return {"value": round(gbs, 1), "unit": "GB/s", "ms": round(ms, 4),
+            "algorithmic_bytes": algo, "launches_per_export": 1,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(gbs / pk["hbm_gbs"], 4),
+                         "peak_kind": "copy bandwidth (%s)" % pk["source"]},
+            "workload": "11 blocks x (Q,K,V,O,fc,proj) d=512 MLP3x int6 + tied emb 1024x512 "
+                        "+ small tensors fp16 passthrough; L2 flushed before each launch"}
+
+
+def measure_core(dev, stream, pk):
+    """3x3 recurrent core at d=640 (QKV/O + MLP 1920), 16x1024 tokens, R=3."""
+    from quantization_aware_tiny_b200 import steps
+    from quantization_aware_tiny_b200 import synthetic as sy
+    c = sy.recurrent_core_case(T=16384)
+    w = {k: torch.from_numpy(c[k]).to(dev) for k in ("Wq", "Wk", "Wv", "Wo", "Wfc", "Wproj")}
+    core = steps.RecurrentCore(w["Wq"], w["Wk"], w["Wv"], w["Wo"], w["Wfc"], w["Wproj"], 6)
+    x0 = c["X"].to(dev)
+    x = x0.clone()
+    for _ in range(3):
+        x.copy_(x0)
+        core.forward(x, 3, stream)
+    times = []
+    for _ in range(10):
+        x.copy_(x0)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        core.forward(x, 3, stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    ms = statistics.median(times)
+    tf = core.flops(16384, 3) / (ms * 1e-3) / 1e12
+    return {"value": round(tf, 1), "unit": "TFLOP/s", "ms": round(ms, 4),
+            "frac": round(tf / pk["bf16_tflops_sustained"], 4),
+            "workload": "3x3 core d=640 8H/4KV hd80, QKV+O+MLP1920, 16384 tokens, R=3, "
+                        "weights quantized once"}
+
+
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_step_time(T, seed=0):
+    """The CPU oracle's version of one step on T tokens (time in seconds)."""
+    import oracle as o
+    from quantization_aware_tiny_b200 import synthetic as sy
+    c = sy.head_mlp_case(T=T, vocab=VOCAB, d=D, H=H, seed=seed)
+    X, dL = c["X"].float().numpy(), c["dLogits"].float().numpy()
+    t0 = time.perf_counter()
+    qe = o.quantize_weight(c["Wemb"], 8)
+    qf = o.quantize_weight(c["Wfc"], 6)
+    qp = o.quantize_weight(c["Wproj"], 6)
+    o.head_mlp_step(qe, qf, qp, X, dL)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(target_s=12.0):
+    """The oracle, as it stands, on a bounded sample of the step's tokens."""
+    t_small = oracle_step_time(512)
+    T = int(min(T_TOKENS, max(512, 512 * target_s / max(t_small, 1e-3))))
+    T = max(512, T // 512 * 512)
+    dt = oracle_step_time(T)
+    flops = 3 * 2.0 * D * (VOCAB + 2 * H) * T
+    return {"value": round(flops / dt / 1e12, 5), "unit": "TFLOP/s", "cores": _threads(),
+            "kind": "oracle",
+            "sample": "one step on %d of the 65536 tokens (quantize + fwd + STE bwd, numpy "
+                      "fp64 GEMMs, scalar C quantizer), %.1f s" % (T, dt)}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    # per-step sample sized so the whole --steps/--warmup run stays within minutes
+    t_small = oracle_step_time(256)
+    per_step = min(6.0, 150.0 / max(1, args.steps + args.warmup))
+    T = int(min(T_TOKENS, max(256, 256 * per_step / max(t_small, 1e-3))))
+    T = max(256, T // 256 * 256)
+    for i in range(args.warmup):
+        oracle_step_time(T, seed=i)
+    tot = 0.0
+    for i in range(args.steps):
+        tot += oracle_step_time(T, seed=100 + i)
+    flops = 3 * 2.0 * D * (VOCAB + 2 * H) * T
+    value = flops * args.steps / tot / 1e12
+    cb = {"value": round(value, 5), "unit": "TFLOP/s", "cores": _threads(), "kind": "oracle",
+          "sample": "%d tokens per step of the 65536-token step (quantize + fwd + STE bwd)" % T}
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(tot / args.steps * 1e3, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "tied int8 head 8192x512 + int6 ReLU^2 MLP 512-2048-512, "
+                               "fwd + STE bwd, 65536 tokens per GPU",
+                   "tokens_per_step_sample": T, "parallelism": "dp%d" % world},
+        "cpu_baseline": cb,
+        "e2e": {"value": round(value, 5), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0}}), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

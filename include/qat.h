@@ -1,0 +1,180 @@
+/*
+ * qat.h -- C ABI of the B200 (sm_100a) int6 quantization-aware linear, ReLU^2
+ * MLP, recurrent-core weight cache and export quantizer.
+ *
+ * Page references used below (title, section):
+ *   [P5] "parameter-golf 16MB 极限压缩实战：11L MLP3x + Int6 QAT + zstd-22 记录详解"
+ *   [P1] "Depth Recurrence + Mixed-Precision Quant" write-up of PR #363
+ *
+ * Conventions shared by every call
+ *   - Every pointer is a caller-owned DEVICE pointer unless stated otherwise,
+ *     row-major and contiguous (a leading-dimension argument says otherwise),
+ *     16-byte aligned.  Nothing is retained after a call returns.
+ *   - bf16 / fp16 tensors are passed as their 16-bit storage (qat_bf16 /
+ *     qat_fp16).  fp32 is IEEE binary32.
+ *   - Every call is asynchronous on the given CUDA stream and never
+ *     synchronizes.  The library never allocates device memory: scratch
+ *     comes from the caller's workspace, sized by qat_workspace_size().
+ *   - Arguments are validated on the host before any launch; on error
+ *     nothing is launched and a QAT_ERR_* code is returned.
+ *   - bits = 6 selects the int6 grid (multiples of 4 in [-128,124], 64
+ *     levels in an int8 container); bits = 8 the int8 grid [-127,127].
+ *   - Shapes: feature dimensions (N, K, d, H, cols) must be multiples of 8
+ *     (16-byte rows for bf16, as the tensor-memory-access engine requires);
+ *     the token count T may be anything >= 0 (T = 0 is a no-op).
+ *   - Bounded device waits: every wait inside a kernel gives up after ~2 s,
+ *     records QAT_ERR_TIMEOUT in a device flag and lets the kernel return;
+ *     qat_device_error() reads and clears that flag.
+ */
+#ifndef QAT_B200_H
+#define QAT_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* qat_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+typedef uint16_t qat_bf16;                /* bfloat16 bit pattern */
+typedef uint16_t qat_fp16;                /* IEEE binary16 bit pattern */
+
+enum {
+  QAT_OK = 0,
+  QAT_ERR_ARG = 1,        /* null pointer, non-positive size, bits not in {6,8} */
+  QAT_ERR_ALIGN = 2,      /* a pointer is not 16-byte aligned */
+  QAT_ERR_SHAPE = 3,      /* a feature dimension is not a multiple of 8, or too large */
+  QAT_ERR_WORKSPACE = 4,  /* workspace missing or smaller than qat_workspace_size() */
+  QAT_ERR_CUDA = 5,       /* a CUDA runtime call or kernel launch failed */
+  QAT_ERR_TIMEOUT = 6,    /* a bounded device wait gave up (see qat_device_error) */
+  QAT_ERR_UNSUPPORTED = 7 /* no sm_100 device, or driver entry point missing */
+};
+
+/* Human-readable text of a QAT_* code (static storage, never NULL). */
+const char* qat_strerror(int code);
+
+/* Number of kernels this library has launched in this process (all streams). */
+int64_t qat_launch_count(void);
+
+/* Synchronizes `stream`, then returns QAT_OK, or QAT_ERR_TIMEOUT if any kernel
+ * of this library recorded a timed-out device wait since the last call
+ * (the flag is cleared), or QAT_ERR_CUDA if the stream reports an error. */
+int qat_device_error(qat_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Quantized weight: the STE forward operand of one weight matrix.
+ * Produced by qat_quantize_weights(); it is also the recurrence cache of [P1]
+ * "税 1" (shared weights are stored once and quantized once, then reused by
+ * every application of the block).
+ *   operand : [N,K] bf16 = bf16_rne(fl32(c * s)), required by every GEMM call
+ *   scales  : [N] fp32 per-row scales s (may be NULL)
+ *   codes   : [N,K] int8 codes c (may be NULL)
+ * ------------------------------------------------------------------------- */
+typedef struct qat_qweight {
+  const qat_bf16* operand;
+  const float* scales;
+  const int8_t* codes;
+  int32_t N, K, bits;
+} qat_qweight;
+
+/* [P5] "训练时的模拟量化": per row i of W [N,K] fp32,
+ *   amax_i = max(max_j |W_ij|, 1e-12)      (floor from [P1] "修复" code)
+ *   s_i    = fl32(amax_i / 127)             (IEEE division)
+ *   int6:  c = clamp(4*rne(rne(fl32(W/s))/4), -128, 124);  int8: clamp(rne(W/s), -127, 127)
+ *   operand = bf16_rne(fl32(c * s))         (the STE forward value cast to bf16)
+ * Outputs: scales [N] (required), codes [N,K] (nullable), operand [N,K] (nullable).
+ * Bit-exact with the CPU oracle. */
+int qat_quantize_weights(const float* W, int32_t N, int32_t K, int32_t bits, int8_t* codes,
+                         float* scales, qat_bf16* operand, qat_stream_t stream);
+
+/* Workspace sizes (bytes) for the calls below.  `raw_weights` != 0 means the
+ * call is given fp32 weights to quantize itself (the workspace then also
+ * holds the bf16 operands and scales); 0 means qat_qweight operands. */
+enum { QAT_OP_LINEAR_FWD = 1, QAT_OP_LINEAR_BWD = 2, QAT_OP_MLP_FWD = 3, QAT_OP_MLP_BWD = 4 };
+size_t qat_workspace_size(int32_t op, int32_t N_or_d, int32_t K_or_H, int64_t T,
+                          int32_t raw_weights);
+
+/* [P5] CastedLinear forward with QAT: Y[T,N] = bf16( X[T,K] . Wq^T (+ residual) ),
+ * fp32 accumulation on the tensor cores.  Weights: either W (fp32 [N,K],
+ * quantized inside the call into the workspace) or qw (pre-quantized; W must
+ * then be NULL).  ldx = row stride of X in elements (0 -> K); residual
+ * (nullable) is [T,N] bf16 and may alias Y exactly. */
+int qat_linear_fwd(const float* W, const qat_qweight* qw, int32_t N, int32_t K, int32_t bits,
+                   const qat_bf16* X, int64_t ldx, int64_t T, const qat_bf16* residual,
+                   qat_bf16* Y, void* workspace, size_t ws_bytes, qat_stream_t stream);
+
+/* STE backward of qat_linear_fwd ([P5]: the forward uses the quantized weight,
+ * the gradient flows to the fp32 weight unchanged):
+ *   dX[T,K] = bf16( dY[T,N] . Wq )            (nullable)
+ *   dW[N,K] (+)= dY^T . X   in fp32            (nullable; accumulate_dW != 0 adds
+ *                                               into dW, e.g. over R recurrent uses)
+ * dX needs W or qw; dW needs neither. */
+int qat_linear_bwd(const float* W, const qat_qweight* qw, int32_t N, int32_t K, int32_t bits,
+                   const qat_bf16* X, const qat_bf16* dY, int64_t T, qat_bf16* dX, float* dW,
+                   int32_t accumulate_dW, void* workspace, size_t ws_bytes, qat_stream_t stream);
+
+/* [P5] "架构" ReLU^2 MLP forward, both linears int6/int8 QAT:
+ *   pre = X . Wfc_q^T  [T,H];  h = relu(pre)^2 (fused in the fc epilogue, from the
+ *   fp32 accumulator);  Y = bf16(h . Wproj_q^T (+ residual))  [T,d].
+ * Weights: (Wfc [H,d], Wproj [d,H]) fp32, or (qfc, qproj).  pre_save [T,H]
+ * (nullable) and h_save [T,H] (nullable; the workspace holds h otherwise)
+ * keep the activations for the backward.  residual may alias Y exactly. */
+int qat_mlp_fwd(const float* Wfc, const float* Wproj, const qat_qweight* qfc,
+                const qat_qweight* qproj, int32_t d, int32_t H, int32_t bits, const qat_bf16* X,
+                int64_t T, const qat_bf16* residual, qat_bf16* Y, qat_bf16* pre_save,
+                qat_bf16* h_save, void* workspace, size_t ws_bytes, qat_stream_t stream);
+
+/* STE backward of qat_mlp_fwd from the saved pre and h:
+ *   dh = dY . Wproj_q;  dpre = dh * 2*relu(pre) (fused in the dh epilogue);
+ *   dWproj (+)= dY^T . h;  dWfc (+)= dpre^T . X;  dX = dpre . Wfc_q.
+ * dX, dWfc, dWproj may each be NULL.  The workspace holds dpre [T,H] bf16. */
+int qat_mlp_bwd(const float* Wfc, const float* Wproj, const qat_qweight* qfc,
+                const qat_qweight* qproj, int32_t d, int32_t H, int32_t bits, const qat_bf16* X,
+                const qat_bf16* pre, const qat_bf16* h, const qat_bf16* dY, int64_t T,
+                qat_bf16* dX, float* dWfc, float* dWproj, int32_t accumulate_dW,
+                void* workspace, size_t ws_bytes, qat_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Export quantizer, [P5] "后训练量化导出".
+ * Per row of W [rows, cols] fp32:
+ *   clip   = linear-interpolated quantile of |w| at q = 0.9999984: sorted
+ *            values v, pos = q*(cols-1) (double), lo = floor(pos), hi = lo+1,
+ *            clip = fl32(v_lo + fl32(fl32(pos-lo) * fl32(v_hi - v_lo)))
+ *   s32    = fl32(max(clip, 1e-12) / 127)
+ *   codes  = the training grid (bits 6 or 8) applied to clamp(w, -clip, clip) with s32
+ *   scales = fp16_rne(s32)
+ * Only the top (cols - lo) order statistics of |w| matter; rows longer than
+ * 625,001 columns (where more than the top two would) return QAT_ERR_SHAPE.
+ * Bit-exact with the CPU oracle.
+ * ------------------------------------------------------------------------- */
+int quantize_rows_export(const float* W, int64_t rows, int64_t cols, int32_t bits,
+                         int8_t* codes, qat_fp16* scales, qat_stream_t stream);
+
+/* One grouped launch over a whole state dict.  `descs` is a HOST array of n
+ * descriptors (n <= QAT_EXPORT_MAX_DESCS); mode 6 or 8 quantizes rows as
+ * above into dst (int8 codes) and scales; mode QAT_EXPORT_FP16 converts src
+ * to fp16 (rne) into dst (the passthrough of non-2D, small and tied-embedding
+ * tensors; scales unused).  The caller applies the passthrough rules. */
+#define QAT_EXPORT_FP16 16
+#define QAT_EXPORT_MAX_DESCS 256
+typedef struct qat_export_desc {
+  const float* src;
+  int64_t rows, cols;
+  int32_t mode;
+  int32_t reserved;
+  void* dst;
+  qat_fp16* scales;
+} qat_export_desc;
+int quantize_export_batch(const qat_export_desc* descs, int32_t n, qat_stream_t stream);
+
+/* Roundtrip dequantize ([P5] "后训练量化导出", roundtrip re-evaluation):
+ *   out = fl32(c * fp32(scale_fp16))  as fp32 (out_dtype 0) or bf16_rne of it (1). */
+enum { QAT_DTYPE_F32 = 0, QAT_DTYPE_BF16 = 1 };
+int dequantize_rows(const int8_t* codes, const qat_fp16* scales, int64_t rows, int64_t cols,
+                    int32_t out_dtype, void* out, qat_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QAT_B200_H */

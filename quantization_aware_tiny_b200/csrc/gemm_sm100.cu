@@ -1,0 +1,483 @@
+// Persistent, warp-specialized tcgen05 GEMM for sm_100a.
+//
+//   warp 0      : TMA producer (one elected lane) filling a STAGES-deep ring of
+//                 128B-swizzled A/B tiles in shared memory
+//   warp 1      : TMEM allocator + MMA issuer (one lane issues tcgen05.mma,
+//                 128 x BN x 16 per instruction, fp32 accumulator in TMEM)
+//   warps 2..5  : epilogue; warp w reads TMEM lanes 32*(w%4)..+31 (its rows),
+//                 applies the fused epilogue and stores to global memory
+//
+// Two accumulator buffers in TMEM (2*BN columns) let the epilogue of tile i
+// overlap the main loop of tile i+1.  Tiles are 128 x BN x 64; split-K (for
+// the long-K weight-gradient GEMMs) adds fp32 partial sums atomically.
+#include <algorithm>
+#include <mutex>
+
+#include "gemm_sm100.cuh"
+#include "sm100_ptx.cuh"
+
+namespace qat {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int kThreads = 192;
+
+template <int BN>
+struct Cfg {
+  static constexpr int STAGES = (BN == 256) ? 4 : 6;
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TMEM_COLS = 2 * BN;  // 256 or 512: powers of two as required
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+};
+
+struct KArgs {
+  int M, N;
+  int num_m_blk, num_n_blk, splits, kblk_total, kblk_per_split, num_tiles;
+  void* D;
+  int64_t ldd;
+  void* D2;
+  int64_t ldd2;
+  const __nv_bfloat16* R;
+  int64_t ldr;
+  int accumulate;
+  int* err;
+};
+
+__device__ __forceinline__ float bf2f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);  // .x = a (low half), .y = b
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Apply the epilogue to 8 consecutive accumulator columns (one 16-byte group
+// of bf16 output) of one row.
+template <int EPI>
+__device__ __forceinline__ void epi_group8(const KArgs& p, int64_t row, int64_t col,
+                                           const float* v) {
+  if constexpr (EPI == EPI_BF16 || EPI == EPI_BF16_RESID || EPI == EPI_DRELU2) {
+    float o[8];
+    if constexpr (EPI == EPI_BF16) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i] = v[i];
+    } else {
+      uint4 rr = *reinterpret_cast<const uint4*>(p.R + row * p.ldr + col);
+      const __nv_bfloat16* r = reinterpret_cast<const __nv_bfloat16*>(&rr);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if constexpr (EPI == EPI_BF16_RESID) {
+          o[i] = __fadd_rn(v[i], bf2f(r[i]));
+        } else {
+          const float t = fmaxf(bf2f(r[i]), 0.0f);
+          o[i] = __fmul_rn(__fmul_rn(v[i], t), 2.0f);
+        }
+      }
+    }
+    uint4 w;
+    w.x = pack_bf16(o[0], o[1]);
+    w.y = pack_bf16(o[2], o[3]);
+    w.z = pack_bf16(o[4], o[5]);
+    w.w = pack_bf16(o[6], o[7]);
+    *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.D) + row * p.ldd + col) = w;
+  } else if constexpr (EPI == EPI_RELU2) {
+    if (p.D != nullptr) {
+      uint4 w;
+      w.x = pack_bf16(v[0], v[1]);
+      w.y = pack_bf16(v[2], v[3]);
+      w.z = pack_bf16(v[4], v[5]);
+      w.w = pack_bf16(v[6], v[7]);
+      *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.D) + row * p.ldd + col) = w;
+    }
+    float h[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float r = fmaxf(v[i], 0.0f);
+      h[i] = __fmul_rn(r, r);
+    }
+    uint4 w;
+    w.x = pack_bf16(h[0], h[1]);
+    w.y = pack_bf16(h[2], h[3]);
+    w.z = pack_bf16(h[4], h[5]);
+    w.w = pack_bf16(h[6], h[7]);
+    *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.D2) + row * p.ldd2 + col) = w;
+  } else if constexpr (EPI == EPI_F32) {
+    float* d = reinterpret_cast<float*>(p.D) + row * p.ldd + col;
+    float4 a = make_float4(v[0], v[1], v[2], v[3]);
+    float4 b = make_float4(v[4], v[5], v[6], v[7]);
+    if (p.accumulate) {
+      const float4 oa = reinterpret_cast<const float4*>(d)[0];
+      const float4 ob = reinterpret_cast<const float4*>(d)[1];
+      a.x = __fadd_rn(a.x, oa.x); a.y = __fadd_rn(a.y, oa.y);
+      a.z = __fadd_rn(a.z, oa.z); a.w = __fadd_rn(a.w, oa.w);
+      b.x = __fadd_rn(b.x, ob.x); b.y = __fadd_rn(b.y, ob.y);
+      b.z = __fadd_rn(b.z, ob.z); b.w = __fadd_rn(b.w, ob.w);
+    }
+    reinterpret_cast<float4*>(d)[0] = a;
+    reinterpret_cast<float4*>(d)[1] = b;
+  } else {  // EPI_F32_ATOMIC
+    float* d = reinterpret_cast<float*>(p.D) + row * p.ldd + col;
+    atomicAdd(reinterpret_cast<float4*>(d), make_float4(v[0], v[1], v[2], v[3]));
+    atomicAdd(reinterpret_cast<float4*>(d) + 1, make_float4(v[4], v[5], v[6], v[7]));
+  }
+}
+
+template <int BN, bool A_MN, bool B_MN, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const KArgs p) {
+  using C = Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + C::STAGES * C::A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* tfull = empty + C::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* mma_done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* prod_pos = const_cast<int*>(abort_flag) + 1;  // producer ring position at exit
+  int* mma_pos = prod_pos + 1;                        // MMA ring position at exit
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    *prod_pos = 0;
+    *mma_pos = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      int stage = 0, pos = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+        const int nb = tile % p.num_n_blk;
+        const int mb = (tile / p.num_n_blk) % p.num_m_blk;
+        const int sp = tile / (p.num_n_blk * p.num_m_blk);
+        const int kb0 = sp * p.kblk_per_split;
+        const int kb1 = min(kb0 + p.kblk_per_split, p.kblk_total);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+          const int k0 = kb * BK;
+          uint8_t* a_dst = sA + stage * C::A_BYTES;
+          uint8_t* b_dst = sB + stage * C::B_BYTES;
+          if constexpr (!A_MN) {
+            tma_load_2d(&tmA, &full[stage], a_dst, k0, mb * BM);
+          } else {
+            tma_load_2d(&tmA, &full[stage], a_dst, mb * BM, k0);
+            tma_load_2d(&tmA, &full[stage], a_dst + 64 * 128, mb * BM + 64, k0);
+          }
+          if constexpr (!B_MN) {
+            tma_load_2d(&tmB, &full[stage], b_dst, k0, nb * BN);
+          } else {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j)
+              tma_load_2d(&tmB, &full[stage], b_dst + j * 64 * 128, nb * BN + j * 64, k0);
+          }
+          ++pos;
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      *prod_pos = pos;
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      constexpr uint32_t IDESC = idesc_bf16(BM, BN, A_MN, B_MN);
+      int stage = 0, pos = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+        const int sp = tile / (p.num_n_blk * p.num_m_blk);
+        const int kb0 = sp * p.kblk_per_split;
+        const int kb1 = min(kb0 + p.kblk_per_split, p.kblk_total);
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, p.err)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sA + stage * C::A_BYTES);
+          const uint32_t b_base = smem_u32(sB + stage * C::B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = A_MN ? sw128_desc(a_base + kk * 2048, 64 * 128, 1024)
+                                     : sw128_desc(a_base + kk * 32, 16, 1024);
+            const uint64_t bd = B_MN ? sw128_desc(b_base + kk * 2048, 64 * 128, 1024)
+                                     : sw128_desc(b_base + kk * 32, 16, 1024);
+            umma_bf16(d_tmem, ad, bd, IDESC, (kb > kb0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[stage]);
+          ++pos;
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      // Wait (bounded) for every MMA this thread issued before TMEM is freed.
+      umma_commit(mma_done);
+      mbar_wait(mma_done, 0, abort_flag, p.err);
+      *mma_pos = pos;
+    }
+  } else {
+    // ------------------------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+      const int nb = tile % p.num_n_blk;
+      const int mb = (tile / p.num_n_blk) % p.num_m_blk;
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err)) break;
+      tc_fence_after();
+      const int64_t row = static_cast<int64_t>(mb) * BM + q * 32 + lane;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(acc * BN);
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(t_row + static_cast<uint32_t>(c0), r);
+        tmem_ld_wait();
+        const int64_t col0 = static_cast<int64_t>(nb) * BN + c0;
+        if (row < p.M) {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const int64_t col = col0 + g * 8;
+            if (col < p.N) epi_group8<EPI>(p, row, col, reinterpret_cast<const float*>(r) + g * 8);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) {
+    // Drain: wait (bounded) for tiles the producer requested but the MMA never
+    // consumed, so no TMA write lands after the block exits.
+    int stage = *mma_pos % C::STAGES;
+    uint32_t phase = static_cast<uint32_t>((*mma_pos / C::STAGES) & 1);
+    const unsigned long long t0 = globaltimer_ns();
+    for (int i = *mma_pos; i < *prod_pos; ++i) {
+      while (!mbar_try_wait(&full[stage], phase))
+        if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+      if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                              const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                              const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn get_encode() {
+  static EncodeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(f);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map: inner dimension `inner` (contiguous), outer `outer`,
+// row stride `ld` elements, box {64, box_outer}, 128-byte swizzle.
+int make_map(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, int64_t ld,
+             int box_outer) {
+  EncodeFn enc = get_encode();
+  if (!enc) return QAT_ERR_UNSUPPORTED;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_outer)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? QAT_OK : QAT_ERR_ARG;
+}
+
+template <int BN, bool A_MN, bool B_MN, int EPI>
+int launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const KArgs& a, cudaStream_t s) {
+  using C = Cfg<BN>;
+  auto kern = gemm_kernel<BN, A_MN, B_MN, EPI>;
+  static bool attr_done = false;  // per instantiation; set before first launch
+  if (!attr_done) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return QAT_ERR_CUDA;
+    attr_done = true;
+  }
+  const int grid = std::max(1, std::min(a.num_tiles, sm_count()));
+  kern<<<grid, kThreads, C::SMEM_BYTES, s>>>(ma, mb, a);
+  count_launch();
+  return cuda_status(cudaGetLastError());
+}
+
+template <int BN>
+int dispatch_bn(const GemmDesc& g, const CUtensorMap& ma, const CUtensorMap& mb, const KArgs& a,
+                int epi, cudaStream_t s) {
+  if (!g.a_mn && !g.b_mn) {
+    switch (epi) {
+      case EPI_BF16: return launch_t<BN, false, false, EPI_BF16>(ma, mb, a, s);
+      case EPI_BF16_RESID: return launch_t<BN, false, false, EPI_BF16_RESID>(ma, mb, a, s);
+      case EPI_RELU2: return launch_t<BN, false, false, EPI_RELU2>(ma, mb, a, s);
+      default: break;
+    }
+  } else if (!g.a_mn && g.b_mn) {
+    switch (epi) {
+      case EPI_BF16: return launch_t<BN, false, true, EPI_BF16>(ma, mb, a, s);
+      case EPI_DRELU2: return launch_t<BN, false, true, EPI_DRELU2>(ma, mb, a, s);
+      default: break;
+    }
+  } else if (g.a_mn && g.b_mn) {
+    switch (epi) {
+      case EPI_F32: return launch_t<BN, true, true, EPI_F32>(ma, mb, a, s);
+      case EPI_F32_ATOMIC: return launch_t<BN, true, true, EPI_F32_ATOMIC>(ma, mb, a, s);
+      default: break;
+    }
+  }
+  return QAT_ERR_ARG;  // combination not instantiated
+}
+
+// Split count for the fp32 weight-gradient GEMMs: minimise the makespan
+// ceil(tiles*s / SMs) * ceil(kblk / s), preferring fewer splits.
+int choose_splits(int tiles, int kblk, int sms) {
+  int best_s = 1;
+  long long best = -1;
+  for (int s = 1; s <= std::min(kblk, 64); ++s) {
+    const long long waves = (static_cast<long long>(tiles) * s + sms - 1) / sms;
+    const long long cost = waves * ((kblk + s - 1) / s);
+    if (best < 0 || cost < best) {
+      best = cost;
+      best_s = s;
+    }
+  }
+  return best_s;
+}
+
+}  // namespace
+
+int launch_gemm(const GemmDesc& g, cudaStream_t stream) {
+  if (g.M < 0 || g.N <= 0 || g.K <= 0) return QAT_ERR_ARG;
+  if (g.M == 0) return QAT_OK;
+  if (!g.A || !g.B || (!g.D && g.epi != EPI_RELU2)) return QAT_ERR_ARG;
+  if (g.epi == EPI_RELU2 && !g.D2) return QAT_ERR_ARG;
+  if ((g.epi == EPI_BF16_RESID || g.epi == EPI_DRELU2) && !g.R) return QAT_ERR_ARG;
+  if (!aligned16(g.A) || !aligned16(g.B) || (g.D && !aligned16(g.D)) || (g.D2 && !aligned16(g.D2)) ||
+      (g.R && !aligned16(g.R)))
+    return QAT_ERR_ALIGN;
+  if ((g.N & 7) || (g.lda & 7) || (g.ldb & 7) || (g.ldd & 7) || (g.D2 && (g.ldd2 & 7)) ||
+      (g.R && (g.ldr & 7)))
+    return QAT_ERR_SHAPE;
+  if (g.M > (1ll << 31) - 256 || g.N > (1 << 30) || g.K > (1ll << 31) - 256) return QAT_ERR_SHAPE;
+
+  // N tile: 256 unless 128 wastes fewer padded columns.
+  const int64_t pad256 = (g.N + 255) / 256 * 256 - g.N;
+  const int64_t pad128 = (g.N + 127) / 128 * 128 - g.N;
+  const int BN = (pad128 < pad256) ? 128 : 256;
+
+  KArgs a{};
+  a.M = static_cast<int>(g.M);
+  a.N = static_cast<int>(g.N);
+  a.num_m_blk = static_cast<int>((g.M + BM - 1) / BM);
+  a.num_n_blk = static_cast<int>((g.N + BN - 1) / BN);
+  a.kblk_total = static_cast<int>((g.K + BK - 1) / BK);
+  a.splits = 1;
+  a.D = g.D;
+  a.ldd = g.ldd;
+  a.D2 = g.D2;
+  a.ldd2 = g.ldd2;
+  a.R = reinterpret_cast<const __nv_bfloat16*>(g.R);
+  a.ldr = g.ldr;
+  a.accumulate = g.accumulate ? 1 : 0;
+  a.err = device_error_ptr();
+
+  int epi = g.epi;
+  if (epi == EPI_F32 || epi == EPI_F32_ATOMIC) {
+    const int tiles = a.num_m_blk * a.num_n_blk;
+    int s = choose_splits(tiles, a.kblk_total, sm_count());
+    a.kblk_per_split = (a.kblk_total + s - 1) / s;
+    s = (a.kblk_total + a.kblk_per_split - 1) / a.kblk_per_split;  // no empty split
+    a.splits = s;
+    if (s > 1) {
+      if (!g.accumulate) {
+        cudaError_t e = (g.ldd == g.N)
+                            ? cudaMemsetAsync(g.D, 0, static_cast<size_t>(g.M * g.N) * 4, stream)
+                            : cudaMemset2DAsync(g.D, static_cast<size_t>(g.ldd) * 4, 0,
+                                                static_cast<size_t>(g.N) * 4,
+                                                static_cast<size_t>(g.M), stream);
+        if (e != cudaSuccess) return QAT_ERR_CUDA;
+      }
+      epi = EPI_F32_ATOMIC;
+    } else {
+      epi = EPI_F32;
+    }
+  } else {
+    a.kblk_per_split = a.kblk_total;
+  }
+  const int64_t tiles64 = static_cast<int64_t>(a.num_m_blk) * a.num_n_blk * a.splits;
+  if (tiles64 > (1ll << 31) - 1) return QAT_ERR_SHAPE;
+  a.num_tiles = static_cast<int>(tiles64);
+
+  CUtensorMap ma, mb;
+  int rc = g.a_mn ? make_map(&ma, g.A, g.M, g.K, g.lda, 64)
+                  : make_map(&ma, g.A, g.K, g.M, g.lda, BM);
+  if (rc) return rc;
+  rc = g.b_mn ? make_map(&mb, g.B, g.N, g.K, g.ldb, 64) : make_map(&mb, g.B, g.K, g.N, g.ldb, BN);
+  if (rc) return rc;
+  return BN == 256 ? dispatch_bn<256>(g, ma, mb, a, epi, stream)
+                   : dispatch_bn<128>(g, ma, mb, a, epi, stream);
+}
+
+}  // namespace qat

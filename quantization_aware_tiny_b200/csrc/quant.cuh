@@ -1,0 +1,40 @@
+// Host interface of the quantizer kernels (not part of the C ABI).
+#pragma once
+
+#include "common.cuh"
+
+namespace qat {
+
+// One export descriptor as the kernel sees it.  Quantized tensors use one
+// warp per row; fp16 passthrough tensors are cut into "rows" of `cols`
+// elements of a flat array of `numel` elements.
+struct ExportDescDev {
+  const float* src;
+  void* dst;
+  __half* scales;
+  int64_t rows, cols, numel;
+  int64_t row_begin;  // first global row of this descriptor
+  int mode;           // 6, 8 or QAT_EXPORT_FP16
+  int m;              // quantile order statistic from the top (1 or 2)
+  float frac;         // quantile interpolation fraction
+  int pad;
+};
+
+struct ExportBatch {
+  int n;
+  int pad;
+  int64_t total_rows;
+  ExportDescDev d[QAT_EXPORT_MAX_DESCS];
+};
+
+// Chunk length of the fp16 passthrough "rows".
+constexpr int64_t kFp16Chunk = 4096;
+
+int launch_quantize_weights(const float* W, int N, int K, int bits, int8_t* codes, float* scales,
+                            __nv_bfloat16* operand, cudaStream_t s);
+int export_quantile_params(int64_t cols, int* m, float* frac);
+int launch_export_batch(const ExportBatch& b, cudaStream_t s);
+int launch_dequant(const int8_t* codes, const __half* scales, int64_t rows, int64_t cols,
+                   int out_bf16, void* out, cudaStream_t s);
+
+}  // namespace qat

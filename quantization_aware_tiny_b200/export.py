@@ -1,0 +1,64 @@
+"""State-dict export through one grouped launch of the export quantizer.
+
+Host-side rules from "parameter-golf 16MB 极限压缩实战：11L MLP3x + Int6 QAT +
+zstd-22 记录详解", section "后训练量化导出":
+  - tensors that are not 2-D, or hold at most 65,536 elements
+    (INT8_KEEP_FLOAT_MAX_NUMEL; "at most" is the reading taken), pass through
+    as fp16;
+  - the tied embedding passes through as fp16 (FP16_EMBED_EXPORT);
+  - other 2-D tensors get per-row codes and fp16 scales: int6 when they
+    belong to a block i with INT6_LAYER_START <= i <= INT6_LAYER_END (both
+    inclusive, -1 = int6 off), else int8.
+The per-row arithmetic all runs in the library's export kernel.
+"""
+import re
+
+import torch
+
+from . import qat
+
+KEEP_FLOAT_MAX_NUMEL = 65536
+_BLOCK = re.compile(r"^blocks\.(\d+)\.")
+
+
+def export_mode(name, shape, numel, int6_range=(0, 10), embed_name="tok_emb.weight"):
+    """Export mode of one tensor: 6, 8 or qat.QAT_EXPORT_FP16."""
+    if len(shape) != 2 or numel <= KEEP_FLOAT_MAX_NUMEL or name == embed_name:
+        return qat.QAT_EXPORT_FP16
+    start, end = int6_range
+    m = _BLOCK.match(name)
+    if m and start >= 0 and end >= 0 and start <= int(m.group(1)) <= end:
+        return 6
+    return 8
+
+
+def plan(state_dict, int6_range=(0, 10), embed_name="tok_emb.weight"):
+    """(name, mode) for every tensor, in order."""
+    return [(n, export_mode(n, tuple(t.shape), t.numel(), int6_range, embed_name))
+            for n, t in state_dict.items()]
+
+
+def export_state_dict(state_dict, int6_range=(0, 10), embed_name="tok_emb.weight", stream=None):
+    """Quantize a dict of fp32 CUDA tensors.  Returns name -> dict with
+    kind 'int6'/'int8' (codes int8 [rows,cols], scale16 fp16 [rows]) or
+    kind 'fp16' (values fp16, original shape).  Launches in chunks of at most
+    QAT_EXPORT_MAX_DESCS descriptors (one launch for a state dict that fits)."""
+    out = {}
+    descs = []
+    for name, mode in plan(state_dict, int6_range, embed_name):
+        t = state_dict[name]
+        if t.dtype != torch.float32 or not t.is_contiguous():
+            raise ValueError("%s: expected a contiguous fp32 tensor" % name)
+        if mode == qat.QAT_EXPORT_FP16:
+            v = torch.empty(t.shape, dtype=torch.float16, device=t.device)
+            out[name] = {"kind": "fp16", "values": v}
+            descs.append((t.reshape(-1), mode, v, None))
+        else:
+            rows, cols = t.shape
+            c = torch.empty((rows, cols), dtype=torch.int8, device=t.device)
+            s = torch.empty(rows, dtype=torch.float16, device=t.device)
+            out[name] = {"kind": "int%d" % mode, "codes": c, "scale16": s}
+            descs.append((t, mode, c, s))
+    for i in range(0, len(descs), qat.QAT_EXPORT_MAX_DESCS):
+        qat.quantize_export_batch(descs[i:i + qat.QAT_EXPORT_MAX_DESCS], stream=stream)
+    return out

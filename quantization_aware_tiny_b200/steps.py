@@ -1,0 +1,113 @@
+"""Multi-call sequences of the C-ABI entry points: the depth-recurrent core and
+the tied-head + MLP training step.  Only sequencing and buffer ownership live
+here; every arithmetic step runs in the library's kernels.
+"""
+import torch
+
+from . import qat
+
+
+class RecurrentCore:
+    """Depth-recurrent core ("Depth Recurrence + Mixed-Precision Quant"
+    write-up, "Stem / Core / Tail" and "税 1"): the block's weights are
+    quantized ONCE (the cache) and its linears are applied R times.
+
+    Per application, attention left out (the O projection reads the query
+    slice of QKV in its place):
+        qkv = x Wqkv^T              (Q|K|V fused: per-row quantization is per
+                                     output row, so concatenation is exact)
+        x1  = x + q Wo^T            (residual fused in the GEMM epilogue)
+        x   = x1 + proj(relu(fc(x1))^2)
+    """
+
+    def __init__(self, Wq, Wk, Wv, Wo, Wfc, Wproj, bits=6, stream=None):
+        self.d = Wq.shape[1]
+        self.H = Wfc.shape[0]
+        self.bits = bits
+        Wqkv = torch.cat([Wq, Wk, Wv], dim=0).contiguous()
+        self.q_qkv = qat.quantize_weight(Wqkv, bits, stream=stream)
+        self.q_o = qat.quantize_weight(Wo.contiguous(), bits, stream=stream)
+        self.q_fc = qat.quantize_weight(Wfc.contiguous(), bits, stream=stream)
+        self.q_proj = qat.quantize_weight(Wproj.contiguous(), bits, stream=stream)
+        self.nqkv = Wqkv.shape[0]
+        self._buf = None
+
+    def _buffers(self, T, device):
+        if self._buf is None or self._buf[0].shape[0] != T:
+            bf = torch.bfloat16
+            self._buf = (torch.empty((T, self.nqkv), dtype=bf, device=device),
+                         torch.empty((T, self.d), dtype=bf, device=device),
+                         torch.empty((T, self.H), dtype=bf, device=device))
+        return self._buf
+
+    def forward(self, x, R, stream=None):
+        """Applies the core R times to x [T,d] bf16 in place; returns x."""
+        T = x.shape[0]
+        qkv, x1, h = self._buffers(T, x.device)
+        for _ in range(R):
+            qat.qat_linear_fwd(x, qkv, self.bits, qw=self.q_qkv, stream=stream)
+            qat.qat_linear_fwd(qkv, x1, self.bits, qw=self.q_o, ldx=self.nqkv, T=T,
+                               residual=x, stream=stream)
+            qat.qat_mlp_fwd(x1, x, self.bits, self.d, self.H, qfc=self.q_fc, qproj=self.q_proj,
+                            residual=x1, h_save=h, stream=stream)
+        return x
+
+    def flops(self, T, R):
+        return 2.0 * T * self.d * (self.nqkv + self.d + 2 * self.H) * R
+
+
+class HeadMlpStep:
+    """One QAT training step of a tied int8 head over an int6 ReLU^2 MLP:
+        quantize (every step: the weights change between steps)
+        Z = MLP(X); logits = Z Wemb^T
+        dZ = dLogits Wemb_q; dWemb = dLogits^T Z; MLP backward -> dX, dWfc, dWproj
+    """
+
+    def __init__(self, Wemb, Wfc, Wproj, T, head_bits=8, mlp_bits=6):
+        dev = Wemb.device
+        self.W = (Wemb, Wfc, Wproj)
+        self.vocab, self.d = Wemb.shape
+        self.H = Wfc.shape[0]
+        self.T = T
+        self.head_bits, self.mlp_bits = head_bits, mlp_bits
+        bf = torch.bfloat16
+        e = lambda *s, dt=bf: torch.empty(s, dtype=dt, device=dev)
+        self.q = [qat.QWeight(e(*w.shape), e(w.shape[0], dt=torch.float32), None, b)
+                  for w, b in ((Wemb, head_bits), (Wfc, mlp_bits), (Wproj, mlp_bits))]
+        self.pre, self.h = e(T, self.H), e(T, self.H)
+        self.Z, self.logits, self.dZ, self.dX = e(T, self.d), e(T, self.vocab), e(T, self.d), e(T, self.d)
+        self.dWemb = e(self.vocab, self.d, dt=torch.float32)
+        self.dWfc = e(self.H, self.d, dt=torch.float32)
+        self.dWproj = e(self.d, self.H, dt=torch.float32)
+        ws = qat.workspace_size(qat.QAT_OP_MLP_BWD, self.d, self.H, T, False)
+        self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
+
+    def quantize(self, stream=None):
+        for w, q in zip(self.W, self.q):
+            qat.qat_quantize_weights(w, q.bits, q.scales, None, q.operand, stream)
+
+    def forward(self, X, stream=None):
+        qe, qf, qp = self.q
+        qat.qat_mlp_fwd(X, self.Z, self.mlp_bits, self.d, self.H, qfc=qf, qproj=qp,
+                        pre_save=self.pre, h_save=self.h, stream=stream)
+        qat.qat_linear_fwd(self.Z, self.logits, self.head_bits, qw=qe, stream=stream)
+
+    def backward(self, X, dLogits, stream=None):
+        qe, qf, qp = self.q
+        qat.qat_linear_bwd(self.Z, dLogits, self.head_bits, qw=qe, dX=self.dZ, dW=self.dWemb,
+                           stream=stream)
+        qat.qat_mlp_bwd(X, self.pre, self.h, self.dZ, self.mlp_bits, self.d, self.H, qfc=qf,
+                        qproj=qp, dX=self.dX, dWfc=self.dWfc, dWproj=self.dWproj,
+                        workspace=self.ws, stream=stream)
+
+    def step(self, X, dLogits, stream=None):
+        self.quantize(stream)
+        self.forward(X, stream)
+        self.backward(X, dLogits, stream)
+
+    def grads(self):
+        return [self.dWemb, self.dWfc, self.dWproj]
+
+    def flops_per_token(self):
+        # forward + two backward GEMMs for the head and for each MLP linear
+        return 3 * 2.0 * self.d * (self.vocab + 2 * self.H)

@@ -1,0 +1,62 @@
+"""GPU parity of the ReLU^2 MLP (fused relu^2 fc epilogue, fused 2*relu(pre)
+backward epilogue) against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as o
+from quantization_aware_tiny_b200 import qat
+from quantization_aware_tiny_b200 import synthetic as sy
+from parity import assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(c, d, H, bits=6, raw=False):
+    X, dY = c["X"].cuda(), c["dY"].cuda()
+    T = X.shape[0]
+    Wfc, Wproj = torch.from_numpy(c["Wfc"]).cuda(), torch.from_numpy(c["Wproj"]).cuda()
+    bf = torch.bfloat16
+    Y, pre, h = (torch.empty((T, n), dtype=bf, device="cuda") for n in (d, H, H))
+    dX = torch.empty((T, d), dtype=bf, device="cuda")
+    dWfc = torch.empty((H, d), dtype=torch.float32, device="cuda")
+    dWproj = torch.empty((d, H), dtype=torch.float32, device="cuda")
+    if raw:
+        kw = {"Wfc": Wfc, "Wproj": Wproj}
+        wsf = torch.empty(qat.workspace_size(qat.QAT_OP_MLP_FWD, d, H, T, True), dtype=torch.uint8, device="cuda")
+        wsb = torch.empty(qat.workspace_size(qat.QAT_OP_MLP_BWD, d, H, T, True), dtype=torch.uint8, device="cuda")
+    else:
+        kw = {"qfc": qat.quantize_weight(Wfc, bits), "qproj": qat.quantize_weight(Wproj, bits)}
+        wsf = None
+        wsb = torch.empty(qat.workspace_size(qat.QAT_OP_MLP_BWD, d, H, T, False), dtype=torch.uint8, device="cuda")
+    qat.qat_mlp_fwd(X, Y, bits, d, H, pre_save=pre, h_save=h, workspace=wsf, **kw)
+    qat.qat_mlp_bwd(X, pre, h, dY, bits, d, H, dX=dX, dWfc=dWfc, dWproj=dWproj, workspace=wsb, **kw)
+    torch.cuda.synchronize()
+    return Y, pre, h, dX, dWfc, dWproj
+
+
+def _check(c, out, bits=6):
+    qf, qp = o.quantize_weight(c["Wfc"], bits), o.quantize_weight(c["Wproj"], bits)
+    X, dY = c["X"].float().numpy(), c["dY"].float().numpy()
+    pre, h, Y = o.mlp_fwd(qf["operand"], qp["operand"], X)
+    dX, dWfc, dWproj = o.mlp_bwd(qf["operand"], qp["operand"], X, pre, h, dY)
+    for name, g, r in zip(("Y", "pre", "h", "dX", "dWfc", "dWproj"), out, (Y, pre, h, dX, dWfc, dWproj)):
+        assert_close(g, r, name)
+
+
+@pytest.mark.parametrize("raw", [False, True])
+def test_mlp_small_ragged(raw):
+    c = sy.mlp_case(T=1000)
+    _check(c, _run(c, 512, 1536, raw=raw))
+
+
+def test_mlp_odd_dims():
+    c = sy.mlp_case(d=136, H=264, T=333, seed=4)
+    _check(c, _run(c, 136, 264))
+
+
+def test_mlp_cfg2_full_size():
+    """The 11-layer record's MLP block at 8x1024 tokens, every element."""
+    c = sy.mlp_case(T=8192)
+    _check(c, _run(c, 512, 1536))
+    assert qat.device_error() == 0

@@ -1,0 +1,100 @@
+"""GPU parity of the quantizer kernels against the CPU oracle: bit-exact codes,
+fp32 scales, bf16 operands, fp16 export scales, fp16 passthrough and the
+dequantized weights."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as o
+from quantization_aware_tiny_b200 import export as qexport
+from quantization_aware_tiny_b200 import qat
+from quantization_aware_tiny_b200 import synthetic as sy
+from parity import bits16
+
+pytestmark = pytest.mark.gpu
+
+
+def _dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def _weights():
+    sd = sy.state_dict_case(n_layers=1)
+    rng = np.random.default_rng(5)
+    cases = {
+        "cfg1_512x512_outliers": sy.linear_case()["W"],
+        "fc_1536x512_heavy": sd["blocks.0.mlp.fc.weight"],
+        "proj_512x1536_heavy": sd["blocks.0.mlp.proj.weight"],
+        "ragged_200x136": (rng.standard_normal((200, 136)) * 0.02).astype(np.float32),
+        "longrow_64x4104": (rng.standard_normal((64, 4104)) * 0.02).astype(np.float32),
+        "head_8192x512": sy.head_mlp_case(T=8)["Wemb"],
+    }
+    z = np.zeros((8, 64), np.float32)
+    z[1, 3] = 1e-30
+    z[2] = 0.5
+    z[3, ::2] = -7.0
+    cases["degenerate_8x64"] = z
+    return cases
+
+
+@pytest.mark.parametrize("bits", [6, 8])
+def test_quantize_weights_bit_exact(bits):
+    for name, W in _weights().items():
+        q = qat.quantize_weight(_dev(W), bits, keep_codes=True)
+        torch.cuda.synchronize()
+        ref = o.quantize_weight(W, bits)
+        assert np.array_equal(q.codes.cpu().numpy(), ref["codes"]), name
+        assert np.array_equal(q.scales.cpu().numpy().view(np.uint32), ref["scales"].view(np.uint32)), name
+        assert np.array_equal(bits16(q.operand), o.operand_bf16_bits(ref["codes"], ref["scales"])), name
+    assert qat.device_error() == 0
+
+
+@pytest.mark.parametrize("bits", [6, 8])
+def test_export_rows_bit_exact(bits):
+    rng = np.random.default_rng(9)
+    ties = np.tile(np.float32([0.01, -0.03, 0.03, 0.002]), (16, 16))  # top two tie
+    for name, W in list(_weights().items()) + [("ties_16x64", ties)]:
+        Wd = _dev(W)
+        codes = torch.empty(W.shape, dtype=torch.int8, device="cuda")
+        s16 = torch.empty(W.shape[0], dtype=torch.float16, device="cuda")
+        qat.quantize_rows_export(Wd, bits, codes, s16)
+        torch.cuda.synchronize()
+        c_ref, s_ref, _ = o.export_rows(W, bits)
+        assert np.array_equal(codes.cpu().numpy(), c_ref), name
+        assert np.array_equal(bits16(s16), s_ref), name
+
+
+def test_export_state_dict_one_launch_bit_exact():
+    """The whole 11-layer d=512 state dict (66 matrices, tied embedding, small
+    tensors) in one grouped launch, against the oracle's tensor-by-tensor export."""
+    sd = sy.state_dict_case()
+    dev = {k: _dev(v) for k, v in sd.items()}
+    n0 = qat.launch_count()
+    out = qexport.export_state_dict(dev)
+    torch.cuda.synchronize()
+    assert qat.launch_count() - n0 == 1
+    ref = o.export_state_dict(sd)
+    for k, r in ref.items():
+        g = out[k]
+        assert g["kind"] == r["kind"], k
+        if r["kind"] == "fp16":
+            assert np.array_equal(bits16(g["values"]).reshape(-1), r["bits16"].reshape(-1)), k
+        else:
+            assert np.array_equal(g["codes"].cpu().numpy(), r["codes"]), k
+            assert np.array_equal(bits16(g["scale16"]), r["scale16"]), k
+
+
+def test_dequantize_rows_bit_exact():
+    sd = sy.state_dict_case(n_layers=1)
+    for name in ("blocks.0.mlp.fc.weight", "blocks.0.attn.c_k.weight"):
+        W = sd[name]
+        c, s16, _ = o.export_rows(W, 6)
+        cd, sd16 = _dev(c), _dev(s16.view(np.float16))
+        out32 = torch.empty(W.shape, dtype=torch.float32, device="cuda")
+        out16 = torch.empty(W.shape, dtype=torch.bfloat16, device="cuda")
+        qat.dequantize_rows(cd, sd16, out32)
+        qat.dequantize_rows(cd, sd16, out16)
+        torch.cuda.synchronize()
+        ref = o.dequant_export(c, s16)
+        assert np.array_equal(out32.cpu().numpy().view(np.uint32), ref.view(np.uint32)), name
+        assert np.array_equal(bits16(out16), o.bf16_bits(ref)), name

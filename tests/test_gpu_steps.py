@@ -1,0 +1,167 @@
+"""GPU parity of the multi-call paths against the oracle: the depth-recurrent
+core (quantize once, apply R=3 times) and the tied-head + MLP training step,
+at small sizes element by element and at the benchmark's full sizes on
+sampled outputs the oracle computes one by one."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as o
+from quantization_aware_tiny_b200 import qat
+from quantization_aware_tiny_b200 import steps
+from quantization_aware_tiny_b200 import synthetic as sy
+from parity import assert_close, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def _core(c, bits=6):
+    dev = {k: torch.from_numpy(c[k]).cuda() for k in ("Wq", "Wk", "Wv", "Wo", "Wfc", "Wproj")}
+    return steps.RecurrentCore(dev["Wq"], dev["Wk"], dev["Wv"], dev["Wo"], dev["Wfc"], dev["Wproj"], bits)
+
+
+def _core_oracle(c, bits=6):
+    q = {"qkv": o.quantize_weight(np.concatenate([c["Wq"], c["Wk"], c["Wv"]]), bits),
+         "o": o.quantize_weight(c["Wo"], bits), "fc": o.quantize_weight(c["Wfc"], bits),
+         "proj": o.quantize_weight(c["Wproj"], bits)}
+    return q
+
+
+def test_recurrent_core_small():
+    c = sy.recurrent_core_case(T=300)
+    core = _core(c)
+    x = c["X"].cuda()
+    n0 = qat.launch_count()
+    core.forward(x, 3)
+    torch.cuda.synchronize()
+    assert qat.launch_count() - n0 == 3 * 4  # no re-quantization inside the loop
+    q = _core_oracle(c)
+    ref = o.recurrent_core_fwd(q["qkv"], q["o"], q["fc"], q["proj"], c["X"].float().numpy(), 3, 640)
+    assert_close(x, ref, "x after 3 applications")
+
+
+def test_recurrent_cache_matches_fresh_quantization():
+    c = sy.recurrent_core_case(T=8)
+    core = _core(c)
+    q = _core_oracle(c)
+    torch.cuda.synchronize()
+    for name, g in (("qkv", core.q_qkv), ("o", core.q_o), ("fc", core.q_fc), ("proj", core.q_proj)):
+        assert np.array_equal(g.operand.cpu().view(torch.int16).numpy().view(np.uint16),
+                              o.bf16_bits(q[name]["operand"].astype(np.float32))), name
+
+
+def test_recurrent_core_full_size_sampled_rows():
+    """3x3 core at d=640, 16x1024 tokens, R=3: rows evolve independently (no
+    attention), so the oracle runs the sampled rows through all three
+    applications."""
+    c = sy.recurrent_core_case(T=16384)
+    core = _core(c)
+    x = c["X"].cuda()
+    core.forward(x, 3)
+    torch.cuda.synchronize()
+    rows = np.random.default_rng(0).choice(16384, 64, replace=False)
+    rows = np.concatenate([rows, [0, 16383]])
+    q = _core_oracle(c)
+    ref = o.recurrent_core_fwd(q["qkv"], q["o"], q["fc"], q["proj"], c["X"].float().numpy()[rows], 3, 640)
+    assert_close(to_np(x)[rows], ref, "sampled rows")
+    assert qat.device_error() == 0
+
+
+def _head_step(c):
+    dev = lambda k: torch.from_numpy(c[k]).cuda()
+    s = steps.HeadMlpStep(dev("Wemb"), dev("Wfc"), dev("Wproj"), c["X"].shape[0])
+    X, dL = c["X"].cuda(), c["dLogits"].cuda()
+    s.step(X, dL)
+    torch.cuda.synchronize()
+    return s
+
+
+def _head_q(c):
+    return o.quantize_weight(c["Wemb"], 8), o.quantize_weight(c["Wfc"], 6), o.quantize_weight(c["Wproj"], 6)
+
+
+def test_head_mlp_step_small():
+    c = sy.head_mlp_case(T=300)
+    s = _head_step(c)
+    qe, qf, qp = _head_q(c)
+    ref = o.head_mlp_step(qe, qf, qp, c["X"].float().numpy(), c["dLogits"].float().numpy())
+    for name, g in (("Z", s.Z), ("logits", s.logits), ("dZ", s.dZ), ("dX", s.dX),
+                    ("dWemb", s.dWemb), ("dWfc", s.dWfc), ("dWproj", s.dWproj)):
+        assert_close(g, ref[name], name)
+
+
+@pytest.fixture(scope="module")
+def full_head():
+    c = sy.head_mlp_case(T=65536)
+    s = _head_step(c)
+    return c, s
+
+
+def test_head_mlp_step_full_size_rows(full_head):
+    """T=65,536 step as the benchmark launches it: per-token outputs on sampled rows."""
+    c, s = full_head
+    qe, qf, qp = _head_q(c)
+    rows = np.concatenate([np.random.default_rng(1).choice(65536, 48, replace=False), [0, 65535]])
+    X = c["X"].float().numpy()[rows]
+    dL = c["dLogits"].float().numpy()[rows]
+    ref = o.head_mlp_step(qe, qf, qp, X, dL)
+    for name, g in (("Z", s.Z), ("logits", s.logits), ("dZ", s.dZ), ("dX", s.dX)):
+        assert_close(to_np(g)[rows], ref[name], name)
+    # dWproj[n, j] = sum_t dZ[t, n] h[t, j]: columns computed over all tokens
+    Xall, dLall = c["X"].float().numpy(), c["dLogits"].float().numpy()
+    ns, js = [0, 17, 511], [0, 1000, 2047]
+    dZ_cols = o.linear_fwd(qe["operand"][:, ns].T, dLall)          # dZ[:, ns] = dL . Wemb_q[:, ns]
+    h_cols = o.relu2(o.linear_fwd(qf["operand"][js], Xall))         # h[:, js]
+    assert_close(to_np(s.dWproj)[np.ix_(ns, js)], dZ_cols.T @ h_cols, "dWproj sampled")
+    assert qat.device_error() == 0
+
+
+def test_head_bwd_full_size_sampled():
+    """Head backward at T=65,536 (the benchmark's launch configuration) on
+    generator inputs: sampled dWemb entries and dX rows."""
+    c = sy.head_mlp_case(T=65536)
+    Z = sy.act_bf16(np.random.default_rng(77), 65536, 512, std=0.25)
+    q = qat.quantize_weight(torch.from_numpy(c["Wemb"]).cuda(), 8)
+    dX = torch.empty((65536, 512), dtype=torch.bfloat16, device="cuda")
+    dW = torch.empty((8192, 512), dtype=torch.float32, device="cuda")
+    qat.qat_linear_bwd(Z.cuda(), c["dLogits"].cuda(), 8, qw=q, dX=dX, dW=dW)
+    torch.cuda.synchronize()
+    op = o.quantize_weight(c["Wemb"], 8)["operand"]
+    dL, Zn = c["dLogits"].float().numpy(), Z.float().numpy()
+    ns, ks = [0, 5, 4095, 8191], [0, 129, 511]
+    assert_close(to_np(dW)[np.ix_(ns, ks)], dL[:, ns].astype(np.float64).T @ Zn[:, ks], "dWemb sampled")
+    rows = [0, 12345, 65535]
+    assert_close(to_np(dX)[rows], o.linear_bwd(op, Zn[rows], dL[rows])[0], "dX rows")
+
+
+def test_mlp_bwd_full_size_sampled():
+    """MLP backward at T=65,536 on generator inputs: sampled dWfc / dWproj entries."""
+    c = sy.head_mlp_case(T=65536)
+    dY = sy.act_bf16(np.random.default_rng(78), 65536, 512, std=0.02)
+    X = c["X"].cuda()
+    qf = qat.quantize_weight(torch.from_numpy(c["Wfc"]).cuda(), 6)
+    qp = qat.quantize_weight(torch.from_numpy(c["Wproj"]).cuda(), 6)
+    bf = torch.bfloat16
+    T, d, H = 65536, 512, 2048
+    Y, pre, h = (torch.empty((T, n), dtype=bf, device="cuda") for n in (d, H, H))
+    dX = torch.empty((T, d), dtype=bf, device="cuda")
+    dWfc = torch.empty((H, d), dtype=torch.float32, device="cuda")
+    dWproj = torch.empty((d, H), dtype=torch.float32, device="cuda")
+    ws = torch.empty(qat.workspace_size(qat.QAT_OP_MLP_BWD, d, H, T, False), dtype=torch.uint8, device="cuda")
+    qat.qat_mlp_fwd(X, Y, 6, d, H, qfc=qf, qproj=qp, pre_save=pre, h_save=h)
+    qat.qat_mlp_bwd(X, pre, h, dY.cuda(), 6, d, H, qfc=qf, qproj=qp, dX=dX, dWfc=dWfc,
+                    dWproj=dWproj, workspace=ws)
+    torch.cuda.synchronize()
+    rf, rp = o.quantize_weight(c["Wfc"], 6), o.quantize_weight(c["Wproj"], 6)
+    Xn, dYn = c["X"].float().numpy(), dY.float().numpy()
+    ns, ks = [0, 777, 2047], [0, 300, 511]
+    pre_c = o.linear_fwd(rf["operand"][ns], Xn)                       # pre[:, ns]
+    dh_c = o.linear_fwd(rp["operand"][:, ns].T, dYn)                  # dh[:, ns] = dY . Wproj_q[:, ns]
+    dpre_c = dh_c * 2.0 * np.maximum(pre_c, 0.0)
+    assert_close(to_np(dWfc)[np.ix_(ns, ks)], dpre_c.T @ Xn[:, ks], "dWfc sampled")
+    h_c = o.relu2(o.linear_fwd(rf["operand"][[5, 1999]], Xn))
+    assert_close(to_np(dWproj)[np.ix_(ks, [5, 1999])], dYn[:, ks].astype(np.float64).T @ h_c, "dWproj sampled")
+    rows = [3, 40000]
+    r = o.mlp_bwd(rf["operand"], rp["operand"], Xn[rows], *o.mlp_fwd(rf["operand"], rp["operand"], Xn[rows])[:2], dYn[rows])
+    assert_close(to_np(dX)[rows], r[0], "dX rows")
+    assert qat.device_error() == 0

@@ -1,0 +1,114 @@
+"""Host-side checks that need no GPU: the C-ABI library loads and exports every
+symbol include/qat.h declares, argument validation rejects bad calls before
+any launch, and the export planner applies the passthrough rules."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle as o
+from quantization_aware_tiny_b200 import build, qat
+from quantization_aware_tiny_b200 import export as qexport
+from quantization_aware_tiny_b200 import synthetic as sy
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "qat.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return qat.lib()
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?(?:int|int64_t|size_t|char\s*\*|const char\s*\*)\s*\*?\s*(\w+)\s*\(",
+                       src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_symbols_exported(L):
+    names = _declared()
+    assert set(names) == set(qat.EXPORTED), names
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_strerror_and_workspace_sizes(L):
+    assert qat.strerror(0) == "ok"
+    assert "aligned" in qat.strerror(qat.QAT_ERR_ALIGN)
+    assert qat.strerror(99) == "unknown error"
+    # raw weights: bf16 operand + fp32 scales, each rounded up to 256 bytes
+    assert qat.workspace_size(qat.QAT_OP_LINEAR_FWD, 512, 512, 256, True) == 512 * 512 * 2 + 2048
+    assert qat.workspace_size(qat.QAT_OP_LINEAR_FWD, 512, 512, 256, False) == 0
+    assert qat.workspace_size(qat.QAT_OP_MLP_BWD, 512, 1536, 8192, False) == 8192 * 1536 * 2
+    assert qat.workspace_size(qat.QAT_OP_MLP_FWD, 0, 1536, 8192, False) == 0
+
+
+P = ctypes.c_void_p
+
+
+def test_argument_validation_before_launch(L):
+    """Bad calls return an error code and launch nothing (no GPU is touched)."""
+    before = qat.launch_count()
+    A16, A_BAD = P(0x10000), P(0x10004)
+    # null activations / outputs
+    assert L.qat_linear_fwd(A16, None, 512, 512, 6, None, 0, 256, None, A16, None, 0, None) == qat.QAT_ERR_ARG
+    # bits outside {6, 8}
+    assert L.qat_linear_fwd(A16, None, 512, 512, 5, A16, 0, 256, None, A16, None, 0, None) == qat.QAT_ERR_ARG
+    # feature dims must be multiples of 8
+    assert L.qat_linear_fwd(A16, None, 500, 512, 6, A16, 0, 256, None, A16, None, 0, None) == qat.QAT_ERR_SHAPE
+    # both W and qw, or neither
+    assert L.qat_linear_fwd(None, None, 512, 512, 6, A16, 0, 256, None, A16, None, 0, None) == qat.QAT_ERR_ARG
+    # misaligned weights
+    assert L.qat_quantize_weights(A_BAD, 512, 512, 6, None, A16, None, None) == qat.QAT_ERR_ALIGN
+    # workspace too small for raw weights
+    assert L.qat_linear_fwd(A16, None, 512, 512, 6, A16, 0, 256, None, A16, A16, 1024, None) == qat.QAT_ERR_WORKSPACE
+    # export: longer rows than the top-2 quantile covers, bad mode, too many descs
+    assert L.quantize_rows_export(A16, 4, 1 << 21, 6, A16, A16, None) == qat.QAT_ERR_SHAPE
+    assert L.quantize_rows_export(A16, 4, 700000, 6, A16, A16, None) == qat.QAT_ERR_SHAPE
+    assert L.quantize_rows_export(A16, 4, 512, 7, A16, A16, None) == qat.QAT_ERR_ARG
+    assert L.quantize_export_batch(None, 1, None) == qat.QAT_ERR_ARG
+    assert L.quantize_export_batch(A16, 257, None) == qat.QAT_ERR_ARG
+    assert L.dequantize_rows(A16, A16, 4, 12, 0, A16, None) == qat.QAT_ERR_SHAPE
+    assert L.dequantize_rows(A16, A16, 4, 16, 3, A16, None) == qat.QAT_ERR_ARG
+    assert L.qat_mlp_bwd(None, None, None, None, 512, 1536, 6, A16, A16, None, A16, 8, None,
+                         None, None, 0, None, 0, None) == qat.QAT_ERR_ARG
+    assert qat.launch_count() == before
+
+
+def test_export_plan_matches_page_rules():
+    """The product planner and the oracle's own rule implementation agree on
+    every tensor of the 11-layer state dict and on the boundary cases."""
+    sd = sy.state_dict_case()
+    sd["blocks.0.edge"] = np.zeros((256, 256), np.float32)      # exactly 65,536
+    sd["blocks.12.big"] = np.ones((300, 256), np.float32)       # outside 0..10
+    sd["flat"] = np.zeros(70000, np.float32)                   # not 2-D
+    kinds = {n: ("fp16" if m == qat.QAT_EXPORT_FP16 else "int%d" % m)
+             for n, m in qexport.plan({k: _Shape(v) for k, v in sd.items()})}
+    oref = o.export_state_dict(sd)
+    assert kinds == {k: v["kind"] for k, v in oref.items()}
+    assert kinds["blocks.3.mlp.fc.weight"] == "int6" and kinds["blocks.12.big"] == "int8"
+    assert kinds["blocks.0.edge"] == "fp16" and kinds["tok_emb.weight"] == "fp16"
+    off = {n: m for n, m in qexport.plan({k: _Shape(v) for k, v in sd.items()}, int6_range=(-1, -1))}
+    assert off["blocks.3.mlp.fc.weight"] == 8
+
+
+class _Shape:
+    def __init__(self, a):
+        self.shape = a.shape
+        self._n = a.size
+
+    def numel(self):
+        return self._n
+
+
+def test_export_quantile_parameters_cover_page_row_lengths():
+    """Rows up to 625,001 columns need only the top-2 order statistics."""
+    for n in (512, 1536, 2048, 625001):
+        pos = 0.9999984 * (n - 1)
+        assert n - int(np.floor(pos)) <= 2
+    assert 700000 - int(np.floor(0.9999984 * 699999)) > 2
