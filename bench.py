@@ -117,9 +117,14 @@ def dist_env():
 
 
 def make_inputs(seed, device):
-    """Synthetic step inputs of one rank, generated on the host and copied in."""
+    """Synthetic step inputs of one rank, generated on the host: the weights
+    are the same on every rank (seed 0, data-parallel replicas), the token
+    shard and its upstream gradient come from the rank's own seed."""
     from quantization_aware_tiny_b200 import synthetic as sy
     c = sy.head_mlp_case(T=T_TOKENS, vocab=VOCAB, d=D, H=H, seed=seed)
+    if seed != 0:
+        w = sy.head_mlp_case(T=1, vocab=VOCAB, d=D, H=H, seed=0)
+        c.update({k: w[k] for k in ("Wemb", "Wfc", "Wproj")})
     return {k: (torch.from_numpy(v) if isinstance(v, np.ndarray) else v) for k, v in c.items()}
 
 
@@ -144,7 +149,7 @@ def timed_calls(step, X, dL, ev_pairs, stream):
 
 
 def run_ours(args):
-    from quantization_aware_tiny_b200 import qat, steps
+    from quantization_aware_tiny_b200 import dp, qat, steps
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -156,7 +161,7 @@ def run_ours(args):
                                 device_id=dev)
         pg = dist
     stream = torch.cuda.current_stream()
-    inp = make_inputs(seed=rank, device=dev)
+    inp = make_inputs(seed=dp.shard_seed(0, rank), device=dev)
     W = {k: inp[k].to(dev) for k in ("Wemb", "Wfc", "Wproj")}
     X, dL = inp["X"].to(dev), inp["dLogits"].to(dev)
     step = steps.HeadMlpStep(W["Wemb"], W["Wfc"], W["Wproj"], T_TOKENS)
@@ -173,8 +178,7 @@ def run_ours(args):
         else:
             step.step(X, dL, stream)
         if pg is not None:
-            for g in step.grads():
-                pg.all_reduce(g)
+            dp.allreduce_grads(step.grads(), pg)
 
     for i in range(args.warmup):
         one(i, False)
@@ -194,9 +198,7 @@ def run_ours(args):
     launches = qat.launch_count() - n0
     ms = start.elapsed_time(end)
     if pg is not None:
-        t = torch.tensor([ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = dp.max_over_ranks(ms, pg, dev)
     err = qat.device_error()
     value = flops_step * world * args.steps / (ms * 1e-3) / 1e12
 
@@ -247,6 +249,7 @@ def run_ours(args):
 
 
 def measure_e2e(step, inp, dev, stream, args, pg, flops_step, world):
+    from quantization_aware_tiny_b200 import dp
     """Same step with the inputs copied from pinned host memory and the weight
     gradients read back every step, inside the timed region."""
     hX = inp["X"].pin_memory()
@@ -261,8 +264,7 @@ def measure_e2e(step, inp, dev, stream, args, pg, flops_step, world):
         dL.copy_(hdL, non_blocking=True)
         step.step(X, dL, stream)
         if pg is not None:
-            for g in step.grads():
-                pg.all_reduce(g)
+            dp.allreduce_grads(step.grads(), pg)
         for h, g in zip(hg, step.grads()):
             h.copy_(g, non_blocking=True)
 
@@ -279,9 +281,7 @@ def measure_e2e(step, inp, dev, stream, args, pg, flops_step, world):
     torch.cuda.synchronize()
     ms = a.elapsed_time(b)
     if pg is not None:
-        t = torch.tensor([ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = dp.max_over_ranks(ms, pg, dev)
     h2d = hX.numel() * 2 + hdL.numel() * 2
     d2h = sum(g.numel() * 4 for g in hg)
     return {"value": round(flops_step * world * steps_e2e / (ms * 1e-3) / 1e12, 2),

@@ -182,15 +182,19 @@ def recurrent_core_fwd(q_qkv, q_o, q_fc, q_proj, X, R, d):
     """Depth-recurrent core (P1 "Stem / Core / Tail", "税 1"): the block's
     linears, quantized once, applied R times.  Attention is left out, so the
     O projection reads the query slice of QKV (reading stated in the design
-    notes).  Per application, in fp64:
-        qkv = x Wqkv^T ; x1 = x + q Wo^T ; x2 = x1 + proj(relu(fc(x1))^2)
-    and x is rounded to bf16 between applications (activations are bf16)."""
-    x = _f64(X)
+    notes).  Per application:
+        qkv = x Wqkv^T ; x1 = x + q Wo^T ; h = relu(x1 Wfc^T)^2 ; x = x1 + h Wproj^T
+    The activations handed from one GEMM to the next (qkv, x1, h and x) are
+    bf16 tensors, as in the bf16 training the pages describe: each is rounded
+    to bf16 once where it is materialised; every sum and product in between
+    is exact (fp64)."""
+    x = bf16_round(_f64(X).astype(np.float32)).astype(np.float64)
+    b = lambda a: bf16_round(a.astype(np.float32)).astype(np.float64)
     for _ in range(R):
-        qkv = x @ q_qkv["operand"].T
-        x1 = x + qkv[:, :d] @ q_o["operand"].T
-        _, _, m = mlp_fwd(q_fc["operand"], q_proj["operand"], x1)
-        x = bf16_round((x1 + m).astype(np.float32)).astype(np.float64)
+        qkv = b(x @ q_qkv["operand"].T)
+        x1 = b(x + qkv[:, :d] @ q_o["operand"].T)
+        h = b(relu2(x1 @ q_fc["operand"].T))
+        x = b(x1 + h @ q_proj["operand"].T)
     return x
 
 

@@ -123,10 +123,10 @@ size_t qat_workspace_size(int32_t op, int32_t N_or_d, int32_t K_or_H, int64_t T,
     case QAT_OP_LINEAR_FWD:
     case QAT_OP_LINEAR_BWD:
       return raw_weights ? operand_bytes(a, b) : 0;
-    case QAT_OP_MLP_FWD:  // h [T,H] when not saved by the caller, + operands
-      return align_up(static_cast<size_t>(T) * b * 2) + (raw_weights ? 2 * operand_bytes(a, b) : 0);
+    case QAT_OP_MLP_FWD:  // h [T,H] when not saved by the caller, + operands of fc [H,d], proj [d,H]
     case QAT_OP_MLP_BWD:  // dpre [T,H] + operands
-      return align_up(static_cast<size_t>(T) * b * 2) + (raw_weights ? 2 * operand_bytes(a, b) : 0);
+      return align_up(static_cast<size_t>(T) * b * 2) +
+             (raw_weights ? operand_bytes(b, a) + operand_bytes(a, b) : 0);
     default:
       return 0;
   }

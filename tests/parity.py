@@ -30,3 +30,17 @@ def assert_close(gpu, ref, what=""):
 
 def bits16(t):
     return t.detach().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def assert_close_chain(gpu, ref, roundings, what=""):
+    """Chained bf16 state (the recurrent core): on top of the single-op
+    tolerance, each of `roundings` bf16 roundings of the state may land on the
+    neighbouring value on one side only -- one bf16 ulp (<= 2^-7 |x|) each."""
+    g = np.asarray(to_np(gpu) if isinstance(gpu, torch.Tensor) else gpu, np.float64)
+    r = np.asarray(ref, np.float64)
+    assert g.shape == r.shape and np.all(np.isfinite(g)), what
+    fro = np.linalg.norm(g - r) / max(np.linalg.norm(r), 1e-30)
+    allow = ABS_REL * (np.abs(r) + 1.0) + roundings * 2.0 ** -7 * np.abs(r)
+    assert fro <= REL_FRO, "%s: relative Frobenius error %.3g" % (what, fro)
+    assert np.all(np.abs(g - r) <= allow), "%s: max excess %.3g" % (what, np.max(np.abs(g - r) - allow))
+    return fro

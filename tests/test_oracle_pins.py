@@ -354,8 +354,13 @@ def test_recurrent_core_is_r_applications():
     for _ in range(3):
         x = o.recurrent_core_fwd(q["qkv"], q["o"], q["fc"], q["proj"], x, 1, 64)
     assert np.array_equal(x3, x)
-    # one application by hand from the definitions
-    x1 = X + (X.astype(np.float64) @ q["qkv"]["operand"].T)[:, :64] @ q["o"]["operand"].T
-    m = np.maximum(x1 @ q["fc"]["operand"].T, 0) ** 2 @ q["proj"]["operand"].T
+    # one application by hand from the definitions, bf16 rounding (torch's)
+    # of each activation handed between GEMMs
+    b = lambda a: torch.from_numpy(np.asarray(a, np.float32)).to(torch.bfloat16).double().numpy()
+    x = b(X)
+    qkv = b(x @ q["qkv"]["operand"].T)
+    x1 = b(x + qkv[:, :64] @ q["o"]["operand"].T)
+    h = b(np.maximum(x1 @ q["fc"]["operand"].T, 0) ** 2)
+    ref = b(x1 + h @ q["proj"]["operand"].T)
     one = o.recurrent_core_fwd(q["qkv"], q["o"], q["fc"], q["proj"], X, 1, 64)
-    assert np.allclose(one, x1 + m, rtol=2 ** -8, atol=1e-6)
+    assert np.array_equal(one, ref)
