@@ -136,6 +136,33 @@ int qat_mlp_bwd(const float* Wfc, const float* Wproj, const qat_qweight* qfc,
                 void* workspace, size_t ws_bytes, qat_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * qat_linear_fwd_noalloc -- the QAT linear forward from fp32 weights that
+ * allocates nothing and takes no workspace.  The pages have no counterpart:
+ * this is a library convenience for callers that cannot allocate device
+ * memory themselves (a plugin inside a framework that owns all device memory
+ * through its own pool, a fixed-budget service that allocates only at
+ * start-up, latency-critical code that cannot afford the synchronization
+ * cudaMalloc / cudaFree may cause).
+ *   Computes exactly what qat_linear_fwd computes when given W (same kernels):
+ *   Y[T,N] = bf16( X[T,K] . bf16(fl32(c*s))^T (+ residual) ).
+ *   Scratch: a fixed device array inside the library holds the bf16 operand and
+ *   the scales -- at most QAT_NOALLOC_MAX_ELEMS weights (N*K) and
+ *   QAT_NOALLOC_MAX_ROWS rows; larger weights return QAT_ERR_SHAPE.  Every GPU
+ *   that loads the library holds this array (8 MiB + 64 KiB) until exit.
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current); make that first call
+ *   before any stream capture.
+ *   All calls share the array and each rewrites what it reads, so nothing
+ *   must start at zero; calls whose kernels overlap on the GPU (other streams
+ *   or host threads on the same device) race on it -- serialize them.
+ * Other arguments, errors and aliasing rules as qat_linear_fwd. */
+#define QAT_NOALLOC_MAX_ELEMS 4194304
+#define QAT_NOALLOC_MAX_ROWS 16384
+int qat_linear_fwd_noalloc(const float* W, int32_t N, int32_t K, int32_t bits,
+                           const qat_bf16* X, int64_t ldx, int64_t T,
+                           const qat_bf16* residual, qat_bf16* Y, qat_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Export quantizer, [P5] "后训练量化导出".
  * Per row of W [rows, cols] fp32:
  *   clip   = linear-interpolated quantile of |w| at q = 0.9999984: sorted

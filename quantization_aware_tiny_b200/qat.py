@@ -25,7 +25,10 @@ QAT_DTYPE_F32, QAT_DTYPE_BF16 = 0, 1
 # every symbol include/qat.h declares
 EXPORTED = ("qat_strerror", "qat_launch_count", "qat_device_error", "qat_quantize_weights",
             "qat_workspace_size", "qat_linear_fwd", "qat_linear_bwd", "qat_mlp_fwd",
-            "qat_mlp_bwd", "quantize_rows_export", "quantize_export_batch", "dequantize_rows")
+            "qat_mlp_bwd", "quantize_rows_export", "quantize_export_batch", "dequantize_rows",
+            "qat_linear_fwd_noalloc")
+QAT_NOALLOC_MAX_ELEMS = 4194304
+QAT_NOALLOC_MAX_ROWS = 16384
 
 
 class QatError(RuntimeError):
@@ -74,6 +77,7 @@ def lib():
         L.quantize_rows_export.argtypes = [P, I64, I64, I32, P, P, P]
         L.quantize_export_batch.argtypes = [P, I32, P]
         L.dequantize_rows.argtypes = [P, P, I64, I64, I32, P, P]
+        L.qat_linear_fwd_noalloc.argtypes = [P, I32, I32, I32, P, I64, I64, P, P, P]
         for name in EXPORTED:
             if name not in ("qat_strerror", "qat_launch_count", "qat_workspace_size"):
                 getattr(L, name).restype = ctypes.c_int
@@ -214,3 +218,13 @@ def dequantize_rows(codes, scales16, out, stream=None):
     dt = QAT_DTYPE_BF16 if out.dtype == torch.bfloat16 else QAT_DTYPE_F32
     _check(lib().dequantize_rows(_p(codes), _p(scales16), rows, cols, dt, _p(out),
                                  _stream(stream)), "dequantize_rows")
+
+
+def qat_linear_fwd_noalloc(W, X, Y, bits, residual=None, ldx=0, T=None, stream=None):
+    """The raw-weight QAT forward without workspace: for callers that cannot
+    allocate device memory (its scratch is a fixed array inside the library)."""
+    N, K = W.shape
+    if T is None:
+        T = X.shape[0]
+    _check(lib().qat_linear_fwd_noalloc(_p(W), N, K, bits, _p(X), ldx, T, _p(residual), _p(Y),
+                                        _stream(stream)), "qat_linear_fwd_noalloc")
