@@ -36,22 +36,42 @@ __device__ __forceinline__ void record_timeout(int* err) {
   if (err) atomicExch(err, QAT_ERR_TIMEOUT);
 }
 
-// IEEE fp32 division and rounding helpers, written so the compiler can
-// neither contract nor approximate them.
+// IEEE fp32 helpers, written so the compiler can neither contract nor
+// approximate them.
 __device__ __forceinline__ float div_rn(float a, float b) { return __fdiv_rn(a, b); }
 __device__ __forceinline__ float mul_rn(float a, float b) { return __fmul_rn(a, b); }
-__device__ __forceinline__ float rne(float x) { return rintf(x); }  // round half to even
 
-// Code of one weight on the int6 / int8 grid (see qat_quantize_weights).
-__device__ __forceinline__ int quant_code(float w, float s, int bits) {
-  float q = rne(div_rn(w, s));
+// fl32(w / s) given r = fl32(1 / s), by Markstein's correction step
+// (P. Markstein, "Computation of elementary functions on the IBM RISC
+// System/6000 processor", IBM J. Res. Develop. 34(1), 1990): q0 = fl(w * r) is
+// within one ulp of w / s, the residual w - s * q0 is exact in one fused
+// multiply-add, and q0 + residual * r rounded once is the correctly rounded
+// quotient.  (Outside the normal range the result may differ from the true
+// quotient only where |w / s| is far below 1/2, where every code is 0.)
+__device__ __forceinline__ float div_by_scale(float w, float s, float r) {
+  const float q0 = __fmul_rn(w, r);
+  const float rem = __fmaf_rn(-q0, s, w);
+  return __fmaf_rn(rem, r, q0);
+}
+
+// Code from the quotient x = fl32(w / s) (see qat_quantize_weights):
+//   k = rne(x) (round half to even, exact for |x| < 2^31);
+//   int6: 4 * rne(k / 4) in integers -- with k = 4m + f, f in 0..3, the result
+//         is 4m for f <= 1, 4m + 4 for f = 3 and the even one of 4m, 4m + 4 for
+//         f = 2, i.e. (k + 1 + (m & 1)) & ~3 -- then clamped to [-128, 124];
+//   int8: k clamped to [-127, 127].
+__device__ __forceinline__ int code_from_quotient(float x, int bits) {
+  int k = __float2int_rn(x);
   if (bits == 6) {
-    q = mul_rn(rne(mul_rn(q, 0.25f)), 4.0f);  // q/4 and *4 are exact in fp32
-    q = fminf(fmaxf(q, -128.0f), 124.0f);
-  } else {
-    q = fminf(fmaxf(q, -127.0f), 127.0f);
+    k = (k + 1 + ((k >> 2) & 1)) & ~3;
+    return min(max(k, -128), 124);
   }
-  return __float2int_rn(q);
+  return min(max(k, -127), 127);
+}
+
+// Code of one weight on the int6 / int8 grid; r = fl32(1 / s).
+__device__ __forceinline__ int quant_code(float w, float s, float r, int bits) {
+  return code_from_quotient(div_by_scale(w, s, r), bits);
 }
 
 }  // namespace qat

@@ -4,12 +4,14 @@
 //                 128B-swizzled A/B tiles in shared memory
 //   warp 1      : TMEM allocator + MMA issuer (one lane issues tcgen05.mma,
 //                 128 x BN x 16 per instruction, fp32 accumulator in TMEM)
-//   warps 2..5  : epilogue; warp w reads TMEM lanes 32*(w%4)..+31 (its rows),
-//                 applies the fused epilogue and stores to global memory
+//   warps 2..5  : epilogue; warp w reads TMEM lanes 32*(w%4)..+31 (its rows)
+//                 32 columns at a time, applies the fused epilogue, writes the
+//                 32x32 chunk into swizzled shared memory and hands it to a TMA
+//                 bulk tensor store (or fp32 reduce-add), double-buffered
 //
 // Two accumulator buffers in TMEM (2*BN columns) let the epilogue of tile i
 // overlap the main loop of tile i+1.  Tiles are 128 x BN x 64; split-K (for
-// the long-K weight-gradient GEMMs) adds fp32 partial sums atomically.
+// the long-K weight-gradient GEMMs) adds fp32 partial sums with TMA reduce-add.
 #include <algorithm>
 #include <mutex>
 
@@ -31,8 +33,9 @@ struct Cfg {
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TMEM_COLS = 2 * BN;  // 256 or 512: powers of two as required
+  static constexpr int STAGING_BYTES = 4 * 8192;  // per epilogue warp: 8 KB of output chunks
   static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + STAGING_BYTES + BAR_BYTES + 1024;
 };
 
 struct KArgs {
@@ -55,80 +58,62 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Apply the epilogue to 8 consecutive accumulator columns (one 16-byte group
-// of bf16 output) of one row.
+// Epilogue of one 32-column chunk of one row (this lane's), staged into the
+// warp's shared-memory chunk buffers:
+//   bf16 outputs: 32 rows x 64 B, 16-byte groups swizzled as TMA's 64-byte
+//                 swizzle expects (group j of row r at j ^ ((r >> 1) & 3));
+//   fp32 outputs: 32 rows x 128 B, 128-byte swizzle (group j at j ^ (r & 7)).
+// Both patterns make each quarter-warp's 16-byte stores hit distinct banks.
 template <int EPI>
-__device__ __forceinline__ void epi_group8(const KArgs& p, int64_t row, int64_t col,
-                                           const float* v) {
-  if constexpr (EPI == EPI_BF16 || EPI == EPI_BF16_RESID || EPI == EPI_DRELU2) {
-    float o[8];
-    if constexpr (EPI == EPI_BF16) {
+__device__ __forceinline__ void stage_chunk(const KArgs& p, const uint32_t (&acc)[32],
+                                            const uint4 (&rin)[4], uint32_t buf0, uint32_t buf1,
+                                            int lane) {
+  const float* v = reinterpret_cast<const float*>(acc);
+  if constexpr (EPI == EPI_F32 || EPI == EPI_F32_ATOMIC) {
+    const uint32_t row = buf0 + static_cast<uint32_t>(lane) * 128u;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) o[i] = v[i];
-    } else {
-      uint4 rr = *reinterpret_cast<const uint4*>(p.R + row * p.ldr + col);
-      const __nv_bfloat16* r = reinterpret_cast<const __nv_bfloat16*>(&rr);
+    for (int j = 0; j < 8; ++j)
+      st_shared_v4(row + ((static_cast<uint32_t>(j ^ (lane & 7))) << 4), acc[4 * j],
+                   acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]);
+  } else {
+    const uint32_t off = static_cast<uint32_t>(lane) * 64u;
+    const int sw = (lane >> 1) & 3;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float o[8];
+      const __nv_bfloat16* r = reinterpret_cast<const __nv_bfloat16*>(&rin[j]);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        if constexpr (EPI == EPI_BF16_RESID) {
-          o[i] = __fadd_rn(v[i], bf2f(r[i]));
-        } else {
-          const float t = fmaxf(bf2f(r[i]), 0.0f);
-          o[i] = __fmul_rn(__fmul_rn(v[i], t), 2.0f);
+        const float a = v[8 * j + i];
+        if constexpr (EPI == EPI_BF16) {
+          o[i] = a;
+        } else if constexpr (EPI == EPI_BF16_RESID) {
+          o[i] = __fadd_rn(a, bf2f(r[i]));
+        } else if constexpr (EPI == EPI_DRELU2) {
+          o[i] = __fmul_rn(__fmul_rn(a, fmaxf(bf2f(r[i]), 0.0f)), 2.0f);
+        } else {  // EPI_RELU2: buf0 <- pre (when kept), buf1 <- relu(acc)^2
+          const float t = fmaxf(a, 0.0f);
+          o[i] = __fmul_rn(t, t);
         }
       }
+      const uint32_t at = off + (static_cast<uint32_t>(j ^ sw) << 4);
+      if constexpr (EPI == EPI_RELU2) {
+        st_shared_v4(buf0 + at, pack_bf16(v[8 * j], v[8 * j + 1]), pack_bf16(v[8 * j + 2], v[8 * j + 3]),
+                     pack_bf16(v[8 * j + 4], v[8 * j + 5]), pack_bf16(v[8 * j + 6], v[8 * j + 7]));
+        st_shared_v4(buf1 + at, pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]), pack_bf16(o[4], o[5]),
+                     pack_bf16(o[6], o[7]));
+      } else {
+        st_shared_v4(buf0 + at, pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]), pack_bf16(o[4], o[5]),
+                     pack_bf16(o[6], o[7]));
+      }
     }
-    uint4 w;
-    w.x = pack_bf16(o[0], o[1]);
-    w.y = pack_bf16(o[2], o[3]);
-    w.z = pack_bf16(o[4], o[5]);
-    w.w = pack_bf16(o[6], o[7]);
-    *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.D) + row * p.ldd + col) = w;
-  } else if constexpr (EPI == EPI_RELU2) {
-    if (p.D != nullptr) {
-      uint4 w;
-      w.x = pack_bf16(v[0], v[1]);
-      w.y = pack_bf16(v[2], v[3]);
-      w.z = pack_bf16(v[4], v[5]);
-      w.w = pack_bf16(v[6], v[7]);
-      *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.D) + row * p.ldd + col) = w;
-    }
-    float h[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float r = fmaxf(v[i], 0.0f);
-      h[i] = __fmul_rn(r, r);
-    }
-    uint4 w;
-    w.x = pack_bf16(h[0], h[1]);
-    w.y = pack_bf16(h[2], h[3]);
-    w.z = pack_bf16(h[4], h[5]);
-    w.w = pack_bf16(h[6], h[7]);
-    *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.D2) + row * p.ldd2 + col) = w;
-  } else if constexpr (EPI == EPI_F32) {
-    float* d = reinterpret_cast<float*>(p.D) + row * p.ldd + col;
-    float4 a = make_float4(v[0], v[1], v[2], v[3]);
-    float4 b = make_float4(v[4], v[5], v[6], v[7]);
-    if (p.accumulate) {
-      const float4 oa = reinterpret_cast<const float4*>(d)[0];
-      const float4 ob = reinterpret_cast<const float4*>(d)[1];
-      a.x = __fadd_rn(a.x, oa.x); a.y = __fadd_rn(a.y, oa.y);
-      a.z = __fadd_rn(a.z, oa.z); a.w = __fadd_rn(a.w, oa.w);
-      b.x = __fadd_rn(b.x, ob.x); b.y = __fadd_rn(b.y, ob.y);
-      b.z = __fadd_rn(b.z, ob.z); b.w = __fadd_rn(b.w, ob.w);
-    }
-    reinterpret_cast<float4*>(d)[0] = a;
-    reinterpret_cast<float4*>(d)[1] = b;
-  } else {  // EPI_F32_ATOMIC
-    float* d = reinterpret_cast<float*>(p.D) + row * p.ldd + col;
-    atomicAdd(reinterpret_cast<float4*>(d), make_float4(v[0], v[1], v[2], v[3]));
-    atomicAdd(reinterpret_cast<float4*>(d) + 1, make_float4(v[4], v[5], v[6], v[7]));
   }
 }
 
 template <int BN, bool A_MN, bool B_MN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmD, const __grid_constant__ CUtensorMap tmD2,
                 const KArgs p) {
   using C = Cfg<BN>;
   extern __shared__ uint8_t smem_raw[];
@@ -136,7 +121,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::STAGES * C::A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint8_t* staging = smem + C::STAGES * C::STAGE_BYTES;  // 1024-aligned
+  uint64_t* full = reinterpret_cast<uint64_t*>(staging + C::STAGING_BYTES);
   uint64_t* empty = full + C::STAGES;
   uint64_t* tfull = empty + C::STAGES;
   uint64_t* tempty = tfull + 2;
@@ -165,6 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmD);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -257,37 +244,70 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------ epilogue (warps 2..5)
+    constexpr bool kF32 = (EPI == EPI_F32 || EPI == EPI_F32_ATOMIC);
     const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const uint32_t wbuf = smem_u32(staging) + static_cast<uint32_t>(q) * 8192u;
+    const bool keep_pre = (EPI == EPI_RELU2) && p.D != nullptr;
     int acc = 0;
     uint32_t acc_phase = 0;
+    uint32_t chunk = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
       const int nb = tile % p.num_n_blk;
       const int mb = (tile / p.num_n_blk) % p.num_m_blk;
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err)) break;
       tc_fence_after();
-      const int64_t row = static_cast<int64_t>(mb) * BM + q * 32 + lane;
+      const int row0 = mb * BM + q * 32;
+      const int64_t row = static_cast<int64_t>(row0) + lane;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
+      const int ncols = min(BN, p.N - nb * BN);
+      const int nchunks = (ncols + 31) / 32;
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(t_row + static_cast<uint32_t>(c0), r);
-        tmem_ld_wait();
-        const int64_t col0 = static_cast<int64_t>(nb) * BN + c0;
-        if (row < p.M) {
+      for (int c = 0; c < nchunks; ++c, ++chunk) {
+        const int col0 = nb * BN + c * 32;
+        uint4 rin[4] = {};
+        if constexpr (EPI == EPI_BF16_RESID || EPI == EPI_DRELU2) {
+          if (row < p.M) {
+            const uint4* src = reinterpret_cast<const uint4*>(p.R + row * p.ldr + col0);
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const int64_t col = col0 + g * 8;
-            if (col < p.N) epi_group8<EPI>(p, row, col, reinterpret_cast<const float*>(r) + g * 8);
+            for (int g = 0; g < 4; ++g)
+              if (col0 + 8 * g < p.N) rin[g] = src[g];
           }
         }
+        uint32_t r[32];
+        tmem_ld32(t_row + static_cast<uint32_t>(c * 32), r);
+        tmem_ld_wait();
+        if (c == nchunks - 1) {  // accumulator fully read: hand it back to the MMA
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[acc]);
+        }
+        const uint32_t b = chunk & 1u;
+        const uint32_t buf0 = kF32 ? wbuf + b * 4096u : wbuf + b * 2048u;
+        const uint32_t buf1 = wbuf + 4096u + b * 2048u;
+        if (lane == 0) bulk_wait_read<1>();  // the store that last used buffer b is done reading
+        __syncwarp();
+        stage_chunk<EPI>(p, r, rin, buf0, buf1, lane);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const uint8_t* s0 = staging + (buf0 - smem_u32(staging));
+          if constexpr (EPI == EPI_F32_ATOMIC) {
+            tma_reduce_add_2d(&tmD, s0, col0, row0);
+          } else if constexpr (EPI == EPI_RELU2) {
+            if (keep_pre) tma_store_2d(&tmD, s0, col0, row0);
+            tma_store_2d(&tmD2, staging + (buf1 - smem_u32(staging)), col0, row0);
+          } else {
+            tma_store_2d(&tmD, s0, col0, row0);
+          }
+          bulk_commit();
+        }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
+    if (lane == 0) bulk_wait_all();  // every output chunk written before the block exits
+    __syncwarp();
   }
 
   __syncthreads();
@@ -347,8 +367,27 @@ int make_map(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, int
   return r == CUDA_SUCCESS ? QAT_OK : QAT_ERR_ARG;
 }
 
+// Output tensor map: inner dimension `inner` (N), outer `outer` (M), row stride
+// `ld` elements, box 32 x 32, bf16 (64-byte swizzle) or fp32 (128-byte swizzle).
+int make_out_map(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, int64_t ld,
+                 bool f32) {
+  EncodeFn enc = get_encode();
+  if (!enc) return QAT_ERR_UNSUPPORTED;
+  const int eb = f32 ? 4 : 2;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * eb};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? QAT_OK : QAT_ERR_ARG;
+}
+
 template <int BN, bool A_MN, bool B_MN, int EPI>
-int launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const KArgs& a, cudaStream_t s) {
+int launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& md,
+             const CUtensorMap& md2, const KArgs& a, cudaStream_t s) {
   using C = Cfg<BN>;
   auto kern = gemm_kernel<BN, A_MN, B_MN, EPI>;
   static bool attr_done = false;  // per instantiation; set before first launch
@@ -359,31 +398,32 @@ int launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const KArgs& a, cudaS
     attr_done = true;
   }
   const int grid = std::max(1, std::min(a.num_tiles, sm_count()));
-  kern<<<grid, kThreads, C::SMEM_BYTES, s>>>(ma, mb, a);
+  kern<<<grid, kThreads, C::SMEM_BYTES, s>>>(ma, mb, md, md2, a);
   count_launch();
   return cuda_status(cudaGetLastError());
 }
 
 template <int BN>
-int dispatch_bn(const GemmDesc& g, const CUtensorMap& ma, const CUtensorMap& mb, const KArgs& a,
-                int epi, cudaStream_t s) {
+int dispatch_bn(const GemmDesc& g, const CUtensorMap& ma, const CUtensorMap& mb,
+                const CUtensorMap& md, const CUtensorMap& md2, const KArgs& a, int epi,
+                cudaStream_t s) {
   if (!g.a_mn && !g.b_mn) {
     switch (epi) {
-      case EPI_BF16: return launch_t<BN, false, false, EPI_BF16>(ma, mb, a, s);
-      case EPI_BF16_RESID: return launch_t<BN, false, false, EPI_BF16_RESID>(ma, mb, a, s);
-      case EPI_RELU2: return launch_t<BN, false, false, EPI_RELU2>(ma, mb, a, s);
+      case EPI_BF16: return launch_t<BN, false, false, EPI_BF16>(ma, mb, md, md2, a, s);
+      case EPI_BF16_RESID: return launch_t<BN, false, false, EPI_BF16_RESID>(ma, mb, md, md2, a, s);
+      case EPI_RELU2: return launch_t<BN, false, false, EPI_RELU2>(ma, mb, md, md2, a, s);
       default: break;
     }
   } else if (!g.a_mn && g.b_mn) {
     switch (epi) {
-      case EPI_BF16: return launch_t<BN, false, true, EPI_BF16>(ma, mb, a, s);
-      case EPI_DRELU2: return launch_t<BN, false, true, EPI_DRELU2>(ma, mb, a, s);
+      case EPI_BF16: return launch_t<BN, false, true, EPI_BF16>(ma, mb, md, md2, a, s);
+      case EPI_DRELU2: return launch_t<BN, false, true, EPI_DRELU2>(ma, mb, md, md2, a, s);
       default: break;
     }
   } else if (g.a_mn && g.b_mn) {
     switch (epi) {
-      case EPI_F32: return launch_t<BN, true, true, EPI_F32>(ma, mb, a, s);
-      case EPI_F32_ATOMIC: return launch_t<BN, true, true, EPI_F32_ATOMIC>(ma, mb, a, s);
+      case EPI_F32: return launch_t<BN, true, true, EPI_F32>(ma, mb, md, md2, a, s);
+      case EPI_F32_ATOMIC: return launch_t<BN, true, true, EPI_F32_ATOMIC>(ma, mb, md, md2, a, s);
       default: break;
     }
   }
@@ -450,7 +490,7 @@ int launch_gemm(const GemmDesc& g, cudaStream_t stream) {
     a.kblk_per_split = (a.kblk_total + s - 1) / s;
     s = (a.kblk_total + a.kblk_per_split - 1) / a.kblk_per_split;  // no empty split
     a.splits = s;
-    if (s > 1) {
+    if (s > 1 || g.accumulate) {
       if (!g.accumulate) {
         cudaError_t e = (g.ldd == g.N)
                             ? cudaMemsetAsync(g.D, 0, static_cast<size_t>(g.M * g.N) * 4, stream)
@@ -476,8 +516,17 @@ int launch_gemm(const GemmDesc& g, cudaStream_t stream) {
   if (rc) return rc;
   rc = g.b_mn ? make_map(&mb, g.B, g.N, g.K, g.ldb, 64) : make_map(&mb, g.B, g.K, g.N, g.ldb, BN);
   if (rc) return rc;
-  return BN == 256 ? dispatch_bn<256>(g, ma, mb, a, epi, stream)
-                   : dispatch_bn<128>(g, ma, mb, a, epi, stream);
+  // Output maps: 32x32 boxes, bf16 with 64-byte swizzle or fp32 with 128-byte swizzle.
+  CUtensorMap md, md2;
+  const bool f32 = (epi == EPI_F32 || epi == EPI_F32_ATOMIC);
+  const void* d_base = g.D ? g.D : g.D2;
+  const int64_t d_ld = g.D ? g.ldd : g.ldd2;
+  rc = make_out_map(&md, d_base, g.N, g.M, d_ld, f32);
+  if (rc) return rc;
+  rc = make_out_map(&md2, g.D2 ? g.D2 : d_base, g.N, g.M, g.D2 ? g.ldd2 : d_ld, false);
+  if (rc) return rc;
+  return BN == 256 ? dispatch_bn<256>(g, ma, mb, md, md2, a, epi, stream)
+                   : dispatch_bn<128>(g, ma, mb, md, md2, a, epi, stream);
 }
 
 }  // namespace qat

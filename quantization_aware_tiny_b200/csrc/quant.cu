@@ -2,13 +2,16 @@
 // operand / recurrence cache), the export quantizer with its per-row quantile
 // clip, fp16 passthrough, and the roundtrip dequantizer.
 //
-// One warp per row: coalesced 16-byte loads (512 B per warp instruction), warp
-// shuffle reductions, rows cached in registers between the reduction pass and
-// the quantization pass (up to 2048 columns; longer rows re-read from L2).
+// Quantization uses one warp per row.  The export kernel stages rows in shared
+// memory with 1-D bulk async copies (the copy engine, completing on an
+// mbarrier) two rows ahead of the row being quantized, so each warp keeps
+// ~12 KB in flight while it computes; the training-time kernel caches the row
+// in registers between its reduction and quantization passes.
 #include <algorithm>
 #include <cmath>
 
 #include "quant.cuh"
+#include "sm100_ptx.cuh"
 
 namespace qat {
 
@@ -64,10 +67,11 @@ __global__ void __launch_bounds__(kQThreads)
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     amax = fmaxf(amax, 1e-12f);
     const float s = div_rn(amax, 127.0f);
+    const float rs = __frcp_rn(s);
     if (lane == 0) scales[row] = s;
     auto emit = [&](int j, float4 v) {
-      const int c0 = quant_code(v.x, s, bits), c1 = quant_code(v.y, s, bits);
-      const int c2 = quant_code(v.z, s, bits), c3 = quant_code(v.w, s, bits);
+      const int c0 = quant_code(v.x, s, rs, bits), c1 = quant_code(v.y, s, rs, bits);
+      const int c2 = quant_code(v.z, s, rs, bits), c3 = quant_code(v.w, s, rs, bits);
       const int64_t e = static_cast<int64_t>(row) * K + 4 * j;
       if (codes) *reinterpret_cast<uint32_t*>(codes + e) = pack_codes(c0, c1, c2, c3);
       if (operand) *reinterpret_cast<uint2*>(operand + e) = operand4(c0, c1, c2, c3, s);
@@ -84,12 +88,9 @@ __global__ void __launch_bounds__(kQThreads)
 // ------------------------------------------------------------------ export
 // Running top-2 of |w| (with multiplicity): t1 >= t2.
 __device__ __forceinline__ void top2_push(float a, float& t1, float& t2) {
-  if (a > t1) {
-    t2 = t1;
-    t1 = a;
-  } else if (a > t2) {
-    t2 = a;
-  }
+  const float lo = fminf(a, t1);
+  t1 = fmaxf(a, t1);
+  t2 = fmaxf(t2, lo);
 }
 __device__ __forceinline__ void top2_push4(float4 v, float& t1, float& t2) {
   top2_push(fabsf(v.x), t1, t2);
@@ -97,94 +98,184 @@ __device__ __forceinline__ void top2_push4(float4 v, float& t1, float& t2) {
   top2_push(fabsf(v.z), t1, t2);
   top2_push(fabsf(v.w), t1, t2);
 }
-
-__device__ __forceinline__ void export_quant_row(const ExportDescDev& d, int64_t row, int lane) {
-  const int64_t cols = d.cols;
-  const int K4 = static_cast<int>(cols >> 2);
-  const float4* r = reinterpret_cast<const float4*>(d.src + row * cols);
-  float4 cache[kRegV4];
-  float t1 = 0.0f, t2 = 0.0f;
-#pragma unroll
-  for (int i = 0; i < kRegV4; ++i) {
-    const int j = lane + 32 * i;
-    if (j < K4) {
-      cache[i] = __ldg(r + j);
-      top2_push4(cache[i], t1, t2);
-    }
-  }
-  for (int j = lane + 32 * kRegV4; j < K4; j += 32) top2_push4(__ldg(r + j), t1, t2);
-  // merge the lanes' top-2 lists
+// Merge the 32 lanes' top-2 lists; every lane ends with the row's top two.
+__device__ __forceinline__ void top2_warp(float& t1, float& t2) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     const float b1 = __shfl_xor_sync(0xffffffffu, t1, o);
     const float b2 = __shfl_xor_sync(0xffffffffu, t2, o);
-    const float n1 = fmaxf(t1, b1);
     const float n2 = fmaxf(fminf(t1, b1), fmaxf(t2, b2));
-    t1 = n1;
+    t1 = fmaxf(t1, b1);
     t2 = n2;
   }
-  // v_hi = largest, v_lo = the (cols - lo)-th largest (top2 = 2, top1 = 1)
+}
+
+struct RowQuant {
+  float clip, s, rs;
+  int bits;
+};
+
+// Clip and scales of one row from its top two |w| (see quantize_rows_export).
+__device__ __forceinline__ RowQuant row_params(const ExportDescDev& d, float t1, float t2) {
   const float v_hi = t1;
   const float v_lo = (d.m == 2) ? t2 : t1;
-  const float clip = __fadd_rn(v_lo, __fmul_rn(d.frac, __fsub_rn(v_hi, v_lo)));
-  const float s = div_rn(fmaxf(clip, 1e-12f), 127.0f);
-  if (lane == 0) d.scales[row] = __float2half_rn(s);
-  int8_t* out = reinterpret_cast<int8_t*>(d.dst) + row * cols;
-  const int bits = d.mode;
-  auto emit = [&](int j, float4 v) {
-    const int c0 = quant_code(fminf(fmaxf(v.x, -clip), clip), s, bits);
-    const int c1 = quant_code(fminf(fmaxf(v.y, -clip), clip), s, bits);
-    const int c2 = quant_code(fminf(fmaxf(v.z, -clip), clip), s, bits);
-    const int c3 = quant_code(fminf(fmaxf(v.w, -clip), clip), s, bits);
-    *reinterpret_cast<uint32_t*>(out + 4 * j) = pack_codes(c0, c1, c2, c3);
-  };
-#pragma unroll
-  for (int i = 0; i < kRegV4; ++i) {
-    const int j = lane + 32 * i;
-    if (j < K4) emit(j, cache[i]);
-  }
-  for (int j = lane + 32 * kRegV4; j < K4; j += 32) emit(j, __ldg(r + j));
+  RowQuant q;
+  q.clip = __fadd_rn(v_lo, __fmul_rn(d.frac, __fsub_rn(v_hi, v_lo)));
+  q.s = div_rn(fmaxf(q.clip, 1e-12f), 127.0f);
+  q.rs = __frcp_rn(q.s);
+  q.bits = d.mode;
+  return q;
+}
+
+__device__ __forceinline__ uint32_t codes4(const RowQuant& q, float4 v) {
+  const float c = q.clip;
+  return pack_codes(quant_code(fminf(fmaxf(v.x, -c), c), q.s, q.rs, q.bits),
+                    quant_code(fminf(fmaxf(v.y, -c), c), q.s, q.rs, q.bits),
+                    quant_code(fminf(fmaxf(v.z, -c), c), q.s, q.rs, q.bits),
+                    quant_code(fminf(fmaxf(v.w, -c), c), q.s, q.rs, q.bits));
+}
+
+// A quantized row staged in shared memory (cols <= kExportMaxStagedCols).
+__device__ __forceinline__ void export_row_smem(const ExportDescDev& d, int64_t row,
+                                                const float4* buf, int lane) {
+  const int K4 = static_cast<int>(d.cols >> 2);
+  float t1 = 0.0f, t2 = 0.0f;
+  for (int j = lane; j < K4; j += 32) top2_push4(buf[j], t1, t2);
+  top2_warp(t1, t2);
+  const RowQuant q = row_params(d, t1, t2);
+  if (lane == 0) d.scales[row] = __float2half_rn(q.s);
+  uint32_t* out = reinterpret_cast<uint32_t*>(reinterpret_cast<int8_t*>(d.dst) + row * d.cols);
+  for (int j = lane; j < K4; j += 32) out[j] = codes4(q, buf[j]);
+}
+
+// A quantized row read from global memory (rows longer than the staging buffer).
+__device__ __forceinline__ void export_row_global(const ExportDescDev& d, int64_t row, int lane) {
+  const int K4 = static_cast<int>(d.cols >> 2);
+  const float4* r = reinterpret_cast<const float4*>(d.src + row * d.cols);
+  float t1 = 0.0f, t2 = 0.0f;
+  for (int j = lane; j < K4; j += 32) top2_push4(__ldg(r + j), t1, t2);
+  top2_warp(t1, t2);
+  const RowQuant q = row_params(d, t1, t2);
+  if (lane == 0) d.scales[row] = __float2half_rn(q.s);
+  uint32_t* out = reinterpret_cast<uint32_t*>(reinterpret_cast<int8_t*>(d.dst) + row * d.cols);
+  for (int j = lane; j < K4; j += 32) out[j] = codes4(q, __ldg(r + j));
 }
 
 // fp16 passthrough of one chunk ("row") of a flat tensor.
 __device__ __forceinline__ void export_fp16_chunk(const ExportDescDev& d, int64_t row, int lane) {
   const int64_t begin = row * d.cols;
   const int64_t end = min(begin + d.cols, d.numel);
-  const float* src = d.src;
-  __half* dst = reinterpret_cast<__half*>(d.dst);
-  // chunk starts are multiples of cols (a multiple of 8), so 8-element groups
-  // are 16-byte aligned in the source and the destination
-  const int64_t n8 = (end - begin) >> 3;
-  for (int64_t g = lane; g < n8; g += 32) {
-    const float4 a = __ldg(reinterpret_cast<const float4*>(src + begin) + 2 * g);
-    const float4 b = __ldg(reinterpret_cast<const float4*>(src + begin) + 2 * g + 1);
-    __half2 h0 = __floats2half2_rn(a.x, a.y), h1 = __floats2half2_rn(a.z, a.w);
-    __half2 h2 = __floats2half2_rn(b.x, b.y), h3 = __floats2half2_rn(b.z, b.w);
-    uint4 w;
-    w.x = *reinterpret_cast<uint32_t*>(&h0);
-    w.y = *reinterpret_cast<uint32_t*>(&h1);
-    w.z = *reinterpret_cast<uint32_t*>(&h2);
-    w.w = *reinterpret_cast<uint32_t*>(&h3);
-    *reinterpret_cast<uint4*>(dst + begin + 8 * g) = w;
+  const float* src = d.src + begin;
+  __half* dst = reinterpret_cast<__half*>(d.dst) + begin;
+  // chunk starts are multiples of cols (a multiple of 8): 8-element groups are
+  // 16-byte aligned in the source and the destination
+  const int n8 = static_cast<int>((end - begin) >> 3);
+  constexpr int U = 4;
+  for (int g0 = lane; g0 < n8; g0 += 32 * U) {
+    float4 a[U], b[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int g = g0 + 32 * u;
+      if (g < n8) {
+        a[u] = __ldg(reinterpret_cast<const float4*>(src) + 2 * g);
+        b[u] = __ldg(reinterpret_cast<const float4*>(src) + 2 * g + 1);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int g = g0 + 32 * u;
+      if (g < n8) {
+        __half2 h0 = __floats2half2_rn(a[u].x, a[u].y), h1 = __floats2half2_rn(a[u].z, a[u].w);
+        __half2 h2 = __floats2half2_rn(b[u].x, b[u].y), h3 = __floats2half2_rn(b[u].z, b[u].w);
+        uint4 w;
+        w.x = *reinterpret_cast<uint32_t*>(&h0);
+        w.y = *reinterpret_cast<uint32_t*>(&h1);
+        w.z = *reinterpret_cast<uint32_t*>(&h2);
+        w.w = *reinterpret_cast<uint32_t*>(&h3);
+        *reinterpret_cast<uint4*>(dst + 8 * g) = w;
+      }
+    }
   }
-  for (int64_t e = begin + 8 * n8 + lane; e < end; e += 32) dst[e] = __float2half_rn(src[e]);
+  for (int64_t e = begin + 8 * static_cast<int64_t>(n8) + lane; e < end; e += 32)
+    reinterpret_cast<__half*>(d.dst)[e] = __float2half_rn(d.src[e]);
 }
 
-__global__ void __launch_bounds__(kQThreads) export_batch_kernel(const ExportBatch b) {
+// Descriptor owning global row g (row_begin is non-decreasing; the last
+// descriptor with row_begin <= g).
+__device__ __forceinline__ int find_desc(const ExportBatch& b, int64_t g) {
+  int lo = 0, hi = b.n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (b.d[mid].row_begin <= g) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ bool staged(const ExportDescDev& d) {
+  return d.mode != QAT_EXPORT_FP16 && d.cols <= kExportMaxStagedCols;
+}
+
+// One launch over all descriptors.  Warp w of the grid takes rows
+// w, w + W, w + 2W, ... (W = warps in the grid); row i of a warp goes to
+// buffer i % kExportBufs, and rows i+1, i+2 are in flight while row i is
+// quantized.  Rows that are not staged still arrive once on their buffer's
+// mbarrier so every buffer's phases stay in step with the row count.
+__global__ void __launch_bounds__(kExportWarps * 32, 1)
+    export_batch_kernel(const __grid_constant__ ExportBatch b, int* err) {
+  extern __shared__ __align__(128) uint8_t xsmem[];
   const int lane = threadIdx.x & 31;
-  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  for (int64_t g = warp; g < b.total_rows; g += nwarps) {
-    // descriptor owning global row g (row_begin is increasing)
-    int lo = 0, hi = b.n - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (b.d[mid].row_begin <= g) lo = mid; else hi = mid - 1;
+  const int wib = threadIdx.x >> 5;
+  float4* bufs = reinterpret_cast<float4*>(xsmem + wib * kExportBufs * kExportBufBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(xsmem + kExportWarps * kExportBufs * kExportBufBytes) +
+                   wib * kExportBufs;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) abort_flag = 0;
+  if (lane == 0) {
+    for (int i = 0; i < kExportBufs; ++i) mbar_init(&bars[i], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  const int64_t W = static_cast<int64_t>(gridDim.x) * kExportWarps;
+  const int64_t gw = static_cast<int64_t>(blockIdx.x) * kExportWarps + wib;
+
+  auto issue = [&](int64_t i) {
+    const int64_t g = gw + i * W;
+    if (g >= b.total_rows || lane != 0) return;
+    const int slot = static_cast<int>(i % kExportBufs);
+    const ExportDescDev& d = b.d[find_desc(b, g)];
+    if (staged(d)) {
+      const uint32_t bytes = static_cast<uint32_t>(d.cols * 4);
+      mbar_arrive_expect_tx(&bars[slot], bytes);
+      bulk_load_1d(bufs + slot * (kExportBufBytes / 16), d.src + (g - d.row_begin) * d.cols, bytes,
+                   &bars[slot]);
+    } else {
+      mbar_arrive(&bars[slot]);
     }
-    const ExportDescDev& d = b.d[lo];
+  };
+
+  for (int i = 0; i < kExportBufs; ++i) issue(i);
+  int64_t i = 0;
+  for (; gw + i * W < b.total_rows; ++i) {
+    const int64_t g = gw + i * W;
+    const int slot = static_cast<int>(i % kExportBufs);
+    const uint32_t parity = static_cast<uint32_t>((i / kExportBufs) & 1);
+    if (!mbar_wait(&bars[slot], parity, &abort_flag, err)) break;
+    const ExportDescDev& d = b.d[find_desc(b, g)];
     const int64_t row = g - d.row_begin;
     if (d.mode == QAT_EXPORT_FP16) export_fp16_chunk(d, row, lane);
-    else export_quant_row(d, row, lane);
+    else if (staged(d)) export_row_smem(d, row, bufs + slot * (kExportBufBytes / 16), lane);
+    else export_row_global(d, row, lane);
+    // the buffer is read; order those reads before the copy engine refills it
+    fence_proxy_async_smem();
+    __syncwarp();
+    issue(i + kExportBufs);
+  }
+  // After a timeout: let the copies this warp still has in flight land (bounded)
+  // before the block's shared memory is released.
+  if (lane == 0 && gw + i * W < b.total_rows) {
+    for (int64_t k = i; k < i + kExportBufs && gw + k * W < b.total_rows; ++k)
+      mbar_drain(&bars[k % kExportBufs], static_cast<uint32_t>((k / kExportBufs) & 1));
   }
 }
 
@@ -253,7 +344,16 @@ int export_quantile_params(int64_t cols, int* m, float* frac) {
 
 int launch_export_batch(const ExportBatch& b, cudaStream_t s) {
   if (b.total_rows == 0) return QAT_OK;
-  export_batch_kernel<<<grid_for_rows(b.total_rows, kQThreads / 32), kQThreads, 0, s>>>(b);
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(export_batch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kExportSmemBytes) != cudaSuccess)
+      return QAT_ERR_CUDA;
+    attr_done = true;
+  }
+  const int64_t want = (b.total_rows + kExportWarps - 1) / kExportWarps;
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, sm_count())));
+  export_batch_kernel<<<grid, kExportWarps * 32, kExportSmemBytes, s>>>(b, device_error_ptr());
   count_launch();
   return cuda_status(cudaGetLastError());
 }

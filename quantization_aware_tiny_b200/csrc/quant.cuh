@@ -30,6 +30,15 @@ struct ExportBatch {
 // Chunk length of the fp16 passthrough "rows".
 constexpr int64_t kFp16Chunk = 4096;
 
+// Export kernel staging: warps per block, row buffers per warp, the longest
+// row staged in shared memory (longer rows are read from global memory).
+constexpr int kExportWarps = 8;
+constexpr int kExportBufs = 3;
+constexpr int64_t kExportMaxStagedCols = 2048;
+constexpr int kExportBufBytes = static_cast<int>(kExportMaxStagedCols) * 4;
+constexpr int kExportSmemBytes =
+    kExportWarps * kExportBufs * kExportBufBytes + kExportWarps * kExportBufs * 8;
+
 int launch_quantize_weights(const float* W, int N, int K, int bits, int8_t* codes, float* scales,
                             __nv_bfloat16* operand, cudaStream_t s);
 int export_quantile_params(int64_t cols, int* m, float* frac);

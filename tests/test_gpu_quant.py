@@ -98,3 +98,44 @@ def test_dequantize_rows_bit_exact():
         ref = o.dequant_export(c, s16)
         assert np.array_equal(out32.cpu().numpy().view(np.uint32), ref.view(np.uint32)), name
         assert np.array_equal(bits16(out16), o.bf16_bits(ref)), name
+
+
+def _near_tie_rows(n_rows=256, cols=512, seed=21):
+    """Rows whose entries sit within a few ulps of (k + 1/2) * s: the code then
+    depends on the correctly rounded quotient w / s (and on ties going to
+    even).  The first two entries carry the row's |w| maximum, so both the
+    training scale and the export clip equal amax / 127."""
+    rng = np.random.default_rng(seed)
+    W = np.empty((n_rows, cols), np.float32)
+    for i in range(n_rows):
+        amax = np.float32(rng.uniform(1e-3, 1e2))
+        s = amax / np.float32(127.0)
+        k = rng.integers(-127, 127, cols).astype(np.float32)
+        base = (k + np.float32(0.5)) * s
+        steps = rng.integers(-3, 4, cols)
+        w = base.copy()
+        for st in range(1, 4):
+            w = np.where(steps >= st, np.nextafter(w, np.float32(np.inf)), w)
+            w = np.where(steps <= -st, np.nextafter(w, np.float32(-np.inf)), w)
+        w = np.clip(w, -amax, amax)
+        w[0], w[1] = amax, -amax
+        W[i] = w
+    return W
+
+
+@pytest.mark.parametrize("bits", [6, 8])
+def test_near_tie_quotients_bit_exact(bits):
+    """Pins the division w / s and the two roundings against the oracle's
+    IEEE fp32 division on adversarial near-tie inputs, for both the training
+    quantizer and the export quantizer."""
+    W = _near_tie_rows()
+    q = qat.quantize_weight(_dev(W), bits, keep_codes=True)
+    codes = torch.empty(W.shape, dtype=torch.int8, device="cuda")
+    s16 = torch.empty(W.shape[0], dtype=torch.float16, device="cuda")
+    qat.quantize_rows_export(_dev(W), bits, codes, s16)
+    torch.cuda.synchronize()
+    ref = o.quantize_weight(W, bits)
+    assert np.array_equal(q.codes.cpu().numpy(), ref["codes"])
+    c_ref, s_ref, _ = o.export_rows(W, bits)
+    assert np.array_equal(codes.cpu().numpy(), c_ref)
+    assert np.array_equal(bits16(s16), s_ref)
