@@ -55,13 +55,16 @@ __device__ __forceinline__ float div_by_scale(float w, float s, float r) {
 }
 
 // Code from the quotient x = fl32(w / s) (see qat_quantize_weights):
-//   k = rne(x) (round half to even, exact for |x| < 2^31);
+//   k = rne(x) (round half to even; |x| <= 128 here);
 //   int6: 4 * rne(k / 4) in integers -- with k = 4m + f, f in 0..3, the result
 //         is 4m for f <= 1, 4m + 4 for f = 3 and the even one of 4m, 4m + 4 for
 //         f = 2, i.e. (k + 1 + (m & 1)) & ~3 -- then clamped to [-128, 124];
 //   int8: k clamped to [-127, 127].
 __device__ __forceinline__ int code_from_quotient(float x, int bits) {
-  int k = __float2int_rn(x);
+  // rne(x) for |x| < 2^22: adding 1.5 * 2^23 gives a float whose ulp is 1, so
+  // the sum is rounded to an integer -- ties to even, as the offset is even --
+  // and its bit pattern minus the offset's is that integer.
+  int k = __float_as_int(__fadd_rn(x, 12582912.0f)) - 0x4B400000;
   if (bits == 6) {
     k = (k + 1 + ((k >> 2) & 1)) & ~3;
     return min(max(k, -128), 124);

@@ -26,11 +26,15 @@ constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int kThreads = 192;
 
-template <int BN>
+// PAIR: the CTA pair of a 2-CTA cluster computes a 256 x BN tile with
+// tcgen05 cta_group::2; each CTA stages 128 rows of A and BN/2 rows of B.
+template <int BN, bool PAIR>
 struct Cfg {
-  static constexpr int STAGES = (BN == 256) ? 4 : 6;
+  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;  // B rows staged by one CTA
+  static constexpr int TILE_M = PAIR ? 2 * BM : BM;
+  static constexpr int STAGES = (B_ROWS == 256) ? 4 : 6;
   static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int B_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TMEM_COLS = 2 * BN;  // 256 or 512: powers of two as required
   static constexpr int STAGING_BYTES = 4 * 8192;  // per epilogue warp: 8 KB of output chunks
@@ -110,12 +114,12 @@ __device__ __forceinline__ void stage_chunk(const KArgs& p, const uint32_t (&acc
   }
 }
 
-template <int BN, bool A_MN, bool B_MN, int EPI>
+template <int BN, bool A_MN, bool B_MN, int EPI, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmD, const __grid_constant__ CUtensorMap tmD2,
                 const KArgs p) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, PAIR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -134,6 +138,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // Position in the CTA pair (PAIR): rank 0 is the leader that issues the MMAs
+  // and owns the full / tmem-empty barriers both CTAs signal.
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = (rank == 0);
+  const int tile0 = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int tile_step = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -142,7 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4);
+      mbar_init(&tempty[b], PAIR ? 8 : 4);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -154,11 +164,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmD);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, C::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) cluster_sync(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -168,30 +183,51 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0, pos = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+      for (int tile = tile0; ok && tile < p.num_tiles; tile += tile_step) {
         const int nb = tile % p.num_n_blk;
         const int mb = (tile / p.num_n_blk) % p.num_m_blk;
         const int sp = tile / (p.num_n_blk * p.num_m_blk);
         const int kb0 = sp * p.kblk_per_split;
         const int kb1 = min(kb0 + p.kblk_per_split, p.kblk_total);
+        const int m0 = mb * C::TILE_M + static_cast<int>(rank) * BM;
+        const int n0 = nb * BN + static_cast<int>(rank) * C::B_ROWS;
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
           const int k0 = kb * BK;
           uint8_t* a_dst = sA + stage * C::A_BYTES;
           uint8_t* b_dst = sB + stage * C::B_BYTES;
-          if constexpr (!A_MN) {
-            tma_load_2d(&tmA, &full[stage], a_dst, k0, mb * BM);
-          } else {
-            tma_load_2d(&tmA, &full[stage], a_dst, mb * BM, k0);
-            tma_load_2d(&tmA, &full[stage], a_dst + 64 * 128, mb * BM + 64, k0);
-          }
-          if constexpr (!B_MN) {
-            tma_load_2d(&tmB, &full[stage], b_dst, k0, nb * BN);
-          } else {
+          if constexpr (PAIR) {
+            // both CTAs' bytes complete on the leader's full barrier
+            const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
+            if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+            if constexpr (!A_MN) {
+              tma_load_2d_pair(&tmA, bar, a_dst, k0, m0);
+            } else {
+              tma_load_2d_pair(&tmA, bar, a_dst, m0, k0);
+              tma_load_2d_pair(&tmA, bar, a_dst + 64 * 128, m0 + 64, k0);
+            }
+            if constexpr (!B_MN) {
+              tma_load_2d_pair(&tmB, bar, b_dst, k0, n0);
+            } else {
 #pragma unroll
-            for (int j = 0; j < BN / 64; ++j)
-              tma_load_2d(&tmB, &full[stage], b_dst + j * 64 * 128, nb * BN + j * 64, k0);
+              for (int j = 0; j < C::B_ROWS / 64; ++j)
+                tma_load_2d_pair(&tmB, bar, b_dst + j * 64 * 128, n0 + j * 64, k0);
+            }
+          } else {
+            mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+            if constexpr (!A_MN) {
+              tma_load_2d(&tmA, &full[stage], a_dst, k0, m0);
+            } else {
+              tma_load_2d(&tmA, &full[stage], a_dst, m0, k0);
+              tma_load_2d(&tmA, &full[stage], a_dst + 64 * 128, m0 + 64, k0);
+            }
+            if constexpr (!B_MN) {
+              tma_load_2d(&tmB, &full[stage], b_dst, k0, n0);
+            } else {
+#pragma unroll
+              for (int j = 0; j < C::B_ROWS / 64; ++j)
+                tma_load_2d(&tmB, &full[stage], b_dst + j * 64 * 128, n0 + j * 64, k0);
+            }
           }
           ++pos;
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
@@ -200,15 +236,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       *prod_pos = pos;
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       // ------------------------------------------------ MMA issuer
-      constexpr uint32_t IDESC = idesc_bf16(BM, BN, A_MN, B_MN);
+      constexpr uint32_t IDESC = idesc_bf16(C::TILE_M, BN, A_MN, B_MN);
       int stage = 0, pos = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+      // Arrive on a barrier of this CTA and (PAIR) the same barrier of the peer.
+      auto commit_both = [&](uint64_t* bar) {
+        if constexpr (PAIR) {
+          umma_commit_pair(smem_u32(bar));
+          umma_commit_pair(mapa_shared(smem_u32(bar), 1));
+        } else {
+          umma_commit(bar);
+        }
+      };
+      for (int tile = tile0; ok && tile < p.num_tiles; tile += tile_step) {
         const int sp = tile / (p.num_n_blk * p.num_m_blk);
         const int kb0 = sp * p.kblk_per_split;
         const int kb1 = min(kb0 + p.kblk_per_split, p.kblk_total);
@@ -226,19 +271,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                                      : sw128_desc(a_base + kk * 32, 16, 1024);
             const uint64_t bd = B_MN ? sw128_desc(b_base + kk * 2048, 64 * 128, 1024)
                                      : sw128_desc(b_base + kk * 32, 16, 1024);
-            umma_bf16(d_tmem, ad, bd, IDESC, (kb > kb0 || kk > 0) ? 1u : 0u);
+            const uint32_t accum = (kb > kb0 || kk > 0) ? 1u : 0u;
+            if constexpr (PAIR) umma_bf16_pair(d_tmem, ad, bd, IDESC, accum);
+            else umma_bf16(d_tmem, ad, bd, IDESC, accum);
           }
-          umma_commit(&empty[stage]);
+          commit_both(&empty[stage]);
           ++pos;
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        umma_commit(&tfull[acc]);
+        commit_both(&tfull[acc]);
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
       // Wait (bounded) for every MMA this thread issued before TMEM is freed.
-      umma_commit(mma_done);
+      if constexpr (PAIR) umma_commit_pair(smem_u32(mma_done)); else umma_commit(mma_done);
       mbar_wait(mma_done, 0, abort_flag, p.err);
       *mma_pos = pos;
     }
@@ -251,12 +298,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     uint32_t chunk = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+    // the leader's tmem-empty barrier, which both CTAs' epilogues release
+    const uint32_t tempty_leader = PAIR ? mapa_shared(smem_u32(tempty), 0) : smem_u32(tempty);
+    for (int tile = tile0; tile < p.num_tiles; tile += tile_step) {
       const int nb = tile % p.num_n_blk;
       const int mb = (tile / p.num_n_blk) % p.num_m_blk;
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err)) break;
       tc_fence_after();
-      const int row0 = mb * BM + q * 32;
+      const int row0 = mb * C::TILE_M + static_cast<int>(rank) * BM + q * 32;
       const int64_t row = static_cast<int64_t>(row0) + lane;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
@@ -280,7 +329,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (c == nchunks - 1) {  // accumulator fully read: hand it back to the MMA
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[acc]);
+          if (lane == 0) {
+            if constexpr (PAIR) mbar_arrive_cluster(tempty_leader + 8u * static_cast<uint32_t>(acc));
+            else mbar_arrive(&tempty[acc]);
+          }
         }
         const uint32_t b = chunk & 1u;
         const uint32_t buf0 = kF32 ? wbuf + b * 4096u : wbuf + b * 2048u;
@@ -323,10 +375,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
     }
   }
-  __syncthreads();
+  // No CTA of a pair leaves while its peer may still signal its barriers.
+  if constexpr (PAIR) cluster_sync(); else __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::TMEM_COLS);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    else tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
 }
 
@@ -385,11 +439,11 @@ int make_out_map(CUtensorMap* m, const void* base, int64_t inner, int64_t outer,
   return r == CUDA_SUCCESS ? QAT_OK : QAT_ERR_ARG;
 }
 
-template <int BN, bool A_MN, bool B_MN, int EPI>
+template <int BN, bool A_MN, bool B_MN, int EPI, bool PAIR>
 int launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& md,
              const CUtensorMap& md2, const KArgs& a, cudaStream_t s) {
-  using C = Cfg<BN>;
-  auto kern = gemm_kernel<BN, A_MN, B_MN, EPI>;
+  using C = Cfg<BN, PAIR>;
+  auto kern = gemm_kernel<BN, A_MN, B_MN, EPI, PAIR>;
   static bool attr_done = false;  // per instantiation; set before first launch
   if (!attr_done) {
     cudaError_t e =
@@ -397,33 +451,48 @@ int launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& md
     if (e != cudaSuccess) return QAT_ERR_CUDA;
     attr_done = true;
   }
-  const int grid = std::max(1, std::min(a.num_tiles, sm_count()));
-  kern<<<grid, kThreads, C::SMEM_BYTES, s>>>(ma, mb, md, md2, a);
+  const int units = PAIR ? sm_count() / 2 : sm_count();
+  const int grid = std::max(1, std::min(a.num_tiles, units)) * (PAIR ? 2 : 1);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = PAIR ? 2 : 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ma, mb, md, md2, a);
   count_launch();
-  return cuda_status(cudaGetLastError());
+  return cuda_status(e == cudaSuccess ? cudaGetLastError() : e);
 }
 
-template <int BN>
+template <int BN, bool PAIR>
 int dispatch_bn(const GemmDesc& g, const CUtensorMap& ma, const CUtensorMap& mb,
                 const CUtensorMap& md, const CUtensorMap& md2, const KArgs& a, int epi,
                 cudaStream_t s) {
   if (!g.a_mn && !g.b_mn) {
     switch (epi) {
-      case EPI_BF16: return launch_t<BN, false, false, EPI_BF16>(ma, mb, md, md2, a, s);
-      case EPI_BF16_RESID: return launch_t<BN, false, false, EPI_BF16_RESID>(ma, mb, md, md2, a, s);
-      case EPI_RELU2: return launch_t<BN, false, false, EPI_RELU2>(ma, mb, md, md2, a, s);
+      case EPI_BF16: return launch_t<BN, false, false, EPI_BF16, PAIR>(ma, mb, md, md2, a, s);
+      case EPI_BF16_RESID:
+        return launch_t<BN, false, false, EPI_BF16_RESID, PAIR>(ma, mb, md, md2, a, s);
+      case EPI_RELU2: return launch_t<BN, false, false, EPI_RELU2, PAIR>(ma, mb, md, md2, a, s);
       default: break;
     }
   } else if (!g.a_mn && g.b_mn) {
     switch (epi) {
-      case EPI_BF16: return launch_t<BN, false, true, EPI_BF16>(ma, mb, md, md2, a, s);
-      case EPI_DRELU2: return launch_t<BN, false, true, EPI_DRELU2>(ma, mb, md, md2, a, s);
+      case EPI_BF16: return launch_t<BN, false, true, EPI_BF16, PAIR>(ma, mb, md, md2, a, s);
+      case EPI_DRELU2: return launch_t<BN, false, true, EPI_DRELU2, PAIR>(ma, mb, md, md2, a, s);
       default: break;
     }
   } else if (g.a_mn && g.b_mn) {
     switch (epi) {
-      case EPI_F32: return launch_t<BN, true, true, EPI_F32>(ma, mb, md, md2, a, s);
-      case EPI_F32_ATOMIC: return launch_t<BN, true, true, EPI_F32_ATOMIC>(ma, mb, md, md2, a, s);
+      case EPI_F32: return launch_t<BN, true, true, EPI_F32, PAIR>(ma, mb, md, md2, a, s);
+      case EPI_F32_ATOMIC:
+        return launch_t<BN, true, true, EPI_F32_ATOMIC, PAIR>(ma, mb, md, md2, a, s);
       default: break;
     }
   }
@@ -466,11 +535,14 @@ int launch_gemm(const GemmDesc& g, cudaStream_t stream) {
   const int64_t pad256 = (g.N + 255) / 256 * 256 - g.N;
   const int64_t pad128 = (g.N + 127) / 128 * 128 - g.N;
   const int BN = (pad128 < pad256) ? 128 : 256;
+  // CTA pairs (256-row tiles, cta_group::2) whenever the 256-wide N tile is used.
+  const bool pair = (BN == 256) && g.M >= 256;
+  const int tile_m = pair ? 2 * BM : BM;
 
   KArgs a{};
   a.M = static_cast<int>(g.M);
   a.N = static_cast<int>(g.N);
-  a.num_m_blk = static_cast<int>((g.M + BM - 1) / BM);
+  a.num_m_blk = static_cast<int>((g.M + tile_m - 1) / tile_m);
   a.num_n_blk = static_cast<int>((g.N + BN - 1) / BN);
   a.kblk_total = static_cast<int>((g.K + BK - 1) / BK);
   a.splits = 1;
@@ -486,7 +558,7 @@ int launch_gemm(const GemmDesc& g, cudaStream_t stream) {
   int epi = g.epi;
   if (epi == EPI_F32 || epi == EPI_F32_ATOMIC) {
     const int tiles = a.num_m_blk * a.num_n_blk;
-    int s = choose_splits(tiles, a.kblk_total, sm_count());
+    int s = choose_splits(tiles, a.kblk_total, pair ? sm_count() / 2 : sm_count());
     a.kblk_per_split = (a.kblk_total + s - 1) / s;
     s = (a.kblk_total + a.kblk_per_split - 1) / a.kblk_per_split;  // no empty split
     a.splits = s;
@@ -511,10 +583,12 @@ int launch_gemm(const GemmDesc& g, cudaStream_t stream) {
   a.num_tiles = static_cast<int>(tiles64);
 
   CUtensorMap ma, mb;
+  const int b_rows = pair ? BN / 2 : BN;  // B rows one CTA stages
   int rc = g.a_mn ? make_map(&ma, g.A, g.M, g.K, g.lda, 64)
                   : make_map(&ma, g.A, g.K, g.M, g.lda, BM);
   if (rc) return rc;
-  rc = g.b_mn ? make_map(&mb, g.B, g.N, g.K, g.ldb, 64) : make_map(&mb, g.B, g.K, g.N, g.ldb, BN);
+  rc = g.b_mn ? make_map(&mb, g.B, g.N, g.K, g.ldb, 64)
+              : make_map(&mb, g.B, g.K, g.N, g.ldb, b_rows);
   if (rc) return rc;
   // Output maps: 32x32 boxes, bf16 with 64-byte swizzle or fp32 with 128-byte swizzle.
   CUtensorMap md, md2;
@@ -525,8 +599,9 @@ int launch_gemm(const GemmDesc& g, cudaStream_t stream) {
   if (rc) return rc;
   rc = make_out_map(&md2, g.D2 ? g.D2 : d_base, g.N, g.M, g.D2 ? g.ldd2 : d_ld, false);
   if (rc) return rc;
-  return BN == 256 ? dispatch_bn<256>(g, ma, mb, md, md2, a, epi, stream)
-                   : dispatch_bn<128>(g, ma, mb, md, md2, a, epi, stream);
+  if (pair) return dispatch_bn<256, true>(g, ma, mb, md, md2, a, epi, stream);
+  return BN == 256 ? dispatch_bn<256, false>(g, ma, mb, md, md2, a, epi, stream)
+                   : dispatch_bn<128, false>(g, ma, mb, md, md2, a, epi, stream);
 }
 
 }  // namespace qat

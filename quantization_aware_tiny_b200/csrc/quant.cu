@@ -4,9 +4,9 @@
 //
 // Quantization uses one warp per row.  The export kernel stages rows in shared
 // memory with 1-D bulk async copies (the copy engine, completing on an
-// mbarrier) two rows ahead of the row being quantized, so each warp keeps
-// ~12 KB in flight while it computes; the training-time kernel caches the row
-// in registers between its reduction and quantization passes.
+// mbarrier) one row ahead of the row being quantized, with up to 16 warps per
+// SM; the training-time kernel caches the row in registers between its
+// reduction and quantization passes.
 #include <algorithm>
 #include <cmath>
 
@@ -127,25 +127,97 @@ __device__ __forceinline__ RowQuant row_params(const ExportDescDev& d, float t1,
   return q;
 }
 
-__device__ __forceinline__ uint32_t codes4(const RowQuant& q, float4 v) {
-  const float c = q.clip;
-  return pack_codes(quant_code(fminf(fmaxf(v.x, -c), c), q.s, q.rs, q.bits),
-                    quant_code(fminf(fmaxf(v.y, -c), c), q.s, q.rs, q.bits),
-                    quant_code(fminf(fmaxf(v.z, -c), c), q.s, q.rs, q.bits),
-                    quant_code(fminf(fmaxf(v.w, -c), c), q.s, q.rs, q.bits));
+// ---- paired fp32 arithmetic (two IEEE round-to-nearest operations per instruction)
+__device__ __forceinline__ uint64_t f2u(float2 v) { return *reinterpret_cast<uint64_t*>(&v); }
+__device__ __forceinline__ float2 u2f(uint64_t v) { return *reinterpret_cast<float2*>(&v); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2u(a)), "l"(f2u(b)));
+  return u2f(d);
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2u(a)), "l"(f2u(b)));
+  return u2f(d);
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f2u(a)), "l"(f2u(b)), "l"(f2u(c)));
+  return u2f(d);
 }
 
-// A quantized row staged in shared memory (cols <= kExportMaxStagedCols).
+// Codes of two clipped weights on the row's grid, the same arithmetic as
+// quant_code (common.cuh) done pairwise: the Markstein-corrected quotient,
+// then the rounding offset 1.5 * 2^23 (see code_from_quotient).  For int6 the
+// second rounding rne(k / 4) is the same trick on k / 4, which
+// fma(k + offset, 1/4, -offset/4) produces exactly; 4 * (bits - offset bits)
+// is formed modulo 2^32.
+template <int BITS>
+__device__ __forceinline__ void codes2(const RowQuant& q, float a, float b, int& ca, int& cb) {
+  constexpr float kOff = 12582912.0f;  // 1.5 * 2^23
+  const float2 w = make_float2(fminf(fmaxf(a, -q.clip), q.clip), fminf(fmaxf(b, -q.clip), q.clip));
+  const float2 s2 = make_float2(-q.s, -q.s), r2 = make_float2(q.rs, q.rs);
+  const float2 q0 = mul2(w, r2);
+  const float2 rem = fma2(q0, s2, w);
+  const float2 x = fma2(rem, r2, q0);
+  const float2 t = add2(x, make_float2(kOff, kOff));  // kOff + rne(x)
+  if constexpr (BITS == 6) {
+    const float2 y = fma2(t, make_float2(0.25f, 0.25f), make_float2(-kOff / 4, -kOff / 4));
+    const float2 u = add2(y, make_float2(kOff, kOff));  // kOff + rne(k / 4)
+    ca = min(max(static_cast<int>(__float_as_uint(u.x) * 4u - 0x2D000000u), -128), 124);
+    cb = min(max(static_cast<int>(__float_as_uint(u.y) * 4u - 0x2D000000u), -128), 124);
+  } else {
+    ca = min(max(__float_as_int(t.x) - 0x4B400000, -127), 127);
+    cb = min(max(__float_as_int(t.y) - 0x4B400000, -127), 127);
+  }
+}
+
+template <int BITS>
+__device__ __forceinline__ uint32_t codes4_t(const RowQuant& q, float4 v) {
+  int c0, c1, c2, c3;
+  codes2<BITS>(q, v.x, v.y, c0, c1);
+  codes2<BITS>(q, v.z, v.w, c2, c3);
+  return pack_codes(c0, c1, c2, c3);
+}
+
+__device__ __forceinline__ uint32_t codes4(const RowQuant& q, float4 v) {
+  return q.bits == 6 ? codes4_t<6>(q, v) : codes4_t<8>(q, v);
+}
+
+template <int BITS>
+__device__ __forceinline__ void quantize_smem_row(const RowQuant& q, const float4* buf, int K4,
+                                                  uint32_t* out, int lane) {
+  int j = lane;
+  for (; j + 32 < K4; j += 64) {
+    const float4 a = buf[j], b = buf[j + 32];
+    const uint32_t ca = codes4_t<BITS>(q, a), cb = codes4_t<BITS>(q, b);
+    out[j] = ca;
+    out[j + 32] = cb;
+  }
+  if (j < K4) out[j] = codes4_t<BITS>(q, buf[j]);
+}
+
+// A quantized row staged in shared memory (cols <= the batch's buffer).
 __device__ __forceinline__ void export_row_smem(const ExportDescDev& d, int64_t row,
                                                 const float4* buf, int lane) {
   const int K4 = static_cast<int>(d.cols >> 2);
-  float t1 = 0.0f, t2 = 0.0f;
-  for (int j = lane; j < K4; j += 32) top2_push4(buf[j], t1, t2);
+  float t1 = 0.0f, t2 = 0.0f, u1 = 0.0f, u2 = 0.0f;
+  int j = lane;
+  for (; j + 32 < K4; j += 64) {
+    top2_push4(buf[j], t1, t2);
+    top2_push4(buf[j + 32], u1, u2);
+  }
+  if (j < K4) top2_push4(buf[j], t1, t2);
+  // merge this lane's two partial lists
+  const float n2 = fmaxf(fminf(t1, u1), fmaxf(t2, u2));
+  t1 = fmaxf(t1, u1);
+  t2 = n2;
   top2_warp(t1, t2);
   const RowQuant q = row_params(d, t1, t2);
   if (lane == 0) d.scales[row] = __float2half_rn(q.s);
   uint32_t* out = reinterpret_cast<uint32_t*>(reinterpret_cast<int8_t*>(d.dst) + row * d.cols);
-  for (int j = lane; j < K4; j += 32) out[j] = codes4(q, buf[j]);
+  if (q.bits == 6) quantize_smem_row<6>(q, buf, K4, out, lane);
+  else quantize_smem_row<8>(q, buf, K4, out, lane);
 }
 
 // A quantized row read from global memory (rows longer than the staging buffer).
@@ -214,19 +286,21 @@ __device__ __forceinline__ int find_desc(const ExportBatch& b, int64_t g) {
 __device__ __forceinline__ bool staged(const ExportDescDev& d) {
   return d.mode != QAT_EXPORT_FP16 && d.cols <= kExportMaxStagedCols;
 }
+// (the host sizes buf_bytes for the longest staged row, so staged rows fit)
 
 // One launch over all descriptors.  Warp w of the grid takes rows
 // w, w + W, w + 2W, ... (W = warps in the grid); row i of a warp goes to
-// buffer i % kExportBufs, and rows i+1, i+2 are in flight while row i is
-// quantized.  Rows that are not staged still arrive once on their buffer's
-// mbarrier so every buffer's phases stay in step with the row count.
-__global__ void __launch_bounds__(kExportWarps * 32, 1)
+// buffer i % kExportBufs, and row i+1 is in flight while row i is quantized.
+// Rows that are not staged still arrive once on their buffer's mbarrier so
+// every buffer's phases stay in step with the row count.
+__global__ void __launch_bounds__(kExportMaxWarps * 32, 1)
     export_batch_kernel(const __grid_constant__ ExportBatch b, int* err) {
   extern __shared__ __align__(128) uint8_t xsmem[];
   const int lane = threadIdx.x & 31;
   const int wib = threadIdx.x >> 5;
-  float4* bufs = reinterpret_cast<float4*>(xsmem + wib * kExportBufs * kExportBufBytes);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(xsmem + kExportWarps * kExportBufs * kExportBufBytes) +
+  const int nw = blockDim.x >> 5;
+  float4* bufs = reinterpret_cast<float4*>(xsmem + wib * kExportBufs * b.buf_bytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(xsmem + nw * kExportBufs * b.buf_bytes) +
                    wib * kExportBufs;
   __shared__ int abort_flag;
   if (threadIdx.x == 0) abort_flag = 0;
@@ -236,8 +310,8 @@ __global__ void __launch_bounds__(kExportWarps * 32, 1)
   }
   __syncthreads();
 
-  const int64_t W = static_cast<int64_t>(gridDim.x) * kExportWarps;
-  const int64_t gw = static_cast<int64_t>(blockIdx.x) * kExportWarps + wib;
+  const int64_t W = static_cast<int64_t>(gridDim.x) * nw;
+  const int64_t gw = static_cast<int64_t>(blockIdx.x) * nw + wib;
 
   auto issue = [&](int64_t i) {
     const int64_t g = gw + i * W;
@@ -247,7 +321,7 @@ __global__ void __launch_bounds__(kExportWarps * 32, 1)
     if (staged(d)) {
       const uint32_t bytes = static_cast<uint32_t>(d.cols * 4);
       mbar_arrive_expect_tx(&bars[slot], bytes);
-      bulk_load_1d(bufs + slot * (kExportBufBytes / 16), d.src + (g - d.row_begin) * d.cols, bytes,
+      bulk_load_1d(bufs + slot * (b.buf_bytes / 16), d.src + (g - d.row_begin) * d.cols, bytes,
                    &bars[slot]);
     } else {
       mbar_arrive(&bars[slot]);
@@ -264,7 +338,7 @@ __global__ void __launch_bounds__(kExportWarps * 32, 1)
     const ExportDescDev& d = b.d[find_desc(b, g)];
     const int64_t row = g - d.row_begin;
     if (d.mode == QAT_EXPORT_FP16) export_fp16_chunk(d, row, lane);
-    else if (staged(d)) export_row_smem(d, row, bufs + slot * (kExportBufBytes / 16), lane);
+    else if (staged(d)) export_row_smem(d, row, bufs + slot * (b.buf_bytes / 16), lane);
     else export_row_global(d, row, lane);
     // the buffer is read; order those reads before the copy engine refills it
     fence_proxy_async_smem();
@@ -342,18 +416,26 @@ int export_quantile_params(int64_t cols, int* m, float* frac) {
   return QAT_OK;
 }
 
-int launch_export_batch(const ExportBatch& b, cudaStream_t s) {
+int launch_export_batch(ExportBatch& b, cudaStream_t s) {
   if (b.total_rows == 0) return QAT_OK;
   static bool attr_done = false;
   if (!attr_done) {
     if (cudaFuncSetAttribute(export_batch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kExportSmemBytes) != cudaSuccess)
+                             kExportSmemBudget) != cudaSuccess)
       return QAT_ERR_CUDA;
     attr_done = true;
   }
-  const int64_t want = (b.total_rows + kExportWarps - 1) / kExportWarps;
+  int64_t longest = 4;  // longest staged row
+  for (int i = 0; i < b.n; ++i)
+    if (b.d[i].mode != QAT_EXPORT_FP16 && b.d[i].cols <= kExportMaxStagedCols)
+      longest = std::max(longest, b.d[i].cols);
+  b.buf_bytes = static_cast<int>((longest * 4 + 127) / 128 * 128);
+  const int per_warp = kExportBufs * (b.buf_bytes + 8);
+  const int warps = std::max(1, std::min(kExportMaxWarps, kExportSmemBudget / per_warp));
+  const int smem = warps * per_warp;
+  const int64_t want = (b.total_rows + warps - 1) / warps;
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, sm_count())));
-  export_batch_kernel<<<grid, kExportWarps * 32, kExportSmemBytes, s>>>(b, device_error_ptr());
+  export_batch_kernel<<<grid, warps * 32, smem, s>>>(b, device_error_ptr());
   count_launch();
   return cuda_status(cudaGetLastError());
 }

@@ -22,7 +22,7 @@ struct ExportDescDev {
 
 struct ExportBatch {
   int n;
-  int pad;
+  int buf_bytes;  // bytes of one row buffer (longest staged row, rounded to 128)
   int64_t total_rows;
   ExportDescDev d[QAT_EXPORT_MAX_DESCS];
 };
@@ -30,19 +30,19 @@ struct ExportBatch {
 // Chunk length of the fp16 passthrough "rows".
 constexpr int64_t kFp16Chunk = 4096;
 
-// Export kernel staging: warps per block, row buffers per warp, the longest
-// row staged in shared memory (longer rows are read from global memory).
-constexpr int kExportWarps = 8;
-constexpr int kExportBufs = 3;
+// Export kernel staging: row buffers per warp, the longest row staged in
+// shared memory (longer rows are read from global memory), the shared memory
+// a block may use and the most warps per block.  Buffers are sized for the
+// longest staged row of the batch, so short-row state dicts get more warps.
+constexpr int kExportBufs = 2;
 constexpr int64_t kExportMaxStagedCols = 2048;
-constexpr int kExportBufBytes = static_cast<int>(kExportMaxStagedCols) * 4;
-constexpr int kExportSmemBytes =
-    kExportWarps * kExportBufs * kExportBufBytes + kExportWarps * kExportBufs * 8;
+constexpr int kExportSmemBudget = 224 * 1024;
+constexpr int kExportMaxWarps = 16;
 
 int launch_quantize_weights(const float* W, int N, int K, int bits, int8_t* codes, float* scales,
                             __nv_bfloat16* operand, cudaStream_t s);
 int export_quantile_params(int64_t cols, int* m, float* frac);
-int launch_export_batch(const ExportBatch& b, cudaStream_t s);
+int launch_export_batch(ExportBatch& b, cudaStream_t s);
 int launch_dequant(const int8_t* codes, const __half* scales, int64_t rows, int64_t cols,
                    int out_bf16, void* out, cudaStream_t s);
 
