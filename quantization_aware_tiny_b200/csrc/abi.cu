@@ -327,9 +327,9 @@ int quantize_rows_export(const float* W, int64_t rows, int64_t cols, int32_t bit
 
 int quantize_export_batch(const qat_export_desc* descs, int32_t n, qat_stream_t stream) {
   if (!descs || n <= 0 || n > QAT_EXPORT_MAX_DESCS) return QAT_ERR_ARG;
-  static thread_local ExportBatch b;  // ~18 KB: kept off the stack
+  static thread_local ExportBatch b;  // ~20 KB: kept off the stack
   b.n = n;
-  b.total_rows = 0;
+  b.total_units = 0;
   for (int i = 0; i < n; ++i) {
     const qat_export_desc& s = descs[i];
     ExportDescDev& d = b.d[i];
@@ -342,23 +342,25 @@ int quantize_export_batch(const qat_export_desc* descs, int32_t n, qat_stream_t 
     d.m = 1;
     d.frac = 0.0f;
     d.pad = 0;
-    d.row_begin = b.total_rows;
+    d.unit_begin = b.total_units;
     if (s.mode == QAT_EXPORT_FP16) {
       d.numel = s.rows * s.cols;
       d.cols = kFp16Chunk;
       d.rows = (d.numel + kFp16Chunk - 1) / kFp16Chunk;
+      d.unit_rows = 1;
     } else if (s.mode == 6 || s.mode == 8) {
       if (!s.scales) return QAT_ERR_ARG;
       if (!dim_ok(s.cols)) return QAT_ERR_SHAPE;
       d.rows = s.rows;
       d.cols = s.cols;
       d.numel = s.rows * s.cols;
+      d.unit_rows = kExportUnitRows;
       const int rc = export_quantile_params(s.cols, &d.m, &d.frac);
       if (rc) return rc;
     } else {
       return QAT_ERR_ARG;
     }
-    b.total_rows += d.rows;
+    b.total_units += (d.rows + d.unit_rows - 1) / d.unit_rows;
   }
   return launch_export_batch(b, stream);
 }

@@ -28,18 +28,25 @@ constexpr int kThreads = 192;
 
 // PAIR: the CTA pair of a 2-CTA cluster computes a 256 x BN tile with
 // tcgen05 cta_group::2; each CTA stages 128 rows of A and BN/2 rows of B.
-template <int BN, bool PAIR>
+// HAS_R: the epilogue reads a bf16 tensor of the output's shape (residual or
+// saved pre-activation), brought in by TMA ahead of use.
+template <int BN, bool PAIR, bool HAS_R = false>
 struct Cfg {
   static constexpr int B_ROWS = PAIR ? BN / 2 : BN;  // B rows staged by one CTA
   static constexpr int TILE_M = PAIR ? 2 * BM : BM;
-  static constexpr int STAGES = (B_ROWS == 256) ? 4 : 6;
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int TMEM_COLS = 2 * BN;  // 256 or 512: powers of two as required
+  static constexpr int TMEM_COLS = (2 * BN <= 256) ? 256 : 512;  // a power of two >= 2*BN
   static constexpr int STAGING_BYTES = 4 * 8192;  // per epilogue warp: 8 KB of output chunks
-  static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + STAGING_BYTES + BAR_BYTES + 1024;
+  static constexpr int R_BUFS = 4;                // R chunks in flight per epilogue warp
+  static constexpr int R_BYTES = HAS_R ? 4 * R_BUFS * 2048 : 0;
+  static constexpr int BAR_BYTES = 512;
+  static constexpr int FIXED = STAGING_BYTES + R_BYTES + BAR_BYTES + 1024;
+  static constexpr int STAGES_FIT = (232448 - FIXED) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + FIXED;
+  static_assert(STAGES >= 3, "pipeline too shallow");
 };
 
 struct KArgs {
@@ -118,20 +125,22 @@ template <int BN, bool A_MN, bool B_MN, int EPI, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmD, const __grid_constant__ CUtensorMap tmD2,
-                const KArgs p) {
-  using C = Cfg<BN, PAIR>;
+                const __grid_constant__ CUtensorMap tmR, const KArgs p) {
+  using C = Cfg<BN, PAIR, (EPI == EPI_BF16_RESID || EPI == EPI_DRELU2)>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::STAGES * C::A_BYTES;
   uint8_t* staging = smem + C::STAGES * C::STAGE_BYTES;  // 1024-aligned
-  uint64_t* full = reinterpret_cast<uint64_t*>(staging + C::STAGING_BYTES);
+  uint8_t* rstage = staging + C::STAGING_BYTES;          // R chunks (HAS_R)
+  uint64_t* full = reinterpret_cast<uint64_t*>(rstage + C::R_BYTES);
   uint64_t* empty = full + C::STAGES;
   uint64_t* tfull = empty + C::STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* mma_done = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* rbar = mma_done + 1;  // 4 epilogue warps x R_BUFS
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rbar + 4 * C::R_BUFS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* prod_pos = const_cast<int*>(abort_flag) + 1;  // producer ring position at exit
   int* mma_pos = prod_pos + 1;                        // MMA ring position at exit
@@ -155,6 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tempty[b], PAIR ? 8 : 4);
     }
     mbar_init(mma_done, 1);
+    for (int i = 0; i < 4 * C::R_BUFS; ++i) mbar_init(&rbar[i], 1);
     *abort_flag = 0;
     *prod_pos = 0;
     *mma_pos = 0;
@@ -162,6 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
     tma_prefetch_desc(&tmD);
+    if constexpr (EPI == EPI_BF16_RESID || EPI == EPI_DRELU2) tma_prefetch_desc(&tmR);
   }
   if (warp == 1) {
     if constexpr (PAIR) {
@@ -292,36 +303,56 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------ epilogue (warps 2..5)
     constexpr bool kF32 = (EPI == EPI_F32 || EPI == EPI_F32_ATOMIC);
+    constexpr bool kR = (EPI == EPI_BF16_RESID || EPI == EPI_DRELU2);
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const uint32_t wbuf = smem_u32(staging) + static_cast<uint32_t>(q) * 8192u;
+    uint8_t* rbuf = rstage + q * C::R_BUFS * 2048;
+    uint64_t* rb = rbar + q * C::R_BUFS;
     const bool keep_pre = (EPI == EPI_RELU2) && p.D != nullptr;
     int acc = 0;
     uint32_t acc_phase = 0;
     uint32_t chunk = 0;
+    uint32_t r_issued = 0, r_used = 0;  // R ring: chunks requested / consumed
     // the leader's tmem-empty barrier, which both CTAs' epilogues release
     const uint32_t tempty_leader = PAIR ? mapa_shared(smem_u32(tempty), 0) : smem_u32(tempty);
     for (int tile = tile0; tile < p.num_tiles; tile += tile_step) {
       const int nb = tile % p.num_n_blk;
       const int mb = (tile / p.num_n_blk) % p.num_m_blk;
-      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err)) break;
-      tc_fence_after();
       const int row0 = mb * C::TILE_M + static_cast<int>(rank) * BM + q * 32;
-      const int64_t row = static_cast<int64_t>(row0) + lane;
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                             static_cast<uint32_t>(acc * BN);
       const int ncols = min(BN, p.N - nb * BN);
       const int nchunks = (ncols + 31) / 32;
+      // Request this tile's first R chunks before waiting for the accumulator.
+      auto issue_r = [&](int c) {
+        if (lane == 0) {
+          const uint32_t slot = r_issued % C::R_BUFS;
+          mbar_arrive_expect_tx(&rb[slot], 2048);
+          tma_load_2d(&tmR, &rb[slot], rbuf + slot * 2048, nb * BN + c * 32, row0);
+        }
+        ++r_issued;
+      };
+      if constexpr (kR) {
+        for (int c = 0; c < nchunks && c < C::R_BUFS; ++c) issue_r(c);
+      }
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err)) break;
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(acc * BN);
+      bool ok = true;
 #pragma unroll 1
       for (int c = 0; c < nchunks; ++c, ++chunk) {
         const int col0 = nb * BN + c * 32;
         uint4 rin[4] = {};
-        if constexpr (EPI == EPI_BF16_RESID || EPI == EPI_DRELU2) {
-          if (row < p.M) {
-            const uint4* src = reinterpret_cast<const uint4*>(p.R + row * p.ldr + col0);
+        if constexpr (kR) {
+          const uint32_t slot = r_used % C::R_BUFS;
+          if (!mbar_wait(&rb[slot], (r_used / C::R_BUFS) & 1u, abort_flag, p.err)) { ok = false; break; }
+          const uint32_t base = smem_u32(rbuf + slot * 2048) + static_cast<uint32_t>(lane) * 64u;
+          const int sw = (lane >> 1) & 3;
 #pragma unroll
-            for (int g = 0; g < 4; ++g)
-              if (col0 + 8 * g < p.N) rin[g] = src[g];
-          }
+          for (int g = 0; g < 4; ++g) rin[g] = ld_shared_v4(base + (static_cast<uint32_t>(g ^ sw) << 4));
+          ++r_used;
+          fence_proxy_async_smem();  // reads done before the slot is refilled by TMA
+          __syncwarp();
+          if (c + C::R_BUFS < nchunks) issue_r(c + C::R_BUFS);
         }
         uint32_t r[32];
         tmem_ld32(t_row + static_cast<uint32_t>(c * 32), r);
@@ -355,8 +386,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           bulk_commit();
         }
       }
+      if (!ok) break;
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
+    }
+    // R chunks requested but not consumed (only after a timeout): let them land.
+    if (kR && lane == 0) {
+      for (uint32_t k = r_used; k < r_issued; ++k)
+        mbar_drain(&rb[k % C::R_BUFS], (k / C::R_BUFS) & 1u);
     }
     if (lane == 0) bulk_wait_all();  // every output chunk written before the block exits
     __syncwarp();
@@ -441,8 +478,8 @@ int make_out_map(CUtensorMap* m, const void* base, int64_t inner, int64_t outer,
 
 template <int BN, bool A_MN, bool B_MN, int EPI, bool PAIR>
 int launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& md,
-             const CUtensorMap& md2, const KArgs& a, cudaStream_t s) {
-  using C = Cfg<BN, PAIR>;
+             const CUtensorMap& md2, const CUtensorMap& mr, const KArgs& a, cudaStream_t s) {
+  using C = Cfg<BN, PAIR, (EPI == EPI_BF16_RESID || EPI == EPI_DRELU2)>;
   auto kern = gemm_kernel<BN, A_MN, B_MN, EPI, PAIR>;
   static bool attr_done = false;  // per instantiation; set before first launch
   if (!attr_done) {
@@ -465,34 +502,44 @@ int launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& md
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ma, mb, md, md2, a);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ma, mb, md, md2, mr, a);
   count_launch();
   return cuda_status(e == cudaSuccess ? cudaGetLastError() : e);
 }
 
 template <int BN, bool PAIR>
 int dispatch_bn(const GemmDesc& g, const CUtensorMap& ma, const CUtensorMap& mb,
-                const CUtensorMap& md, const CUtensorMap& md2, const KArgs& a, int epi,
-                cudaStream_t s) {
+                const CUtensorMap& md, const CUtensorMap& md2, const CUtensorMap& mr,
+                const KArgs& a, int epi, cudaStream_t s) {
+  if constexpr (BN % 128 != 0) {  // 160 / 192: forward (K-major B) epilogues only
+    if (g.a_mn || g.b_mn) return QAT_ERR_ARG;
+    switch (epi) {
+      case EPI_BF16: return launch_t<BN, false, false, EPI_BF16, PAIR>(ma, mb, md, md2, mr, a, s);
+      case EPI_BF16_RESID:
+        return launch_t<BN, false, false, EPI_BF16_RESID, PAIR>(ma, mb, md, md2, mr, a, s);
+      case EPI_RELU2: return launch_t<BN, false, false, EPI_RELU2, PAIR>(ma, mb, md, md2, mr, a, s);
+      default: return QAT_ERR_ARG;
+    }
+  }
   if (!g.a_mn && !g.b_mn) {
     switch (epi) {
-      case EPI_BF16: return launch_t<BN, false, false, EPI_BF16, PAIR>(ma, mb, md, md2, a, s);
+      case EPI_BF16: return launch_t<BN, false, false, EPI_BF16, PAIR>(ma, mb, md, md2, mr, a, s);
       case EPI_BF16_RESID:
-        return launch_t<BN, false, false, EPI_BF16_RESID, PAIR>(ma, mb, md, md2, a, s);
-      case EPI_RELU2: return launch_t<BN, false, false, EPI_RELU2, PAIR>(ma, mb, md, md2, a, s);
+        return launch_t<BN, false, false, EPI_BF16_RESID, PAIR>(ma, mb, md, md2, mr, a, s);
+      case EPI_RELU2: return launch_t<BN, false, false, EPI_RELU2, PAIR>(ma, mb, md, md2, mr, a, s);
       default: break;
     }
   } else if (!g.a_mn && g.b_mn) {
     switch (epi) {
-      case EPI_BF16: return launch_t<BN, false, true, EPI_BF16, PAIR>(ma, mb, md, md2, a, s);
-      case EPI_DRELU2: return launch_t<BN, false, true, EPI_DRELU2, PAIR>(ma, mb, md, md2, a, s);
+      case EPI_BF16: return launch_t<BN, false, true, EPI_BF16, PAIR>(ma, mb, md, md2, mr, a, s);
+      case EPI_DRELU2: return launch_t<BN, false, true, EPI_DRELU2, PAIR>(ma, mb, md, md2, mr, a, s);
       default: break;
     }
   } else if (g.a_mn && g.b_mn) {
     switch (epi) {
-      case EPI_F32: return launch_t<BN, true, true, EPI_F32, PAIR>(ma, mb, md, md2, a, s);
+      case EPI_F32: return launch_t<BN, true, true, EPI_F32, PAIR>(ma, mb, md, md2, mr, a, s);
       case EPI_F32_ATOMIC:
-        return launch_t<BN, true, true, EPI_F32_ATOMIC, PAIR>(ma, mb, md, md2, a, s);
+        return launch_t<BN, true, true, EPI_F32_ATOMIC, PAIR>(ma, mb, md, md2, mr, a, s);
       default: break;
     }
   }
@@ -531,12 +578,21 @@ int launch_gemm(const GemmDesc& g, cudaStream_t stream) {
     return QAT_ERR_SHAPE;
   if (g.M > (1ll << 31) - 256 || g.N > (1 << 30) || g.K > (1ll << 31) - 256) return QAT_ERR_SHAPE;
 
-  // N tile: 256 unless 128 wastes fewer padded columns.
-  const int64_t pad256 = (g.N + 255) / 256 * 256 - g.N;
-  const int64_t pad128 = (g.N + 127) / 128 * 128 - g.N;
-  const int BN = (pad128 < pad256) ? 128 : 256;
-  // CTA pairs (256-row tiles, cta_group::2) whenever the 256-wide N tile is used.
-  const bool pair = (BN == 256) && g.M >= 256;
+  // N tile.  Forward GEMMs (K-major B) with at least 256 rows run on CTA pairs
+  // with the widest of 256 / 192 / 160 that divides N, else 256; the other
+  // GEMMs take 256 (paired when M >= 256) unless 128 wastes fewer columns.
+  int BN;
+  bool pair;
+  const bool kmajor_fwd = !g.a_mn && !g.b_mn && g.epi != EPI_F32 && g.epi != EPI_F32_ATOMIC;
+  if (kmajor_fwd && g.M >= 256 && g.N >= 160) {
+    pair = true;
+    BN = (g.N % 256 == 0) ? 256 : (g.N % 192 == 0) ? 192 : (g.N % 160 == 0) ? 160 : 256;
+  } else {
+    const int64_t pad256 = (g.N + 255) / 256 * 256 - g.N;
+    const int64_t pad128 = (g.N + 127) / 128 * 128 - g.N;
+    BN = (pad128 < pad256) ? 128 : 256;
+    pair = (BN == 256) && g.M >= 256;
+  }
   const int tile_m = pair ? 2 * BM : BM;
 
   KArgs a{};
@@ -599,9 +655,20 @@ int launch_gemm(const GemmDesc& g, cudaStream_t stream) {
   if (rc) return rc;
   rc = make_out_map(&md2, g.D2 ? g.D2 : d_base, g.N, g.M, g.D2 ? g.ldd2 : d_ld, false);
   if (rc) return rc;
-  if (pair) return dispatch_bn<256, true>(g, ma, mb, md, md2, a, epi, stream);
-  return BN == 256 ? dispatch_bn<256, false>(g, ma, mb, md, md2, a, epi, stream)
-                   : dispatch_bn<128, false>(g, ma, mb, md, md2, a, epi, stream);
+  CUtensorMap mr = md;
+  if (g.epi == EPI_BF16_RESID || g.epi == EPI_DRELU2) {
+    rc = make_out_map(&mr, g.R, g.N, g.M, g.ldr, false);
+    if (rc) return rc;
+  }
+  if (pair) {
+    switch (BN) {
+      case 160: return dispatch_bn<160, true>(g, ma, mb, md, md2, mr, a, epi, stream);
+      case 192: return dispatch_bn<192, true>(g, ma, mb, md, md2, mr, a, epi, stream);
+      default: return dispatch_bn<256, true>(g, ma, mb, md, md2, mr, a, epi, stream);
+    }
+  }
+  return BN == 256 ? dispatch_bn<256, false>(g, ma, mb, md, md2, mr, a, epi, stream)
+                   : dispatch_bn<128, false>(g, ma, mb, md, md2, mr, a, epi, stream);
 }
 
 }  // namespace qat

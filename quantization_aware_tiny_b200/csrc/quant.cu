@@ -99,16 +99,22 @@ __device__ __forceinline__ void top2_push4(float4 v, float& t1, float& t2) {
   top2_push(fabsf(v.w), t1, t2);
 }
 // Merge the 32 lanes' top-2 lists; every lane ends with the row's top two.
+// The values are >= 0, so their bit patterns order like unsigned integers and
+// one warp-wide integer max finds the largest, M.  The second largest (with
+// multiplicity) is M when two lanes hold M, else the largest of every lane's
+// list with one M removed.
 __device__ __forceinline__ void top2_warp(float& t1, float& t2) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float b1 = __shfl_xor_sync(0xffffffffu, t1, o);
-    const float b2 = __shfl_xor_sync(0xffffffffu, t2, o);
-    const float n2 = fmaxf(fminf(t1, b1), fmaxf(t2, b2));
-    t1 = fmaxf(t1, b1);
-    t2 = n2;
-  }
+  const uint32_t m = __reduce_max_sync(0xffffffffu, __float_as_uint(t1));
+  const bool has = __float_as_uint(t1) == m;
+  const uint32_t holders = __ballot_sync(0xffffffffu, has);
+  const uint32_t cand = __float_as_uint(has ? t2 : t1);
+  const uint32_t second = __reduce_max_sync(0xffffffffu, cand);
+  t1 = __uint_as_float(m);
+  t2 = __popc(holders) >= 2 ? t1 : __uint_as_float(second);
 }
+
+// fl32(1 / 127), correctly rounded (0x3C010204).
+constexpr float kRcp127 = 0.00787401571869850158691406f;
 
 struct RowQuant {
   float clip, s, rs;
@@ -121,7 +127,7 @@ __device__ __forceinline__ RowQuant row_params(const ExportDescDev& d, float t1,
   const float v_lo = (d.m == 2) ? t2 : t1;
   RowQuant q;
   q.clip = __fadd_rn(v_lo, __fmul_rn(d.frac, __fsub_rn(v_hi, v_lo)));
-  q.s = div_rn(fmaxf(q.clip, 1e-12f), 127.0f);
+  q.s = div_by_scale(fmaxf(q.clip, 1e-12f), 127.0f, kRcp127);
   q.rs = __frcp_rn(q.s);
   q.bits = d.mode;
   return q;
@@ -146,22 +152,32 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
   return u2f(d);
 }
 
-// Codes of two clipped weights on the row's grid, the same arithmetic as
-// quant_code (common.cuh) done pairwise: the Markstein-corrected quotient,
-// then the rounding offset 1.5 * 2^23 (see code_from_quotient).  For int6 the
-// second rounding rne(k / 4) is the same trick on k / 4, which
+// Codes of two weights on the row's grid, the same arithmetic as quant_code
+// (common.cuh) done pairwise: the Markstein-corrected quotient, then the
+// rounding offset 1.5 * 2^23 (see code_from_quotient).  For int6 the second
+// rounding rne(k / 4) is the same trick on k / 4, which
 // fma(k + offset, 1/4, -offset/4) produces exactly; 4 * (bits - offset bits)
 // is formed modulo 2^32.
-template <int BITS>
+//
+// CLIP = false skips clamping w to [-clip, clip].  That is exact when
+// clip >= v_hi / 2 (always so for rows up to 32,768 columns, where the
+// interpolation fraction exceeds 0.947): only entries with |w| > clip differ,
+// their quotient |w / s| then lies in (127, 254], and after the grid's clamp
+// their code equals the code of +-clip itself (+124 / -128 for int6,
+// +-127 for int8); the offset trick stays exact for |x| < 2^22.
+template <int BITS, bool CLIP>
 __device__ __forceinline__ void codes2(const RowQuant& q, float a, float b, int& ca, int& cb) {
   constexpr float kOff = 12582912.0f;  // 1.5 * 2^23
-  const float2 w = make_float2(fminf(fmaxf(a, -q.clip), q.clip), fminf(fmaxf(b, -q.clip), q.clip));
+  const float2 w = CLIP ? make_float2(fminf(fmaxf(a, -q.clip), q.clip),
+                                      fminf(fmaxf(b, -q.clip), q.clip))
+                        : make_float2(a, b);
   const float2 s2 = make_float2(-q.s, -q.s), r2 = make_float2(q.rs, q.rs);
   const float2 q0 = mul2(w, r2);
   const float2 rem = fma2(q0, s2, w);
   const float2 x = fma2(rem, r2, q0);
   const float2 t = add2(x, make_float2(kOff, kOff));  // kOff + rne(x)
   if constexpr (BITS == 6) {
+    // k = rne(x) >= -254 gives 4 rne(k / 4) >= -256: both clamps can bind
     const float2 y = fma2(t, make_float2(0.25f, 0.25f), make_float2(-kOff / 4, -kOff / 4));
     const float2 u = add2(y, make_float2(kOff, kOff));  // kOff + rne(k / 4)
     ca = min(max(static_cast<int>(__float_as_uint(u.x) * 4u - 0x2D000000u), -128), 124);
@@ -172,52 +188,82 @@ __device__ __forceinline__ void codes2(const RowQuant& q, float a, float b, int&
   }
 }
 
-template <int BITS>
+// Four codes packed little-endian into a word (byte permutes).
+__device__ __forceinline__ uint32_t pack4(int c0, int c1, int c2, int c3) {
+  const uint32_t lo = __byte_perm(static_cast<uint32_t>(c0), static_cast<uint32_t>(c1), 0x0040);
+  const uint32_t hi = __byte_perm(static_cast<uint32_t>(c2), static_cast<uint32_t>(c3), 0x0040);
+  return __byte_perm(lo, hi, 0x5410);
+}
+
+template <int BITS, bool CLIP>
 __device__ __forceinline__ uint32_t codes4_t(const RowQuant& q, float4 v) {
   int c0, c1, c2, c3;
-  codes2<BITS>(q, v.x, v.y, c0, c1);
-  codes2<BITS>(q, v.z, v.w, c2, c3);
-  return pack_codes(c0, c1, c2, c3);
+  codes2<BITS, CLIP>(q, v.x, v.y, c0, c1);
+  codes2<BITS, CLIP>(q, v.z, v.w, c2, c3);
+  return pack4(c0, c1, c2, c3);
 }
 
 __device__ __forceinline__ uint32_t codes4(const RowQuant& q, float4 v) {
-  return q.bits == 6 ? codes4_t<6>(q, v) : codes4_t<8>(q, v);
+  return q.bits == 6 ? codes4_t<6, true>(q, v) : codes4_t<8, true>(q, v);
 }
 
-template <int BITS>
+#ifndef QAT_EXPORT_UNROLL
+#define QAT_EXPORT_UNROLL 4
+#endif
+// float4 groups per lane and loop iteration in the shared-memory passes: more
+// independent dependency chains per warp.
+constexpr int kUnroll = QAT_EXPORT_UNROLL;
+
+template <int BITS, bool CLIP>
 __device__ __forceinline__ void quantize_smem_row(const RowQuant& q, const float4* buf, int K4,
                                                   uint32_t* out, int lane) {
   int j = lane;
-  for (; j + 32 < K4; j += 64) {
-    const float4 a = buf[j], b = buf[j + 32];
-    const uint32_t ca = codes4_t<BITS>(q, a), cb = codes4_t<BITS>(q, b);
-    out[j] = ca;
-    out[j + 32] = cb;
+  for (; j + 32 * (kUnroll - 1) < K4; j += 32 * kUnroll) {
+    float4 v[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) v[u] = buf[j + 32 * u];
+    uint32_t c[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) c[u] = codes4_t<BITS, CLIP>(q, v[u]);
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) out[j + 32 * u] = c[u];
   }
-  if (j < K4) out[j] = codes4_t<BITS>(q, buf[j]);
+  for (; j < K4; j += 32) out[j] = codes4_t<BITS, CLIP>(q, buf[j]);
 }
 
 // A quantized row staged in shared memory (cols <= the batch's buffer).
 __device__ __forceinline__ void export_row_smem(const ExportDescDev& d, int64_t row,
                                                 const float4* buf, int lane) {
   const int K4 = static_cast<int>(d.cols >> 2);
-  float t1 = 0.0f, t2 = 0.0f, u1 = 0.0f, u2 = 0.0f;
+  float t1[kUnroll], t2[kUnroll];
+#pragma unroll
+  for (int u = 0; u < kUnroll; ++u) t1[u] = t2[u] = 0.0f;
   int j = lane;
-  for (; j + 32 < K4; j += 64) {
-    top2_push4(buf[j], t1, t2);
-    top2_push4(buf[j + 32], u1, u2);
+  for (; j + 32 * (kUnroll - 1) < K4; j += 32 * kUnroll) {
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) top2_push4(buf[j + 32 * u], t1[u], t2[u]);
   }
-  if (j < K4) top2_push4(buf[j], t1, t2);
-  // merge this lane's two partial lists
-  const float n2 = fmaxf(fminf(t1, u1), fmaxf(t2, u2));
-  t1 = fmaxf(t1, u1);
-  t2 = n2;
-  top2_warp(t1, t2);
-  const RowQuant q = row_params(d, t1, t2);
+  for (; j < K4; j += 32) top2_push4(buf[j], t1[0], t2[0]);
+  // merge this lane's partial lists
+#pragma unroll
+  for (int u = 1; u < kUnroll; ++u) {
+    const float n2 = fmaxf(fminf(t1[0], t1[u]), fmaxf(t2[0], t2[u]));
+    t1[0] = fmaxf(t1[0], t1[u]);
+    t2[0] = n2;
+  }
+  float a1 = t1[0], a2 = t2[0];
+  top2_warp(a1, a2);
+  const RowQuant q = row_params(d, a1, a2);
   if (lane == 0) d.scales[row] = __float2half_rn(q.s);
   uint32_t* out = reinterpret_cast<uint32_t*>(reinterpret_cast<int8_t*>(d.dst) + row * d.cols);
-  if (q.bits == 6) quantize_smem_row<6>(q, buf, K4, out, lane);
-  else quantize_smem_row<8>(q, buf, K4, out, lane);
+  const bool clip = a1 > 2.0f * q.clip;  // see codes2: clamping needed only then
+  if (q.bits == 6) {
+    if (clip) quantize_smem_row<6, true>(q, buf, K4, out, lane);
+    else quantize_smem_row<6, false>(q, buf, K4, out, lane);
+  } else {
+    if (clip) quantize_smem_row<8, true>(q, buf, K4, out, lane);
+    else quantize_smem_row<8, false>(q, buf, K4, out, lane);
+  }
 }
 
 // A quantized row read from global memory (rows longer than the staging buffer).
@@ -272,13 +318,13 @@ __device__ __forceinline__ void export_fp16_chunk(const ExportDescDev& d, int64_
     reinterpret_cast<__half*>(d.dst)[e] = __float2half_rn(d.src[e]);
 }
 
-// Descriptor owning global row g (row_begin is non-decreasing; the last
-// descriptor with row_begin <= g).
-__device__ __forceinline__ int find_desc(const ExportBatch& b, int64_t g) {
+// Descriptor owning work unit u (unit_begin is non-decreasing; the last
+// descriptor with unit_begin <= u).
+__device__ __forceinline__ int find_desc(const ExportBatch& b, int64_t u) {
   int lo = 0, hi = b.n - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (b.d[mid].row_begin <= g) lo = mid; else hi = mid - 1;
+    if (b.d[mid].unit_begin <= u) lo = mid; else hi = mid - 1;
   }
   return lo;
 }
@@ -288,11 +334,41 @@ __device__ __forceinline__ bool staged(const ExportDescDev& d) {
 }
 // (the host sizes buf_bytes for the longest staged row, so staged rows fit)
 
-// One launch over all descriptors.  Warp w of the grid takes rows
-// w, w + W, w + 2W, ... (W = warps in the grid); row i of a warp goes to
-// buffer i % kExportBufs, and row i+1 is in flight while row i is quantized.
-// Rows that are not staged still arrive once on their buffer's mbarrier so
-// every buffer's phases stay in step with the row count.
+// A warp's position in its sequence of rows: the row `row` (of [row, row_end)
+// in work unit `unit`) of descriptor `d`; d < 0 once the sequence is done.
+struct RowPos {
+  int64_t unit, row, row_end;
+  int d;
+};
+
+__device__ __forceinline__ RowPos unit_start(const ExportBatch& b, int64_t u) {
+  RowPos p;
+  p.unit = u;
+  if (u >= b.total_units) {
+    p.d = -1;
+    p.row = p.row_end = 0;
+    return p;
+  }
+  p.d = find_desc(b, u);
+  const ExportDescDev& d = b.d[p.d];
+  p.row = (u - d.unit_begin) * d.unit_rows;
+  p.row_end = min(p.row + d.unit_rows, d.rows);
+  return p;
+}
+
+__device__ __forceinline__ RowPos next_row(const ExportBatch& b, RowPos p, int64_t W) {
+  if (p.d < 0) return p;
+  if (++p.row < p.row_end) return p;
+  return unit_start(b, p.unit + W);
+}
+
+// One launch over all descriptors.  Work units are runs of up to
+// kExportUnitRows consecutive rows of one tensor (one chunk for fp16
+// passthrough); warp w of the grid takes units w, w + W, ... (W = warps in the
+// grid) and streams their rows through kExportBufs shared-memory buffers: the
+// next rows are in flight while this one is quantized.  Rows that are not staged still
+// arrive once on their buffer's mbarrier so every buffer's phases stay in
+// step with the row count.
 __global__ void __launch_bounds__(kExportMaxWarps * 32, 1)
     export_batch_kernel(const __grid_constant__ ExportBatch b, int* err) {
   extern __shared__ __align__(128) uint8_t xsmem[];
@@ -312,44 +388,49 @@ __global__ void __launch_bounds__(kExportMaxWarps * 32, 1)
 
   const int64_t W = static_cast<int64_t>(gridDim.x) * nw;
   const int64_t gw = static_cast<int64_t>(blockIdx.x) * nw + wib;
+  const int stride = b.buf_bytes / 16;
 
-  auto issue = [&](int64_t i) {
-    const int64_t g = gw + i * W;
-    if (g >= b.total_rows || lane != 0) return;
-    const int slot = static_cast<int>(i % kExportBufs);
-    const ExportDescDev& d = b.d[find_desc(b, g)];
+  auto issue = [&](const RowPos& p, int slot) {
+    if (p.d < 0 || lane != 0) return;
+    const ExportDescDev& d = b.d[p.d];
     if (staged(d)) {
       const uint32_t bytes = static_cast<uint32_t>(d.cols * 4);
       mbar_arrive_expect_tx(&bars[slot], bytes);
-      bulk_load_1d(bufs + slot * (b.buf_bytes / 16), d.src + (g - d.row_begin) * d.cols, bytes,
-                   &bars[slot]);
+      bulk_load_1d(bufs + slot * stride, d.src + p.row * d.cols, bytes, &bars[slot]);
     } else {
       mbar_arrive(&bars[slot]);
     }
   };
 
-  for (int i = 0; i < kExportBufs; ++i) issue(i);
-  int64_t i = 0;
-  for (; gw + i * W < b.total_rows; ++i) {
-    const int64_t g = gw + i * W;
-    const int slot = static_cast<int>(i % kExportBufs);
-    const uint32_t parity = static_cast<uint32_t>((i / kExportBufs) & 1);
-    if (!mbar_wait(&bars[slot], parity, &abort_flag, err)) break;
-    const ExportDescDev& d = b.d[find_desc(b, g)];
-    const int64_t row = g - d.row_begin;
-    if (d.mode == QAT_EXPORT_FP16) export_fp16_chunk(d, row, lane);
-    else if (staged(d)) export_row_smem(d, row, bufs + slot * (b.buf_bytes / 16), lane);
-    else export_row_global(d, row, lane);
+  // ring of kExportBufs rows: pos[k] is the row in buffer (i + k) % kExportBufs
+  RowPos pos[kExportBufs];
+  pos[0] = unit_start(b, gw);
+  for (int k = 1; k < kExportBufs; ++k) pos[k] = next_row(b, pos[k - 1], W);
+  for (int k = 0; k < kExportBufs; ++k) issue(pos[k], k);
+  int i = 0;
+  for (; pos[0].d >= 0; ++i) {
+    const int slot = i % kExportBufs;
+    if (!mbar_wait(&bars[slot], static_cast<uint32_t>((i / kExportBufs) & 1), &abort_flag, err))
+      break;
+    const ExportDescDev& d = b.d[pos[0].d];
+    if (d.mode == QAT_EXPORT_FP16) export_fp16_chunk(d, pos[0].row, lane);
+    else if (staged(d)) export_row_smem(d, pos[0].row, bufs + slot * stride, lane);
+    else export_row_global(d, pos[0].row, lane);
     // the buffer is read; order those reads before the copy engine refills it
     fence_proxy_async_smem();
     __syncwarp();
-    issue(i + kExportBufs);
+    const RowPos nn = next_row(b, pos[kExportBufs - 1], W);
+    issue(nn, slot);
+#pragma unroll
+    for (int k = 0; k + 1 < kExportBufs; ++k) pos[k] = pos[k + 1];
+    pos[kExportBufs - 1] = nn;
   }
   // After a timeout: let the copies this warp still has in flight land (bounded)
   // before the block's shared memory is released.
-  if (lane == 0 && gw + i * W < b.total_rows) {
-    for (int64_t k = i; k < i + kExportBufs && gw + k * W < b.total_rows; ++k)
-      mbar_drain(&bars[k % kExportBufs], static_cast<uint32_t>((k / kExportBufs) & 1));
+  if (lane == 0) {
+    for (int k = 0; k < kExportBufs; ++k)
+      if (pos[k].d >= 0)
+        mbar_drain(&bars[(i + k) % kExportBufs], static_cast<uint32_t>(((i + k) / kExportBufs) & 1));
   }
 }
 
@@ -417,7 +498,7 @@ int export_quantile_params(int64_t cols, int* m, float* frac) {
 }
 
 int launch_export_batch(ExportBatch& b, cudaStream_t s) {
-  if (b.total_rows == 0) return QAT_OK;
+  if (b.total_units == 0) return QAT_OK;
   static bool attr_done = false;
   if (!attr_done) {
     if (cudaFuncSetAttribute(export_batch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -433,7 +514,7 @@ int launch_export_batch(ExportBatch& b, cudaStream_t s) {
   const int per_warp = kExportBufs * (b.buf_bytes + 8);
   const int warps = std::max(1, std::min(kExportMaxWarps, kExportSmemBudget / per_warp));
   const int smem = warps * per_warp;
-  const int64_t want = (b.total_rows + warps - 1) / warps;
+  const int64_t want = (b.total_units + warps - 1) / warps;
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, sm_count())));
   export_batch_kernel<<<grid, warps * 32, smem, s>>>(b, device_error_ptr());
   count_launch();

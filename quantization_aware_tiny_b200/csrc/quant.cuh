@@ -13,7 +13,8 @@ struct ExportDescDev {
   void* dst;
   __half* scales;
   int64_t rows, cols, numel;
-  int64_t row_begin;  // first global row of this descriptor
+  int64_t unit_begin;  // first global work unit of this descriptor
+  int64_t unit_rows;   // rows per work unit
   int mode;           // 6, 8 or QAT_EXPORT_FP16
   int m;              // quantile order statistic from the top (1 or 2)
   float frac;         // quantile interpolation fraction
@@ -23,7 +24,7 @@ struct ExportDescDev {
 struct ExportBatch {
   int n;
   int buf_bytes;  // bytes of one row buffer (longest staged row, rounded to 128)
-  int64_t total_rows;
+  int64_t total_units;
   ExportDescDev d[QAT_EXPORT_MAX_DESCS];
 };
 
@@ -34,7 +35,11 @@ constexpr int64_t kFp16Chunk = 4096;
 // shared memory (longer rows are read from global memory), the shared memory
 // a block may use and the most warps per block.  Buffers are sized for the
 // longest staged row of the batch, so short-row state dicts get more warps.
-constexpr int kExportBufs = 2;
+#ifndef QAT_EXPORT_BUFS
+#define QAT_EXPORT_BUFS 2
+#endif
+constexpr int kExportBufs = QAT_EXPORT_BUFS;
+constexpr int64_t kExportUnitRows = 4;  // rows per work unit of a quantized tensor
 constexpr int64_t kExportMaxStagedCols = 2048;
 constexpr int kExportSmemBudget = 224 * 1024;
 constexpr int kExportMaxWarps = 16;
