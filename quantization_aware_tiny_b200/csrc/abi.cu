@@ -1,5 +1,6 @@
 // extern "C" entry points declared in include/qat.h: argument checks on the
 // host, workspace carving, and the sequencing of quantizer and GEMM launches.
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 
@@ -354,7 +355,10 @@ int quantize_export_batch(const qat_export_desc* descs, int32_t n, qat_stream_t 
       d.rows = s.rows;
       d.cols = s.cols;
       d.numel = s.rows * s.cols;
-      d.unit_rows = kExportUnitRows;
+      // staged rows travel in units of as many rows as fit kExportUnitBytes
+      d.unit_rows = (s.cols <= kExportMaxStagedCols)
+                        ? std::max<int64_t>(1, kExportUnitBytes / (s.cols * 4))
+                        : 1;
       const int rc = export_quantile_params(s.cols, &d.m, &d.frac);
       if (rc) return rc;
     } else {

@@ -9,6 +9,7 @@
 // reduction and quantization passes.
 #include <algorithm>
 #include <cmath>
+#include <type_traits>
 
 #include "quant.cuh"
 #include "sm100_ptx.cuh"
@@ -207,12 +208,9 @@ __device__ __forceinline__ uint32_t codes4(const RowQuant& q, float4 v) {
   return q.bits == 6 ? codes4_t<6, true>(q, v) : codes4_t<8, true>(q, v);
 }
 
-#ifndef QAT_EXPORT_UNROLL
-#define QAT_EXPORT_UNROLL 4
-#endif
 // float4 groups per lane and loop iteration in the shared-memory passes: more
 // independent dependency chains per warp.
-constexpr int kUnroll = QAT_EXPORT_UNROLL;
+constexpr int kUnroll = 4;
 
 template <int BITS, bool CLIP>
 __device__ __forceinline__ void quantize_smem_row(const RowQuant& q, const float4* buf, int K4,
@@ -263,6 +261,73 @@ __device__ __forceinline__ void export_row_smem(const ExportDescDev& d, int64_t 
   } else {
     if (clip) quantize_smem_row<8, true>(q, buf, K4, out, lane);
     else quantize_smem_row<8, false>(q, buf, K4, out, lane);
+  }
+}
+
+// Two rows of the same tensor staged in shared memory, processed together so
+// their top-2 passes, warp merges, scale computations and quantization passes
+// interleave (two independent dependency chains through every phase).
+__device__ __forceinline__ void export_two_rows_smem(const ExportDescDev& d, int64_t row,
+                                                     const float4* bufA, const float4* bufB,
+                                                     int lane) {
+  const int K4 = static_cast<int>(d.cols >> 2);
+  float a1 = 0.0f, a2 = 0.0f, b1 = 0.0f, b2 = 0.0f, c1 = 0.0f, c2 = 0.0f, e1 = 0.0f, e2 = 0.0f;
+  int j = lane;
+  for (; j + 32 < K4; j += 64) {
+    top2_push4(bufA[j], a1, a2);
+    top2_push4(bufB[j], b1, b2);
+    top2_push4(bufA[j + 32], c1, c2);
+    top2_push4(bufB[j + 32], e1, e2);
+  }
+  if (j < K4) {
+    top2_push4(bufA[j], a1, a2);
+    top2_push4(bufB[j], b1, b2);
+  }
+  {
+    const float n2 = fmaxf(fminf(a1, c1), fmaxf(a2, c2));
+    a1 = fmaxf(a1, c1);
+    a2 = n2;
+    const float m2 = fmaxf(fminf(b1, e1), fmaxf(b2, e2));
+    b1 = fmaxf(b1, e1);
+    b2 = m2;
+  }
+  top2_warp(a1, a2);
+  top2_warp(b1, b2);
+  const RowQuant qa = row_params(d, a1, a2);
+  const RowQuant qb = row_params(d, b1, b2);
+  if (lane == 0) {
+    d.scales[row] = __float2half_rn(qa.s);
+    d.scales[row + 1] = __float2half_rn(qb.s);
+  }
+  uint32_t* outA = reinterpret_cast<uint32_t*>(reinterpret_cast<int8_t*>(d.dst) + row * d.cols);
+  uint32_t* outB = outA + K4;
+  const bool clip = (a1 > 2.0f * qa.clip) || (b1 > 2.0f * qb.clip);
+  auto run = [&](auto bits_tag, auto clip_tag) {
+    constexpr int BITS = decltype(bits_tag)::value;
+    constexpr bool CLIP = decltype(clip_tag)::value;
+    int k = lane;
+    for (; k + 32 < K4; k += 64) {
+      const float4 v0 = bufA[k], v1 = bufB[k], v2 = bufA[k + 32], v3 = bufB[k + 32];
+      const uint32_t c0 = codes4_t<BITS, CLIP>(qa, v0), c1v = codes4_t<BITS, CLIP>(qb, v1);
+      const uint32_t c2v = codes4_t<BITS, CLIP>(qa, v2), c3 = codes4_t<BITS, CLIP>(qb, v3);
+      outA[k] = c0;
+      outB[k] = c1v;
+      outA[k + 32] = c2v;
+      outB[k + 32] = c3;
+    }
+    if (k < K4) {
+      outA[k] = codes4_t<BITS, CLIP>(qa, bufA[k]);
+      outB[k] = codes4_t<BITS, CLIP>(qb, bufB[k]);
+    }
+  };
+  using T6 = std::integral_constant<int, 6>;
+  using T8 = std::integral_constant<int, 8>;
+  using TT = std::true_type;
+  using TF = std::false_type;
+  if (qa.bits == 6) {
+    if (clip) run(T6{}, TT{}); else run(T6{}, TF{});
+  } else {
+    if (clip) run(T8{}, TT{}); else run(T8{}, TF{});
   }
 }
 
@@ -334,41 +399,38 @@ __device__ __forceinline__ bool staged(const ExportDescDev& d) {
 }
 // (the host sizes buf_bytes for the longest staged row, so staged rows fit)
 
-// A warp's position in its sequence of rows: the row `row` (of [row, row_end)
-// in work unit `unit`) of descriptor `d`; d < 0 once the sequence is done.
-struct RowPos {
-  int64_t unit, row, row_end;
+// A work unit: rows [row0, row0 + nrows) of descriptor d (d < 0: no more work).
+struct UnitPos {
+  int64_t row0;
+  int nrows;
   int d;
 };
 
-__device__ __forceinline__ RowPos unit_start(const ExportBatch& b, int64_t u) {
-  RowPos p;
-  p.unit = u;
+// Unit u of the batch, or d < 0 past the last unit.
+__device__ __forceinline__ UnitPos unit_at(const ExportBatch& b, int64_t u) {
+  UnitPos p;
   if (u >= b.total_units) {
     p.d = -1;
-    p.row = p.row_end = 0;
+    p.row0 = 0;
+    p.nrows = 0;
     return p;
   }
   p.d = find_desc(b, u);
   const ExportDescDev& d = b.d[p.d];
-  p.row = (u - d.unit_begin) * d.unit_rows;
-  p.row_end = min(p.row + d.unit_rows, d.rows);
+  p.row0 = (u - d.unit_begin) * d.unit_rows;
+  p.nrows = static_cast<int>(min(d.unit_rows, d.rows - p.row0));
   return p;
 }
 
-__device__ __forceinline__ RowPos next_row(const ExportBatch& b, RowPos p, int64_t W) {
-  if (p.d < 0) return p;
-  if (++p.row < p.row_end) return p;
-  return unit_start(b, p.unit + W);
-}
-
-// One launch over all descriptors.  Work units are runs of up to
-// kExportUnitRows consecutive rows of one tensor (one chunk for fp16
-// passthrough); warp w of the grid takes units w, w + W, ... (W = warps in the
-// grid) and streams their rows through kExportBufs shared-memory buffers: the
-// next rows are in flight while this one is quantized.  Rows that are not staged still
-// arrive once on their buffer's mbarrier so every buffer's phases stay in
-// step with the row count.
+// One launch over all descriptors.  Work units are runs of consecutive rows of
+// one tensor -- as many as fit kExportUnitBytes for rows staged in shared
+// memory, one row otherwise, one chunk of about the same bytes for fp16
+// passthrough -- so units cost about the same.  Warp w of the grid takes units
+// w, w + W, w + 2W, ... (W = warps in the grid; a static assignment: one
+// shared work counter would serialise the warps on its atomics); a staged unit
+// arrives in one bulk copy into one of the warp's kExportBufs buffers while
+// the warp quantizes the previous one.  Units that are not staged still arrive once on their buffer's
+// mbarrier so every buffer's phases stay in step with the unit count.
 __global__ void __launch_bounds__(kExportMaxWarps * 32, 1)
     export_batch_kernel(const __grid_constant__ ExportBatch b, int* err) {
   extern __shared__ __align__(128) uint8_t xsmem[];
@@ -390,44 +452,57 @@ __global__ void __launch_bounds__(kExportMaxWarps * 32, 1)
   const int64_t gw = static_cast<int64_t>(blockIdx.x) * nw + wib;
   const int stride = b.buf_bytes / 16;
 
-  auto issue = [&](const RowPos& p, int slot) {
+  auto issue = [&](const UnitPos& p, int slot) {
     if (p.d < 0 || lane != 0) return;
     const ExportDescDev& d = b.d[p.d];
     if (staged(d)) {
-      const uint32_t bytes = static_cast<uint32_t>(d.cols * 4);
+      const uint32_t bytes = static_cast<uint32_t>(p.nrows * d.cols * 4);
       mbar_arrive_expect_tx(&bars[slot], bytes);
-      bulk_load_1d(bufs + slot * stride, d.src + p.row * d.cols, bytes, &bars[slot]);
+      bulk_load_1d(bufs + slot * stride, d.src + p.row0 * d.cols, bytes, &bars[slot]);
     } else {
       mbar_arrive(&bars[slot]);
     }
   };
 
-  // ring of kExportBufs rows: pos[k] is the row in buffer (i + k) % kExportBufs
-  RowPos pos[kExportBufs];
-  pos[0] = unit_start(b, gw);
-  for (int k = 1; k < kExportBufs; ++k) pos[k] = next_row(b, pos[k - 1], W);
-  for (int k = 0; k < kExportBufs; ++k) issue(pos[k], k);
+  // ring of kExportBufs units: pos[k] is the unit in buffer (i + k) % kExportBufs
+  UnitPos pos[kExportBufs];
+  int64_t next_u = gw;
+  for (int k = 0; k < kExportBufs; ++k) {
+    pos[k] = unit_at(b, next_u);
+    next_u += W;
+    issue(pos[k], k);
+  }
   int i = 0;
   for (; pos[0].d >= 0; ++i) {
     const int slot = i % kExportBufs;
     if (!mbar_wait(&bars[slot], static_cast<uint32_t>((i / kExportBufs) & 1), &abort_flag, err))
       break;
     const ExportDescDev& d = b.d[pos[0].d];
-    if (d.mode == QAT_EXPORT_FP16) export_fp16_chunk(d, pos[0].row, lane);
-    else if (staged(d)) export_row_smem(d, pos[0].row, bufs + slot * stride, lane);
-    else export_row_global(d, pos[0].row, lane);
+    if (d.mode == QAT_EXPORT_FP16) {
+      export_fp16_chunk(d, pos[0].row0, lane);
+    } else if (staged(d)) {
+      const int K4 = static_cast<int>(d.cols >> 2);
+      const float4* ub = bufs + slot * stride;
+      int r = 0;
+      for (; r + 1 < pos[0].nrows; r += 2)
+        export_two_rows_smem(d, pos[0].row0 + r, ub + r * K4, ub + (r + 1) * K4, lane);
+      if (r < pos[0].nrows) export_row_smem(d, pos[0].row0 + r, ub + r * K4, lane);
+    } else {
+      export_row_global(d, pos[0].row0, lane);
+    }
     // the buffer is read; order those reads before the copy engine refills it
     fence_proxy_async_smem();
     __syncwarp();
-    const RowPos nn = next_row(b, pos[kExportBufs - 1], W);
+    const UnitPos nn = unit_at(b, next_u);
+    next_u += W;
     issue(nn, slot);
 #pragma unroll
     for (int k = 0; k + 1 < kExportBufs; ++k) pos[k] = pos[k + 1];
     pos[kExportBufs - 1] = nn;
   }
-  // After a timeout: let the copies this warp still has in flight land (bounded)
-  // before the block's shared memory is released.
   if (lane == 0) {
+    // After a timeout: let the copies this warp still has in flight land
+    // (bounded) before the block's shared memory is released.
     for (int k = 0; k < kExportBufs; ++k)
       if (pos[k].d >= 0)
         mbar_drain(&bars[(i + k) % kExportBufs], static_cast<uint32_t>(((i + k) / kExportBufs) & 1));
@@ -506,11 +581,11 @@ int launch_export_batch(ExportBatch& b, cudaStream_t s) {
       return QAT_ERR_CUDA;
     attr_done = true;
   }
-  int64_t longest = 4;  // longest staged row
+  int64_t longest = 16;  // bytes of the longest staged unit
   for (int i = 0; i < b.n; ++i)
     if (b.d[i].mode != QAT_EXPORT_FP16 && b.d[i].cols <= kExportMaxStagedCols)
-      longest = std::max(longest, b.d[i].cols);
-  b.buf_bytes = static_cast<int>((longest * 4 + 127) / 128 * 128);
+      longest = std::max(longest, b.d[i].unit_rows * b.d[i].cols * 4);
+  b.buf_bytes = static_cast<int>((longest + 127) / 128 * 128);
   const int per_warp = kExportBufs * (b.buf_bytes + 8);
   const int warps = std::max(1, std::min(kExportMaxWarps, kExportSmemBudget / per_warp));
   const int smem = warps * per_warp;

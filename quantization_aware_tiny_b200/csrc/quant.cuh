@@ -28,8 +28,8 @@ struct ExportBatch {
   ExportDescDev d[QAT_EXPORT_MAX_DESCS];
 };
 
-// Chunk length of the fp16 passthrough "rows".
-constexpr int64_t kFp16Chunk = 4096;
+// Chunk length of the fp16 passthrough "rows" (6 KB of fp32, like a staged unit).
+constexpr int64_t kFp16Chunk = 1536;
 
 // Export kernel staging: row buffers per warp, the longest row staged in
 // shared memory (longer rows are read from global memory), the shared memory
@@ -39,7 +39,7 @@ constexpr int64_t kFp16Chunk = 4096;
 #define QAT_EXPORT_BUFS 2
 #endif
 constexpr int kExportBufs = QAT_EXPORT_BUFS;
-constexpr int64_t kExportUnitRows = 4;  // rows per work unit of a quantized tensor
+constexpr int64_t kExportUnitBytes = 6144;  // staged bytes per work unit (whole rows)
 constexpr int64_t kExportMaxStagedCols = 2048;
 constexpr int kExportSmemBudget = 224 * 1024;
 constexpr int kExportMaxWarps = 16;

@@ -202,15 +202,23 @@ def quantize_rows_export(W, bits, codes, scales, stream=None):
                                       _stream(stream)), "quantize_rows_export")
 
 
-def quantize_export_batch(descs, stream=None):
-    """descs: list of (src, mode, dst, scales) with src a 2-D (or flat) fp32
-    device tensor, mode 6 / 8 / QAT_EXPORT_FP16."""
+def export_descs(descs):
+    """Marshal (src, mode, dst, scales) tuples into the C descriptor array once;
+    the result can be passed to quantize_export_batch repeatedly."""
     arr = (_ExportDesc * len(descs))()
     for i, (src, mode, dst, scales) in enumerate(descs):
         rows, cols = (src.shape if src.dim() == 2 else (1, src.numel()))
         arr[i] = _ExportDesc(src.data_ptr(), rows, cols, mode, 0, dst.data_ptr(),
                              scales.data_ptr() if scales is not None else None)
-    _check(lib().quantize_export_batch(arr, len(descs), _stream(stream)), "quantize_export_batch")
+    return arr
+
+
+def quantize_export_batch(descs, stream=None):
+    """descs: list of (src, mode, dst, scales) with src a 2-D (or flat) fp32
+    device tensor, mode 6 / 8 / QAT_EXPORT_FP16 -- or an array from
+    export_descs() (the tensors it points to must stay alive)."""
+    arr = descs if isinstance(descs, ctypes.Array) else export_descs(descs)
+    _check(lib().quantize_export_batch(arr, len(arr), _stream(stream)), "quantize_export_batch")
 
 
 def dequantize_rows(codes, scales16, out, stream=None):
