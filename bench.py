@@ -32,9 +32,13 @@ METRIC = "QAT linear/MLP TFLOP/s (% B200 bf16 peak); export quantizer GB/s (% HB
 T_TOKENS = 65536
 VOCAB, D, H = 8192, 512, 2048
 
-# DRAM bytes per launch of the logits GEMM from an ncu capture, with the hash
-# of the GEMM sources it was taken on (reported only while they still match).
-NCU_TRAFFIC = {"kernel_hash": None, "bytes_per_launch": None}
+# DRAM bytes (read + write) per launch of the head GEMMs from one ncu capture
+# each at 16,384 tokens, scaled by 4 to the 65,536-token launch (the traffic
+# grows with the token count), with the hash of the GEMM sources the captures
+# were taken on: reported only while the sources still match.
+NCU_TRAFFIC = {"kernel_hash": "2c05f7b683b6a621",
+               "bytes_per_launch": {"logits_fwd": 4 * (25.281024e6 + 215.121664e6),
+                                    "head_dW": 4 * (303.659520e6 + 9.542912e6)}}
 
 
 def gemm_source_hash():
@@ -71,7 +75,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -217,7 +221,7 @@ def run_ours(args):
               "head_dW": 2.0 * T_TOKENS * VOCAB * D}
     pk = peaks()
     achieved = kflops[dom] / (kt[dom] * 1e-3) / 1e12
-    traffic = (NCU_TRAFFIC["bytes_per_launch"]
+    traffic = (NCU_TRAFFIC["bytes_per_launch"].get(dom)
                if NCU_TRAFFIC["kernel_hash"] == gemm_source_hash() else None)
     roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1),
                 "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",

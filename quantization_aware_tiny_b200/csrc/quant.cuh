@@ -21,11 +21,14 @@ struct ExportDescDev {
   int pad;
 };
 
+#ifndef QAT_EXPORT_BATCH_CAP
+#define QAT_EXPORT_BATCH_CAP QAT_EXPORT_MAX_DESCS
+#endif
 struct ExportBatch {
   int n;
   int buf_bytes;  // bytes of one row buffer (longest staged row, rounded to 128)
   int64_t total_units;
-  ExportDescDev d[QAT_EXPORT_MAX_DESCS];
+  ExportDescDev d[QAT_EXPORT_BATCH_CAP];
 };
 
 // Chunk length of the fp16 passthrough "rows" (6 KB of fp32, like a staged unit).
