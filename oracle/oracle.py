@@ -41,6 +41,8 @@ def _c():
         lib.oracle_dequant_export.argtypes = [P, P, I64, I64, P]
         lib.oracle_fp16_array.argtypes = [P, I64, P]
         lib.oracle_bf16_array.argtypes = [P, I64, P]
+        lib.oracle_philox4x32_10.argtypes = [P, P, P]
+        lib.oracle_noisy_operand.argtypes = [P, I64, I64, ctypes.c_uint64, ctypes.c_uint64, P, P, P]
         _lib = lib
     return _lib
 
@@ -133,6 +135,32 @@ def quantize_weight(W, bits):
     c = qat_codes(W, s, bits)
     op = bf16_bits_to_f32(operand_bf16_bits(c, s)).astype(np.float64)
     return {"codes": c, "scales": s, "wq": dequant(c, s), "operand": op}
+
+
+# ------------------------------------------------ Noisy QAT (P1 "幸存发现 1")
+
+def philox4x32_10(counter, key):
+    """Philox-4x32-10 block (Salmon et al., SC'11) of a 4-word counter and a
+    2-word key, as 4 uint32."""
+    c = np.ascontiguousarray(counter, np.uint32)
+    k = np.ascontiguousarray(key, np.uint32)
+    out = np.empty(4, np.uint32)
+    _c().oracle_philox4x32_10(_ptr(c), _ptr(k), _ptr(out))
+    return out
+
+
+def noisy_weight(W, seed, offset=0):
+    """P1 "幸存发现 1 Noisy QAT": w + (u - 0.5) * max(amax,1e-12)/127 per row, u from
+    Philox-4x32-10 (counter = element // 4 and offset, key = seed).  Returns the
+    fp32 scales, the noisy fp32 weight and its bf16 operand (float64 values)."""
+    W = _f32(W)
+    N, K = W.shape
+    s = np.empty(N, np.float32)
+    noisy = np.empty((N, K), np.float32)
+    op = np.empty((N, K), np.uint16)
+    _c().oracle_noisy_operand(_ptr(W), N, K, int(seed), int(offset), _ptr(s), _ptr(noisy), _ptr(op))
+    return {"scales": s, "noisy": noisy, "operand_bits": op,
+            "operand": bf16_bits_to_f32(op).astype(np.float64)}
 
 
 # -------------------------------------------------------- dense algebra (fp64)

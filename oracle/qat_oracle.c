@@ -246,3 +246,60 @@ void oracle_fp16_array(const float* in, int64_t n, uint16_t* out) {
 void oracle_bf16_array(const float* in, int64_t n, uint16_t* out) {
   for (int64_t j = 0; j < n; ++j) out[j] = oracle_bf16_rne(in[j]);
 }
+
+/* ---- Noisy QAT (training-time noise for depth-recurrent cores) ------------ */
+/* Source: "Depth Recurrence + Mixed-Precision Quant" write-up (PR #363),
+ * section "幸存发现 1 Noisy QAT": for the shared core blocks the forward weight
+ * is w + (U(0,1) - 0.5) * amax/127 (per-row amax clamped at 1e-12), the noise
+ * drawn without gradient, so the backward is the identity in w.
+ *
+ * The uniform draws come from Philox-4x32-10 (J. K. Salmon, M. A. Moraes,
+ * R. O. Dror, D. E. Shaw, "Parallel random numbers: as easy as 1, 2, 3",
+ * SC'11), written here from that definition: ten rounds of
+ *   (c0,c1,c2,c3) -> (hi(M1*c2) ^ c1 ^ k0, lo(M1*c2), hi(M0*c0) ^ c3 ^ k1, lo(M0*c0))
+ * with M0 = 0xD2511F53, M1 = 0xCD9E8D57, the key bumped by
+ * (0x9E3779B9, 0xBB67AE85) before every round after the first.
+ * Element e of the row-major [N,K] weight uses output word e % 4 of the block
+ * with counter (g, g >> 32, offset, offset >> 32), g = e / 4, and key
+ * (seed, seed >> 32); the word x becomes u = (x >> 8) * 2^-24 in [0, 1). */
+void oracle_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]) {
+  uint32_t c0 = ctr[0], c1 = ctr[1], c2 = ctr[2], c3 = ctr[3];
+  uint32_t k0 = key[0], k1 = key[1];
+  for (int r = 0; r < 10; ++r) {
+    if (r > 0) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    uint64_t p0 = (uint64_t)0xD2511F53u * (uint64_t)c0;
+    uint64_t p1 = (uint64_t)0xCD9E8D57u * (uint64_t)c2;
+    uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+    uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+    uint32_t n0 = hi1 ^ c1 ^ k0, n1 = lo1, n2 = hi0 ^ c3 ^ k1, n3 = lo0;
+    c0 = n0; c1 = n1; c2 = n2; c3 = n3;
+  }
+  out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
+}
+
+/* Noisy forward weight of every element and its bf16 operand:
+ *   s = fl32(max(amax, 1e-12) / 127);  noise = fl32(fl32(u - 0.5) * s);
+ *   w' = fl32(w + noise);  operand = bf16_rne(w').  (u - 0.5 is exact.) */
+void oracle_noisy_operand(const float* W, int64_t N, int64_t K, uint64_t seed, uint64_t offset,
+                          float* scale, float* noisy, uint16_t* operand) {
+  oracle_qat_scales(W, N, K, scale);
+  uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+  for (int64_t i = 0; i < N; ++i) {
+    for (int64_t j = 0; j < K; ++j) {
+      int64_t e = i * K + j;
+      uint64_t g = (uint64_t)e >> 2;
+      uint32_t ctr[4] = {(uint32_t)g, (uint32_t)(g >> 32), (uint32_t)offset,
+                         (uint32_t)(offset >> 32)};
+      uint32_t x[4];
+      oracle_philox4x32_10(ctr, key, x);
+      float u = (float)(x[e & 3] >> 8) * 5.9604644775390625e-08f;
+      float noise = (u - 0.5f) * scale[i];
+      float w = W[e] + noise;
+      if (noisy) noisy[e] = w;
+      if (operand) operand[e] = oracle_bf16_rne(w);
+    }
+  }
+}

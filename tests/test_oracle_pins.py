@@ -364,3 +364,50 @@ def test_recurrent_core_is_r_applications():
     ref = b(x1 + h @ q["proj"]["operand"].T)
     one = o.recurrent_core_fwd(q["qkv"], q["o"], q["fc"], q["proj"], X, 1, 64)
     assert np.array_equal(one, ref)
+
+
+# ------------------------------------------------------------- Noisy QAT
+
+def test_philox_known_answers():
+    """Philox-4x32-10 against the known-answer vectors published with the
+    generator (Salmon et al., SC'11, Random123 distribution)."""
+    kat = [([0, 0, 0, 0], [0, 0], [0x6627e8d5, 0xe169c58d, 0xbc57ac4c, 0x9b00dbd8]),
+           ([0xffffffff] * 4, [0xffffffff] * 2, [0x408f276d, 0x41c83b0e, 0xa20bc7c6, 0x6d5451fd]),
+           ([0x243f6a88, 0x85a308d3, 0x13198a2e, 0x03707344], [0xa4093822, 0x299f31d0],
+            [0xd16cfe09, 0x94fdcceb, 0x5001e420, 0x24126ea1])]
+    for ctr, key, want in kat:
+        assert o.philox4x32_10(ctr, key).tolist() == want
+
+
+def test_noisy_weight_bounds_statistics_and_determinism():
+    """P1 "幸存发现 1 Noisy QAT": the noise is (u - 0.5) * s with s the per-row
+    int8 step amax/127, so |w' - w| <= s/2 (+ the fp32 rounding of the add);
+    u is uniform (mean 1/2, variance 1/12, Kolmogorov-Smirnov against U(0,1));
+    the same (seed, offset) gives the same weights, another offset others."""
+    from scipy import stats
+    W = sy.linear_case(N=512, K=512, seed=4)["W"]
+    r = o.noisy_weight(W, seed=1234, offset=7)
+    s = r["scales"].astype(np.float64)
+    assert np.array_equal(r["scales"], o.qat_scales(W))
+    d = (r["noisy"].astype(np.float64) - W.astype(np.float64)) / s[:, None]
+    ulp = np.spacing(np.abs(r["noisy"])).astype(np.float64) / s[:, None]
+    assert np.all(np.abs(d) <= 0.5 + ulp)
+    u = (d + 0.5).ravel()
+    assert abs(u.mean() - 0.5) < 0.005 and abs(u.var() - 1.0 / 12) < 0.002
+    assert stats.kstest(np.clip(u, 0, 1), "uniform").pvalue > 1e-3
+    assert np.array_equal(o.noisy_weight(W, 1234, 7)["noisy"], r["noisy"])
+    assert not np.array_equal(o.noisy_weight(W, 1234, 8)["noisy"], r["noisy"])
+    ref = torch.from_numpy(r["noisy"]).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(r["operand"].astype(np.float32), ref)
+
+
+def test_noisy_uses_documented_counter_layout():
+    """Element e takes word e % 4 of the Philox block at counter (e // 4, offset)."""
+    W = np.zeros((2, 8), np.float32)
+    W[:, 0] = 127.0  # s = 1 in both rows
+    r = o.noisy_weight(W, seed=(5 << 32) | 9, offset=(3 << 32) | 11)
+    for e in (1, 2, 5, 9, 14):
+        g = e // 4
+        x = o.philox4x32_10([g, 0, 11, 3], [9, 5])[e % 4]
+        u = np.float32(x >> 8) * np.float32(2.0 ** -24)
+        assert r["noisy"].ravel()[e] == np.float32(u - np.float32(0.5))
