@@ -88,6 +88,20 @@ typedef struct qat_qweight {
 int qat_quantize_weights(const float* W, int32_t N, int32_t K, int32_t bits, int8_t* codes,
                          float* scales, qat_bf16* operand, qat_stream_t stream);
 
+/* Noisy QAT for the shared blocks of a depth-recurrent core ([P1] "幸存发现 1
+ * Noisy QAT"): instead of the STE fake quantization, the forward weight is
+ *   w' = fl32(w + fl32(fl32(u - 1/2) * s)),  s = fl32(max(amax_row, 1e-12) / 127),
+ * u uniform in [0,1), and the gradient flows through w' to w unchanged (the
+ * noise carries none), so the backward is qat_linear_bwd with this operand.
+ * u comes from Philox-4x32-10 (Salmon et al., SC'11): element e of the
+ * row-major [N,K] weight uses word e % 4 of the block with counter
+ * (e/4 low, e/4 high, offset low, offset high) and key (seed low, seed high);
+ * u = (word >> 8) * 2^-24.  Outputs: operand [N,K] bf16 = bf16_rne(w')
+ * (required; pass it as qat_qweight.operand), scales [N] fp32 (nullable).
+ * Bit-exact with the CPU oracle.  Use a fresh offset per draw. */
+int qat_noisy_operand(const float* W, int32_t N, int32_t K, uint64_t seed, uint64_t offset,
+                      float* scales, qat_bf16* operand, qat_stream_t stream);
+
 /* Workspace sizes (bytes) for the calls below.  `raw_weights` != 0 means the
  * call is given fp32 weights to quantize itself (the workspace then also
  * holds the bf16 operands and scales); 0 means qat_qweight operands. */

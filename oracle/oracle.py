@@ -226,6 +226,18 @@ def recurrent_core_fwd(q_qkv, q_o, q_fc, q_proj, X, R, d):
     return x
 
 
+def recurrent_core_fwd_noisy(Ws, X, R, d, seed, offset):
+    """The recurrent core under Noisy QAT (P1 "幸存发现 1"): application r uses
+    the noisy operands of the four weights (qkv, o, fc, proj -> k = 0..3) drawn
+    at Philox offset offset + 4*r + k, composed exactly as recurrent_core_fwd."""
+    x = X
+    for r in range(R):
+        q = [{"operand": noisy_weight(w, seed, offset + 4 * r + k)["operand"]}
+             for k, w in enumerate(Ws)]
+        x = recurrent_core_fwd(q[0], q[1], q[2], q[3], x, 1, d)
+    return x
+
+
 def head_mlp_step(q_emb, q_fc, q_proj, X, dLogits):
     """Tied-head throughput step: Z = MLP(X), logits = Z Wemb^T, then the STE
     backward of both from the upstream gradient dLogits."""

@@ -116,6 +116,15 @@ int qat_device_error(qat_stream_t stream) {
   return v;
 }
 
+int qat_noisy_operand(const float* W, int32_t N, int32_t K, uint64_t seed, uint64_t offset,
+                      float* scales, qat_bf16* operand, qat_stream_t stream) {
+  if (!W || !operand || N <= 0) return QAT_ERR_ARG;
+  if (!dim_ok(K)) return QAT_ERR_SHAPE;
+  if (!aligned16(W) || !aligned16(operand)) return QAT_ERR_ALIGN;
+  return launch_noisy_operand(W, N, K, seed, offset, scales,
+                              reinterpret_cast<__nv_bfloat16*>(operand), stream);
+}
+
 size_t qat_workspace_size(int32_t op, int32_t N_or_d, int32_t K_or_H, int64_t T,
                           int32_t raw_weights) {
   const int64_t a = N_or_d, b = K_or_H;

@@ -86,6 +86,83 @@ __global__ void __launch_bounds__(kQThreads)
   }
 }
 
+// ------------------------------------------------------------------ Noisy QAT
+// Philox-4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as
+// easy as 1, 2, 3", SC'11): ten rounds of the multiply-xor round function on a
+// 4-word counter under a 2-word key bumped by the Weyl constants each round.
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r > 0) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint32_t hi0 = __umulhi(0xD2511F53u, c.x), lo0 = 0xD2511F53u * c.x;
+    const uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z), lo1 = 0xCD9E8D57u * c.z;
+    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+  }
+  return c;
+}
+
+// fl32(w + fl32(fl32(u - 1/2) * s)) with u = (x >> 8) * 2^-24 in [0, 1).
+__device__ __forceinline__ float noisy_value(float w, uint32_t x, float s) {
+  const float u = __uint2float_rn(x >> 8) * 5.9604644775390625e-08f;  // exact
+  return __fadd_rn(w, __fmul_rn(__fsub_rn(u, 0.5f), s));
+}
+
+// Noisy-QAT forward operand ("Depth Recurrence + Mixed-Precision Quant",
+// "幸存发现 1 Noisy QAT"): per row s = max(amax, 1e-12) / 127, every weight
+// gets (u - 1/2) * s of uniform noise, the result is cast to bf16.  Element e
+// of the row-major weight takes word e % 4 of the Philox block with counter
+// (e / 4, offset) and key seed.  One warp per row, the row cached in registers
+// between the amax and the noise passes.
+__global__ void __launch_bounds__(kQThreads)
+    noisy_operand_kernel(const float* __restrict__ W, int N, int K, uint64_t seed,
+                         uint64_t offset, float* __restrict__ scales,
+                         __nv_bfloat16* __restrict__ operand) {
+  const int lane = threadIdx.x & 31;
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  const int K4 = K >> 2;
+  const uint32_t k0 = static_cast<uint32_t>(seed), k1 = static_cast<uint32_t>(seed >> 32);
+  const uint32_t o0 = static_cast<uint32_t>(offset), o1 = static_cast<uint32_t>(offset >> 32);
+  for (int row = warp; row < N; row += nwarps) {
+    const float4* r = reinterpret_cast<const float4*>(W + static_cast<int64_t>(row) * K);
+    float4 cache[kRegV4];
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kRegV4; ++i) {
+      const int j = lane + 32 * i;
+      if (j < K4) {
+        cache[i] = __ldg(r + j);
+        amax = fmaxf(amax, amax4(cache[i]));
+      }
+    }
+    for (int j = lane + 32 * kRegV4; j < K4; j += 32) amax = fmaxf(amax, amax4(__ldg(r + j)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float s = div_rn(fmaxf(amax, 1e-12f), 127.0f);
+    if (lane == 0 && scales) scales[row] = s;
+    auto emit = [&](int j, float4 v) {
+      const uint64_t g = static_cast<uint64_t>(row) * static_cast<uint64_t>(K4) + j;  // e / 4
+      const uint4 x = philox4x32_10(
+          make_uint4(static_cast<uint32_t>(g), static_cast<uint32_t>(g >> 32), o0, o1), k0, k1);
+      __nv_bfloat162 lo = __floats2bfloat162_rn(noisy_value(v.x, x.x, s), noisy_value(v.y, x.y, s));
+      __nv_bfloat162 hi = __floats2bfloat162_rn(noisy_value(v.z, x.z, s), noisy_value(v.w, x.w, s));
+      uint2 o;
+      o.x = *reinterpret_cast<uint32_t*>(&lo);
+      o.y = *reinterpret_cast<uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(operand + static_cast<int64_t>(row) * K + 4 * j) = o;
+    };
+#pragma unroll
+    for (int i = 0; i < kRegV4; ++i) {
+      const int j = lane + 32 * i;
+      if (j < K4) emit(j, cache[i]);
+    }
+    for (int j = lane + 32 * kRegV4; j < K4; j += 32) emit(j, __ldg(r + j));
+  }
+}
+
 // ------------------------------------------------------------------ export
 // Running top-2 of |w| (with multiplicity): t1 >= t2.
 __device__ __forceinline__ void top2_push(float a, float& t1, float& t2) {
@@ -554,6 +631,14 @@ int launch_quantize_weights(const float* W, int N, int K, int bits, int8_t* code
                             __nv_bfloat16* operand, cudaStream_t s) {
   quantize_weights_kernel<<<grid_for_rows(N, kQThreads / 32), kQThreads, 0, s>>>(
       W, N, K, bits, codes, scales, operand);
+  count_launch();
+  return cuda_status(cudaGetLastError());
+}
+
+int launch_noisy_operand(const float* W, int N, int K, uint64_t seed, uint64_t offset,
+                         float* scales, __nv_bfloat16* operand, cudaStream_t s) {
+  noisy_operand_kernel<<<grid_for_rows(N, kQThreads / 32), kQThreads, 0, s>>>(
+      W, N, K, seed, offset, scales, operand);
   count_launch();
   return cuda_status(cudaGetLastError());
 }

@@ -26,7 +26,7 @@ QAT_DTYPE_F32, QAT_DTYPE_BF16 = 0, 1
 EXPORTED = ("qat_strerror", "qat_launch_count", "qat_device_error", "qat_quantize_weights",
             "qat_workspace_size", "qat_linear_fwd", "qat_linear_bwd", "qat_mlp_fwd",
             "qat_mlp_bwd", "quantize_rows_export", "quantize_export_batch", "dequantize_rows",
-            "qat_linear_fwd_noalloc")
+            "qat_linear_fwd_noalloc", "qat_noisy_operand")
 QAT_NOALLOC_MAX_ELEMS = 4194304
 QAT_NOALLOC_MAX_ROWS = 16384
 
@@ -78,6 +78,7 @@ def lib():
         L.quantize_export_batch.argtypes = [P, I32, P]
         L.dequantize_rows.argtypes = [P, P, I64, I64, I32, P, P]
         L.qat_linear_fwd_noalloc.argtypes = [P, I32, I32, I32, P, I64, I64, P, P, P]
+        L.qat_noisy_operand.argtypes = [P, I32, I32, ctypes.c_uint64, ctypes.c_uint64, P, P, P]
         for name in EXPORTED:
             if name not in ("qat_strerror", "qat_launch_count", "qat_workspace_size"):
                 getattr(L, name).restype = ctypes.c_int
@@ -157,6 +158,22 @@ def quantize_weight(W, bits, keep_codes=False, stream=None):
     codes = torch.empty((N, K), dtype=torch.int8, device=W.device) if keep_codes else None
     qat_quantize_weights(W, bits, scales, codes, operand, stream)
     return QWeight(operand, scales, codes, bits)
+
+
+def qat_noisy_operand(W, seed, offset, operand, scales=None, stream=None):
+    """Noisy-QAT forward operand bf16(w + (u - 1/2) * amax/127) of W [N,K]."""
+    N, K = W.shape
+    _check(lib().qat_noisy_operand(_p(W), N, K, int(seed), int(offset), _p(scales), _p(operand),
+                                   _stream(stream)), "qat_noisy_operand")
+
+
+def noisy_weight(W, seed, offset, stream=None):
+    """A new QWeight holding the Noisy-QAT operand of W (bits recorded as 0)."""
+    N, K = W.shape
+    scales = torch.empty(N, dtype=torch.float32, device=W.device)
+    operand = torch.empty((N, K), dtype=torch.bfloat16, device=W.device)
+    qat_noisy_operand(W, seed, offset, operand, scales, stream)
+    return QWeight(operand, scales, None, 0)
 
 
 def qat_linear_fwd(X, Y, bits, W=None, qw=None, residual=None, workspace=None, N=None, K=None,

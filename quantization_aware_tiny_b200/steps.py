@@ -25,10 +25,9 @@ class RecurrentCore:
         self.H = Wfc.shape[0]
         self.bits = bits
         Wqkv = torch.cat([Wq, Wk, Wv], dim=0).contiguous()
-        self.q_qkv = qat.quantize_weight(Wqkv, bits, stream=stream)
-        self.q_o = qat.quantize_weight(Wo.contiguous(), bits, stream=stream)
-        self.q_fc = qat.quantize_weight(Wfc.contiguous(), bits, stream=stream)
-        self.q_proj = qat.quantize_weight(Wproj.contiguous(), bits, stream=stream)
+        self.W = (Wqkv, Wo.contiguous(), Wfc.contiguous(), Wproj.contiguous())
+        self.q_qkv, self.q_o, self.q_fc, self.q_proj = (
+            qat.quantize_weight(w, bits, stream=stream) for w in self.W)
         self.nqkv = Wqkv.shape[0]
         self._buf = None
 
@@ -40,16 +39,30 @@ class RecurrentCore:
                          torch.empty((T, self.H), dtype=bf, device=device))
         return self._buf
 
-    def forward(self, x, R, stream=None):
-        """Applies the core R times to x [T,d] bf16 in place; returns x."""
+    def forward(self, x, R, stream=None, noise=None):
+        """Applies the core R times to x [T,d] bf16 in place; returns x.
+
+        noise = (seed, offset) switches to Noisy QAT ("Depth Recurrence +
+        Mixed-Precision Quant", "幸存发现 1"): every application draws fresh
+        uniform noise at the int8 step for each of the four weights, with
+        Philox offsets offset + 4*r + k (r = application, k = qkv, o, fc,
+        proj), instead of reusing the once-quantized operands."""
         T = x.shape[0]
         qkv, x1, h = self._buffers(T, x.device)
-        for _ in range(R):
-            qat.qat_linear_fwd(x, qkv, self.bits, qw=self.q_qkv, stream=stream)
-            qat.qat_linear_fwd(qkv, x1, self.bits, qw=self.q_o, ldx=self.nqkv, T=T,
-                               residual=x, stream=stream)
-            qat.qat_mlp_fwd(x1, x, self.bits, self.d, self.H, qfc=self.q_fc, qproj=self.q_proj,
-                            residual=x1, h_save=h, stream=stream)
+        ops = (self.q_qkv, self.q_o, self.q_fc, self.q_proj)
+        if noise is not None:
+            ops = tuple(qat.QWeight(torch.empty_like(q.operand), None, None, 0) for q in ops)
+        for r in range(R):
+            if noise is not None:
+                seed, offset = noise
+                for k, (w, q) in enumerate(zip(self.W, ops)):
+                    qat.qat_noisy_operand(w, seed, offset + 4 * r + k, q.operand, stream=stream)
+            q_qkv, q_o, q_fc, q_proj = ops
+            bits = self.bits
+            qat.qat_linear_fwd(x, qkv, bits, qw=q_qkv, stream=stream)
+            qat.qat_linear_fwd(qkv, x1, bits, qw=q_o, ldx=self.nqkv, T=T, residual=x, stream=stream)
+            qat.qat_mlp_fwd(x1, x, bits, self.d, self.H, qfc=q_fc, qproj=q_proj, residual=x1,
+                            h_save=h, stream=stream)
         return x
 
     def flops(self, T, R):

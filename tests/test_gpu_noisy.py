@@ -1,0 +1,61 @@
+"""GPU parity of Noisy QAT ("Depth Recurrence + Mixed-Precision Quant",
+"幸存发现 1"): the noisy bf16 operand bit-exact against the oracle's Philox and
+fp32 arithmetic, the linear forward / backward through it, and the recurrent
+core with fresh noise per application."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as o
+from quantization_aware_tiny_b200 import qat, steps
+from quantization_aware_tiny_b200 import synthetic as sy
+from parity import assert_close, assert_close_chain, bits16
+
+pytestmark = pytest.mark.gpu
+
+SEEDS = [(0, 0), (1234, 7), ((0xDEADBEEF << 32) | 0x1234567, (0xFFFFFFFF << 32) | 3)]
+
+
+@pytest.mark.parametrize("seed,offset", SEEDS)
+def test_noisy_operand_bit_exact(seed, offset):
+    rng = np.random.default_rng(31)
+    for shape in ((512, 512), (200, 136), (64, 4104), (1280, 640)):
+        W = (rng.standard_normal(shape) * 0.02).astype(np.float32)
+        q = qat.noisy_weight(torch.from_numpy(W).cuda(), seed, offset)
+        torch.cuda.synchronize()
+        ref = o.noisy_weight(W, seed, offset)
+        assert np.array_equal(bits16(q.operand), ref["operand_bits"]), shape
+        assert np.array_equal(q.scales.cpu().numpy(), ref["scales"]), shape
+    assert qat.device_error() == 0
+
+
+def test_noisy_linear_fwd_bwd():
+    c = sy.linear_case(N=512, K=512, T=300, seed=2, with_dy=True)
+    W = torch.from_numpy(c["W"]).cuda()
+    q = qat.noisy_weight(W, 99, 5)
+    T = 300
+    Y = torch.empty((T, 512), dtype=torch.bfloat16, device="cuda")
+    dX = torch.empty((T, 512), dtype=torch.bfloat16, device="cuda")
+    dW = torch.empty((512, 512), dtype=torch.float32, device="cuda")
+    qat.qat_linear_fwd(c["X"].cuda(), Y, 8, qw=q)
+    qat.qat_linear_bwd(c["X"].cuda(), c["dY"].cuda(), 8, qw=q, dX=dX, dW=dW)
+    torch.cuda.synchronize()
+    op = o.noisy_weight(c["W"], 99, 5)["operand"]
+    X, dY = c["X"].float().numpy(), c["dY"].float().numpy()
+    assert_close(Y, o.linear_fwd(op, X), "Y")
+    rdX, rdW = o.linear_bwd(op, X, dY)
+    assert_close(dX, rdX, "dX")
+    assert_close(dW, rdW, "dW")
+
+
+def test_noisy_recurrent_core():
+    c = sy.recurrent_core_case(T=300)
+    dev = {k: torch.from_numpy(c[k]).cuda() for k in ("Wq", "Wk", "Wv", "Wo", "Wfc", "Wproj")}
+    core = steps.RecurrentCore(dev["Wq"], dev["Wk"], dev["Wv"], dev["Wo"], dev["Wfc"], dev["Wproj"])
+    x = c["X"].cuda()
+    core.forward(x, 3, noise=(2024, 100))
+    torch.cuda.synchronize()
+    Ws = [np.concatenate([c["Wq"], c["Wk"], c["Wv"]]), c["Wo"], c["Wfc"], c["Wproj"]]
+    ref = o.recurrent_core_fwd_noisy(Ws, c["X"].float().numpy(), 3, 640, 2024, 100)
+    assert_close_chain(x, ref, 6, "noisy core, 3 applications")
+    assert qat.device_error() == 0

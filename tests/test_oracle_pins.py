@@ -411,3 +411,17 @@ def test_noisy_uses_documented_counter_layout():
         x = o.philox4x32_10([g, 0, 11, 3], [9, 5])[e % 4]
         u = np.float32(x >> 8) * np.float32(2.0 ** -24)
         assert r["noisy"].ravel()[e] == np.float32(u - np.float32(0.5))
+
+
+def test_noisy_recurrent_core_draws_per_application():
+    """Application r of the noisy core uses offsets offset + 4r + (0..3); two
+    applications equal one application of each draw chained."""
+    c = sy.recurrent_core_case(d=64, H=192, T=8)
+    Ws = [np.concatenate([c["Wq"], c["Wk"], c["Wv"]]), c["Wo"], c["Wfc"], c["Wproj"]]
+    X = c["X"].float().numpy()
+    two = o.recurrent_core_fwd_noisy(Ws, X, 2, 64, 3, 10)
+    x = X
+    for r in range(2):
+        q = [{"operand": o.noisy_weight(w, 3, 10 + 4 * r + k)["operand"]} for k, w in enumerate(Ws)]
+        x = o.recurrent_core_fwd(q[0], q[1], q[2], q[3], x, 1, 64)
+    assert np.array_equal(two, x)
