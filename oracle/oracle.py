@@ -30,6 +30,7 @@ def _c():
         P = ctypes.c_void_p
         I64 = ctypes.c_int64
         lib.oracle_qat_scales.argtypes = [P, I64, I64, P]
+        lib.oracle_qat_scales_bits.argtypes = [P, I64, I64, ctypes.c_int, P]
         lib.oracle_qat_codes.argtypes = [P, I64, I64, P, ctypes.c_int, P]
         lib.oracle_qat_codes.restype = ctypes.c_int
         lib.oracle_dequant_f32.argtypes = [P, P, I64, I64, P]
@@ -42,7 +43,8 @@ def _c():
         lib.oracle_fp16_array.argtypes = [P, I64, P]
         lib.oracle_bf16_array.argtypes = [P, I64, P]
         lib.oracle_philox4x32_10.argtypes = [P, P, P]
-        lib.oracle_noisy_operand.argtypes = [P, I64, I64, ctypes.c_uint64, ctypes.c_uint64, P, P, P]
+        lib.oracle_noisy_operand.argtypes = [P, I64, I64, ctypes.c_int, ctypes.c_uint64,
+                                             ctypes.c_uint64, P, P, P]
         _lib = lib
     return _lib
 
@@ -84,25 +86,26 @@ def fp16_bits(x):
 
 # ------------------------------------------------- QAT fake quantization (P5)
 
-def qat_scales(W):
-    """P5 "训练时的模拟量化": s_i = max(max_j |W_ij|, 1e-12) / 127 (fp32)."""
+def qat_scales(W, bits=8):
+    """P5 "训练时的模拟量化": s_i = max(max_j |W_ij|, 1e-12) / 127 (fp32); for
+    bits = 5 the divisor is 15 (P1 "更多算力下…": the int5 step amax / 15)."""
     W = _f32(W)
     N, K = W.shape
     s = np.empty(N, np.float32)
-    _c().oracle_qat_scales(_ptr(W), N, K, _ptr(s))
+    _c().oracle_qat_scales_bits(_ptr(W), N, K, int(bits), _ptr(s))
     return s
 
 
 def qat_codes(W, scales, bits):
     """P5 "训练时的模拟量化": int6 c = clamp(4*rne(rne(w/s)/4), -128, 124);
-    int8 c = clamp(rne(w/s), -127, 127)."""
+    int8 c = clamp(rne(w/s), -127, 127); int5 c = clamp(rne(w/s), -15, 15)."""
     W = _f32(W)
     s = _f32(scales)
     N, K = W.shape
     c = np.empty((N, K), np.int8)
     rc = _c().oracle_qat_codes(_ptr(W), N, K, _ptr(s), int(bits), _ptr(c))
     if rc != 0:
-        raise ValueError("bits must be 6 or 8")
+        raise ValueError("bits must be 5, 6 or 8")
     return c
 
 
@@ -131,7 +134,7 @@ def quantize_weight(W, bits):
     """Quantize once (also the recurrence cache: P1 "税 1", shared weights are
     stored once and quantized once).  Returns codes, scales, the fp32 STE
     value and the bf16 operand (as float64 for the algebra)."""
-    s = qat_scales(W)
+    s = qat_scales(W, bits)
     c = qat_codes(W, s, bits)
     op = bf16_bits_to_f32(operand_bf16_bits(c, s)).astype(np.float64)
     return {"codes": c, "scales": s, "wq": dequant(c, s), "operand": op}
@@ -149,16 +152,18 @@ def philox4x32_10(counter, key):
     return out
 
 
-def noisy_weight(W, seed, offset=0):
-    """P1 "幸存发现 1 Noisy QAT": w + (u - 0.5) * max(amax,1e-12)/127 per row, u from
-    Philox-4x32-10 (counter = element // 4 and offset, key = seed).  Returns the
-    fp32 scales, the noisy fp32 weight and its bf16 operand (float64 values)."""
+def noisy_weight(W, seed, offset=0, bits=8):
+    """P1 "幸存发现 1 Noisy QAT": w + (u - 0.5) * max(amax,1e-12)/127 per row (the
+    int8 step; bits = 5 uses the int5 step amax/15), u from Philox-4x32-10
+    (counter = element // 4 and offset, key = seed).  Returns the fp32 scales,
+    the noisy fp32 weight and its bf16 operand (float64 values)."""
     W = _f32(W)
     N, K = W.shape
     s = np.empty(N, np.float32)
     noisy = np.empty((N, K), np.float32)
     op = np.empty((N, K), np.uint16)
-    _c().oracle_noisy_operand(_ptr(W), N, K, int(seed), int(offset), _ptr(s), _ptr(noisy), _ptr(op))
+    _c().oracle_noisy_operand(_ptr(W), N, K, int(bits), int(seed), int(offset), _ptr(s),
+                              _ptr(noisy), _ptr(op))
     return {"scales": s, "noisy": noisy, "operand_bits": op,
             "operand": bf16_bits_to_f32(op).astype(np.float64)}
 
@@ -187,19 +192,36 @@ def relu2(x):
     return r * r
 
 
-def mlp_fwd(Wfc_op, Wproj_op, X):
-    """P5 "架构": MLP(x) = proj(relu(fc(x))^2).  Returns pre, h, Y."""
+def leaky2(x):
+    """LeakyReLU(0.5)^2 (P1 negative result #9; P4 leaderboard "LeakyReLU²")."""
+    x = _f64(x)
+    l = np.where(x > 0, x, 0.5 * x)
+    return l * l
+
+
+def mlp_fwd(Wfc_op, Wproj_op, X, act="relu2"):
+    """P5 "架构": MLP(x) = proj(relu(fc(x))^2) (act = "leaky2": proj(leaky_relu(fc(x), 0.5)^2)).
+    Returns pre, h, Y."""
     pre = _f64(X) @ _f64(Wfc_op).T
-    h = relu2(pre)
+    h = relu2(pre) if act == "relu2" else leaky2(pre)
     return pre, h, h @ _f64(Wproj_op).T
 
 
-def mlp_bwd(Wfc_op, Wproj_op, X, pre, h, dY):
-    """Chain rule through proj, relu^2 (derivative 2*relu(pre)) and fc, with the
-    STE making the quantized weights' gradients the weights' gradients."""
+def act_grad(pre, act="relu2"):
+    """d(act(pre))/d(pre): relu^2 -> 2 relu(pre); leaky(0.5)^2 -> 2x (x>0), x/2 (x<0)."""
+    pre = _f64(pre)
+    if act == "relu2":
+        return 2.0 * np.maximum(pre, 0.0)
+    return np.where(pre > 0, 2.0 * pre, 0.5 * pre)
+
+
+def mlp_bwd(Wfc_op, Wproj_op, X, pre, h, dY, act="relu2"):
+    """Chain rule through proj, the activation (relu^2: derivative 2*relu(pre))
+    and fc, with the STE making the quantized weights' gradients the weights'
+    gradients."""
     dY = _f64(dY)
     dh = dY @ _f64(Wproj_op)
-    dpre = dh * 2.0 * np.maximum(_f64(pre), 0.0)
+    dpre = dh * act_grad(pre, act)
     dWproj = dY.T @ _f64(h)
     dWfc = dpre.T @ _f64(X)
     dX = dpre @ _f64(Wfc_op)
@@ -268,7 +290,7 @@ def export_rows(W, bits, q=EXPORT_CLIP_Q):
     rc = _c().oracle_export_rows(_ptr(W), rows, cols, int(bits), float(q), _ptr(c),
                                  _ptr(s16), _ptr(s32))
     if rc != 0:
-        raise ValueError("bits must be 6 or 8")
+        raise ValueError("bits must be 5, 6 or 8")
     return c, s16, s32
 
 
@@ -286,12 +308,15 @@ _BLOCK_RE = re.compile(r"^blocks\.(\d+)\.")
 
 
 def export_state_dict(sd, int6_start=0, int6_end=10, fp16_embed_name="tok_emb.weight",
-                      keep_float_max=KEEP_FLOAT_MAX_NUMEL):
+                      keep_float_max=KEEP_FLOAT_MAX_NUMEL, mlp_int5=False, attn_int5=False):
     """P5 "后训练量化导出" rules, tensor by tensor:
     non-2D or numel <= keep_float_max -> fp16 passthrough; the tied embedding
     -> fp16 passthrough; other 2D tensors -> per-row codes, int6 when the
     tensor belongs to block i with int6_start <= i <= int6_end (inclusive,
-    -1 switches int6 off), else int8."""
+    -1 switches int6 off), else int8.
+    P1 reproduction commands (MLP_INT5 / ATTN_INT5): with mlp_int5 every block
+    MLP weight ("blocks.<i>.mlp."), with attn_int5 every block attention weight
+    ("blocks.<i>.attn.") is exported int5 instead (the mixed int5/int6 export)."""
     out = {}
     for name, t in sd.items():
         t = _f32(t)
@@ -304,6 +329,8 @@ def export_state_dict(sd, int6_start=0, int6_end=10, fp16_embed_name="tok_emb.we
             i = int(m.group(1))
             if int6_start <= i <= int6_end:
                 bits = 6
+        if m and ((mlp_int5 and ".mlp." in name) or (attn_int5 and ".attn." in name)):
+            bits = 5
         c, s16, _ = export_rows(t, bits)
         out[name] = {"kind": "int%d" % bits, "codes": c, "scale16": s16}
     return out

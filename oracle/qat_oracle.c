@@ -122,8 +122,14 @@ float oracle_fp16_to_f32(uint16_t h) {
 
 /* ---- QAT fake quantization (training-time simulated quantization) -------- */
 
-/* Per-row amax clamped below at 1e-12, scale = amax / 127. */
-void oracle_qat_scales(const float* W, int64_t N, int64_t K, float* scale) {
+/* Levels of a grid: the scale is amax / levels.  int6 and int8 use 127 (the
+ * int6 grid is every fourth int8 level); int5 uses 15 (reading of the page-1
+ * remark that an int5-calibrated step would be amax / 15: codes in [-15, 15]). */
+static float oracle_levels(int bits) { return bits == 5 ? 15.0f : 127.0f; }
+
+/* Per-row amax clamped below at 1e-12, scale = amax / levels. */
+void oracle_qat_scales_bits(const float* W, int64_t N, int64_t K, int bits, float* scale) {
+  const float levels = oracle_levels(bits);
   for (int64_t i = 0; i < N; ++i) {
     float amax = 0.0f;
     for (int64_t j = 0; j < K; ++j) {
@@ -131,16 +137,27 @@ void oracle_qat_scales(const float* W, int64_t N, int64_t K, float* scale) {
       if (a > amax) amax = a;
     }
     if (amax < ORACLE_AMAX_FLOOR) amax = ORACLE_AMAX_FLOOR;
-    scale[i] = amax / 127.0f;
+    scale[i] = amax / levels;
   }
+}
+
+/* The int6 / int8 scale, amax / 127. */
+void oracle_qat_scales(const float* W, int64_t N, int64_t K, float* scale) {
+  oracle_qat_scales_bits(W, N, K, 8, scale);
 }
 
 /* One code from a weight value and its row scale.
  * bits == 6: rne(rne(w/s)/4)*4 clamped to [-128, 124] (64 levels, multiples
  *            of 4 stored in an int8);
- * bits == 8: rne(w/s) clamped to [-127, 127]. */
+ * bits == 8: rne(w/s) clamped to [-127, 127];
+ * bits == 5: rne(w/s) clamped to [-15, 15] (s = amax / 15). */
 static int oracle_code(float w, float s, int bits) {
   float q_raw = nearbyintf(w / s);
+  if (bits == 5) {
+    if (q_raw < -15.0f) q_raw = -15.0f;
+    if (q_raw > 15.0f) q_raw = 15.0f;
+    return (int)q_raw;
+  }
   if (bits == 6) {
     float q = nearbyintf(q_raw / 4.0f) * 4.0f;
     if (q < -128.0f) q = -128.0f;
@@ -154,7 +171,7 @@ static int oracle_code(float w, float s, int bits) {
 
 int oracle_qat_codes(const float* W, int64_t N, int64_t K, const float* scale, int bits,
                      int8_t* codes) {
-  if (bits != 6 && bits != 8) return -1;
+  if (bits != 5 && bits != 6 && bits != 8) return -1;
   for (int64_t i = 0; i < N; ++i)
     for (int64_t j = 0; j < K; ++j)
       codes[i * K + j] = (int8_t)oracle_code(W[i * K + j], scale[i], bits);
@@ -211,12 +228,12 @@ float oracle_row_quantile_abs(const float* row, int64_t n, double qf) {
  * stored scale fp16_rne(s).  scale32 may be NULL. */
 int oracle_export_rows(const float* W, int64_t rows, int64_t cols, int bits, double qf,
                        int8_t* codes, uint16_t* scale16, float* scale32) {
-  if (bits != 6 && bits != 8) return -1;
+  if (bits != 5 && bits != 6 && bits != 8) return -1;
   for (int64_t i = 0; i < rows; ++i) {
     const float* r = W + i * cols;
     float clip = oracle_row_quantile_abs(r, cols, qf);
     float c = clip < ORACLE_AMAX_FLOOR ? ORACLE_AMAX_FLOOR : clip;
-    float s = c / 127.0f;
+    float s = c / oracle_levels(bits);
     for (int64_t j = 0; j < cols; ++j) {
       float w = r[j];
       if (w > clip) w = clip;
@@ -281,11 +298,13 @@ void oracle_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t
 }
 
 /* Noisy forward weight of every element and its bf16 operand:
- *   s = fl32(max(amax, 1e-12) / 127);  noise = fl32(fl32(u - 0.5) * s);
+ *   s = fl32(max(amax, 1e-12) / levels), levels 127 (noise at the int8 step, as
+ *   the page's code) or 15 (bits == 5: at the int5 step, the page's remark);
+ *   noise = fl32(fl32(u - 0.5) * s);
  *   w' = fl32(w + noise);  operand = bf16_rne(w').  (u - 0.5 is exact.) */
-void oracle_noisy_operand(const float* W, int64_t N, int64_t K, uint64_t seed, uint64_t offset,
-                          float* scale, float* noisy, uint16_t* operand) {
-  oracle_qat_scales(W, N, K, scale);
+void oracle_noisy_operand(const float* W, int64_t N, int64_t K, int bits, uint64_t seed,
+                          uint64_t offset, float* scale, float* noisy, uint16_t* operand) {
+  oracle_qat_scales_bits(W, N, K, bits, scale);
   uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
   for (int64_t i = 0; i < N; ++i) {
     for (int64_t j = 0; j < K; ++j) {

@@ -42,6 +42,42 @@ def test_worked_example_int6_int8():
     assert o.qat_codes(W, s, 8)[0].tolist() == [int(v) for v in g["int8"]]
 
 
+def test_int5_worked_example():
+    """P1 "幸存发现 1 Noisy QAT" (int5 step amax / 15) and the MLP_INT5 /
+    ATTN_INT5 switches: hand-derived codes, ties to even."""
+    g = _golden("int5_worked_example.txt")
+    for r in ("W", "V"):
+        W = np.array([g[r]], dtype=np.float32)
+        s = o.qat_scales(W, 5)
+        assert s[0] == np.float32(g[r + "_scale"][0])
+        assert o.qat_codes(W, s, 5)[0].tolist() == [int(v) for v in g[r + "_int5"]]
+    A = np.array([g["A"]], np.float32)
+    c5, s16, _ = o.export_rows(A, 5)
+    assert c5[0].tolist() == [int(v) for v in g["A_int5"]]
+    assert int(s16[0]) == int(g["A_scale16"][0])
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_int5_grid_and_error_bound(seed):
+    """int5: s = fl32(amax/15) (numpy IEEE division), codes in [-15, 15], the
+    code is numpy's rne of the IEEE quotient, |w - c*s| <= s/2 (+ fp32
+    roundings), and every row's amax element saturates to +-15."""
+    W = sy.linear_case(seed=seed)["W"]
+    s = o.qat_scales(W, 5)
+    amax = np.abs(W).max(axis=1)
+    assert np.array_equal(s, amax / np.float32(15.0))
+    c = o.qat_codes(W, s, 5).astype(np.int32)
+    assert c.min() >= -15 and c.max() <= 15
+    assert np.array_equal(c, np.clip(np.rint(W / s[:, None]), -15, 15).astype(np.int32))
+    err = np.abs(W.astype(np.float64) - o.dequant(c.astype(np.int8), s).astype(np.float64))
+    assert np.all(err / s[:, None].astype(np.float64) <= 0.5 + 64 * 2.0 ** -24)
+    im = np.argmax(np.abs(W), axis=1)
+    cm = c[np.arange(W.shape[0]), im]
+    assert np.array_equal(np.abs(cm), np.full(W.shape[0], 15))
+    wq = o.dequant(c.astype(np.int8), s)
+    assert np.array_equal(o.qat_codes(wq, s, 5), c.astype(np.int8))
+
+
 def test_scale_is_ieee_division_and_floor():
     """s = fl32(max(amax, 1e-12) / 127) -- numpy float32 division is IEEE."""
     c = sy.linear_case()
@@ -261,6 +297,13 @@ def test_export_passthrough_and_layer_range():
                      "tok_emb.weight": "fp16"}
     off = o.export_state_dict(sd, int6_start=-1, int6_end=-1)
     assert off["blocks.0.b"]["kind"] == "int8"
+    sd5 = {"blocks.1.mlp.fc.weight": sd["blocks.0.b"], "blocks.12.attn.c_q.weight": sd["blocks.0.b"],
+           "blocks.1.attn.c_q.weight": sd["blocks.0.b"]}
+    k5 = {k: v["kind"] for k, v in o.export_state_dict(sd5, mlp_int5=True).items()}
+    assert k5 == {"blocks.1.mlp.fc.weight": "int5", "blocks.12.attn.c_q.weight": "int8",
+                  "blocks.1.attn.c_q.weight": "int6"}
+    k5 = {k: v["kind"] for k, v in o.export_state_dict(sd5, mlp_int5=True, attn_int5=True).items()}
+    assert set(k5.values()) == {"int5"}
     assert np.array_equal(out["vec"]["bits16"], sd["vec"].astype(np.float16).view(np.uint16))
 
 
@@ -309,6 +352,22 @@ def test_mlp_relu2_and_bwd_finite_differences():
     assert np.abs(pre).min() > 1e-3  # keep finite differences off the kink
     L = lambda: float(np.sum(dY * o.mlp_fwd(Wfc, Wproj, X)[2]))
     dX, dWfc, dWproj = o.mlp_bwd(Wfc, Wproj, X, pre, h, dY)
+    assert np.allclose(dX, _fd(L, X), atol=1e-5)
+    assert np.allclose(dWfc, _fd(L, Wfc), atol=1e-5)
+    assert np.allclose(dWproj, _fd(L, Wproj), atol=1e-5)
+
+
+def test_mlp_leaky2_and_bwd_finite_differences():
+    """LeakyReLU(0.5)^2 (P1 negative result #9) is x*x for x>0 and x*x/4
+    otherwise; its backward matches central differences."""
+    rng = np.random.default_rng(15)
+    X, Wfc, Wproj = rng.standard_normal((3, 4)), rng.standard_normal((8, 4)), rng.standard_normal((4, 8))
+    dY = rng.standard_normal((3, 4))
+    pre, h, Y = o.mlp_fwd(Wfc, Wproj, X, act="leaky2")
+    assert np.array_equal(h, np.where(pre > 0, pre * pre, 0.25 * pre * pre))
+    assert (pre < 0).any() and (pre > 0).any() and np.abs(pre).min() > 1e-3
+    L = lambda: float(np.sum(dY * o.mlp_fwd(Wfc, Wproj, X, act="leaky2")[2]))
+    dX, dWfc, dWproj = o.mlp_bwd(Wfc, Wproj, X, pre, h, dY, act="leaky2")
     assert np.allclose(dX, _fd(L, X), atol=1e-5)
     assert np.allclose(dWfc, _fd(L, Wfc), atol=1e-5)
     assert np.allclose(dWproj, _fd(L, Wproj), atol=1e-5)
@@ -411,6 +470,26 @@ def test_noisy_uses_documented_counter_layout():
         x = o.philox4x32_10([g, 0, 11, 3], [9, 5])[e % 4]
         u = np.float32(x >> 8) * np.float32(2.0 ** -24)
         assert r["noisy"].ravel()[e] == np.float32(u - np.float32(0.5))
+
+
+def test_noisy_int5_step_shares_the_draws():
+    """bits = 5 scales the same uniform draws by the int5 step amax/15: a row
+    of amax 15 (s = 1) gets noise u - 1/2 from the documented counter layout,
+    and every |w' - w| <= s5/2."""
+    W = np.zeros((2, 8), np.float32)
+    W[:, 0] = 15.0
+    r = o.noisy_weight(W, seed=(5 << 32) | 9, offset=(3 << 32) | 11, bits=5)
+    assert np.all(r["scales"] == 1.0)
+    for e in (1, 2, 5, 9, 14):
+        x = o.philox4x32_10([e // 4, 0, 11, 3], [9, 5])[e % 4]
+        u = np.float32(x >> 8) * np.float32(2.0 ** -24)
+        assert r["noisy"].ravel()[e] == np.float32(u - np.float32(0.5))
+    W = sy.linear_case(N=64, K=256, seed=6)["W"]
+    r = o.noisy_weight(W, 77, 1, bits=5)
+    s = r["scales"].astype(np.float64)
+    assert np.array_equal(r["scales"], o.qat_scales(W, 5))
+    d = np.abs(r["noisy"].astype(np.float64) - W.astype(np.float64)) / s[:, None]
+    assert np.all(d <= 0.5 + np.spacing(np.abs(r["noisy"])).astype(np.float64) / s[:, None])
 
 
 def test_noisy_recurrent_core_draws_per_application():
