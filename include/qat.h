@@ -1,10 +1,12 @@
 /*
  * qat.h -- C ABI of the B200 (sm_100a) int6 quantization-aware linear, ReLU^2
- * MLP, recurrent-core weight cache and export quantizer.
+ * MLP, recurrent-core weight cache and export quantizer (with the int5 grid,
+ * Noisy QAT and the LeakyReLU(0.5)^2 MLP of the depth-recurrence write-up).
  *
  * Page references used below (title, section):
  *   [P5] "parameter-golf 16MB 极限压缩实战：11L MLP3x + Int6 QAT + zstd-22 记录详解"
  *   [P1] "Depth Recurrence + Mixed-Precision Quant" write-up of PR #363
+ *   [P4] "openai/parameter-golf" README mirror, leaderboard table
  *
  * Conventions shared by every call
  *   - Every pointer is a caller-owned DEVICE pointer unless stated otherwise,
@@ -18,7 +20,10 @@
  *   - Arguments are validated on the host before any launch; on error
  *     nothing is launched and a QAT_ERR_* code is returned.
  *   - bits = 6 selects the int6 grid (multiples of 4 in [-128,124], 64
- *     levels in an int8 container); bits = 8 the int8 grid [-127,127].
+ *     levels in an int8 container); bits = 8 the int8 grid [-127,127];
+ *     bits = 5 the int5 grid [-15,15] with scale amax/15 ([P1] "幸存发现 1
+ *     Noisy QAT" gives amax/15 as the int5 step; its reproduction commands
+ *     switch MLP and attention weights to int5 with MLP_INT5 / ATTN_INT5).
  *   - Shapes: feature dimensions (N, K, d, H, cols) must be multiples of 8
  *     (16-byte rows for bf16, as the tensor-memory-access engine requires);
  *     the token count T may be anything >= 0 (T = 0 is a no-op).
@@ -42,7 +47,7 @@ typedef uint16_t qat_fp16;                /* IEEE binary16 bit pattern */
 
 enum {
   QAT_OK = 0,
-  QAT_ERR_ARG = 1,        /* null pointer, non-positive size, bits not in {6,8} */
+  QAT_ERR_ARG = 1,        /* null pointer, non-positive size, bits not in {5,6,8} */
   QAT_ERR_ALIGN = 2,      /* a pointer is not 16-byte aligned */
   QAT_ERR_SHAPE = 3,      /* a feature dimension is not a multiple of 8, or too large */
   QAT_ERR_WORKSPACE = 4,  /* workspace missing or smaller than qat_workspace_size() */
@@ -80,8 +85,9 @@ typedef struct qat_qweight {
 
 /* [P5] "训练时的模拟量化": per row i of W [N,K] fp32,
  *   amax_i = max(max_j |W_ij|, 1e-12)      (floor from [P1] "修复" code)
- *   s_i    = fl32(amax_i / 127)             (IEEE division)
+ *   s_i    = fl32(amax_i / 127)             (IEEE division; / 15 for int5)
  *   int6:  c = clamp(4*rne(rne(fl32(W/s))/4), -128, 124);  int8: clamp(rne(W/s), -127, 127)
+ *   int5:  c = clamp(rne(fl32(W/s)), -15, 15)
  *   operand = bf16_rne(fl32(c * s))         (the STE forward value cast to bf16)
  * Outputs: scales [N] (required), codes [N,K] (nullable), operand [N,K] (nullable).
  * Bit-exact with the CPU oracle. */
@@ -90,7 +96,9 @@ int qat_quantize_weights(const float* W, int32_t N, int32_t K, int32_t bits, int
 
 /* Noisy QAT for the shared blocks of a depth-recurrent core ([P1] "幸存发现 1
  * Noisy QAT"): instead of the STE fake quantization, the forward weight is
- *   w' = fl32(w + fl32(fl32(u - 1/2) * s)),  s = fl32(max(amax_row, 1e-12) / 127),
+ *   w' = fl32(w + fl32(fl32(u - 1/2) * s)),  s = fl32(max(amax_row, 1e-12) / L),
+ * L = 127 (the int8 step of the page's code) for bits 6 or 8, L = 15 for
+ * bits = 5 (the int5-matched step the page proposes for an int5 export),
  * u uniform in [0,1), and the gradient flows through w' to w unchanged (the
  * noise carries none), so the backward is qat_linear_bwd with this operand.
  * u comes from Philox-4x32-10 (Salmon et al., SC'11): element e of the
@@ -99,8 +107,8 @@ int qat_quantize_weights(const float* W, int32_t N, int32_t K, int32_t bits, int
  * u = (word >> 8) * 2^-24.  Outputs: operand [N,K] bf16 = bf16_rne(w')
  * (required; pass it as qat_qweight.operand), scales [N] fp32 (nullable).
  * Bit-exact with the CPU oracle.  Use a fresh offset per draw. */
-int qat_noisy_operand(const float* W, int32_t N, int32_t K, uint64_t seed, uint64_t offset,
-                      float* scales, qat_bf16* operand, qat_stream_t stream);
+int qat_noisy_operand(const float* W, int32_t N, int32_t K, int32_t bits, uint64_t seed,
+                      uint64_t offset, float* scales, qat_bf16* operand, qat_stream_t stream);
 
 /* Workspace sizes (bytes) for the calls below.  `raw_weights` != 0 means the
  * call is given fp32 weights to quantize itself (the workspace then also
@@ -128,25 +136,32 @@ int qat_linear_bwd(const float* W, const qat_qweight* qw, int32_t N, int32_t K, 
                    const qat_bf16* X, const qat_bf16* dY, int64_t T, qat_bf16* dX, float* dW,
                    int32_t accumulate_dW, void* workspace, size_t ws_bytes, qat_stream_t stream);
 
-/* [P5] "架构" ReLU^2 MLP forward, both linears int6/int8 QAT:
- *   pre = X . Wfc_q^T  [T,H];  h = relu(pre)^2 (fused in the fc epilogue, from the
- *   fp32 accumulator);  Y = bf16(h . Wproj_q^T (+ residual))  [T,d].
+/* MLP activations: [P5] "架构" relu(x)^2, and leaky_relu(x, 0.5)^2 ([P1]
+ * negative result #9 "LeakyReLU(0.5)²"; [P4] leaderboard entries use it). */
+enum { QAT_ACT_RELU2 = 0, QAT_ACT_LEAKY_RELU2 = 1 };
+
+/* [P5] "架构" ReLU^2 MLP forward, both linears int5/int6/int8 QAT:
+ *   pre = X . Wfc_q^T  [T,H];  h = act(pre) (fused in the fc epilogue, from the
+ *   fp32 accumulator: relu(pre)^2, or for QAT_ACT_LEAKY_RELU2 t^2 with t = pre
+ *   (pre > 0) else pre/2);  Y = bf16(h . Wproj_q^T (+ residual))  [T,d].
  * Weights: (Wfc [H,d], Wproj [d,H]) fp32, or (qfc, qproj).  pre_save [T,H]
  * (nullable) and h_save [T,H] (nullable; the workspace holds h otherwise)
  * keep the activations for the backward.  residual may alias Y exactly. */
 int qat_mlp_fwd(const float* Wfc, const float* Wproj, const qat_qweight* qfc,
-                const qat_qweight* qproj, int32_t d, int32_t H, int32_t bits, const qat_bf16* X,
-                int64_t T, const qat_bf16* residual, qat_bf16* Y, qat_bf16* pre_save,
-                qat_bf16* h_save, void* workspace, size_t ws_bytes, qat_stream_t stream);
+                const qat_qweight* qproj, int32_t d, int32_t H, int32_t bits, int32_t act,
+                const qat_bf16* X, int64_t T, const qat_bf16* residual, qat_bf16* Y,
+                qat_bf16* pre_save, qat_bf16* h_save, void* workspace, size_t ws_bytes,
+                qat_stream_t stream);
 
 /* STE backward of qat_mlp_fwd from the saved pre and h:
- *   dh = dY . Wproj_q;  dpre = dh * 2*relu(pre) (fused in the dh epilogue);
+ *   dh = dY . Wproj_q;  dpre = dh * act'(pre) (fused in the dh epilogue:
+ *   2*relu(pre), or for QAT_ACT_LEAKY_RELU2 2*pre (pre > 0) else pre/2);
  *   dWproj (+)= dY^T . h;  dWfc (+)= dpre^T . X;  dX = dpre . Wfc_q.
  * dX, dWfc, dWproj may each be NULL.  The workspace holds dpre [T,H] bf16. */
 int qat_mlp_bwd(const float* Wfc, const float* Wproj, const qat_qweight* qfc,
-                const qat_qweight* qproj, int32_t d, int32_t H, int32_t bits, const qat_bf16* X,
-                const qat_bf16* pre, const qat_bf16* h, const qat_bf16* dY, int64_t T,
-                qat_bf16* dX, float* dWfc, float* dWproj, int32_t accumulate_dW,
+                const qat_qweight* qproj, int32_t d, int32_t H, int32_t bits, int32_t act,
+                const qat_bf16* X, const qat_bf16* pre, const qat_bf16* h, const qat_bf16* dY,
+                int64_t T, qat_bf16* dX, float* dWfc, float* dWproj, int32_t accumulate_dW,
                 void* workspace, size_t ws_bytes, qat_stream_t stream);
 
 /* ---------------------------------------------------------------------------
@@ -182,8 +197,8 @@ int qat_linear_fwd_noalloc(const float* W, int32_t N, int32_t K, int32_t bits,
  *   clip   = linear-interpolated quantile of |w| at q = 0.9999984: sorted
  *            values v, pos = q*(cols-1) (double), lo = floor(pos), hi = lo+1,
  *            clip = fl32(v_lo + fl32(fl32(pos-lo) * fl32(v_hi - v_lo)))
- *   s32    = fl32(max(clip, 1e-12) / 127)
- *   codes  = the training grid (bits 6 or 8) applied to clamp(w, -clip, clip) with s32
+ *   s32    = fl32(max(clip, 1e-12) / 127)   (/ 15 for bits = 5)
+ *   codes  = the training grid (bits 5, 6 or 8) applied to clamp(w, -clip, clip) with s32
  *   scales = fp16_rne(s32)
  * Only the top (cols - lo) order statistics of |w| matter; rows longer than
  * 625,001 columns (where more than the top two would) return QAT_ERR_SHAPE.
@@ -193,7 +208,7 @@ int quantize_rows_export(const float* W, int64_t rows, int64_t cols, int32_t bit
                          int8_t* codes, qat_fp16* scales, qat_stream_t stream);
 
 /* One grouped launch over a whole state dict.  `descs` is a HOST array of n
- * descriptors (n <= QAT_EXPORT_MAX_DESCS); mode 6 or 8 quantizes rows as
+ * descriptors (n <= QAT_EXPORT_MAX_DESCS); mode 5, 6 or 8 quantizes rows as
  * above into dst (int8 codes) and scales; mode QAT_EXPORT_FP16 converts src
  * to fp16 (rne) into dst (the passthrough of non-2D, small and tied-embedding
  * tensors; scales unused).  The caller applies the passthrough rules. */

@@ -228,7 +228,7 @@ def mlp_bwd(Wfc_op, Wproj_op, X, pre, h, dY, act="relu2"):
     return dX, dWfc, dWproj
 
 
-def recurrent_core_fwd(q_qkv, q_o, q_fc, q_proj, X, R, d):
+def recurrent_core_fwd(q_qkv, q_o, q_fc, q_proj, X, R, d, act="relu2"):
     """Depth-recurrent core (P1 "Stem / Core / Tail", "税 1"): the block's
     linears, quantized once, applied R times.  Attention is left out, so the
     O projection reads the query slice of QKV (reading stated in the design
@@ -243,30 +243,32 @@ def recurrent_core_fwd(q_qkv, q_o, q_fc, q_proj, X, R, d):
     for _ in range(R):
         qkv = b(x @ q_qkv["operand"].T)
         x1 = b(x + qkv[:, :d] @ q_o["operand"].T)
-        h = b(relu2(x1 @ q_fc["operand"].T))
+        pre = x1 @ q_fc["operand"].T
+        h = b(relu2(pre) if act == "relu2" else leaky2(pre))
         x = b(x1 + h @ q_proj["operand"].T)
     return x
 
 
-def recurrent_core_fwd_noisy(Ws, X, R, d, seed, offset):
+def recurrent_core_fwd_noisy(Ws, X, R, d, seed, offset, bits=6, act="relu2"):
     """The recurrent core under Noisy QAT (P1 "幸存发现 1"): application r uses
     the noisy operands of the four weights (qkv, o, fc, proj -> k = 0..3) drawn
-    at Philox offset offset + 4*r + k, composed exactly as recurrent_core_fwd."""
+    at Philox offset offset + 4*r + k (noise at the int8 step, or at the int5
+    step for bits = 5), composed exactly as recurrent_core_fwd."""
     x = X
     for r in range(R):
-        q = [{"operand": noisy_weight(w, seed, offset + 4 * r + k)["operand"]}
+        q = [{"operand": noisy_weight(w, seed, offset + 4 * r + k, bits)["operand"]}
              for k, w in enumerate(Ws)]
-        x = recurrent_core_fwd(q[0], q[1], q[2], q[3], x, 1, d)
+        x = recurrent_core_fwd(q[0], q[1], q[2], q[3], x, 1, d, act)
     return x
 
 
-def head_mlp_step(q_emb, q_fc, q_proj, X, dLogits):
+def head_mlp_step(q_emb, q_fc, q_proj, X, dLogits, act="relu2"):
     """Tied-head throughput step: Z = MLP(X), logits = Z Wemb^T, then the STE
     backward of both from the upstream gradient dLogits."""
-    pre, h, Z = mlp_fwd(q_fc["operand"], q_proj["operand"], X)
+    pre, h, Z = mlp_fwd(q_fc["operand"], q_proj["operand"], X, act)
     logits = Z @ q_emb["operand"].T
     dZ, dWemb = linear_bwd(q_emb["operand"], Z, dLogits)
-    dX, dWfc, dWproj = mlp_bwd(q_fc["operand"], q_proj["operand"], X, pre, h, dZ)
+    dX, dWfc, dWproj = mlp_bwd(q_fc["operand"], q_proj["operand"], X, pre, h, dZ, act)
     return {"pre": pre, "h": h, "Z": Z, "logits": logits, "dZ": dZ, "dWemb": dWemb,
             "dX": dX, "dWfc": dWfc, "dWproj": dWproj}
 

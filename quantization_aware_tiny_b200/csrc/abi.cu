@@ -59,7 +59,8 @@ struct Carver {
 
 inline size_t operand_bytes(int64_t N, int64_t K) { return align_up(N * K * 2) + align_up(N * 4); }
 
-bool bits_ok(int bits) { return bits == 6 || bits == 8; }
+bool bits_ok(int bits) { return bits == 5 || bits == 6 || bits == 8; }
+bool act_ok(int act) { return act == QAT_ACT_RELU2 || act == QAT_ACT_LEAKY_RELU2; }
 bool dim_ok(int64_t x) { return x > 0 && (x & 7) == 0 && x <= (1 << 20); }
 
 // The bf16 operand of a weight: taken from `qw`, or produced from fp32 `W`
@@ -116,12 +117,12 @@ int qat_device_error(qat_stream_t stream) {
   return v;
 }
 
-int qat_noisy_operand(const float* W, int32_t N, int32_t K, uint64_t seed, uint64_t offset,
-                      float* scales, qat_bf16* operand, qat_stream_t stream) {
-  if (!W || !operand || N <= 0) return QAT_ERR_ARG;
+int qat_noisy_operand(const float* W, int32_t N, int32_t K, int32_t bits, uint64_t seed,
+                      uint64_t offset, float* scales, qat_bf16* operand, qat_stream_t stream) {
+  if (!W || !operand || N <= 0 || !bits_ok(bits)) return QAT_ERR_ARG;
   if (!dim_ok(K)) return QAT_ERR_SHAPE;
   if (!aligned16(W) || !aligned16(operand)) return QAT_ERR_ALIGN;
-  return launch_noisy_operand(W, N, K, seed, offset, scales,
+  return launch_noisy_operand(W, N, K, bits, seed, offset, scales,
                               reinterpret_cast<__nv_bfloat16*>(operand), stream);
 }
 
@@ -214,10 +215,11 @@ int qat_linear_bwd(const float* W, const qat_qweight* qw, int32_t N, int32_t K, 
 }
 
 int qat_mlp_fwd(const float* Wfc, const float* Wproj, const qat_qweight* qfc,
-                const qat_qweight* qproj, int32_t d, int32_t H, int32_t bits, const qat_bf16* X,
-                int64_t T, const qat_bf16* residual, qat_bf16* Y, qat_bf16* pre_save,
-                qat_bf16* h_save, void* workspace, size_t ws_bytes, qat_stream_t stream) {
-  if ((T > 0 && (!X || !Y)) || T < 0 || !bits_ok(bits)) return QAT_ERR_ARG;
+                const qat_qweight* qproj, int32_t d, int32_t H, int32_t bits, int32_t act,
+                const qat_bf16* X, int64_t T, const qat_bf16* residual, qat_bf16* Y,
+                qat_bf16* pre_save, qat_bf16* h_save, void* workspace, size_t ws_bytes,
+                qat_stream_t stream) {
+  if ((T > 0 && (!X || !Y)) || T < 0 || !bits_ok(bits) || !act_ok(act)) return QAT_ERR_ARG;
   if (!dim_ok(d) || !dim_ok(H)) return QAT_ERR_SHAPE;
   if ((pre_save && !aligned16(pre_save)) || (h_save && !aligned16(h_save))) return QAT_ERR_ALIGN;
   Carver ws(workspace, ws_bytes);
@@ -232,11 +234,11 @@ int qat_mlp_fwd(const float* Wfc, const float* Wproj, const qat_qweight* qfc,
     h = ws.take(static_cast<size_t>(T) * H * 2);
     if (!h) return QAT_ERR_WORKSPACE;
   }
-  GemmDesc g1;  // pre = X . Wfc^T ; h = relu(pre)^2
+  GemmDesc g1;  // pre = X . Wfc^T ; h = act(pre)
   g1.A = X; g1.lda = d;
   g1.B = op_fc; g1.ldb = d;
   g1.M = T; g1.N = H; g1.K = d;
-  g1.epi = EPI_RELU2;
+  g1.epi = act == QAT_ACT_RELU2 ? EPI_RELU2 : EPI_LRELU2;
   g1.D = pre_save; g1.ldd = H;
   g1.D2 = h; g1.ldd2 = H;
   rc = launch_gemm(g1, stream);
@@ -252,11 +254,12 @@ int qat_mlp_fwd(const float* Wfc, const float* Wproj, const qat_qweight* qfc,
 }
 
 int qat_mlp_bwd(const float* Wfc, const float* Wproj, const qat_qweight* qfc,
-                const qat_qweight* qproj, int32_t d, int32_t H, int32_t bits, const qat_bf16* X,
-                const qat_bf16* pre, const qat_bf16* h, const qat_bf16* dY, int64_t T,
-                qat_bf16* dX, float* dWfc, float* dWproj, int32_t accumulate_dW,
+                const qat_qweight* qproj, int32_t d, int32_t H, int32_t bits, int32_t act,
+                const qat_bf16* X, const qat_bf16* pre, const qat_bf16* h, const qat_bf16* dY,
+                int64_t T, qat_bf16* dX, float* dWfc, float* dWproj, int32_t accumulate_dW,
                 void* workspace, size_t ws_bytes, qat_stream_t stream) {
-  if ((T > 0 && (!X || !pre || !h || !dY)) || T < 0 || !bits_ok(bits)) return QAT_ERR_ARG;
+  if ((T > 0 && (!X || !pre || !h || !dY)) || T < 0 || !bits_ok(bits) || !act_ok(act))
+    return QAT_ERR_ARG;
   if (!dim_ok(d) || !dim_ok(H)) return QAT_ERR_SHAPE;
   Carver ws(workspace, ws_bytes);
   const __nv_bfloat16 *op_fc = nullptr, *op_proj = nullptr;
@@ -286,12 +289,12 @@ int qat_mlp_bwd(const float* Wfc, const float* Wproj, const qat_qweight* qfc,
     rc = launch_gemm(g, stream);
     if (rc) return rc;
   }
-  {  // dpre[T,H] = (dY . Wproj_q) * 2 relu(pre)
+  {  // dpre[T,H] = (dY . Wproj_q) * act'(pre)
     GemmDesc g;
     g.A = dY; g.lda = d;
     g.B = op_proj; g.ldb = H; g.b_mn = true;
     g.M = T; g.N = H; g.K = d;
-    g.epi = EPI_DRELU2;
+    g.epi = act == QAT_ACT_RELU2 ? EPI_DRELU2 : EPI_DLRELU2;
     g.D = dpre; g.ldd = H;
     g.R = pre; g.ldr = H;
     rc = launch_gemm(g, stream);
@@ -331,7 +334,7 @@ int quantize_rows_export(const float* W, int64_t rows, int64_t cols, int32_t bit
   d.reserved = 0;
   d.dst = codes;
   d.scales = scales;
-  if (bits != 6 && bits != 8) return QAT_ERR_ARG;
+  if (!bits_ok(bits)) return QAT_ERR_ARG;
   return quantize_export_batch(&d, 1, stream);
 }
 
@@ -358,7 +361,7 @@ int quantize_export_batch(const qat_export_desc* descs, int32_t n, qat_stream_t 
       d.cols = kFp16Chunk;
       d.rows = (d.numel + kFp16Chunk - 1) / kFp16Chunk;
       d.unit_rows = 1;
-    } else if (s.mode == 6 || s.mode == 8) {
+    } else if (bits_ok(s.mode)) {
       if (!s.scales) return QAT_ERR_ARG;
       if (!dim_ok(s.cols)) return QAT_ERR_SHAPE;
       d.rows = s.rows;

@@ -59,7 +59,8 @@ __device__ __forceinline__ float div_by_scale(float w, float s, float r) {
 //   int6: 4 * rne(k / 4) in integers -- with k = 4m + f, f in 0..3, the result
 //         is 4m for f <= 1, 4m + 4 for f = 3 and the even one of 4m, 4m + 4 for
 //         f = 2, i.e. (k + 1 + (m & 1)) & ~3 -- then clamped to [-128, 124];
-//   int8: k clamped to [-127, 127].
+//   int8: k clamped to [-127, 127];
+//   int5: k clamped to [-15, 15] (the scale is then amax / 15).
 __device__ __forceinline__ int code_from_quotient(float x, int bits) {
   // rne(x) for |x| < 2^22: adding 1.5 * 2^23 gives a float whose ulp is 1, so
   // the sum is rounded to an integer -- ties to even, as the offset is even --
@@ -69,10 +70,15 @@ __device__ __forceinline__ int code_from_quotient(float x, int bits) {
     k = (k + 1 + ((k >> 2) & 1)) & ~3;
     return min(max(k, -128), 124);
   }
+  if (bits == 5) return min(max(k, -15), 15);
   return min(max(k, -127), 127);
 }
 
-// Code of one weight on the int6 / int8 grid; r = fl32(1 / s).
+// Levels of a grid's scale, s = amax / levels: 15 for int5, 127 for int6 and
+// int8 (the int6 grid is every fourth int8 level).
+__device__ __forceinline__ float grid_levels(int bits) { return bits == 5 ? 15.0f : 127.0f; }
+
+// Code of one weight on the int5 / int6 / int8 grid; r = fl32(1 / s).
 __device__ __forceinline__ int quant_code(float w, float s, float r, int bits) {
   return code_from_quotient(div_by_scale(w, s, r), bits);
 }

@@ -102,13 +102,20 @@ __device__ __forceinline__ void stage_chunk(const KArgs& p, const uint32_t (&acc
           o[i] = __fadd_rn(a, bf2f(r[i]));
         } else if constexpr (EPI == EPI_DRELU2) {
           o[i] = __fmul_rn(__fmul_rn(a, fmaxf(bf2f(r[i]), 0.0f)), 2.0f);
+        } else if constexpr (EPI == EPI_DLRELU2) {
+          // d/dx leaky(x, 0.5)^2 = 2x (x > 0), x/2 (x <= 0): the scalings are exact
+          const float pre = bf2f(r[i]);
+          o[i] = __fmul_rn(a, pre > 0.0f ? __fmul_rn(pre, 2.0f) : __fmul_rn(pre, 0.5f));
+        } else if constexpr (EPI == EPI_LRELU2) {  // buf1 <- leaky_relu(acc, 0.5)^2
+          const float t = a > 0.0f ? a : __fmul_rn(a, 0.5f);
+          o[i] = __fmul_rn(t, t);
         } else {  // EPI_RELU2: buf0 <- pre (when kept), buf1 <- relu(acc)^2
           const float t = fmaxf(a, 0.0f);
           o[i] = __fmul_rn(t, t);
         }
       }
       const uint32_t at = off + (static_cast<uint32_t>(j ^ sw) << 4);
-      if constexpr (EPI == EPI_RELU2) {
+      if constexpr (epi_act_fwd(EPI)) {
         st_shared_v4(buf0 + at, pack_bf16(v[8 * j], v[8 * j + 1]), pack_bf16(v[8 * j + 2], v[8 * j + 3]),
                      pack_bf16(v[8 * j + 4], v[8 * j + 5]), pack_bf16(v[8 * j + 6], v[8 * j + 7]));
         st_shared_v4(buf1 + at, pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]), pack_bf16(o[4], o[5]),
@@ -126,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmD, const __grid_constant__ CUtensorMap tmD2,
                 const __grid_constant__ CUtensorMap tmR, const KArgs p) {
-  using C = Cfg<BN, PAIR, (EPI == EPI_BF16_RESID || EPI == EPI_DRELU2)>;
+  using C = Cfg<BN, PAIR, epi_reads_r(EPI)>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -172,7 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
     tma_prefetch_desc(&tmD);
-    if constexpr (EPI == EPI_BF16_RESID || EPI == EPI_DRELU2) tma_prefetch_desc(&tmR);
+    if constexpr (epi_reads_r(EPI)) tma_prefetch_desc(&tmR);
   }
   if (warp == 1) {
     if constexpr (PAIR) {
@@ -303,12 +310,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------ epilogue (warps 2..5)
     constexpr bool kF32 = (EPI == EPI_F32 || EPI == EPI_F32_ATOMIC);
-    constexpr bool kR = (EPI == EPI_BF16_RESID || EPI == EPI_DRELU2);
+    constexpr bool kR = epi_reads_r(EPI);
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const uint32_t wbuf = smem_u32(staging) + static_cast<uint32_t>(q) * 8192u;
     uint8_t* rbuf = rstage + q * C::R_BUFS * 2048;
     uint64_t* rb = rbar + q * C::R_BUFS;
-    const bool keep_pre = (EPI == EPI_RELU2) && p.D != nullptr;
+    const bool keep_pre = epi_act_fwd(EPI) && p.D != nullptr;
     int acc = 0;
     uint32_t acc_phase = 0;
     uint32_t chunk = 0;
@@ -377,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint8_t* s0 = staging + (buf0 - smem_u32(staging));
           if constexpr (EPI == EPI_F32_ATOMIC) {
             tma_reduce_add_2d(&tmD, s0, col0, row0);
-          } else if constexpr (EPI == EPI_RELU2) {
+          } else if constexpr (epi_act_fwd(EPI)) {
             if (keep_pre) tma_store_2d(&tmD, s0, col0, row0);
             tma_store_2d(&tmD2, staging + (buf1 - smem_u32(staging)), col0, row0);
           } else {
@@ -479,7 +486,7 @@ int make_out_map(CUtensorMap* m, const void* base, int64_t inner, int64_t outer,
 template <int BN, bool A_MN, bool B_MN, int EPI, bool PAIR>
 int launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& md,
              const CUtensorMap& md2, const CUtensorMap& mr, const KArgs& a, cudaStream_t s) {
-  using C = Cfg<BN, PAIR, (EPI == EPI_BF16_RESID || EPI == EPI_DRELU2)>;
+  using C = Cfg<BN, PAIR, epi_reads_r(EPI)>;
   auto kern = gemm_kernel<BN, A_MN, B_MN, EPI, PAIR>;
   static bool attr_done = false;  // per instantiation; set before first launch
   if (!attr_done) {
@@ -518,6 +525,8 @@ int dispatch_bn(const GemmDesc& g, const CUtensorMap& ma, const CUtensorMap& mb,
       case EPI_BF16_RESID:
         return launch_t<BN, false, false, EPI_BF16_RESID, PAIR>(ma, mb, md, md2, mr, a, s);
       case EPI_RELU2: return launch_t<BN, false, false, EPI_RELU2, PAIR>(ma, mb, md, md2, mr, a, s);
+      case EPI_LRELU2:
+        return launch_t<BN, false, false, EPI_LRELU2, PAIR>(ma, mb, md, md2, mr, a, s);
       default: return QAT_ERR_ARG;
     }
   }
@@ -527,12 +536,16 @@ int dispatch_bn(const GemmDesc& g, const CUtensorMap& ma, const CUtensorMap& mb,
       case EPI_BF16_RESID:
         return launch_t<BN, false, false, EPI_BF16_RESID, PAIR>(ma, mb, md, md2, mr, a, s);
       case EPI_RELU2: return launch_t<BN, false, false, EPI_RELU2, PAIR>(ma, mb, md, md2, mr, a, s);
+      case EPI_LRELU2:
+        return launch_t<BN, false, false, EPI_LRELU2, PAIR>(ma, mb, md, md2, mr, a, s);
       default: break;
     }
   } else if (!g.a_mn && g.b_mn) {
     switch (epi) {
       case EPI_BF16: return launch_t<BN, false, true, EPI_BF16, PAIR>(ma, mb, md, md2, mr, a, s);
       case EPI_DRELU2: return launch_t<BN, false, true, EPI_DRELU2, PAIR>(ma, mb, md, md2, mr, a, s);
+      case EPI_DLRELU2:
+        return launch_t<BN, false, true, EPI_DLRELU2, PAIR>(ma, mb, md, md2, mr, a, s);
       default: break;
     }
   } else if (g.a_mn && g.b_mn) {
@@ -567,9 +580,9 @@ int choose_splits(int tiles, int kblk, int sms) {
 int launch_gemm(const GemmDesc& g, cudaStream_t stream) {
   if (g.M < 0 || g.N <= 0 || g.K <= 0) return QAT_ERR_ARG;
   if (g.M == 0) return QAT_OK;
-  if (!g.A || !g.B || (!g.D && g.epi != EPI_RELU2)) return QAT_ERR_ARG;
-  if (g.epi == EPI_RELU2 && !g.D2) return QAT_ERR_ARG;
-  if ((g.epi == EPI_BF16_RESID || g.epi == EPI_DRELU2) && !g.R) return QAT_ERR_ARG;
+  if (!g.A || !g.B || (!g.D && !epi_act_fwd(g.epi))) return QAT_ERR_ARG;
+  if (epi_act_fwd(g.epi) && !g.D2) return QAT_ERR_ARG;
+  if (epi_reads_r(g.epi) && !g.R) return QAT_ERR_ARG;
   if (!aligned16(g.A) || !aligned16(g.B) || (g.D && !aligned16(g.D)) || (g.D2 && !aligned16(g.D2)) ||
       (g.R && !aligned16(g.R)))
     return QAT_ERR_ALIGN;
@@ -656,7 +669,7 @@ int launch_gemm(const GemmDesc& g, cudaStream_t stream) {
   rc = make_out_map(&md2, g.D2 ? g.D2 : d_base, g.N, g.M, g.D2 ? g.ldd2 : d_ld, false);
   if (rc) return rc;
   CUtensorMap mr = md;
-  if (g.epi == EPI_BF16_RESID || g.epi == EPI_DRELU2) {
+  if (epi_reads_r(g.epi)) {
     rc = make_out_map(&mr, g.R, g.N, g.M, g.ldr, false);
     if (rc) return rc;
   }

@@ -13,7 +13,15 @@ enum Epi : int {
   EPI_DRELU2 = 3,      // D = bf16(acc * 2*relu(R))     (R = saved pre-activation)
   EPI_F32 = 4,         // D = acc (+ D if accumulate), single writer per element
   EPI_F32_ATOMIC = 5,  // D += acc with atomics (split-K partial sums)
+  EPI_LRELU2 = 6,      // D = bf16(acc) (optional), D2 = bf16(leaky_relu(acc, 0.5)^2)
+  EPI_DLRELU2 = 7,     // D = bf16(acc * g(R)), g = 2R for R > 0 else R/2 (its derivative)
 };
+
+// Epilogues that read a bf16 tile R, and those that write the activation pair.
+constexpr bool epi_reads_r(int e) {
+  return e == EPI_BF16_RESID || e == EPI_DRELU2 || e == EPI_DLRELU2;
+}
+constexpr bool epi_act_fwd(int e) { return e == EPI_RELU2 || e == EPI_LRELU2; }
 
 // D[M,N] = A[M,K] . B[N,K]^T with bf16 operands and fp32 accumulation.
 // A is K-major (row m contiguous along K, row stride lda) unless a_mn, in which

@@ -55,7 +55,7 @@ extern "C" int qat_linear_fwd_noalloc(const float* W, int32_t N, int32_t K, int3
                                       const qat_bf16* X, int64_t ldx, int64_t T,
                                       const qat_bf16* residual, qat_bf16* Y, qat_stream_t stream) {
   using namespace qat;
-  if (!W || (T > 0 && (!X || !Y)) || T < 0 || (bits != 6 && bits != 8)) return QAT_ERR_ARG;
+  if (!W || (T > 0 && (!X || !Y)) || T < 0 || (bits != 5 && bits != 6 && bits != 8)) return QAT_ERR_ARG;
   if (N <= 0 || K <= 0 || (N & 7) || (K & 7)) return QAT_ERR_SHAPE;
   if (static_cast<int64_t>(N) * K > QAT_NOALLOC_MAX_ELEMS || N > QAT_NOALLOC_MAX_ROWS)
     return QAT_ERR_SHAPE;

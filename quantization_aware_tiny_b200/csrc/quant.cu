@@ -67,7 +67,7 @@ __global__ void __launch_bounds__(kQThreads)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     amax = fmaxf(amax, 1e-12f);
-    const float s = div_rn(amax, 127.0f);
+    const float s = div_rn(amax, grid_levels(bits));
     const float rs = __frcp_rn(s);
     if (lane == 0) scales[row] = s;
     auto emit = [&](int j, float4 v) {
@@ -111,13 +111,14 @@ __device__ __forceinline__ float noisy_value(float w, uint32_t x, float s) {
 }
 
 // Noisy-QAT forward operand ("Depth Recurrence + Mixed-Precision Quant",
-// "幸存发现 1 Noisy QAT"): per row s = max(amax, 1e-12) / 127, every weight
-// gets (u - 1/2) * s of uniform noise, the result is cast to bf16.  Element e
+// "幸存发现 1 Noisy QAT"): per row s = max(amax, 1e-12) / 127 (the int8 step;
+// amax / 15, the int5 step, for bits = 5), every weight gets (u - 1/2) * s of
+// uniform noise, the result is cast to bf16.  Element e
 // of the row-major weight takes word e % 4 of the Philox block with counter
 // (e / 4, offset) and key seed.  One warp per row, the row cached in registers
 // between the amax and the noise passes.
 __global__ void __launch_bounds__(kQThreads)
-    noisy_operand_kernel(const float* __restrict__ W, int N, int K, uint64_t seed,
+    noisy_operand_kernel(const float* __restrict__ W, int N, int K, int bits, uint64_t seed,
                          uint64_t offset, float* __restrict__ scales,
                          __nv_bfloat16* __restrict__ operand) {
   const int lane = threadIdx.x & 31;
@@ -141,7 +142,7 @@ __global__ void __launch_bounds__(kQThreads)
     for (int j = lane + 32 * kRegV4; j < K4; j += 32) amax = fmaxf(amax, amax4(__ldg(r + j)));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    const float s = div_rn(fmaxf(amax, 1e-12f), 127.0f);
+    const float s = div_rn(fmaxf(amax, 1e-12f), grid_levels(bits));
     if (lane == 0 && scales) scales[row] = s;
     auto emit = [&](int j, float4 v) {
       const uint64_t g = static_cast<uint64_t>(row) * static_cast<uint64_t>(K4) + j;  // e / 4
@@ -191,8 +192,9 @@ __device__ __forceinline__ void top2_warp(float& t1, float& t2) {
   t2 = __popc(holders) >= 2 ? t1 : __uint_as_float(second);
 }
 
-// fl32(1 / 127), correctly rounded (0x3C010204).
+// fl32(1 / 127) and fl32(1 / 15), correctly rounded (0x3C010204, 0x3D888889).
 constexpr float kRcp127 = 0.00787401571869850158691406f;
+constexpr float kRcp15 = 0.066666670143604278564453125f;
 
 struct RowQuant {
   float clip, s, rs;
@@ -205,7 +207,8 @@ __device__ __forceinline__ RowQuant row_params(const ExportDescDev& d, float t1,
   const float v_lo = (d.m == 2) ? t2 : t1;
   RowQuant q;
   q.clip = __fadd_rn(v_lo, __fmul_rn(d.frac, __fsub_rn(v_hi, v_lo)));
-  q.s = div_by_scale(fmaxf(q.clip, 1e-12f), 127.0f, kRcp127);
+  q.s = d.mode == 5 ? div_by_scale(fmaxf(q.clip, 1e-12f), 15.0f, kRcp15)
+                    : div_by_scale(fmaxf(q.clip, 1e-12f), 127.0f, kRcp127);
   q.rs = __frcp_rn(q.s);
   q.bits = d.mode;
   return q;
@@ -240,9 +243,10 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
 // CLIP = false skips clamping w to [-clip, clip].  That is exact when
 // clip >= v_hi / 2 (always so for rows up to 32,768 columns, where the
 // interpolation fraction exceeds 0.947): only entries with |w| > clip differ,
-// their quotient |w / s| then lies in (127, 254], and after the grid's clamp
-// their code equals the code of +-clip itself (+124 / -128 for int6,
-// +-127 for int8); the offset trick stays exact for |x| < 2^22.
+// their quotient |w / s| then lies in (L, 2L] (L = 127, or 15 for int5), and
+// after the grid's clamp their code equals the code of +-clip itself (+124 /
+// -128 for int6, +-127 for int8, +-15 for int5); the offset trick stays exact
+// for |x| < 2^22.
 template <int BITS, bool CLIP>
 __device__ __forceinline__ void codes2(const RowQuant& q, float a, float b, int& ca, int& cb) {
   constexpr float kOff = 12582912.0f;  // 1.5 * 2^23
@@ -261,8 +265,24 @@ __device__ __forceinline__ void codes2(const RowQuant& q, float a, float b, int&
     ca = min(max(static_cast<int>(__float_as_uint(u.x) * 4u - 0x2D000000u), -128), 124);
     cb = min(max(static_cast<int>(__float_as_uint(u.y) * 4u - 0x2D000000u), -128), 124);
   } else {
-    ca = min(max(__float_as_int(t.x) - 0x4B400000, -127), 127);
-    cb = min(max(__float_as_int(t.y) - 0x4B400000, -127), 127);
+    constexpr int L = BITS == 5 ? 15 : 127;
+    ca = min(max(__float_as_int(t.x) - 0x4B400000, -L), L);
+    cb = min(max(__float_as_int(t.y) - 0x4B400000, -L), L);
+  }
+}
+
+// Calls f(integral_constant<int, bits>, bool_constant<clip>) for a row's grid.
+template <typename F>
+__device__ __forceinline__ void with_grid(int bits, bool clip, F&& f) {
+  using T5 = std::integral_constant<int, 5>;
+  using T6 = std::integral_constant<int, 6>;
+  using T8 = std::integral_constant<int, 8>;
+  if (bits == 6) {
+    if (clip) f(T6{}, std::true_type{}); else f(T6{}, std::false_type{});
+  } else if (bits == 5) {
+    if (clip) f(T5{}, std::true_type{}); else f(T5{}, std::false_type{});
+  } else {
+    if (clip) f(T8{}, std::true_type{}); else f(T8{}, std::false_type{});
   }
 }
 
@@ -282,7 +302,8 @@ __device__ __forceinline__ uint32_t codes4_t(const RowQuant& q, float4 v) {
 }
 
 __device__ __forceinline__ uint32_t codes4(const RowQuant& q, float4 v) {
-  return q.bits == 6 ? codes4_t<6, true>(q, v) : codes4_t<8, true>(q, v);
+  if (q.bits == 6) return codes4_t<6, true>(q, v);
+  return q.bits == 5 ? codes4_t<5, true>(q, v) : codes4_t<8, true>(q, v);
 }
 
 // float4 groups per lane and loop iteration in the shared-memory passes: more
@@ -332,13 +353,9 @@ __device__ __forceinline__ void export_row_smem(const ExportDescDev& d, int64_t 
   if (lane == 0) d.scales[row] = __float2half_rn(q.s);
   uint32_t* out = reinterpret_cast<uint32_t*>(reinterpret_cast<int8_t*>(d.dst) + row * d.cols);
   const bool clip = a1 > 2.0f * q.clip;  // see codes2: clamping needed only then
-  if (q.bits == 6) {
-    if (clip) quantize_smem_row<6, true>(q, buf, K4, out, lane);
-    else quantize_smem_row<6, false>(q, buf, K4, out, lane);
-  } else {
-    if (clip) quantize_smem_row<8, true>(q, buf, K4, out, lane);
-    else quantize_smem_row<8, false>(q, buf, K4, out, lane);
-  }
+  with_grid(q.bits, clip, [&](auto bits_tag, auto clip_tag) {
+    quantize_smem_row<decltype(bits_tag)::value, decltype(clip_tag)::value>(q, buf, K4, out, lane);
+  });
 }
 
 // Two rows of the same tensor staged in shared memory, processed together so
@@ -397,15 +414,7 @@ __device__ __forceinline__ void export_two_rows_smem(const ExportDescDev& d, int
       outB[k] = codes4_t<BITS, CLIP>(qb, bufB[k]);
     }
   };
-  using T6 = std::integral_constant<int, 6>;
-  using T8 = std::integral_constant<int, 8>;
-  using TT = std::true_type;
-  using TF = std::false_type;
-  if (qa.bits == 6) {
-    if (clip) run(T6{}, TT{}); else run(T6{}, TF{});
-  } else {
-    if (clip) run(T8{}, TT{}); else run(T8{}, TF{});
-  }
+  with_grid(qa.bits, clip, run);
 }
 
 // A quantized row read from global memory (rows longer than the staging buffer).
@@ -635,10 +644,10 @@ int launch_quantize_weights(const float* W, int N, int K, int bits, int8_t* code
   return cuda_status(cudaGetLastError());
 }
 
-int launch_noisy_operand(const float* W, int N, int K, uint64_t seed, uint64_t offset,
+int launch_noisy_operand(const float* W, int N, int K, int bits, uint64_t seed, uint64_t offset,
                          float* scales, __nv_bfloat16* operand, cudaStream_t s) {
   noisy_operand_kernel<<<grid_for_rows(N, kQThreads / 32), kQThreads, 0, s>>>(
-      W, N, K, seed, offset, scales, operand);
+      W, N, K, bits, seed, offset, scales, operand);
   count_launch();
   return cuda_status(cudaGetLastError());
 }

@@ -49,7 +49,7 @@ constexpr int kExportMaxWarps = 16;
 
 int launch_quantize_weights(const float* W, int N, int K, int bits, int8_t* codes, float* scales,
                             __nv_bfloat16* operand, cudaStream_t s);
-int launch_noisy_operand(const float* W, int N, int K, uint64_t seed, uint64_t offset,
+int launch_noisy_operand(const float* W, int N, int K, int bits, uint64_t seed, uint64_t offset,
                          float* scales, __nv_bfloat16* operand, cudaStream_t s);
 int export_quantile_params(int64_t cols, int* m, float* frac);
 int launch_export_batch(ExportBatch& b, cudaStream_t s);

@@ -9,6 +9,10 @@ zstd-22 记录详解", section "后训练量化导出":
   - other 2-D tensors get per-row codes and fp16 scales: int6 when they
     belong to a block i with INT6_LAYER_START <= i <= INT6_LAYER_END (both
     inclusive, -1 = int6 off), else int8.
+From "Depth Recurrence + Mixed-Precision Quant", reproduction commands
+(MLP_INT5 / ATTN_INT5): with mlp_int5 every block MLP weight
+("blocks.<i>.mlp."), with attn_int5 every block attention weight
+("blocks.<i>.attn."), is exported on the int5 grid instead.
 The per-row arithmetic all runs in the library's export kernel.
 """
 import re
@@ -21,31 +25,37 @@ KEEP_FLOAT_MAX_NUMEL = 65536
 _BLOCK = re.compile(r"^blocks\.(\d+)\.")
 
 
-def export_mode(name, shape, numel, int6_range=(0, 10), embed_name="tok_emb.weight"):
-    """Export mode of one tensor: 6, 8 or qat.QAT_EXPORT_FP16."""
+def export_mode(name, shape, numel, int6_range=(0, 10), embed_name="tok_emb.weight",
+                mlp_int5=False, attn_int5=False):
+    """Export mode of one tensor: 5, 6, 8 or qat.QAT_EXPORT_FP16."""
     if len(shape) != 2 or numel <= KEEP_FLOAT_MAX_NUMEL or name == embed_name:
         return qat.QAT_EXPORT_FP16
-    start, end = int6_range
     m = _BLOCK.match(name)
+    if m and ((mlp_int5 and ".mlp." in name) or (attn_int5 and ".attn." in name)):
+        return 5
+    start, end = int6_range
     if m and start >= 0 and end >= 0 and start <= int(m.group(1)) <= end:
         return 6
     return 8
 
 
-def plan(state_dict, int6_range=(0, 10), embed_name="tok_emb.weight"):
+def plan(state_dict, int6_range=(0, 10), embed_name="tok_emb.weight", mlp_int5=False,
+         attn_int5=False):
     """(name, mode) for every tensor, in order."""
-    return [(n, export_mode(n, tuple(t.shape), t.numel(), int6_range, embed_name))
+    return [(n, export_mode(n, tuple(t.shape), t.numel(), int6_range, embed_name, mlp_int5,
+                            attn_int5))
             for n, t in state_dict.items()]
 
 
-def export_state_dict(state_dict, int6_range=(0, 10), embed_name="tok_emb.weight", stream=None):
+def export_state_dict(state_dict, int6_range=(0, 10), embed_name="tok_emb.weight", stream=None,
+                      mlp_int5=False, attn_int5=False):
     """Quantize a dict of fp32 CUDA tensors.  Returns name -> dict with
-    kind 'int6'/'int8' (codes int8 [rows,cols], scale16 fp16 [rows]) or
+    kind 'int5'/'int6'/'int8' (codes int8 [rows,cols], scale16 fp16 [rows]) or
     kind 'fp16' (values fp16, original shape).  Launches in chunks of at most
     QAT_EXPORT_MAX_DESCS descriptors (one launch for a state dict that fits)."""
     out = {}
     descs = []
-    for name, mode in plan(state_dict, int6_range, embed_name):
+    for name, mode in plan(state_dict, int6_range, embed_name, mlp_int5, attn_int5):
         t = state_dict[name]
         if t.dtype != torch.float32 or not t.is_contiguous():
             raise ValueError("%s: expected a contiguous fp32 tensor" % name)

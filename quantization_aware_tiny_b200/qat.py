@@ -27,6 +27,9 @@ EXPORTED = ("qat_strerror", "qat_launch_count", "qat_device_error", "qat_quantiz
             "qat_workspace_size", "qat_linear_fwd", "qat_linear_bwd", "qat_mlp_fwd",
             "qat_mlp_bwd", "quantize_rows_export", "quantize_export_batch", "dequantize_rows",
             "qat_linear_fwd_noalloc", "qat_noisy_operand")
+QAT_ACT_RELU2 = 0
+QAT_ACT_LEAKY_RELU2 = 1
+_ACTS = {"relu2": QAT_ACT_RELU2, "leaky2": QAT_ACT_LEAKY_RELU2}
 QAT_NOALLOC_MAX_ELEMS = 4194304
 QAT_NOALLOC_MAX_ROWS = 16384
 
@@ -71,14 +74,15 @@ def lib():
         L.qat_workspace_size.restype = SZ
         L.qat_linear_fwd.argtypes = [P, P, I32, I32, I32, P, I64, I64, P, P, P, SZ, P]
         L.qat_linear_bwd.argtypes = [P, P, I32, I32, I32, P, P, I64, P, P, I32, P, SZ, P]
-        L.qat_mlp_fwd.argtypes = [P, P, P, P, I32, I32, I32, P, I64, P, P, P, P, P, SZ, P]
-        L.qat_mlp_bwd.argtypes = [P, P, P, P, I32, I32, I32, P, P, P, P, I64, P, P, P, I32, P,
+        L.qat_mlp_fwd.argtypes = [P, P, P, P, I32, I32, I32, I32, P, I64, P, P, P, P, P, SZ, P]
+        L.qat_mlp_bwd.argtypes = [P, P, P, P, I32, I32, I32, I32, P, P, P, P, I64, P, P, P, I32, P,
                                   SZ, P]
         L.quantize_rows_export.argtypes = [P, I64, I64, I32, P, P, P]
         L.quantize_export_batch.argtypes = [P, I32, P]
         L.dequantize_rows.argtypes = [P, P, I64, I64, I32, P, P]
         L.qat_linear_fwd_noalloc.argtypes = [P, I32, I32, I32, P, I64, I64, P, P, P]
-        L.qat_noisy_operand.argtypes = [P, I32, I32, ctypes.c_uint64, ctypes.c_uint64, P, P, P]
+        L.qat_noisy_operand.argtypes = [P, I32, I32, I32, ctypes.c_uint64, ctypes.c_uint64, P, P,
+                                        P]
         for name in EXPORTED:
             if name not in ("qat_strerror", "qat_launch_count", "qat_workspace_size"):
                 getattr(L, name).restype = ctypes.c_int
@@ -160,19 +164,20 @@ def quantize_weight(W, bits, keep_codes=False, stream=None):
     return QWeight(operand, scales, codes, bits)
 
 
-def qat_noisy_operand(W, seed, offset, operand, scales=None, stream=None):
-    """Noisy-QAT forward operand bf16(w + (u - 1/2) * amax/127) of W [N,K]."""
+def qat_noisy_operand(W, seed, offset, operand, scales=None, stream=None, bits=8):
+    """Noisy-QAT forward operand bf16(w + (u - 1/2) * amax/L) of W [N,K]; L = 127
+    (the int8 step) for bits 6 / 8, 15 (the int5 step) for bits 5."""
     N, K = W.shape
-    _check(lib().qat_noisy_operand(_p(W), N, K, int(seed), int(offset), _p(scales), _p(operand),
-                                   _stream(stream)), "qat_noisy_operand")
+    _check(lib().qat_noisy_operand(_p(W), N, K, int(bits), int(seed), int(offset), _p(scales),
+                                   _p(operand), _stream(stream)), "qat_noisy_operand")
 
 
-def noisy_weight(W, seed, offset, stream=None):
+def noisy_weight(W, seed, offset, stream=None, bits=8):
     """A new QWeight holding the Noisy-QAT operand of W (bits recorded as 0)."""
     N, K = W.shape
     scales = torch.empty(N, dtype=torch.float32, device=W.device)
     operand = torch.empty((N, K), dtype=torch.bfloat16, device=W.device)
-    qat_noisy_operand(W, seed, offset, operand, scales, stream)
+    qat_noisy_operand(W, seed, offset, operand, scales, stream, bits=bits)
     return QWeight(operand, scales, None, 0)
 
 
@@ -198,17 +203,21 @@ def qat_linear_bwd(X, dY, bits, W=None, qw=None, dX=None, dW=None, accumulate_dW
 
 
 def qat_mlp_fwd(X, Y, bits, d, H, Wfc=None, Wproj=None, qfc=None, qproj=None, residual=None,
-                pre_save=None, h_save=None, workspace=None, stream=None):
+                pre_save=None, h_save=None, workspace=None, stream=None, act="relu2"):
+    """act = "relu2" (relu(x)^2) or "leaky2" (leaky_relu(x, 0.5)^2)."""
     ws, wsb = _ws(workspace)
-    _check(lib().qat_mlp_fwd(_p(Wfc), _p(Wproj), _qref(qfc), _qref(qproj), d, H, bits, _p(X),
+    _check(lib().qat_mlp_fwd(_p(Wfc), _p(Wproj), _qref(qfc), _qref(qproj), d, H, bits,
+                             _ACTS[act], _p(X),
                              X.shape[0], _p(residual), _p(Y), _p(pre_save), _p(h_save), ws, wsb,
                              _stream(stream)), "qat_mlp_fwd")
 
 
 def qat_mlp_bwd(X, pre, h, dY, bits, d, H, Wfc=None, Wproj=None, qfc=None, qproj=None, dX=None,
-                dWfc=None, dWproj=None, accumulate_dW=False, workspace=None, stream=None):
+                dWfc=None, dWproj=None, accumulate_dW=False, workspace=None, stream=None,
+                act="relu2"):
     ws, wsb = _ws(workspace)
-    _check(lib().qat_mlp_bwd(_p(Wfc), _p(Wproj), _qref(qfc), _qref(qproj), d, H, bits, _p(X),
+    _check(lib().qat_mlp_bwd(_p(Wfc), _p(Wproj), _qref(qfc), _qref(qproj), d, H, bits,
+                             _ACTS[act], _p(X),
                              _p(pre), _p(h), _p(dY), X.shape[0], _p(dX), _p(dWfc), _p(dWproj),
                              int(bool(accumulate_dW)), ws, wsb, _stream(stream)), "qat_mlp_bwd")
 

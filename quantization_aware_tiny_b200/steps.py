@@ -17,13 +17,16 @@ class RecurrentCore:
         qkv = x Wqkv^T              (Q|K|V fused: per-row quantization is per
                                      output row, so concatenation is exact)
         x1  = x + q Wo^T            (residual fused in the GEMM epilogue)
-        x   = x1 + proj(relu(fc(x1))^2)
+        x   = x1 + proj(act(fc(x1)))
+    act = relu^2, or leaky_relu(., 0.5)^2 with act="leaky2"; bits = 5 selects
+    the int5 grid (the write-up's MLP_INT5 / ATTN_INT5 configuration).
     """
 
-    def __init__(self, Wq, Wk, Wv, Wo, Wfc, Wproj, bits=6, stream=None):
+    def __init__(self, Wq, Wk, Wv, Wo, Wfc, Wproj, bits=6, stream=None, act="relu2"):
         self.d = Wq.shape[1]
         self.H = Wfc.shape[0]
         self.bits = bits
+        self.act = act
         Wqkv = torch.cat([Wq, Wk, Wv], dim=0).contiguous()
         self.W = (Wqkv, Wo.contiguous(), Wfc.contiguous(), Wproj.contiguous())
         self.q_qkv, self.q_o, self.q_fc, self.q_proj = (
@@ -44,7 +47,8 @@ class RecurrentCore:
 
         noise = (seed, offset) switches to Noisy QAT ("Depth Recurrence +
         Mixed-Precision Quant", "幸存发现 1"): every application draws fresh
-        uniform noise at the int8 step for each of the four weights, with
+        uniform noise at the int8 step (the int5 step when bits = 5) for each
+        of the four weights, with
         Philox offsets offset + 4*r + k (r = application, k = qkv, o, fc,
         proj), instead of reusing the once-quantized operands."""
         T = x.shape[0]
@@ -56,13 +60,14 @@ class RecurrentCore:
             if noise is not None:
                 seed, offset = noise
                 for k, (w, q) in enumerate(zip(self.W, ops)):
-                    qat.qat_noisy_operand(w, seed, offset + 4 * r + k, q.operand, stream=stream)
+                    qat.qat_noisy_operand(w, seed, offset + 4 * r + k, q.operand, stream=stream,
+                                          bits=self.bits)
             q_qkv, q_o, q_fc, q_proj = ops
             bits = self.bits
             qat.qat_linear_fwd(x, qkv, bits, qw=q_qkv, stream=stream)
             qat.qat_linear_fwd(qkv, x1, bits, qw=q_o, ldx=self.nqkv, T=T, residual=x, stream=stream)
             qat.qat_mlp_fwd(x1, x, bits, self.d, self.H, qfc=q_fc, qproj=q_proj, residual=x1,
-                            h_save=h, stream=stream)
+                            h_save=h, stream=stream, act=self.act)
         return x
 
     def flops(self, T, R):
@@ -76,13 +81,14 @@ class HeadMlpStep:
         dZ = dLogits Wemb_q; dWemb = dLogits^T Z; MLP backward -> dX, dWfc, dWproj
     """
 
-    def __init__(self, Wemb, Wfc, Wproj, T, head_bits=8, mlp_bits=6):
+    def __init__(self, Wemb, Wfc, Wproj, T, head_bits=8, mlp_bits=6, act="relu2"):
         dev = Wemb.device
         self.W = (Wemb, Wfc, Wproj)
         self.vocab, self.d = Wemb.shape
         self.H = Wfc.shape[0]
         self.T = T
         self.head_bits, self.mlp_bits = head_bits, mlp_bits
+        self.act = act
         bf = torch.bfloat16
         e = lambda *s, dt=bf: torch.empty(s, dtype=dt, device=dev)
         self.q = [qat.QWeight(e(*w.shape), e(w.shape[0], dt=torch.float32), None, b)
@@ -102,7 +108,7 @@ class HeadMlpStep:
     def forward(self, X, stream=None):
         qe, qf, qp = self.q
         qat.qat_mlp_fwd(X, self.Z, self.mlp_bits, self.d, self.H, qfc=qf, qproj=qp,
-                        pre_save=self.pre, h_save=self.h, stream=stream)
+                        pre_save=self.pre, h_save=self.h, stream=stream, act=self.act)
         qat.qat_linear_fwd(self.Z, self.logits, self.head_bits, qw=qe, stream=stream)
 
     def backward(self, X, dLogits, stream=None):
@@ -111,7 +117,7 @@ class HeadMlpStep:
                            stream=stream)
         qat.qat_mlp_bwd(X, self.pre, self.h, self.dZ, self.mlp_bits, self.d, self.H, qfc=qf,
                         qproj=qp, dX=self.dX, dWfc=self.dWfc, dWproj=self.dWproj,
-                        workspace=self.ws, stream=stream)
+                        workspace=self.ws, stream=stream, act=self.act)
 
     def step(self, X, dLogits, stream=None):
         self.quantize(stream)

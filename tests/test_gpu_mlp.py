@@ -1,5 +1,6 @@
 """GPU parity of the ReLU^2 MLP (fused relu^2 fc epilogue, fused 2*relu(pre)
-backward epilogue) against the fp64 oracle."""
+backward epilogue) and of its LeakyReLU(0.5)^2 variant, on the int5 / int6 /
+int8 grids, against the fp64 oracle."""
 import numpy as np
 import pytest
 import torch
@@ -12,7 +13,7 @@ from parity import assert_close
 pytestmark = pytest.mark.gpu
 
 
-def _run(c, d, H, bits=6, raw=False):
+def _run(c, d, H, bits=6, raw=False, act="relu2"):
     X, dY = c["X"].cuda(), c["dY"].cuda()
     T = X.shape[0]
     Wfc, Wproj = torch.from_numpy(c["Wfc"]).cuda(), torch.from_numpy(c["Wproj"]).cuda()
@@ -29,17 +30,18 @@ def _run(c, d, H, bits=6, raw=False):
         kw = {"qfc": qat.quantize_weight(Wfc, bits), "qproj": qat.quantize_weight(Wproj, bits)}
         wsf = None
         wsb = torch.empty(qat.workspace_size(qat.QAT_OP_MLP_BWD, d, H, T, False), dtype=torch.uint8, device="cuda")
-    qat.qat_mlp_fwd(X, Y, bits, d, H, pre_save=pre, h_save=h, workspace=wsf, **kw)
-    qat.qat_mlp_bwd(X, pre, h, dY, bits, d, H, dX=dX, dWfc=dWfc, dWproj=dWproj, workspace=wsb, **kw)
+    qat.qat_mlp_fwd(X, Y, bits, d, H, pre_save=pre, h_save=h, workspace=wsf, act=act, **kw)
+    qat.qat_mlp_bwd(X, pre, h, dY, bits, d, H, dX=dX, dWfc=dWfc, dWproj=dWproj, workspace=wsb,
+                    act=act, **kw)
     torch.cuda.synchronize()
     return Y, pre, h, dX, dWfc, dWproj
 
 
-def _check(c, out, bits=6):
+def _check(c, out, bits=6, act="relu2"):
     qf, qp = o.quantize_weight(c["Wfc"], bits), o.quantize_weight(c["Wproj"], bits)
     X, dY = c["X"].float().numpy(), c["dY"].float().numpy()
-    pre, h, Y = o.mlp_fwd(qf["operand"], qp["operand"], X)
-    dX, dWfc, dWproj = o.mlp_bwd(qf["operand"], qp["operand"], X, pre, h, dY)
+    pre, h, Y = o.mlp_fwd(qf["operand"], qp["operand"], X, act)
+    dX, dWfc, dWproj = o.mlp_bwd(qf["operand"], qp["operand"], X, pre, h, dY, act)
     for name, g, r in zip(("Y", "pre", "h", "dX", "dWfc", "dWproj"), out, (Y, pre, h, dX, dWfc, dWproj)):
         assert_close(g, r, name)
 
@@ -59,4 +61,22 @@ def test_mlp_cfg2_full_size():
     """The 11-layer record's MLP block at 8x1024 tokens, every element."""
     c = sy.mlp_case(T=8192)
     _check(c, _run(c, 512, 1536))
+    assert qat.device_error() == 0
+
+
+@pytest.mark.parametrize("bits", [5, 8])
+@pytest.mark.parametrize("act", ["relu2", "leaky2"])
+def test_mlp_bits_and_activation(bits, act):
+    """int5 / int8 grids and LeakyReLU(0.5)^2, raw fp32 weights and cached
+    operands, ragged token count spanning several tiles."""
+    c = sy.mlp_case(T=1000, seed=7)
+    _check(c, _run(c, 512, 1536, bits=bits, act=act), bits=bits, act=act)
+    _check(c, _run(c, 512, 1536, bits=bits, raw=True, act=act), bits=bits, act=act)
+
+
+def test_mlp_leaky2_full_size():
+    """LeakyReLU(0.5)^2 MLP at 8x1024 tokens (int5, the all-int5 configuration),
+    every element."""
+    c = sy.mlp_case(T=8192, seed=8)
+    _check(c, _run(c, 512, 1536, bits=5, act="leaky2"), bits=5, act="leaky2")
     assert qat.device_error() == 0

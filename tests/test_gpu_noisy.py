@@ -17,13 +17,15 @@ SEEDS = [(0, 0), (1234, 7), ((0xDEADBEEF << 32) | 0x1234567, (0xFFFFFFFF << 32) 
 
 
 @pytest.mark.parametrize("seed,offset", SEEDS)
-def test_noisy_operand_bit_exact(seed, offset):
+@pytest.mark.parametrize("bits", [8, 5])
+def test_noisy_operand_bit_exact(seed, offset, bits):
+    """Noise at the int8 step (bits 8) and at the int5 step (bits 5)."""
     rng = np.random.default_rng(31)
     for shape in ((512, 512), (200, 136), (64, 4104), (1280, 640)):
         W = (rng.standard_normal(shape) * 0.02).astype(np.float32)
-        q = qat.noisy_weight(torch.from_numpy(W).cuda(), seed, offset)
+        q = qat.noisy_weight(torch.from_numpy(W).cuda(), seed, offset, bits=bits)
         torch.cuda.synchronize()
-        ref = o.noisy_weight(W, seed, offset)
+        ref = o.noisy_weight(W, seed, offset, bits)
         assert np.array_equal(bits16(q.operand), ref["operand_bits"]), shape
         assert np.array_equal(q.scales.cpu().numpy(), ref["scales"]), shape
     assert qat.device_error() == 0
@@ -58,4 +60,21 @@ def test_noisy_recurrent_core():
     Ws = [np.concatenate([c["Wq"], c["Wk"], c["Wv"]]), c["Wo"], c["Wfc"], c["Wproj"]]
     ref = o.recurrent_core_fwd_noisy(Ws, c["X"].float().numpy(), 3, 640, 2024, 100)
     assert_close_chain(x, ref, 6, "noisy core, 3 applications")
+    assert qat.device_error() == 0
+
+
+def test_noisy_recurrent_core_int5_leaky2():
+    """An all-int5 core (noise at the int5 step, as the write-up proposes for an
+    int5 export) with the LeakyReLU(0.5)^2 MLP."""
+    c = sy.recurrent_core_case(T=300, seed=3)
+    dev = {k: torch.from_numpy(c[k]).cuda() for k in ("Wq", "Wk", "Wv", "Wo", "Wfc", "Wproj")}
+    core = steps.RecurrentCore(dev["Wq"], dev["Wk"], dev["Wv"], dev["Wo"], dev["Wfc"], dev["Wproj"],
+                               bits=5, act="leaky2")
+    x = c["X"].cuda()
+    core.forward(x, 2, noise=(77, 4))
+    torch.cuda.synchronize()
+    Ws = [np.concatenate([c["Wq"], c["Wk"], c["Wv"]]), c["Wo"], c["Wfc"], c["Wproj"]]
+    ref = o.recurrent_core_fwd_noisy(Ws, c["X"].float().numpy(), 2, 640, 77, 4, bits=5,
+                                     act="leaky2")
+    assert_close_chain(x, ref, 6, "noisy int5 leaky core, 2 applications")
     assert qat.device_error() == 0

@@ -1,4 +1,5 @@
-"""GPU parity of the quantizer kernels against the CPU oracle: bit-exact codes,
+"""GPU parity of the quantizer kernels (int5, int6, int8 grids) against the CPU
+oracle: bit-exact codes,
 fp32 scales, bf16 operands, fp16 export scales, fp16 passthrough and the
 dequantized weights."""
 import numpy as np
@@ -37,7 +38,7 @@ def _weights():
     return cases
 
 
-@pytest.mark.parametrize("bits", [6, 8])
+@pytest.mark.parametrize("bits", [5, 6, 8])
 def test_quantize_weights_bit_exact(bits):
     for name, W in _weights().items():
         q = qat.quantize_weight(_dev(W), bits, keep_codes=True)
@@ -49,7 +50,7 @@ def test_quantize_weights_bit_exact(bits):
     assert qat.device_error() == 0
 
 
-@pytest.mark.parametrize("bits", [6, 8])
+@pytest.mark.parametrize("bits", [5, 6, 8])
 def test_export_rows_bit_exact(bits):
     rng = np.random.default_rng(9)
     ties = np.tile(np.float32([0.01, -0.03, 0.03, 0.002]), (16, 16))  # top two tie
@@ -84,6 +85,25 @@ def test_export_state_dict_one_launch_bit_exact():
             assert np.array_equal(bits16(g["scale16"]), r["scale16"]), k
 
 
+@pytest.mark.parametrize("flags", [{"mlp_int5": True}, {"mlp_int5": True, "attn_int5": True}])
+def test_export_state_dict_mixed_int5_bit_exact(flags):
+    """Mixed int5 / int6 export (MLP_INT5, ATTN_INT5) of a 3-layer state dict in
+    one launch, against the oracle."""
+    sd = sy.state_dict_case(n_layers=3, seed=2)
+    out = qexport.export_state_dict({k: _dev(v) for k, v in sd.items()}, **flags)
+    torch.cuda.synchronize()
+    ref = o.export_state_dict(sd, **flags)
+    assert "int5" in {r["kind"] for r in ref.values()}
+    for k, r in ref.items():
+        g = out[k]
+        assert g["kind"] == r["kind"], k
+        if r["kind"] == "fp16":
+            assert np.array_equal(bits16(g["values"]).reshape(-1), r["bits16"].reshape(-1)), k
+        else:
+            assert np.array_equal(g["codes"].cpu().numpy(), r["codes"]), k
+            assert np.array_equal(bits16(g["scale16"]), r["scale16"]), k
+
+
 def test_dequantize_rows_bit_exact():
     sd = sy.state_dict_case(n_layers=1)
     for name in ("blocks.0.mlp.fc.weight", "blocks.0.attn.c_k.weight"):
@@ -100,17 +120,17 @@ def test_dequantize_rows_bit_exact():
         assert np.array_equal(bits16(out16), o.bf16_bits(ref)), name
 
 
-def _near_tie_rows(n_rows=256, cols=512, seed=21):
+def _near_tie_rows(n_rows=256, cols=512, seed=21, levels=127):
     """Rows whose entries sit within a few ulps of (k + 1/2) * s: the code then
     depends on the correctly rounded quotient w / s (and on ties going to
     even).  The first two entries carry the row's |w| maximum, so both the
-    training scale and the export clip equal amax / 127."""
+    training scale and the export clip equal amax / levels."""
     rng = np.random.default_rng(seed)
     W = np.empty((n_rows, cols), np.float32)
     for i in range(n_rows):
         amax = np.float32(rng.uniform(1e-3, 1e2))
-        s = amax / np.float32(127.0)
-        k = rng.integers(-127, 127, cols).astype(np.float32)
+        s = amax / np.float32(levels)
+        k = rng.integers(-levels, levels, cols).astype(np.float32)
         base = (k + np.float32(0.5)) * s
         steps = rng.integers(-3, 4, cols)
         w = base.copy()
@@ -123,12 +143,12 @@ def _near_tie_rows(n_rows=256, cols=512, seed=21):
     return W
 
 
-@pytest.mark.parametrize("bits", [6, 8])
+@pytest.mark.parametrize("bits", [5, 6, 8])
 def test_near_tie_quotients_bit_exact(bits):
     """Pins the division w / s and the two roundings against the oracle's
     IEEE fp32 division on adversarial near-tie inputs, for both the training
     quantizer and the export quantizer."""
-    W = _near_tie_rows()
+    W = _near_tie_rows(levels=15 if bits == 5 else 127)
     q = qat.quantize_weight(_dev(W), bits, keep_codes=True)
     codes = torch.empty(W.shape, dtype=torch.int8, device="cuda")
     s16 = torch.empty(W.shape[0], dtype=torch.float16, device="cuda")

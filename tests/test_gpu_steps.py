@@ -15,9 +15,10 @@ from parity import assert_close, assert_close_chain, to_np
 pytestmark = pytest.mark.gpu
 
 
-def _core(c, bits=6):
+def _core(c, bits=6, act="relu2"):
     dev = {k: torch.from_numpy(c[k]).cuda() for k in ("Wq", "Wk", "Wv", "Wo", "Wfc", "Wproj")}
-    return steps.RecurrentCore(dev["Wq"], dev["Wk"], dev["Wv"], dev["Wo"], dev["Wfc"], dev["Wproj"], bits)
+    return steps.RecurrentCore(dev["Wq"], dev["Wk"], dev["Wv"], dev["Wo"], dev["Wfc"], dev["Wproj"], bits,
+                               act=act)
 
 
 def _core_oracle(c, bits=6):
@@ -37,6 +38,20 @@ def test_recurrent_core_small():
     assert qat.launch_count() - n0 == 3 * 4  # no re-quantization inside the loop
     q = _core_oracle(c)
     ref = o.recurrent_core_fwd(q["qkv"], q["o"], q["fc"], q["proj"], c["X"].float().numpy(), 3, 640)
+    assert_close_chain(x, ref, 6, "x after 3 applications")
+
+
+@pytest.mark.parametrize("bits,act", [(5, "relu2"), (5, "leaky2"), (6, "leaky2")])
+def test_recurrent_core_int5_and_leaky2(bits, act):
+    """The all-int5 core (MLP_INT5 + ATTN_INT5) and the LeakyReLU(0.5)^2 MLP."""
+    c = sy.recurrent_core_case(T=300, seed=5)
+    core = _core(c, bits, act)
+    x = c["X"].cuda()
+    core.forward(x, 3)
+    torch.cuda.synchronize()
+    q = _core_oracle(c, bits)
+    ref = o.recurrent_core_fwd(q["qkv"], q["o"], q["fc"], q["proj"], c["X"].float().numpy(), 3, 640,
+                               act)
     assert_close_chain(x, ref, 6, "x after 3 applications")
 
 

@@ -57,8 +57,9 @@ def test_argument_validation_before_launch(L):
     A16, A_BAD = P(0x10000), P(0x10004)
     # null activations / outputs
     assert L.qat_linear_fwd(A16, None, 512, 512, 6, None, 0, 256, None, A16, None, 0, None) == qat.QAT_ERR_ARG
-    # bits outside {6, 8}
-    assert L.qat_linear_fwd(A16, None, 512, 512, 5, A16, 0, 256, None, A16, None, 0, None) == qat.QAT_ERR_ARG
+    # bits outside {5, 6, 8}
+    assert L.qat_linear_fwd(A16, None, 512, 512, 7, A16, 0, 256, None, A16, None, 0, None) == qat.QAT_ERR_ARG
+    assert L.qat_linear_fwd(A16, None, 512, 512, 4, A16, 0, 256, None, A16, None, 0, None) == qat.QAT_ERR_ARG
     # feature dims must be multiples of 8
     assert L.qat_linear_fwd(A16, None, 500, 512, 6, A16, 0, 256, None, A16, None, 0, None) == qat.QAT_ERR_SHAPE
     # both W and qw, or neither
@@ -75,8 +76,12 @@ def test_argument_validation_before_launch(L):
     assert L.quantize_export_batch(A16, 257, None) == qat.QAT_ERR_ARG
     assert L.dequantize_rows(A16, A16, 4, 12, 0, A16, None) == qat.QAT_ERR_SHAPE
     assert L.dequantize_rows(A16, A16, 4, 16, 3, A16, None) == qat.QAT_ERR_ARG
-    assert L.qat_mlp_bwd(None, None, None, None, 512, 1536, 6, A16, A16, None, A16, 8, None,
+    assert L.qat_mlp_bwd(None, None, None, None, 512, 1536, 6, 0, A16, A16, None, A16, 8, None,
                          None, None, 0, None, 0, None) == qat.QAT_ERR_ARG
+    # activation outside {relu^2, leaky^2}; bits 7
+    assert L.qat_mlp_fwd(None, None, None, None, 512, 1536, 6, 2, A16, 8, None, A16, None, None,
+                         None, 0, None) == qat.QAT_ERR_ARG
+    assert L.qat_noisy_operand(A16, 4, 512, 7, 1, 0, None, A16, None) == qat.QAT_ERR_ARG
     assert qat.launch_count() == before
 
 
@@ -95,6 +100,12 @@ def test_export_plan_matches_page_rules():
     assert kinds["blocks.0.edge"] == "fp16" and kinds["tok_emb.weight"] == "fp16"
     off = {n: m for n, m in qexport.plan({k: _Shape(v) for k, v in sd.items()}, int6_range=(-1, -1))}
     assert off["blocks.3.mlp.fc.weight"] == 8
+    for flags in ({"mlp_int5": True}, {"attn_int5": True}, {"mlp_int5": True, "attn_int5": True}):
+        k5 = {n: ("fp16" if m == qat.QAT_EXPORT_FP16 else "int%d" % m)
+              for n, m in qexport.plan({k: _Shape(v) for k, v in sd.items()}, **flags)}
+        assert k5 == {k: v["kind"] for k, v in o.export_state_dict(sd, **flags).items()}
+        assert (k5["blocks.3.mlp.fc.weight"] == "int5") == ("mlp_int5" in flags)
+        assert (k5["blocks.3.attn.c_q.weight"] == "int5") == ("attn_int5" in flags)
 
 
 class _Shape:
