@@ -31,6 +31,8 @@ def _c():
         I64 = ctypes.c_int64
         lib.oracle_qat_scales.argtypes = [P, I64, I64, P]
         lib.oracle_qat_scales_bits.argtypes = [P, I64, I64, ctypes.c_int, P]
+        lib.oracle_pack6.argtypes = [P, I64, ctypes.c_int, P]
+        lib.oracle_unpack6.argtypes = [P, I64, ctypes.c_int, P]
         lib.oracle_qat_codes.argtypes = [P, I64, I64, P, ctypes.c_int, P]
         lib.oracle_qat_codes.restype = ctypes.c_int
         lib.oracle_dequant_f32.argtypes = [P, P, I64, I64, P]
@@ -303,6 +305,26 @@ def dequant_export(codes, scale16_bits):
     rows, cols = c.shape
     out = np.empty((rows, cols), np.float32)
     _c().oracle_dequant_export(_ptr(c), _ptr(s), rows, cols, _ptr(out))
+    return out
+
+
+def pack6(codes, bits):
+    """6-bit packing of int6 / int5 codes (P1 Day 0 "bit-packing"): field c/4
+    (int6) or c (int5), 6 bits two's complement, little-endian bit stream,
+    4 codes -> 3 bytes.  Returns uint8 [3*n/4] for the flattened codes."""
+    c = np.ascontiguousarray(codes, np.int8).reshape(-1)
+    out = np.empty(3 * c.size // 4, np.uint8)
+    if _c().oracle_pack6(_ptr(c), c.size, int(bits), _ptr(out)) != 0:
+        raise ValueError("pack6 needs bits 5 or 6 and a multiple of 4 codes")
+    return out
+
+
+def unpack6(packed, n, bits):
+    """Inverse of pack6: n int8 codes."""
+    p = np.ascontiguousarray(packed, np.uint8).reshape(-1)
+    out = np.empty(n, np.int8)
+    if _c().oracle_unpack6(_ptr(p), n, int(bits), _ptr(out)) != 0:
+        raise ValueError("unpack6 needs bits 5 or 6 and a multiple of 4 codes")
     return out
 
 

@@ -247,6 +247,45 @@ int oracle_export_rows(const float* W, int64_t rows, int64_t cols, int bits, dou
 }
 
 /* Roundtrip dequantize: fl32(c * fp32(scale16)). */
+/* 6-bit packing of int6 / int5 codes (the bit-packing of the depth-recurrence
+ * write-up's Day 0 compression study, which puts int6 codes at about 2.94
+ * bits of entropy each; the pages give no format).  Reading: each code
+ * becomes one 6-bit two's-complement field -- c / 4 for int6 (codes are
+ * multiples of 4 in [-128, 124], so c / 4 is in [-32, 31]), c itself for int5
+ * ([-15, 15]) -- and field i occupies bits 6i .. 6i+5 of a little-endian bit
+ * stream: bit k of the stream is bit (k mod 8) of byte k / 8.  n codes (n a
+ * multiple of 4) give 3n/4 bytes.  Written bit by bit, as the definition. */
+int oracle_pack6(const int8_t* codes, int64_t n, int bits, uint8_t* out) {
+  if ((bits != 5 && bits != 6) || n % 4 != 0) return -1;
+  for (int64_t b = 0; b < 3 * n / 4; ++b) out[b] = 0;
+  for (int64_t i = 0; i < n; ++i) {
+    const int c = codes[i];
+    const int v = bits == 6 ? c / 4 : c;            /* exact: c is a multiple of 4 */
+    const unsigned field = (unsigned)v & 63u;       /* two's complement, 6 bits */
+    for (int k = 0; k < 6; ++k) {
+      const int64_t pos = 6 * i + k;
+      if ((field >> k) & 1u) out[pos / 8] |= (uint8_t)(1u << (pos % 8));
+    }
+  }
+  return 0;
+}
+
+/* Inverse of oracle_pack6: field i read back bit by bit, sign-extended from 6
+ * bits, times 4 for int6. */
+int oracle_unpack6(const uint8_t* in, int64_t n, int bits, int8_t* codes) {
+  if ((bits != 5 && bits != 6) || n % 4 != 0) return -1;
+  for (int64_t i = 0; i < n; ++i) {
+    unsigned field = 0;
+    for (int k = 0; k < 6; ++k) {
+      const int64_t pos = 6 * i + k;
+      field |= (unsigned)((in[pos / 8] >> (pos % 8)) & 1u) << k;
+    }
+    const int v = field >= 32u ? (int)field - 64 : (int)field;
+    codes[i] = (int8_t)(bits == 6 ? 4 * v : v);
+  }
+  return 0;
+}
+
 void oracle_dequant_export(const int8_t* codes, const uint16_t* scale16, int64_t rows,
                            int64_t cols, float* out) {
   for (int64_t i = 0; i < rows; ++i) {

@@ -307,6 +307,35 @@ def test_export_passthrough_and_layer_range():
     assert np.array_equal(out["vec"]["bits16"], sd["vec"].astype(np.float16).view(np.uint16))
 
 
+def test_pack6_worked_example():
+    """P1 Day 0 bit-packing, read as 6-bit little-endian fields: hand-derived bytes."""
+    g = _golden("pack6_worked_example.txt")
+    for bits in (6, 5):
+        c = np.array([int(v) for v in g["int%d_codes" % bits]], np.int8)
+        assert o.pack6(c, bits).tolist() == [int(v) for v in g["int%d_bytes" % bits]]
+
+
+@pytest.mark.parametrize("bits", [5, 6])
+def test_pack6_against_numpy_packbits_and_roundtrip(bits):
+    """The packed stream equals numpy.packbits (little bit order) of the
+    fields' bits; unpack inverts pack on every code of the grid and on export
+    codes of a real row set; 4 codes take 3 bytes."""
+    grid = np.arange(-128, 125, 4) if bits == 6 else np.arange(-15, 16)
+    rng = np.random.default_rng(bits)
+    c = rng.choice(grid, 4096).astype(np.int8)
+    c[:len(grid)] = grid
+    f = (c.astype(np.int32) // (4 if bits == 6 else 1)) & 63
+    bitstream = ((f[:, None] >> np.arange(6)[None, :]) & 1).astype(np.uint8).reshape(-1)
+    ref = np.packbits(bitstream, bitorder="little")
+    p = o.pack6(c, bits)
+    assert p.size == 3 * c.size // 4
+    assert np.array_equal(p, ref)
+    assert np.array_equal(o.unpack6(p, c.size, bits), c)
+    W = sy.linear_case(N=64, K=256, seed=9)["W"]
+    ce, _, _ = o.export_rows(W, bits)
+    assert np.array_equal(o.unpack6(o.pack6(ce, bits), ce.size, bits).reshape(ce.shape), ce)
+
+
 # ------------------------------------------------------------------ algebra
 
 def test_linear_fwd_brute_force():
