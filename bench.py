@@ -252,6 +252,7 @@ def run_ours(args):
         out["e2e"] = e2e
         if world == 1:
             out["export"] = measure_export(dev, stream, pk)
+            out["export_pack6"] = measure_export(dev, stream, pk, pack6=True)
             out["recurrent_core"] = measure_core(dev, stream, pk)
             out["cpu_baseline"] = cpu_baseline()
         print(json.dumps(out), flush=True)
@@ -308,14 +309,15 @@ def flush_l2(buf, clean):
     clean.sum()
 
 
-def measure_export(dev, stream, pk):
+def measure_export(dev, stream, pk, pack6=False):
     """Export quantizer over the 11-layer d=512 state dict: one grouped launch,
-    L2 flushed (256 MB write) before every timed launch."""
+    L2 flushed (256 MB write) before every timed launch.  pack6: the int6 codes
+    are stored 6-bit packed (3 bytes per 4 codes)."""
     from quantization_aware_tiny_b200 import export as qexport
     from quantization_aware_tiny_b200 import qat
     from quantization_aware_tiny_b200 import synthetic as sy
     sd = {k: torch.from_numpy(v).to(dev) for k, v in sy.state_dict_case().items()}
-    out = qexport.export_state_dict(sd)  # allocates outputs once
+    out = qexport.export_state_dict(sd, pack6=pack6)  # allocates outputs once
     descs = []
     algo = 0
     for name, mode in qexport.plan(sd):
@@ -324,6 +326,9 @@ def measure_export(dev, stream, pk):
         if mode == qat.QAT_EXPORT_FP16:
             descs.append((t.reshape(-1), mode, o["values"], None))
             algo += t.numel() * (4 + 2)
+        elif "packed" in o:
+            descs.append((t, mode, o["packed"], o["scale16"], qat.QAT_EXPORT_PACK6))
+            algo += t.numel() * 4 + t.numel() * 3 // 4 + t.shape[0] * 2
         else:
             descs.append((t, mode, o["codes"], o["scale16"]))
             algo += t.numel() * (4 + 1) + t.shape[0] * 2
@@ -347,8 +352,9 @@ def measure_export(dev, stream, pk):
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"],
                          "unit": "GB/s", "frac": round(gbs / pk["hbm_gbs"], 4),
                          "peak_kind": "copy bandwidth (%s)" % pk["source"]},
-            "workload": "11 blocks x (Q,K,V,O,fc,proj) d=512 MLP3x int6 + tied emb 1024x512 "
-                        "+ small tensors fp16 passthrough; L2 flushed (256 MB written, 256 MB read) before each launch"}
+            "workload": "11 blocks x (Q,K,V,O,fc,proj) d=512 MLP3x int6%s + tied emb 1024x512 "
+                        "+ small tensors fp16 passthrough; L2 flushed (256 MB written, 256 MB read) "
+                        "before each launch" % (" 6-bit packed" if pack6 else "")}
 
 
 def measure_core(dev, stream, pk):

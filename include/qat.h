@@ -211,18 +211,32 @@ int quantize_rows_export(const float* W, int64_t rows, int64_t cols, int32_t bit
  * descriptors (n <= QAT_EXPORT_MAX_DESCS); mode 5, 6 or 8 quantizes rows as
  * above into dst (int8 codes) and scales; mode QAT_EXPORT_FP16 converts src
  * to fp16 (rne) into dst (the passthrough of non-2D, small and tied-embedding
- * tensors; scales unused).  The caller applies the passthrough rules. */
+ * tensors; scales unused).  The caller applies the passthrough rules.
+ * flags: 0, or QAT_EXPORT_PACK6 with mode 5 or 6 -- dst then receives the codes
+ * 6-bit packed (see unpack_codes6), rows*cols*3/4 bytes, row r at byte
+ * r*cols*3/4 (the bit-packing of [P1] Day 0; the format is this library's:
+ * one 6-bit two's-complement field per code, c/4 for int6 and c for int5,
+ * field i at bits 6i..6i+5 of a little-endian bit stream).  Other flags, or
+ * PACK6 with another mode, return QAT_ERR_ARG. */
 #define QAT_EXPORT_FP16 16
 #define QAT_EXPORT_MAX_DESCS 256
+#define QAT_EXPORT_PACK6 1
 typedef struct qat_export_desc {
   const float* src;
   int64_t rows, cols;
   int32_t mode;
-  int32_t reserved;
+  int32_t flags;
   void* dst;
   qat_fp16* scales;
 } qat_export_desc;
 int quantize_export_batch(const qat_export_desc* descs, int32_t n, qat_stream_t stream);
+
+/* Unpacks n 6-bit packed codes (QAT_EXPORT_PACK6 layout, 3n/4 bytes at
+ * `packed`) into n int8 codes: the field sign-extended, times 4 for bits = 6.
+ * n must be a multiple of 8 (QAT_ERR_SHAPE otherwise); bits 5 or 6.  Both
+ * pointers are device pointers, 16-byte aligned.  Bit-exact with the oracle. */
+int unpack_codes6(const uint8_t* packed, int64_t n, int32_t bits, int8_t* codes,
+                  qat_stream_t stream);
 
 /* Roundtrip dequantize ([P5] "后训练量化导出", roundtrip re-evaluation):
  *   out = fl32(c * fp32(scale_fp16))  as fp32 (out_dtype 0) or bf16_rne of it (1). */

@@ -331,7 +331,7 @@ int quantize_rows_export(const float* W, int64_t rows, int64_t cols, int32_t bit
   d.rows = rows;
   d.cols = cols;
   d.mode = bits;
-  d.reserved = 0;
+  d.flags = 0;
   d.dst = codes;
   d.scales = scales;
   if (!bits_ok(bits)) return QAT_ERR_ARG;
@@ -354,7 +354,9 @@ int quantize_export_batch(const qat_export_desc* descs, int32_t n, qat_stream_t 
     d.mode = s.mode;
     d.m = 1;
     d.frac = 0.0f;
-    d.pad = 0;
+    if (s.flags & ~QAT_EXPORT_PACK6) return QAT_ERR_ARG;
+    d.pack6 = (s.flags & QAT_EXPORT_PACK6) != 0;
+    if (d.pack6 && s.mode != 5 && s.mode != 6) return QAT_ERR_ARG;
     d.unit_begin = b.total_units;
     if (s.mode == QAT_EXPORT_FP16) {
       d.numel = s.rows * s.cols;
@@ -379,6 +381,14 @@ int quantize_export_batch(const qat_export_desc* descs, int32_t n, qat_stream_t 
     b.total_units += (d.rows + d.unit_rows - 1) / d.unit_rows;
   }
   return launch_export_batch(b, stream);
+}
+
+int unpack_codes6(const uint8_t* packed, int64_t n, int32_t bits, int8_t* codes,
+                  qat_stream_t stream) {
+  if (!packed || !codes || n < 0 || (bits != 5 && bits != 6)) return QAT_ERR_ARG;
+  if (n % 8 != 0) return QAT_ERR_SHAPE;
+  if (!aligned16(packed) || !aligned16(codes)) return QAT_ERR_ALIGN;
+  return launch_unpack6(packed, n, bits, codes, stream);
 }
 
 int dequantize_rows(const int8_t* codes, const qat_fp16* scales, int64_t rows, int64_t cols,

@@ -306,6 +306,46 @@ __device__ __forceinline__ uint32_t codes4(const RowQuant& q, float4 v) {
   return q.bits == 5 ? codes4_t<5, true>(q, v) : codes4_t<8, true>(q, v);
 }
 
+// ---- 6-bit packing of int6 / int5 codes: one 6-bit two's-complement field per
+// code (c / 4 for int6, c for int5), field i at bits 6i .. 6i+5 of a
+// little-endian bit stream; four codes make 24 bits, three bytes.
+
+// The 24 packed bits of the four codes in the bytes of x (byte i = code i).
+template <int BITS>
+__device__ __forceinline__ uint32_t pack24(uint32_t x) {
+  // per byte: the field in bits 0..5 (int6: the byte's bits 2..7, i.e. c / 4)
+  const uint32_t y = (BITS == 6 ? (x >> 2) : x) & 0x3F3F3F3Fu;
+  return (y & 0x3Fu) | ((y >> 2) & 0xFC0u) | ((y >> 4) & 0x3F000u) | ((y >> 6) & 0xFC0000u);
+}
+
+// Stores the 24-bit values p of the warp's first n lanes (n even, <= 32) as
+// 3n contiguous bytes at dst (2-byte aligned).  Output word w (of 32 or 16
+// bits) starts at stream bit 32w (16w), inside lane a = 4w / 3 (2w / 3)'s
+// value at bit offset `off`; its remaining high bits come from lane a + 1.
+// Full 32-lane chunks at 4-byte aligned addresses go out as 24 words, the
+// rest as 16-bit halves.  Every lane must call this (shuffles).
+__device__ __forceinline__ void store_pack6_chunk(uint8_t* dst, uint32_t p, int n, int lane) {
+  if (n == 32 && (reinterpret_cast<uintptr_t>(dst) & 3u) == 0) {
+    const int a = (4 * lane) / 3;
+    const int off = 8 * (4 * lane - 3 * a);  // 0, 8 or 16
+    const uint32_t lo = __shfl_sync(0xffffffffu, p, a & 31);
+    const uint32_t hi = __shfl_sync(0xffffffffu, p, (a + 1) & 31);
+    if (lane < 24) reinterpret_cast<uint32_t*>(dst)[lane] = (lo >> off) | (hi << (24 - off));
+  } else {
+    const int halves = 3 * n / 2;
+    for (int h0 = 0; h0 < halves; h0 += 32) {
+      const int h = h0 + lane;
+      const int a = (2 * h) / 3;
+      const int off = 8 * (2 * h - 3 * a);  // 0, 8 or 16
+      const uint32_t lo = __shfl_sync(0xffffffffu, p, a & 31);
+      const uint32_t hi = __shfl_sync(0xffffffffu, p, (a + 1) & 31);
+      if (h < halves)
+        reinterpret_cast<uint16_t*>(dst)[h] =
+            static_cast<uint16_t>((lo >> off) | (hi << (24 - off)));
+    }
+  }
+}
+
 // float4 groups per lane and loop iteration in the shared-memory passes: more
 // independent dependency chains per warp.
 constexpr int kUnroll = 4;
@@ -325,6 +365,28 @@ __device__ __forceinline__ void quantize_smem_row(const RowQuant& q, const float
     for (int u = 0; u < kUnroll; ++u) out[j + 32 * u] = c[u];
   }
   for (; j < K4; j += 32) out[j] = codes4_t<BITS, CLIP>(q, buf[j]);
+}
+
+// The same codes stored 6-bit packed: row bytes [3 * K4) at out (2-byte
+// aligned: K4 is even).  Chunks of 32 float4 groups are warp-uniform, so the
+// packing shuffles see every lane.
+template <int BITS, bool CLIP, typename Src>
+__device__ __forceinline__ void quantize_row_pack6(const RowQuant& q, Src src, int K4,
+                                                   uint8_t* out, int lane) {
+  constexpr int U = 2;
+  for (int base = 0; base < K4; base += 32 * U) {
+    uint32_t p[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int j = base + 32 * u + lane;
+      p[u] = j < K4 ? pack24<BITS>(codes4_t<BITS, CLIP>(q, src(j))) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c0 = base + 32 * u;
+      if (c0 < K4) store_pack6_chunk(out + 3 * c0, p[u], min(32, K4 - c0), lane);
+    }
+  }
 }
 
 // A quantized row staged in shared memory (cols <= the batch's buffer).
@@ -351,8 +413,18 @@ __device__ __forceinline__ void export_row_smem(const ExportDescDev& d, int64_t 
   top2_warp(a1, a2);
   const RowQuant q = row_params(d, a1, a2);
   if (lane == 0) d.scales[row] = __float2half_rn(q.s);
-  uint32_t* out = reinterpret_cast<uint32_t*>(reinterpret_cast<int8_t*>(d.dst) + row * d.cols);
   const bool clip = a1 > 2.0f * q.clip;  // see codes2: clamping needed only then
+  if (d.pack6) {
+    uint8_t* out = reinterpret_cast<uint8_t*>(d.dst) + row * 3 * K4;
+    with_grid(q.bits, clip, [&](auto bits_tag, auto clip_tag) {
+      constexpr int B = decltype(bits_tag)::value;
+      if constexpr (B != 8)
+        quantize_row_pack6<B, decltype(clip_tag)::value>(
+            q, [&](int j) { return buf[j]; }, K4, out, lane);
+    });
+    return;
+  }
+  uint32_t* out = reinterpret_cast<uint32_t*>(reinterpret_cast<int8_t*>(d.dst) + row * d.cols);
   with_grid(q.bits, clip, [&](auto bits_tag, auto clip_tag) {
     quantize_smem_row<decltype(bits_tag)::value, decltype(clip_tag)::value>(q, buf, K4, out, lane);
   });
@@ -393,9 +465,21 @@ __device__ __forceinline__ void export_two_rows_smem(const ExportDescDev& d, int
     d.scales[row] = __float2half_rn(qa.s);
     d.scales[row + 1] = __float2half_rn(qb.s);
   }
+  const bool clip = (a1 > 2.0f * qa.clip) || (b1 > 2.0f * qb.clip);
+  if (d.pack6) {
+    uint8_t* outA = reinterpret_cast<uint8_t*>(d.dst) + row * 3 * K4;
+    with_grid(qa.bits, clip, [&](auto bits_tag, auto clip_tag) {
+      constexpr int B = decltype(bits_tag)::value;
+      constexpr bool C = decltype(clip_tag)::value;
+      if constexpr (B != 8) {
+        quantize_row_pack6<B, C>(qa, [&](int j) { return bufA[j]; }, K4, outA, lane);
+        quantize_row_pack6<B, C>(qb, [&](int j) { return bufB[j]; }, K4, outA + 3 * K4, lane);
+      }
+    });
+    return;
+  }
   uint32_t* outA = reinterpret_cast<uint32_t*>(reinterpret_cast<int8_t*>(d.dst) + row * d.cols);
   uint32_t* outB = outA + K4;
-  const bool clip = (a1 > 2.0f * qa.clip) || (b1 > 2.0f * qb.clip);
   auto run = [&](auto bits_tag, auto clip_tag) {
     constexpr int BITS = decltype(bits_tag)::value;
     constexpr bool CLIP = decltype(clip_tag)::value;
@@ -426,6 +510,16 @@ __device__ __forceinline__ void export_row_global(const ExportDescDev& d, int64_
   top2_warp(t1, t2);
   const RowQuant q = row_params(d, t1, t2);
   if (lane == 0) d.scales[row] = __float2half_rn(q.s);
+  if (d.pack6) {
+    uint8_t* out = reinterpret_cast<uint8_t*>(d.dst) + row * 3 * K4;
+    with_grid(q.bits, true, [&](auto bits_tag, auto clip_tag) {
+      constexpr int B = decltype(bits_tag)::value;
+      if constexpr (B != 8)
+        quantize_row_pack6<B, decltype(clip_tag)::value>(
+            q, [&](int j) { return __ldg(r + j); }, K4, out, lane);
+    });
+    return;
+  }
   uint32_t* out = reinterpret_cast<uint32_t*>(reinterpret_cast<int8_t*>(d.dst) + row * d.cols);
   for (int j = lane; j < K4; j += 32) out[j] = codes4(q, __ldg(r + j));
 }
@@ -628,6 +722,27 @@ __global__ void __launch_bounds__(kQThreads)
   }
 }
 
+// 6-bit packed codes back to int8 codes: thread per 8 codes (6 bytes read as
+// three 16-bit halves, 2-byte aligned; 8 codes written as one 8-byte word).
+__global__ void __launch_bounds__(kQThreads)
+    unpack6_kernel(const uint16_t* __restrict__ packed, int64_t n8, int bits,
+                   uint2* __restrict__ codes) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint64_t v = static_cast<uint64_t>(packed[3 * i]) |
+                       (static_cast<uint64_t>(packed[3 * i + 1]) << 16) |
+                       (static_cast<uint64_t>(packed[3 * i + 2]) << 32);
+    uint32_t w[2] = {0u, 0u};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int f = static_cast<int>((v >> (6 * k)) & 63u);
+      const int c = (f >= 32 ? f - 64 : f) * (bits == 6 ? 4 : 1);
+      w[k >> 2] |= (static_cast<uint32_t>(c) & 0xFFu) << (8 * (k & 3));
+    }
+    codes[i] = make_uint2(w[0], w[1]);
+  }
+}
+
 int grid_for_rows(int64_t rows_or_items, int items_per_block) {
   const int64_t want = (rows_or_items + items_per_block - 1) / items_per_block;
   const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
@@ -696,6 +811,15 @@ int launch_dequant(const int8_t* codes, const __half* scales, int64_t rows, int6
   if (items == 0) return QAT_OK;
   dequant_kernel<<<grid_for_rows(items, kQThreads), kQThreads, 0, s>>>(codes, scales, rows, cols,
                                                                        out_bf16, out);
+  count_launch();
+  return cuda_status(cudaGetLastError());
+}
+
+int launch_unpack6(const uint8_t* packed, int64_t n, int bits, int8_t* codes, cudaStream_t s) {
+  const int64_t n8 = n / 8;
+  if (n8 == 0) return QAT_OK;
+  unpack6_kernel<<<grid_for_rows(n8, kQThreads), kQThreads, 0, s>>>(
+      reinterpret_cast<const uint16_t*>(packed), n8, bits, reinterpret_cast<uint2*>(codes));
   count_launch();
   return cuda_status(cudaGetLastError());
 }

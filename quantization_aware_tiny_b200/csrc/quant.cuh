@@ -15,10 +15,10 @@ struct ExportDescDev {
   int64_t rows, cols, numel;
   int64_t unit_begin;  // first global work unit of this descriptor
   int64_t unit_rows;   // rows per work unit
-  int mode;           // 6, 8 or QAT_EXPORT_FP16
+  int mode;           // 5, 6, 8 or QAT_EXPORT_FP16
   int m;              // quantile order statistic from the top (1 or 2)
   float frac;         // quantile interpolation fraction
-  int pad;
+  int pack6;          // codes stored as 6-bit fields, 4 codes in 3 bytes
 };
 
 #ifndef QAT_EXPORT_BATCH_CAP
@@ -55,5 +55,6 @@ int export_quantile_params(int64_t cols, int* m, float* frac);
 int launch_export_batch(ExportBatch& b, cudaStream_t s);
 int launch_dequant(const int8_t* codes, const __half* scales, int64_t rows, int64_t cols,
                    int out_bf16, void* out, cudaStream_t s);
+int launch_unpack6(const uint8_t* packed, int64_t n, int bits, int8_t* codes, cudaStream_t s);
 
 }  // namespace qat

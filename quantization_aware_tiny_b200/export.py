@@ -48,10 +48,12 @@ def plan(state_dict, int6_range=(0, 10), embed_name="tok_emb.weight", mlp_int5=F
 
 
 def export_state_dict(state_dict, int6_range=(0, 10), embed_name="tok_emb.weight", stream=None,
-                      mlp_int5=False, attn_int5=False):
+                      mlp_int5=False, attn_int5=False, pack6=False):
     """Quantize a dict of fp32 CUDA tensors.  Returns name -> dict with
     kind 'int5'/'int6'/'int8' (codes int8 [rows,cols], scale16 fp16 [rows]) or
-    kind 'fp16' (values fp16, original shape).  Launches in chunks of at most
+    kind 'fp16' (values fp16, original shape).  With pack6, int5 / int6 tensors
+    hold 'packed' (uint8 [rows, cols*3/4], the 6-bit packed codes; see
+    qat.unpack_codes6) in place of 'codes'.  Launches in chunks of at most
     QAT_EXPORT_MAX_DESCS descriptors (one launch for a state dict that fits)."""
     out = {}
     descs = []
@@ -65,10 +67,15 @@ def export_state_dict(state_dict, int6_range=(0, 10), embed_name="tok_emb.weight
             descs.append((t.reshape(-1), mode, v, None))
         else:
             rows, cols = t.shape
-            c = torch.empty((rows, cols), dtype=torch.int8, device=t.device)
             s = torch.empty(rows, dtype=torch.float16, device=t.device)
-            out[name] = {"kind": "int%d" % mode, "codes": c, "scale16": s}
-            descs.append((t, mode, c, s))
+            if pack6 and mode in (5, 6):
+                p = torch.empty((rows, cols * 3 // 4), dtype=torch.uint8, device=t.device)
+                out[name] = {"kind": "int%d" % mode, "packed": p, "scale16": s}
+                descs.append((t, mode, p, s, qat.QAT_EXPORT_PACK6))
+            else:
+                c = torch.empty((rows, cols), dtype=torch.int8, device=t.device)
+                out[name] = {"kind": "int%d" % mode, "codes": c, "scale16": s}
+                descs.append((t, mode, c, s))
     for i in range(0, len(descs), qat.QAT_EXPORT_MAX_DESCS):
         qat.quantize_export_batch(descs[i:i + qat.QAT_EXPORT_MAX_DESCS], stream=stream)
     return out

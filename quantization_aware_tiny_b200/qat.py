@@ -26,7 +26,8 @@ QAT_DTYPE_F32, QAT_DTYPE_BF16 = 0, 1
 EXPORTED = ("qat_strerror", "qat_launch_count", "qat_device_error", "qat_quantize_weights",
             "qat_workspace_size", "qat_linear_fwd", "qat_linear_bwd", "qat_mlp_fwd",
             "qat_mlp_bwd", "quantize_rows_export", "quantize_export_batch", "dequantize_rows",
-            "qat_linear_fwd_noalloc", "qat_noisy_operand")
+            "qat_linear_fwd_noalloc", "qat_noisy_operand", "unpack_codes6")
+QAT_EXPORT_PACK6 = 1
 QAT_ACT_RELU2 = 0
 QAT_ACT_LEAKY_RELU2 = 1
 _ACTS = {"relu2": QAT_ACT_RELU2, "leaky2": QAT_ACT_LEAKY_RELU2}
@@ -48,7 +49,7 @@ class _QWeight(ctypes.Structure):
 
 class _ExportDesc(ctypes.Structure):
     _fields_ = [("src", ctypes.c_void_p), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
-                ("mode", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("mode", ctypes.c_int32), ("flags", ctypes.c_int32),
                 ("dst", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
 
 
@@ -80,6 +81,7 @@ def lib():
         L.quantize_rows_export.argtypes = [P, I64, I64, I32, P, P, P]
         L.quantize_export_batch.argtypes = [P, I32, P]
         L.dequantize_rows.argtypes = [P, P, I64, I64, I32, P, P]
+        L.unpack_codes6.argtypes = [P, I64, I32, P, P]
         L.qat_linear_fwd_noalloc.argtypes = [P, I32, I32, I32, P, I64, I64, P, P, P]
         L.qat_noisy_operand.argtypes = [P, I32, I32, I32, ctypes.c_uint64, ctypes.c_uint64, P, P,
                                         P]
@@ -229,22 +231,31 @@ def quantize_rows_export(W, bits, codes, scales, stream=None):
 
 
 def export_descs(descs):
-    """Marshal (src, mode, dst, scales) tuples into the C descriptor array once;
-    the result can be passed to quantize_export_batch repeatedly."""
+    """Marshal (src, mode, dst, scales[, flags]) tuples into the C descriptor
+    array once; the result can be passed to quantize_export_batch repeatedly."""
     arr = (_ExportDesc * len(descs))()
-    for i, (src, mode, dst, scales) in enumerate(descs):
+    for i, dsc in enumerate(descs):
+        src, mode, dst, scales = dsc[:4]
+        flags = dsc[4] if len(dsc) > 4 else 0
         rows, cols = (src.shape if src.dim() == 2 else (1, src.numel()))
-        arr[i] = _ExportDesc(src.data_ptr(), rows, cols, mode, 0, dst.data_ptr(),
+        arr[i] = _ExportDesc(src.data_ptr(), rows, cols, mode, flags, dst.data_ptr(),
                              scales.data_ptr() if scales is not None else None)
     return arr
 
 
 def quantize_export_batch(descs, stream=None):
-    """descs: list of (src, mode, dst, scales) with src a 2-D (or flat) fp32
-    device tensor, mode 6 / 8 / QAT_EXPORT_FP16 -- or an array from
-    export_descs() (the tensors it points to must stay alive)."""
+    """descs: list of (src, mode, dst, scales[, flags]) with src a 2-D (or flat)
+    fp32 device tensor, mode 5 / 6 / 8 / QAT_EXPORT_FP16, flags 0 or
+    QAT_EXPORT_PACK6 -- or an array from export_descs() (the tensors it points
+    to must stay alive)."""
     arr = descs if isinstance(descs, ctypes.Array) else export_descs(descs)
     _check(lib().quantize_export_batch(arr, len(arr), _stream(stream)), "quantize_export_batch")
+
+
+def unpack_codes6(packed, n, bits, codes, stream=None):
+    """n 6-bit packed codes (uint8 device tensor of 3n/4 bytes) into int8 codes."""
+    _check(lib().unpack_codes6(_p(packed), int(n), int(bits), _p(codes), _stream(stream)),
+           "unpack_codes6")
 
 
 def dequantize_rows(codes, scales16, out, stream=None):

@@ -104,6 +104,53 @@ def test_export_state_dict_mixed_int5_bit_exact(flags):
             assert np.array_equal(bits16(g["scale16"]), r["scale16"]), k
 
 
+@pytest.mark.parametrize("bits", [5, 6])
+def test_export_pack6_bit_exact(bits):
+    """6-bit packed export codes (word stores for aligned full chunks, 16-bit
+    stores for odd-offset rows and ragged tails, rows read from global memory
+    beyond the staging buffer) equal the oracle's bit-serial packing of its
+    codes; unpack_codes6 returns the oracle's codes."""
+    for name, W in _weights().items():
+        rows, cols = W.shape
+        packed = torch.full((rows, cols * 3 // 4), 0xA5, dtype=torch.uint8, device="cuda")
+        s16 = torch.empty(rows, dtype=torch.float16, device="cuda")
+        Wd = _dev(W)
+        qat.quantize_export_batch([(Wd, bits, packed, s16, qat.QAT_EXPORT_PACK6)])
+        codes = torch.empty((rows, cols), dtype=torch.int8, device="cuda")
+        qat.unpack_codes6(packed, rows * cols, bits, codes)
+        torch.cuda.synchronize()
+        c_ref, s_ref, _ = o.export_rows(W, bits)
+        assert np.array_equal(packed.cpu().numpy().reshape(-1), o.pack6(c_ref, bits)), name
+        assert np.array_equal(bits16(s16), s_ref), name
+        assert np.array_equal(codes.cpu().numpy(), c_ref), name
+
+
+def test_export_state_dict_pack6_one_launch():
+    """The all-int5 / int6 mixed state dict exported packed in one launch:
+    packed bytes equal the oracle's packing of its codes; int8 tensors are
+    unpacked codes as before."""
+    sd = sy.state_dict_case(n_layers=2, seed=4)
+    sd["blocks.0.attn.c_q.weight"] = sd["blocks.0.attn.c_q.weight"][:, :136].copy()  # odd row bytes
+    n0 = qat.launch_count()
+    out = qexport.export_state_dict({k: _dev(v) for k, v in sd.items()}, mlp_int5=True,
+                                    int6_range=(0, 0), pack6=True)
+    torch.cuda.synchronize()
+    assert qat.launch_count() - n0 == 1
+    ref = o.export_state_dict(sd, mlp_int5=True, int6_start=0, int6_end=0)
+    kinds = set()
+    for k, r in ref.items():
+        g = out[k]
+        kinds.add(r["kind"])
+        assert g["kind"] == r["kind"], k
+        if r["kind"] in ("int5", "int6"):
+            assert np.array_equal(g["packed"].cpu().numpy().reshape(-1),
+                                  o.pack6(r["codes"], int(r["kind"][3:]))), k
+            assert np.array_equal(bits16(g["scale16"]), r["scale16"]), k
+        elif r["kind"] == "int8":
+            assert np.array_equal(g["codes"].cpu().numpy(), r["codes"]), k
+    assert {"int5", "int6", "int8", "fp16"} <= kinds
+
+
 def test_dequantize_rows_bit_exact():
     sd = sy.state_dict_case(n_layers=1)
     for name in ("blocks.0.mlp.fc.weight", "blocks.0.attn.c_k.weight"):
