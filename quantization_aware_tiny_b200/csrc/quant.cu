@@ -367,24 +367,32 @@ __device__ __forceinline__ void quantize_smem_row(const RowQuant& q, const float
   for (; j < K4; j += 32) out[j] = codes4_t<BITS, CLIP>(q, buf[j]);
 }
 
-// The same codes stored 6-bit packed: row bytes [3 * K4) at out (2-byte
-// aligned: K4 is even).  Chunks of 32 float4 groups are warp-uniform, so the
-// packing shuffles see every lane.
-template <int BITS, bool CLIP, typename Src>
-__device__ __forceinline__ void quantize_row_pack6(const RowQuant& q, Src src, int K4,
-                                                   uint8_t* out, int lane) {
-  constexpr int U = 2;
+// The same codes stored 6-bit packed: NR rows of K4 float4 groups (K4 even),
+// row k read through src(k, j) and written to bytes [3 * K4) at out[k] (2-byte
+// aligned).  The rows are interleaved, 4 / NR chunks of 32 groups each per
+// iteration, so every lane has four independent groups in flight; chunks are
+// warp-uniform, so the packing shuffles see every lane.
+template <int BITS, bool CLIP, int NR, typename Src>
+__device__ __forceinline__ void quantize_rows_pack6(const RowQuant (&q)[NR], Src src, int K4,
+                                                    uint8_t* const (&out)[NR], int lane) {
+  constexpr int U = 4 / NR;
   for (int base = 0; base < K4; base += 32 * U) {
-    uint32_t p[U];
+    uint32_t p[NR][U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int j = base + 32 * u + lane;
-      p[u] = j < K4 ? pack24<BITS>(codes4_t<BITS, CLIP>(q, src(j))) : 0u;
+#pragma unroll
+      for (int k = 0; k < NR; ++k)
+        p[k][u] = j < K4 ? pack24<BITS>(codes4_t<BITS, CLIP>(q[k], src(k, j))) : 0u;
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int c0 = base + 32 * u;
-      if (c0 < K4) store_pack6_chunk(out + 3 * c0, p[u], min(32, K4 - c0), lane);
+      if (c0 < K4) {
+#pragma unroll
+        for (int k = 0; k < NR; ++k)
+          store_pack6_chunk(out[k] + 3 * c0, p[k][u], min(32, K4 - c0), lane);
+      }
     }
   }
 }
@@ -415,12 +423,13 @@ __device__ __forceinline__ void export_row_smem(const ExportDescDev& d, int64_t 
   if (lane == 0) d.scales[row] = __float2half_rn(q.s);
   const bool clip = a1 > 2.0f * q.clip;  // see codes2: clamping needed only then
   if (d.pack6) {
-    uint8_t* out = reinterpret_cast<uint8_t*>(d.dst) + row * 3 * K4;
+    const RowQuant qs[1] = {q};
+    uint8_t* const out[1] = {reinterpret_cast<uint8_t*>(d.dst) + row * 3 * K4};
     with_grid(q.bits, clip, [&](auto bits_tag, auto clip_tag) {
       constexpr int B = decltype(bits_tag)::value;
       if constexpr (B != 8)
-        quantize_row_pack6<B, decltype(clip_tag)::value>(
-            q, [&](int j) { return buf[j]; }, K4, out, lane);
+        quantize_rows_pack6<B, decltype(clip_tag)::value, 1>(
+            qs, [&](int, int j) { return buf[j]; }, K4, out, lane);
     });
     return;
   }
@@ -467,14 +476,14 @@ __device__ __forceinline__ void export_two_rows_smem(const ExportDescDev& d, int
   }
   const bool clip = (a1 > 2.0f * qa.clip) || (b1 > 2.0f * qb.clip);
   if (d.pack6) {
-    uint8_t* outA = reinterpret_cast<uint8_t*>(d.dst) + row * 3 * K4;
+    const RowQuant qs[2] = {qa, qb};
+    uint8_t* const outA = reinterpret_cast<uint8_t*>(d.dst) + row * 3 * K4;
+    uint8_t* const out[2] = {outA, outA + 3 * K4};
     with_grid(qa.bits, clip, [&](auto bits_tag, auto clip_tag) {
       constexpr int B = decltype(bits_tag)::value;
-      constexpr bool C = decltype(clip_tag)::value;
-      if constexpr (B != 8) {
-        quantize_row_pack6<B, C>(qa, [&](int j) { return bufA[j]; }, K4, outA, lane);
-        quantize_row_pack6<B, C>(qb, [&](int j) { return bufB[j]; }, K4, outA + 3 * K4, lane);
-      }
+      if constexpr (B != 8)
+        quantize_rows_pack6<B, decltype(clip_tag)::value, 2>(
+            qs, [&](int k, int j) { return k == 0 ? bufA[j] : bufB[j]; }, K4, out, lane);
     });
     return;
   }
@@ -511,12 +520,13 @@ __device__ __forceinline__ void export_row_global(const ExportDescDev& d, int64_
   const RowQuant q = row_params(d, t1, t2);
   if (lane == 0) d.scales[row] = __float2half_rn(q.s);
   if (d.pack6) {
-    uint8_t* out = reinterpret_cast<uint8_t*>(d.dst) + row * 3 * K4;
+    const RowQuant qs[1] = {q};
+    uint8_t* const out[1] = {reinterpret_cast<uint8_t*>(d.dst) + row * 3 * K4};
     with_grid(q.bits, true, [&](auto bits_tag, auto clip_tag) {
       constexpr int B = decltype(bits_tag)::value;
       if constexpr (B != 8)
-        quantize_row_pack6<B, decltype(clip_tag)::value>(
-            q, [&](int j) { return __ldg(r + j); }, K4, out, lane);
+        quantize_rows_pack6<B, decltype(clip_tag)::value, 1>(
+            qs, [&](int, int j) { return __ldg(r + j); }, K4, out, lane);
     });
     return;
   }
