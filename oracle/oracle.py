@@ -32,6 +32,8 @@ def _c():
         lib.oracle_qat_scales.argtypes = [P, I64, I64, P]
         lib.oracle_qat_scales_bits.argtypes = [P, I64, I64, ctypes.c_int, P]
         lib.oracle_pack6.argtypes = [P, I64, ctypes.c_int, P]
+        lib.oracle_export_rows_search.argtypes = [P, I64, I64, ctypes.c_int, P, ctypes.c_int,
+                                                  P, P, P, P, P]
         lib.oracle_unpack6.argtypes = [P, I64, ctypes.c_int, P]
         lib.oracle_qat_codes.argtypes = [P, I64, I64, P, ctypes.c_int, P]
         lib.oracle_qat_codes.restype = ctypes.c_int
@@ -296,6 +298,33 @@ def export_rows(W, bits, q=EXPORT_CLIP_Q):
     if rc != 0:
         raise ValueError("bits must be 5, 6 or 8")
     return c, s16, s32
+
+
+# Clip-search candidates (reading of "GPTQ-lite 裁剪搜索"; the pages give no
+# list): the row maximum, the export's own 99.99984 percentile, then four
+# tighter clips; the first of equal errors (the widest clip) is kept.
+CLIP_CANDIDATES = (1.0, 0.9999984, 0.99999, 0.9999, 0.9995, 0.999)
+
+
+def export_rows_search(W, bits, cand=CLIP_CANDIDATES):
+    """P4 leaderboard "GPTQ-lite 裁剪搜索" (undefined there): per row, export at
+    every candidate clip quantile and keep the one whose stored row (codes times
+    the fp16 scale) has the least squared error against w.  Returns codes,
+    fp16 scale bits, fp32 scales, the kept candidate index per row and the
+    errors [rows, len(cand)]."""
+    W = _f32(W)
+    rows, cols = W.shape
+    cd = np.ascontiguousarray(cand, np.float64)
+    c = np.empty((rows, cols), np.int8)
+    s16 = np.empty(rows, np.uint16)
+    s32 = np.empty(rows, np.float32)
+    ch = np.empty(rows, np.int32)
+    errs = np.empty((rows, cd.size), np.float64)
+    rc = _c().oracle_export_rows_search(_ptr(W), rows, cols, int(bits), _ptr(cd), cd.size,
+                                        _ptr(c), _ptr(s16), _ptr(s32), _ptr(ch), _ptr(errs))
+    if rc != 0:
+        raise ValueError("bits must be 5, 6 or 8")
+    return c, s16, s32, ch, errs
 
 
 def dequant_export(codes, scale16_bits):

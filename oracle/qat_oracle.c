@@ -226,27 +226,76 @@ float oracle_row_quantile_abs(const float* row, int64_t n, double qf) {
 /* Export one matrix: per row clip, fp32 scale s = max(clip,1e-12)/127,
  * codes of clamp(w, -clip, clip) with the same rounding as training,
  * stored scale fp16_rne(s).  scale32 may be NULL. */
+static void export_one_row(const float* r, int64_t cols, int bits, double qf, int8_t* codes,
+                           uint16_t* scale16, float* scale32) {
+  float clip = oracle_row_quantile_abs(r, cols, qf);
+  float c = clip < ORACLE_AMAX_FLOOR ? ORACLE_AMAX_FLOOR : clip;
+  float s = c / oracle_levels(bits);
+  for (int64_t j = 0; j < cols; ++j) {
+    float w = r[j];
+    if (w > clip) w = clip;
+    if (w < -clip) w = -clip;
+    codes[j] = (int8_t)oracle_code(w, s, bits);
+  }
+  *scale16 = oracle_fp16_rne(s);
+  *scale32 = s;
+}
+
 int oracle_export_rows(const float* W, int64_t rows, int64_t cols, int bits, double qf,
                        int8_t* codes, uint16_t* scale16, float* scale32) {
   if (bits != 5 && bits != 6 && bits != 8) return -1;
   for (int64_t i = 0; i < rows; ++i) {
-    const float* r = W + i * cols;
-    float clip = oracle_row_quantile_abs(r, cols, qf);
-    float c = clip < ORACLE_AMAX_FLOOR ? ORACLE_AMAX_FLOOR : clip;
-    float s = c / oracle_levels(bits);
-    for (int64_t j = 0; j < cols; ++j) {
-      float w = r[j];
-      if (w > clip) w = clip;
-      if (w < -clip) w = -clip;
-      codes[i * cols + j] = (int8_t)oracle_code(w, s, bits);
-    }
-    scale16[i] = oracle_fp16_rne(s);
-    if (scale32) scale32[i] = s;
+    float s32;
+    export_one_row(W + i * cols, cols, bits, qf, codes + i * cols, scale16 + i, &s32);
+    if (scale32) scale32[i] = s32;
   }
   return 0;
 }
 
-/* Roundtrip dequantize: fl32(c * fp32(scale16)). */
+/* Clip search of the export ("GPTQ-lite 裁剪搜索" of the parameter-golf
+ * leaderboard, record "11L EMA + GPTQ-lite + warmdown3500"; the pages name it
+ * without defining it).  Reading: per row, each candidate quantile q_k of
+ * `cand` (n_cand of them, in the order given) is exported exactly as above;
+ * its reconstruction error is E_k = sum_j (w_j - c_j * s16_k)^2, with s16_k
+ * the stored fp16 scale read back as fp32 -- what a dequantizing reader gets
+ * -- evaluated in double; the row keeps the first candidate of smallest
+ * E_k.  Outputs the kept codes and scales, the kept index and every E_k
+ * (errs [rows, n_cand]; nullable). */
+int oracle_export_rows_search(const float* W, int64_t rows, int64_t cols, int bits,
+                              const double* cand, int n_cand, int8_t* codes, uint16_t* scale16,
+                              float* scale32, int32_t* chosen, double* errs) {
+  if (bits != 5 && bits != 6 && bits != 8) return -1;
+  if (n_cand < 1) return -1;
+  int8_t* tmp = (int8_t*)malloc((size_t)cols);
+  for (int64_t i = 0; i < rows; ++i) {
+    const float* r = W + i * cols;
+    double best = 0.0;
+    int kbest = -1;
+    for (int k = 0; k < n_cand; ++k) {
+      uint16_t h;
+      float s32;
+      export_one_row(r, cols, bits, cand[k], tmp, &h, &s32);
+      const double sh = (double)oracle_fp16_to_f32(h);
+      double e = 0.0;
+      for (int64_t j = 0; j < cols; ++j) {
+        const double d = (double)r[j] - (double)tmp[j] * sh;
+        e += d * d;
+      }
+      if (errs) errs[i * n_cand + k] = e;
+      if (kbest < 0 || e < best) {
+        best = e;
+        kbest = k;
+        for (int64_t j = 0; j < cols; ++j) codes[i * cols + j] = tmp[j];
+        scale16[i] = h;
+        if (scale32) scale32[i] = s32;
+      }
+    }
+    if (chosen) chosen[i] = kbest;
+  }
+  free(tmp);
+  return 0;
+}
+
 /* 6-bit packing of int6 / int5 codes (the bit-packing of the depth-recurrence
  * write-up's Day 0 compression study, which puts int6 codes at about 2.94
  * bits of entropy each; the pages give no format).  Reading: each code
@@ -286,6 +335,7 @@ int oracle_unpack6(const uint8_t* in, int64_t n, int bits, int8_t* codes) {
   return 0;
 }
 
+/* Roundtrip dequantize: fl32(c * fp32(scale16)). */
 void oracle_dequant_export(const int8_t* codes, const uint16_t* scale16, int64_t rows,
                            int64_t cols, float* out) {
   for (int64_t i = 0; i < rows; ++i) {

@@ -336,6 +336,55 @@ def test_pack6_against_numpy_packbits_and_roundtrip(bits):
     assert np.array_equal(o.unpack6(o.pack6(ce, bits), ce.size, bits).reshape(ce.shape), ce)
 
 
+def _exact_err(w, c, s16):
+    from fractions import Fraction
+    sh = Fraction(float(np.uint16(s16).view(np.float16)))
+    return sum((Fraction(float(x)) - int(k) * sh) ** 2 for x, k in zip(w, c))
+
+
+@pytest.mark.parametrize("bits", [5, 6, 8])
+def test_clip_search_minimises_exact_error(bits):
+    """The clip search keeps, per row, the candidate whose stored row has the
+    least squared error, checked with exact rational arithmetic on codes and
+    scales produced by the plain export at each candidate quantile; the kept
+    codes and scale are that export's."""
+    sd = sy.state_dict_case(n_layers=1, seed=3)
+    W = np.concatenate([sd["blocks.0.mlp.fc.weight"][:6], sd["blocks.0.mlp.proj.weight"][:3, :512]])
+    W = np.ascontiguousarray(W)
+    c, s16, s32, ch, errs = o.export_rows_search(W, bits)
+    for i in range(W.shape[0]):
+        exact = []
+        for q in o.CLIP_CANDIDATES:
+            ck, hk, _ = o.export_rows(W[i:i + 1], bits, q=q)
+            exact.append(_exact_err(W[i], ck[0], hk[0]))
+        best = min(exact)
+        k = ch[i]
+        assert exact[k] == best or float(exact[k] - best) <= 1e-12 * float(best), (i, k)
+        assert all(e > exact[k] or j >= k for j, e in enumerate(exact) if e == exact[k])
+        for j, e in enumerate(exact):
+            assert abs(errs[i, j] - float(e)) <= 1e-9 * float(e) + 1e-30
+        ck, hk, sk = o.export_rows(W[i:i + 1], bits, q=o.CLIP_CANDIDATES[k])
+        assert np.array_equal(c[i], ck[0]) and s16[i] == hk[0] and s32[i] == sk[0]
+    assert np.all(errs[np.arange(len(ch)), ch] <= errs[:, 1])   # never worse than the plain export
+
+
+def test_clip_search_exact_row_and_outlier_row():
+    """A row already on the int8 grid with a power-of-two scale keeps the row
+    maximum at zero error; a row with one 10-sigma outlier gives up part of
+    it for a finer grid on the rest when the grid is coarse (int5: a tight
+    candidate wins by a wide margin)."""
+    on_grid = np.array([np.arange(-127, 129, 2)[:128]], np.float32)   # amax 127 -> s = 1
+    on_grid[0, 0] = 127.0
+    c, s16, _, ch, errs = o.export_rows_search(on_grid, 8)
+    assert ch[0] == 0 and errs[0, 0] == 0.0
+    assert np.array_equal(c[0].astype(np.float32), on_grid[0])
+    rng = np.random.default_rng(4)
+    row = (rng.standard_normal((1, 4096)) * 0.01).astype(np.float32)
+    row[0, 7] = 0.1
+    _, _, _, ch, errs = o.export_rows_search(row, 5)
+    assert ch[0] >= 3 and errs[0, ch[0]] < 0.5 * errs[0, 0]
+
+
 # ------------------------------------------------------------------ algebra
 
 def test_linear_fwd_brute_force():
