@@ -216,11 +216,20 @@ int quantize_rows_export(const float* W, int64_t rows, int64_t cols, int32_t bit
  * 6-bit packed (see unpack_codes6), rows*cols*3/4 bytes, row r at byte
  * r*cols*3/4 (the bit-packing of [P1] Day 0; the format is this library's:
  * one 6-bit two's-complement field per code, c/4 for int6 and c for int5,
- * field i at bits 6i..6i+5 of a little-endian bit stream).  Other flags, or
- * PACK6 with another mode, return QAT_ERR_ARG. */
+ * field i at bits 6i..6i+5 of a little-endian bit stream).
+ * QAT_EXPORT_CLIP_SEARCH (modes 5, 6, 8; may be combined with PACK6): instead
+ * of the fixed 99.99984 percentile, each row tries the clip quantiles
+ * q = 1.0, 0.9999984, 0.99999, 0.9999, 0.9995, 0.999 (in this order; each
+ * exported as above) and keeps the first whose stored row has the least
+ * squared error sum_j (w_j - c_j * fp32(scale_fp16))^2, computed in fp32 (the
+ * [P4] leaderboard's "GPTQ-lite" clip search, which the pages do not define;
+ * this is the library's reading).  Rows of more than 2048 columns return
+ * QAT_ERR_SHAPE.  Other flags, or PACK6 with another mode, return
+ * QAT_ERR_ARG. */
 #define QAT_EXPORT_FP16 16
 #define QAT_EXPORT_MAX_DESCS 256
 #define QAT_EXPORT_PACK6 1
+#define QAT_EXPORT_CLIP_SEARCH 2
 typedef struct qat_export_desc {
   const float* src;
   int64_t rows, cols;

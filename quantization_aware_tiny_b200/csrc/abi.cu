@@ -354,9 +354,13 @@ int quantize_export_batch(const qat_export_desc* descs, int32_t n, qat_stream_t 
     d.mode = s.mode;
     d.m = 1;
     d.frac = 0.0f;
-    if (s.flags & ~QAT_EXPORT_PACK6) return QAT_ERR_ARG;
+    if (s.flags & ~(QAT_EXPORT_PACK6 | QAT_EXPORT_CLIP_SEARCH)) return QAT_ERR_ARG;
     d.pack6 = (s.flags & QAT_EXPORT_PACK6) != 0;
+    d.search = (s.flags & QAT_EXPORT_CLIP_SEARCH) != 0;
+    d.pad = 0;
     if (d.pack6 && s.mode != 5 && s.mode != 6) return QAT_ERR_ARG;
+    if (d.search && !bits_ok(s.mode)) return QAT_ERR_ARG;
+    if (d.search && !clip_search_supported(s.cols)) return QAT_ERR_SHAPE;
     d.unit_begin = b.total_units;
     if (s.mode == QAT_EXPORT_FP16) {
       d.numel = s.rows * s.cols;

@@ -510,6 +510,153 @@ __device__ __forceinline__ void export_two_rows_smem(const ExportDescDev& d, int
   with_grid(qa.bits, clip, run);
 }
 
+// ---- clip search (the leaderboard's "GPTQ-lite" clip search, read as: per row,
+// export at each candidate quantile and keep the first candidate of least
+// squared error of the stored row, sum_j (w_j - c_j * fp16(s))^2).
+
+// The candidate quantiles, in search order (the same values on the host).
+__device__ __forceinline__ double clip_candidate(int k) {
+  switch (k) {
+    case 0: return 1.0;
+    case 1: return 0.9999984;
+    case 2: return 0.99999;
+    case 3: return 0.9999;
+    case 4: return 0.9995;
+    default: return 0.999;
+  }
+}
+
+// Running top-4 of |w| (with multiplicity), t[0] >= t[1] >= t[2] >= t[3].
+__device__ __forceinline__ void top4_push(float a, float (&t)[kClipSearchTop]) {
+#pragma unroll
+  for (int i = 0; i < kClipSearchTop; ++i) {
+    const float hi = fmaxf(a, t[i]);
+    a = fminf(a, t[i]);
+    t[i] = hi;
+  }
+}
+
+// The row's top four from the lanes' sorted lists: four rounds, each taking
+// the warp-wide largest head (values >= 0 order like their bit patterns) and
+// popping it from one lane that holds it.
+__device__ __forceinline__ void top4_warp(float (&t)[kClipSearchTop], float (&top)[kClipSearchTop],
+                                          int lane) {
+#pragma unroll
+  for (int r = 0; r < kClipSearchTop; ++r) {
+    const uint32_t m = __reduce_max_sync(0xffffffffu, __float_as_uint(t[0]));
+    const uint32_t holders = __ballot_sync(0xffffffffu, __float_as_uint(t[0]) == m);
+    if (lane == __ffs(holders) - 1) {
+#pragma unroll
+      for (int i = 0; i + 1 < kClipSearchTop; ++i) t[i] = t[i + 1];
+      t[kClipSearchTop - 1] = 0.0f;
+    }
+    top[r] = __uint_as_float(m);
+  }
+}
+
+__device__ __forceinline__ float top_at(const float (&top)[kClipSearchTop], int64_t k) {
+  return k == 0 ? top[0] : k == 1 ? top[1] : k == 2 ? top[2] : top[3];
+}
+
+// Grid parameters of candidate k for a row of n entries with top four `top`:
+// the quantile as in quantize_rows_export (pos = q (n - 1) in double, linear
+// interpolation in three fp32 roundings), then the row's scales.
+__device__ __forceinline__ RowQuant candidate_params(const float (&top)[kClipSearchTop], int64_t n,
+                                                     int k, int bits) {
+  const double pos = clip_candidate(k) * static_cast<double>(n - 1);
+  int64_t lo = static_cast<int64_t>(floor(pos));
+  lo = lo < 0 ? 0 : (lo > n - 1 ? n - 1 : lo);
+  const int64_t hi = lo + 1 < n ? lo + 1 : lo;
+  const float frac = static_cast<float>(pos - static_cast<double>(lo));
+  const float v_lo = top_at(top, n - 1 - lo), v_hi = top_at(top, n - 1 - hi);
+  RowQuant q;
+  q.clip = __fadd_rn(v_lo, __fmul_rn(frac, __fsub_rn(v_hi, v_lo)));
+  q.s = bits == 5 ? div_by_scale(fmaxf(q.clip, 1e-12f), 15.0f, kRcp15)
+                  : div_by_scale(fmaxf(q.clip, 1e-12f), 127.0f, kRcp127);
+  q.rs = __frcp_rn(q.s);
+  q.bits = bits;
+  return q;
+}
+
+// Squared error of four weights against their codes times the stored scale sh.
+template <int BITS>
+__device__ __forceinline__ float sq_err4(const RowQuant& q, float sh, float4 v, float e) {
+  int c0, c1, c2, c3;
+  codes2<BITS, true>(q, v.x, v.y, c0, c1);
+  codes2<BITS, true>(q, v.z, v.w, c2, c3);
+  const float d0 = __fmaf_rn(-static_cast<float>(c0), sh, v.x);
+  const float d1 = __fmaf_rn(-static_cast<float>(c1), sh, v.y);
+  const float d2 = __fmaf_rn(-static_cast<float>(c2), sh, v.z);
+  const float d3 = __fmaf_rn(-static_cast<float>(c3), sh, v.w);
+  e = __fmaf_rn(d0, d0, e);
+  e = __fmaf_rn(d1, d1, e);
+  e = __fmaf_rn(d2, d2, e);
+  return __fmaf_rn(d3, d3, e);
+}
+
+// One staged row under the clip search: top four of |w|, the candidates'
+// errors in one pass (fp32, per-lane sums reduced by a butterfly so every
+// lane holds the same totals and takes the same decision), then the row
+// quantized with the kept candidate.
+template <int BITS>
+__device__ __forceinline__ void export_row_search_t(const ExportDescDev& d, int64_t row,
+                                                    const float4* buf, int lane) {
+  const int K4 = static_cast<int>(d.cols >> 2);
+  float t[kClipSearchTop] = {0.0f, 0.0f, 0.0f, 0.0f};
+  for (int j = lane; j < K4; j += 32) {
+    const float4 v = buf[j];
+    top4_push(fabsf(v.x), t);
+    top4_push(fabsf(v.y), t);
+    top4_push(fabsf(v.z), t);
+    top4_push(fabsf(v.w), t);
+  }
+  float top[kClipSearchTop];
+  top4_warp(t, top, lane);
+  RowQuant q[kClipCandidates];
+  float sh[kClipCandidates], e[kClipCandidates];
+#pragma unroll
+  for (int k = 0; k < kClipCandidates; ++k) {
+    q[k] = candidate_params(top, d.cols, k, BITS);
+    sh[k] = __half2float(__float2half_rn(q[k].s));
+    e[k] = 0.0f;
+  }
+  for (int j = lane; j < K4; j += 32) {
+    const float4 v = buf[j];
+#pragma unroll
+    for (int k = 0; k < kClipCandidates; ++k) e[k] = sq_err4<BITS>(q[k], sh[k], v, e[k]);
+  }
+  int best = 0;
+  float best_e = 0.0f;
+#pragma unroll
+  for (int k = 0; k < kClipCandidates; ++k) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) e[k] += __shfl_xor_sync(0xffffffffu, e[k], o);
+    if (k == 0 || e[k] < best_e) {
+      best_e = e[k];
+      best = k;
+    }
+  }
+  const RowQuant qb = candidate_params(top, d.cols, best, BITS);
+  if (lane == 0) d.scales[row] = __float2half_rn(qb.s);
+  if (d.pack6) {
+    if constexpr (BITS != 8) {
+      const RowQuant qs[1] = {qb};
+      uint8_t* const out[1] = {reinterpret_cast<uint8_t*>(d.dst) + row * 3 * K4};
+      quantize_rows_pack6<BITS, true, 1>(qs, [&](int, int j) { return buf[j]; }, K4, out, lane);
+    }
+    return;
+  }
+  uint32_t* out = reinterpret_cast<uint32_t*>(reinterpret_cast<int8_t*>(d.dst) + row * d.cols);
+  quantize_smem_row<BITS, true>(qb, buf, K4, out, lane);
+}
+
+__device__ __forceinline__ void export_row_search(const ExportDescDev& d, int64_t row,
+                                                  const float4* buf, int lane) {
+  if (d.mode == 6) export_row_search_t<6>(d, row, buf, lane);
+  else if (d.mode == 5) export_row_search_t<5>(d, row, buf, lane);
+  else export_row_search_t<8>(d, row, buf, lane);
+}
+
 // A quantized row read from global memory (rows longer than the staging buffer).
 __device__ __forceinline__ void export_row_global(const ExportDescDev& d, int64_t row, int lane) {
   const int K4 = static_cast<int>(d.cols >> 2);
@@ -621,6 +768,7 @@ __device__ __forceinline__ UnitPos unit_at(const ExportBatch& b, int64_t u) {
 // arrives in one bulk copy into one of the warp's kExportBufs buffers while
 // the warp quantizes the previous one.  Units that are not staged still arrive once on their buffer's
 // mbarrier so every buffer's phases stay in step with the unit count.
+template <bool SEARCH>
 __global__ void __launch_bounds__(kExportMaxWarps * 32, 1)
     export_batch_kernel(const __grid_constant__ ExportBatch b, int* err) {
   extern __shared__ __align__(128) uint8_t xsmem[];
@@ -674,9 +822,13 @@ __global__ void __launch_bounds__(kExportMaxWarps * 32, 1)
       const int K4 = static_cast<int>(d.cols >> 2);
       const float4* ub = bufs + slot * stride;
       int r = 0;
-      for (; r + 1 < pos[0].nrows; r += 2)
-        export_two_rows_smem(d, pos[0].row0 + r, ub + r * K4, ub + (r + 1) * K4, lane);
-      if (r < pos[0].nrows) export_row_smem(d, pos[0].row0 + r, ub + r * K4, lane);
+      if (SEARCH && d.search) {
+        for (; r < pos[0].nrows; ++r) export_row_search(d, pos[0].row0 + r, ub + r * K4, lane);
+      } else {
+        for (; r + 1 < pos[0].nrows; r += 2)
+          export_two_rows_smem(d, pos[0].row0 + r, ub + r * K4, ub + (r + 1) * K4, lane);
+        if (r < pos[0].nrows) export_row_smem(d, pos[0].row0 + r, ub + r * K4, lane);
+      }
     } else {
       export_row_global(d, pos[0].row0, lane);
     }
@@ -791,11 +943,28 @@ int export_quantile_params(int64_t cols, int* m, float* frac) {
   return QAT_OK;
 }
 
+// Whether the clip search covers rows of `cols` entries: the row is staged in
+// shared memory and every candidate's quantile needs only the top four order
+// statistics (the same double arithmetic as the kernel's).
+int clip_search_supported(int64_t cols) {
+  if (cols < 2 || cols > kExportMaxStagedCols) return 0;
+  static const double cand[kClipCandidates] = {1.0, 0.9999984, 0.99999, 0.9999, 0.9995, 0.999};
+  for (int k = 0; k < kClipCandidates; ++k) {
+    const int64_t lo = static_cast<int64_t>(std::floor(cand[k] * static_cast<double>(cols - 1)));
+    if (cols - 1 - lo > kClipSearchTop - 1) return 0;
+  }
+  return 1;
+}
+
 int launch_export_batch(ExportBatch& b, cudaStream_t s) {
   if (b.total_units == 0) return QAT_OK;
   static bool attr_done = false;
   if (!attr_done) {
-    if (cudaFuncSetAttribute(export_batch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(export_batch_kernel<false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kExportSmemBudget) != cudaSuccess ||
+        cudaFuncSetAttribute(export_batch_kernel<true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kExportSmemBudget) != cudaSuccess)
       return QAT_ERR_CUDA;
     attr_done = true;
@@ -810,7 +979,13 @@ int launch_export_batch(ExportBatch& b, cudaStream_t s) {
   const int smem = warps * per_warp;
   const int64_t want = (b.total_units + warps - 1) / warps;
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, sm_count())));
-  export_batch_kernel<<<grid, warps * 32, smem, s>>>(b, device_error_ptr());
+  bool search = false;
+  for (int i = 0; i < b.n; ++i) search = search || b.d[i].search;
+  // the search's registers stay out of the plain export kernel
+  if (search)
+    export_batch_kernel<true><<<grid, warps * 32, smem, s>>>(b, device_error_ptr());
+  else
+    export_batch_kernel<false><<<grid, warps * 32, smem, s>>>(b, device_error_ptr());
   count_launch();
   return cuda_status(cudaGetLastError());
 }

@@ -19,7 +19,15 @@ struct ExportDescDev {
   int m;              // quantile order statistic from the top (1 or 2)
   float frac;         // quantile interpolation fraction
   int pack6;          // codes stored as 6-bit fields, 4 codes in 3 bytes
+  int search;         // per-row clip search over kClipCandidates
+  int pad;
 };
+
+// Clip-search candidates (quantiles of |w|): the row maximum, the export's
+// 99.99984 percentile, then four tighter clips.  Only the top four order
+// statistics of a row are needed for rows of up to kExportMaxStagedCols.
+constexpr int kClipCandidates = 6;
+constexpr int kClipSearchTop = 4;
 
 #ifndef QAT_EXPORT_BATCH_CAP
 #define QAT_EXPORT_BATCH_CAP QAT_EXPORT_MAX_DESCS
@@ -52,6 +60,7 @@ int launch_quantize_weights(const float* W, int N, int K, int bits, int8_t* code
 int launch_noisy_operand(const float* W, int N, int K, int bits, uint64_t seed, uint64_t offset,
                          float* scales, __nv_bfloat16* operand, cudaStream_t s);
 int export_quantile_params(int64_t cols, int* m, float* frac);
+int clip_search_supported(int64_t cols);
 int launch_export_batch(ExportBatch& b, cudaStream_t s);
 int launch_dequant(const int8_t* codes, const __half* scales, int64_t rows, int64_t cols,
                    int out_bf16, void* out, cudaStream_t s);

@@ -48,12 +48,15 @@ def plan(state_dict, int6_range=(0, 10), embed_name="tok_emb.weight", mlp_int5=F
 
 
 def export_state_dict(state_dict, int6_range=(0, 10), embed_name="tok_emb.weight", stream=None,
-                      mlp_int5=False, attn_int5=False, pack6=False):
+                      mlp_int5=False, attn_int5=False, pack6=False, clip_search=False):
     """Quantize a dict of fp32 CUDA tensors.  Returns name -> dict with
     kind 'int5'/'int6'/'int8' (codes int8 [rows,cols], scale16 fp16 [rows]) or
     kind 'fp16' (values fp16, original shape).  With pack6, int5 / int6 tensors
     hold 'packed' (uint8 [rows, cols*3/4], the 6-bit packed codes; see
-    qat.unpack_codes6) in place of 'codes'.  Launches in chunks of at most
+    qat.unpack_codes6) in place of 'codes'.  clip_search: every quantized row
+    keeps the clip quantile of least reconstruction error among the library's
+    candidates (the leaderboard's "GPTQ-lite" clip search, read as a data-free
+    per-row search).  Launches in chunks of at most
     QAT_EXPORT_MAX_DESCS descriptors (one launch for a state dict that fits)."""
     out = {}
     descs = []
@@ -68,14 +71,15 @@ def export_state_dict(state_dict, int6_range=(0, 10), embed_name="tok_emb.weight
         else:
             rows, cols = t.shape
             s = torch.empty(rows, dtype=torch.float16, device=t.device)
+            flags = qat.QAT_EXPORT_CLIP_SEARCH if clip_search else 0
             if pack6 and mode in (5, 6):
                 p = torch.empty((rows, cols * 3 // 4), dtype=torch.uint8, device=t.device)
                 out[name] = {"kind": "int%d" % mode, "packed": p, "scale16": s}
-                descs.append((t, mode, p, s, qat.QAT_EXPORT_PACK6))
+                descs.append((t, mode, p, s, flags | qat.QAT_EXPORT_PACK6))
             else:
                 c = torch.empty((rows, cols), dtype=torch.int8, device=t.device)
                 out[name] = {"kind": "int%d" % mode, "codes": c, "scale16": s}
-                descs.append((t, mode, c, s))
+                descs.append((t, mode, c, s, flags))
     for i in range(0, len(descs), qat.QAT_EXPORT_MAX_DESCS):
         qat.quantize_export_batch(descs[i:i + qat.QAT_EXPORT_MAX_DESCS], stream=stream)
     return out

@@ -28,6 +28,7 @@ EXPORTED = ("qat_strerror", "qat_launch_count", "qat_device_error", "qat_quantiz
             "qat_mlp_bwd", "quantize_rows_export", "quantize_export_batch", "dequantize_rows",
             "qat_linear_fwd_noalloc", "qat_noisy_operand", "unpack_codes6")
 QAT_EXPORT_PACK6 = 1
+QAT_EXPORT_CLIP_SEARCH = 2
 QAT_ACT_RELU2 = 0
 QAT_ACT_LEAKY_RELU2 = 1
 _ACTS = {"relu2": QAT_ACT_RELU2, "leaky2": QAT_ACT_LEAKY_RELU2}
@@ -245,9 +246,9 @@ def export_descs(descs):
 
 def quantize_export_batch(descs, stream=None):
     """descs: list of (src, mode, dst, scales[, flags]) with src a 2-D (or flat)
-    fp32 device tensor, mode 5 / 6 / 8 / QAT_EXPORT_FP16, flags 0 or
-    QAT_EXPORT_PACK6 -- or an array from export_descs() (the tensors it points
-    to must stay alive)."""
+    fp32 device tensor, mode 5 / 6 / 8 / QAT_EXPORT_FP16, flags 0 or an OR of
+    QAT_EXPORT_PACK6 / QAT_EXPORT_CLIP_SEARCH -- or an array from export_descs()
+    (the tensors it points to must stay alive)."""
     arr = descs if isinstance(descs, ctypes.Array) else export_descs(descs)
     _check(lib().quantize_export_batch(arr, len(arr), _stream(stream)), "quantize_export_batch")
 

@@ -151,6 +151,59 @@ def test_export_state_dict_pack6_one_launch():
     assert {"int5", "int6", "int8", "fp16"} <= kinds
 
 
+def _search_check(W, bits, codes, s16, rows_ok=1.0):
+    """Rows whose kept candidate matches the oracle's are bit-exact; a row may
+    keep another candidate only where the two candidates' errors tie to fp32
+    summation accuracy (1e-5 relative), and then holds exactly that
+    candidate's export."""
+    c_ref, s_ref, _, ch, errs = o.export_rows_search(W, bits)
+    same = (codes == c_ref).all(axis=1) & (s16 == s_ref)
+    for i in np.nonzero(~same)[0]:
+        alt = [k for k, q in enumerate(o.CLIP_CANDIDATES)
+               if (lambda r: np.array_equal(r[0][0], codes[i]) and r[1][0] == s16[i])(
+                   o.export_rows(W[i:i + 1], bits, q=q))]
+        assert alt, "row %d: not the export of any candidate" % i
+        assert min(abs(errs[i, k] - errs[i, ch[i]]) for k in alt) <= 1e-5 * errs[i, ch[i]], i
+    assert same.mean() >= rows_ok
+    return ch
+
+
+@pytest.mark.parametrize("bits", [5, 6, 8])
+def test_export_clip_search(bits):
+    """Clip search on heavy-tailed rows of 512 and 1536 columns, a ragged
+    136-column matrix and degenerate rows: bit-exact against the oracle's
+    search (see _search_check for near-ties)."""
+    sd = sy.state_dict_case(n_layers=1, seed=3)
+    rng = np.random.default_rng(12)
+    cases = [sd["blocks.0.mlp.fc.weight"], sd["blocks.0.mlp.proj.weight"],
+             (rng.standard_normal((200, 136)) * 0.02).astype(np.float32), _weights()["degenerate_8x64"]]
+    chosen = []
+    for W in cases:
+        rows, cols = W.shape
+        codes = torch.empty((rows, cols), dtype=torch.int8, device="cuda")
+        s16 = torch.empty(rows, dtype=torch.float16, device="cuda")
+        qat.quantize_export_batch([(_dev(W), bits, codes, s16, qat.QAT_EXPORT_CLIP_SEARCH)])
+        torch.cuda.synchronize()
+        chosen.append(_search_check(W, bits, codes.cpu().numpy(), bits16(s16), rows_ok=0.99))
+    assert len(np.unique(np.concatenate(chosen))) >= 4   # the search is not a no-op
+    assert qat.device_error() == 0
+
+
+def test_export_state_dict_clip_search_packed():
+    """A whole state dict with clip search and 6-bit packing in one launch."""
+    sd = sy.state_dict_case(n_layers=2, seed=6)
+    out = qexport.export_state_dict({k: _dev(v) for k, v in sd.items()}, pack6=True,
+                                    clip_search=True)
+    torch.cuda.synchronize()
+    for k, r in o.export_state_dict(sd).items():
+        g = out[k]
+        if r["kind"] == "int6":
+            codes = o.unpack6(g["packed"].cpu().numpy(), sd[k].size, 6).reshape(sd[k].shape)
+            _search_check(sd[k], 6, codes, bits16(g["scale16"]), rows_ok=0.99)
+        elif r["kind"] == "int8":
+            _search_check(sd[k], 8, g["codes"].cpu().numpy(), bits16(g["scale16"]), rows_ok=0.99)
+
+
 def test_dequantize_rows_bit_exact():
     sd = sy.state_dict_case(n_layers=1)
     for name in ("blocks.0.mlp.fc.weight", "blocks.0.attn.c_k.weight"):

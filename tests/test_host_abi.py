@@ -77,10 +77,18 @@ def test_argument_validation_before_launch(L):
     assert L.dequantize_rows(A16, A16, 4, 12, 0, A16, None) == qat.QAT_ERR_SHAPE
     # 6-bit packing: only int5 / int6, unknown flags refused, n a multiple of 8
     bad = (qat._ExportDesc * 3)(qat._ExportDesc(0x10000, 4, 512, 8, qat.QAT_EXPORT_PACK6, 0x10000, 0x10000),
-                                qat._ExportDesc(0x10000, 4, 512, 6, 2, 0x10000, 0x10000),
+                                qat._ExportDesc(0x10000, 4, 512, 6, 8, 0x10000, 0x10000),
                                 qat._ExportDesc(0x10000, 4, 512, qat.QAT_EXPORT_FP16, 1, 0x10000, 0))
     for i in range(3):
         assert L.quantize_export_batch(ctypes.byref(bad[i]), 1, None) == qat.QAT_ERR_ARG
+    # clip search: not for fp16 passthrough, rows of at most 2048 columns, unknown flag 4
+    srch = (qat._ExportDesc * 3)(
+        qat._ExportDesc(0x10000, 4, 512, qat.QAT_EXPORT_FP16, qat.QAT_EXPORT_CLIP_SEARCH, 0x10000, 0),
+        qat._ExportDesc(0x10000, 4, 4096, 6, qat.QAT_EXPORT_CLIP_SEARCH, 0x10000, 0x10000),
+        qat._ExportDesc(0x10000, 4, 512, 6, 4, 0x10000, 0x10000))
+    assert L.quantize_export_batch(ctypes.byref(srch[0]), 1, None) == qat.QAT_ERR_ARG
+    assert L.quantize_export_batch(ctypes.byref(srch[1]), 1, None) == qat.QAT_ERR_SHAPE
+    assert L.quantize_export_batch(ctypes.byref(srch[2]), 1, None) == qat.QAT_ERR_ARG
     assert L.unpack_codes6(A16, 12, 6, A16, None) == qat.QAT_ERR_SHAPE
     assert L.unpack_codes6(A16, 16, 8, A16, None) == qat.QAT_ERR_ARG
     assert L.unpack_codes6(A_BAD, 16, 6, A16, None) == qat.QAT_ERR_ALIGN
