@@ -4,10 +4,12 @@
 //                 128B-swizzled A/B tiles in shared memory
 //   warp 1      : TMEM allocator + MMA issuer (one lane issues tcgen05.mma,
 //                 128 x BN x 16 per instruction, fp32 accumulator in TMEM)
-//   warps 2..5  : epilogue; warp w reads TMEM lanes 32*(w%4)..+31 (its rows)
-//                 32 columns at a time, applies the fused epilogue, writes the
-//                 32x32 chunk into swizzled shared memory and hands it to a TMA
-//                 bulk tensor store (or fp32 reduce-add), double-buffered
+//   warps 2..   : epilogue, 8 warps for bf16 outputs (4 for fp32); warp w
+//                 reads TMEM lanes 32*(w%4)..+31 (its rows) -- two warps share
+//                 a lane quarter and take alternate 32-column chunks -- applies
+//                 the fused epilogue, writes the 32x32 chunk into swizzled
+//                 shared memory and hands it to a TMA bulk tensor store (or
+//                 fp32 reduce-add), double-buffered
 //
 // Two accumulator buffers in TMEM (2*BN columns) let the epilogue of tile i
 // overlap the main loop of tile i+1.  Tiles are 128 x BN x 64; split-K (for
@@ -24,29 +26,39 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int kThreads = 192;
 
 // PAIR: the CTA pair of a 2-CTA cluster computes a 256 x BN tile with
 // tcgen05 cta_group::2; each CTA stages 128 rows of A and BN/2 rows of B.
-// HAS_R: the epilogue reads a bf16 tensor of the output's shape (residual or
-// saved pre-activation), brought in by TMA ahead of use.
-template <int BN, bool PAIR, bool HAS_R = false>
+// Epilogues that read a bf16 tensor of the output's shape (residual or saved
+// pre-activation) bring it in by TMA ahead of use (R).  bf16-output epilogues
+// run 8 warps (their HBM traffic per FLOP is high: a lone warp per lane
+// quarter left the tensor pipe idle), the fp32 split-K ones 4.
+template <int BN, bool PAIR, int EPI>
 struct Cfg {
+  static constexpr bool F32 = (EPI == EPI_F32 || EPI == EPI_F32_ATOMIC);
+  static constexpr bool HAS_R = epi_reads_r(EPI);
+  static constexpr int EW = F32 ? 4 : 8;              // epilogue warps
+  static constexpr int THREADS = 64 + 32 * EW;
   static constexpr int B_ROWS = PAIR ? BN / 2 : BN;  // B rows staged by one CTA
   static constexpr int TILE_M = PAIR ? 2 * BM : BM;
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TMEM_COLS = (2 * BN <= 256) ? 256 : 512;  // a power of two >= 2*BN
-  static constexpr int STAGING_BYTES = 4 * 8192;  // per epilogue warp: 8 KB of output chunks
-  static constexpr int R_BUFS = 4;                // R chunks in flight per epilogue warp
-  static constexpr int R_BYTES = HAS_R ? 4 * R_BUFS * 2048 : 0;
+  // per epilogue warp: two buffers of one or two 32x32 output chunks
+  static constexpr int WBUF = (F32 || epi_act_fwd(EPI)) ? 8192 : 4096;
+  static constexpr int STAGING_BYTES = EW * WBUF;
+  static constexpr int R_BUFS = EW == 8 ? 2 : 4;  // R chunks in flight per epilogue warp
+  static constexpr int R_BYTES = HAS_R ? EW * R_BUFS * 2048 : 0;
   static constexpr int BAR_BYTES = 512;
   static constexpr int FIXED = STAGING_BYTES + R_BYTES + BAR_BYTES + 1024;
   static constexpr int STAGES_FIT = (232448 - FIXED) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + FIXED;
   static_assert(STAGES >= 3, "pipeline too shallow");
+  // barriers (full/empty per stage, tfull/tempty x2, mma_done, R ring per
+  // epilogue warp) followed by tmem_slot, abort flag and two ring positions
+  static_assert((2 * STAGES + 5 + EW * R_BUFS) * 8 + 16 <= BAR_BYTES, "barrier block overflow");
 };
 
 struct KArgs {
@@ -129,11 +141,11 @@ __device__ __forceinline__ void stage_chunk(const KArgs& p, const uint32_t (&acc
 }
 
 template <int BN, bool A_MN, bool B_MN, int EPI, bool PAIR>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<BN, PAIR, EPI>::THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmD, const __grid_constant__ CUtensorMap tmD2,
                 const __grid_constant__ CUtensorMap tmR, const KArgs p) {
-  using C = Cfg<BN, PAIR, epi_reads_r(EPI)>;
+  using C = Cfg<BN, PAIR, EPI>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -146,8 +158,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* tfull = empty + C::STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* mma_done = tempty + 2;
-  uint64_t* rbar = mma_done + 1;  // 4 epilogue warps x R_BUFS
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rbar + 4 * C::R_BUFS);
+  uint64_t* rbar = mma_done + 1;  // EW epilogue warps x R_BUFS
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rbar + C::EW * C::R_BUFS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* prod_pos = const_cast<int*>(abort_flag) + 1;  // producer ring position at exit
   int* mma_pos = prod_pos + 1;                        // MMA ring position at exit
@@ -168,10 +180,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], PAIR ? 8 : 4);
+      mbar_init(&tempty[b], PAIR ? 2 * C::EW : C::EW);
     }
     mbar_init(mma_done, 1);
-    for (int i = 0; i < 4 * C::R_BUFS; ++i) mbar_init(&rbar[i], 1);
+    for (int i = 0; i < C::EW * C::R_BUFS; ++i) mbar_init(&rbar[i], 1);
     *abort_flag = 0;
     *prod_pos = 0;
     *mma_pos = 0;
@@ -308,13 +320,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       *mma_pos = pos;
     }
   } else {
-    // ------------------------------------------------ epilogue (warps 2..5)
-    constexpr bool kF32 = (EPI == EPI_F32 || EPI == EPI_F32_ATOMIC);
-    constexpr bool kR = epi_reads_r(EPI);
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
-    const uint32_t wbuf = smem_u32(staging) + static_cast<uint32_t>(q) * 8192u;
-    uint8_t* rbuf = rstage + q * C::R_BUFS * 2048;
-    uint64_t* rb = rbar + q * C::R_BUFS;
+    // ------------------------------------------------ epilogue (warps 2..)
+    constexpr bool kF32 = C::F32;
+    constexpr bool kR = C::HAS_R;
+    constexpr int kSplit = C::EW / 4;  // warps sharing one TMEM lane quarter
+    const int q = warp & 3;            // TMEM lane quarter this warp may access
+    const int ew = warp - 2;           // epilogue warp index
+    const int h = ew >> 2;             // this warp's chunks: h, h + kSplit, ...
+    const uint32_t wbuf = smem_u32(staging) + static_cast<uint32_t>(ew * C::WBUF);
+    uint8_t* rbuf = rstage + ew * C::R_BUFS * 2048;
+    uint64_t* rb = rbar + ew * C::R_BUFS;
     const bool keep_pre = epi_act_fwd(EPI) && p.D != nullptr;
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -328,25 +343,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row0 = mb * C::TILE_M + static_cast<int>(rank) * BM + q * 32;
       const int ncols = min(BN, p.N - nb * BN);
       const int nchunks = (ncols + 31) / 32;
-      // Request this tile's first R chunks before waiting for the accumulator.
-      auto issue_r = [&](int c) {
+      const int mine = nchunks > h ? (nchunks - h + kSplit - 1) / kSplit : 0;
+      // Request this warp's first R chunks before waiting for the accumulator.
+      auto issue_r = [&](int i) {
         if (lane == 0) {
           const uint32_t slot = r_issued % C::R_BUFS;
           mbar_arrive_expect_tx(&rb[slot], 2048);
-          tma_load_2d(&tmR, &rb[slot], rbuf + slot * 2048, nb * BN + c * 32, row0);
+          tma_load_2d(&tmR, &rb[slot], rbuf + slot * 2048, nb * BN + (h + i * kSplit) * 32, row0);
         }
         ++r_issued;
       };
       if constexpr (kR) {
-        for (int c = 0; c < nchunks && c < C::R_BUFS; ++c) issue_r(c);
+        for (int i = 0; i < mine && i < C::R_BUFS; ++i) issue_r(i);
       }
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
+      auto release_acc = [&]() {  // this warp's part of the accumulator is read
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (PAIR) mbar_arrive_cluster(tempty_leader + 8u * static_cast<uint32_t>(acc));
+          else mbar_arrive(&tempty[acc]);
+        }
+      };
+      if (mine == 0) release_acc();
       bool ok = true;
 #pragma unroll 1
-      for (int c = 0; c < nchunks; ++c, ++chunk) {
+      for (int i = 0; i < mine; ++i, ++chunk) {
+        const int c = h + i * kSplit;
         const int col0 = nb * BN + c * 32;
         uint4 rin[4] = {};
         if constexpr (kR) {
@@ -359,19 +385,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++r_used;
           fence_proxy_async_smem();  // reads done before the slot is refilled by TMA
           __syncwarp();
-          if (c + C::R_BUFS < nchunks) issue_r(c + C::R_BUFS);
+          if (i + C::R_BUFS < mine) issue_r(i + C::R_BUFS);
         }
         uint32_t r[32];
         tmem_ld32(t_row + static_cast<uint32_t>(c * 32), r);
         tmem_ld_wait();
-        if (c == nchunks - 1) {  // accumulator fully read: hand it back to the MMA
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) {
-            if constexpr (PAIR) mbar_arrive_cluster(tempty_leader + 8u * static_cast<uint32_t>(acc));
-            else mbar_arrive(&tempty[acc]);
-          }
-        }
+        if (i == mine - 1) release_acc();  // hand the accumulator back to the MMA
         const uint32_t b = chunk & 1u;
         const uint32_t buf0 = kF32 ? wbuf + b * 4096u : wbuf + b * 2048u;
         const uint32_t buf1 = wbuf + 4096u + b * 2048u;
@@ -486,7 +505,7 @@ int make_out_map(CUtensorMap* m, const void* base, int64_t inner, int64_t outer,
 template <int BN, bool A_MN, bool B_MN, int EPI, bool PAIR>
 int launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& md,
              const CUtensorMap& md2, const CUtensorMap& mr, const KArgs& a, cudaStream_t s) {
-  using C = Cfg<BN, PAIR, epi_reads_r(EPI)>;
+  using C = Cfg<BN, PAIR, EPI>;
   auto kern = gemm_kernel<BN, A_MN, B_MN, EPI, PAIR>;
   static bool attr_done = false;  // per instantiation; set before first launch
   if (!attr_done) {
@@ -499,7 +518,7 @@ int launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& md
   const int grid = std::max(1, std::min(a.num_tiles, units)) * (PAIR ? 2 : 1);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(C::THREADS);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -529,31 +548,32 @@ int dispatch_bn(const GemmDesc& g, const CUtensorMap& ma, const CUtensorMap& mb,
         return launch_t<BN, false, false, EPI_LRELU2, PAIR>(ma, mb, md, md2, mr, a, s);
       default: return QAT_ERR_ARG;
     }
-  }
-  if (!g.a_mn && !g.b_mn) {
-    switch (epi) {
-      case EPI_BF16: return launch_t<BN, false, false, EPI_BF16, PAIR>(ma, mb, md, md2, mr, a, s);
-      case EPI_BF16_RESID:
-        return launch_t<BN, false, false, EPI_BF16_RESID, PAIR>(ma, mb, md, md2, mr, a, s);
-      case EPI_RELU2: return launch_t<BN, false, false, EPI_RELU2, PAIR>(ma, mb, md, md2, mr, a, s);
-      case EPI_LRELU2:
-        return launch_t<BN, false, false, EPI_LRELU2, PAIR>(ma, mb, md, md2, mr, a, s);
-      default: break;
-    }
-  } else if (!g.a_mn && g.b_mn) {
-    switch (epi) {
-      case EPI_BF16: return launch_t<BN, false, true, EPI_BF16, PAIR>(ma, mb, md, md2, mr, a, s);
-      case EPI_DRELU2: return launch_t<BN, false, true, EPI_DRELU2, PAIR>(ma, mb, md, md2, mr, a, s);
-      case EPI_DLRELU2:
-        return launch_t<BN, false, true, EPI_DLRELU2, PAIR>(ma, mb, md, md2, mr, a, s);
-      default: break;
-    }
-  } else if (g.a_mn && g.b_mn) {
-    switch (epi) {
-      case EPI_F32: return launch_t<BN, true, true, EPI_F32, PAIR>(ma, mb, md, md2, mr, a, s);
-      case EPI_F32_ATOMIC:
-        return launch_t<BN, true, true, EPI_F32_ATOMIC, PAIR>(ma, mb, md, md2, mr, a, s);
-      default: break;
+  } else {
+    if (!g.a_mn && !g.b_mn) {
+      switch (epi) {
+        case EPI_BF16: return launch_t<BN, false, false, EPI_BF16, PAIR>(ma, mb, md, md2, mr, a, s);
+        case EPI_BF16_RESID:
+          return launch_t<BN, false, false, EPI_BF16_RESID, PAIR>(ma, mb, md, md2, mr, a, s);
+        case EPI_RELU2: return launch_t<BN, false, false, EPI_RELU2, PAIR>(ma, mb, md, md2, mr, a, s);
+        case EPI_LRELU2:
+          return launch_t<BN, false, false, EPI_LRELU2, PAIR>(ma, mb, md, md2, mr, a, s);
+        default: break;
+      }
+    } else if (!g.a_mn && g.b_mn) {
+      switch (epi) {
+        case EPI_BF16: return launch_t<BN, false, true, EPI_BF16, PAIR>(ma, mb, md, md2, mr, a, s);
+        case EPI_DRELU2: return launch_t<BN, false, true, EPI_DRELU2, PAIR>(ma, mb, md, md2, mr, a, s);
+        case EPI_DLRELU2:
+          return launch_t<BN, false, true, EPI_DLRELU2, PAIR>(ma, mb, md, md2, mr, a, s);
+        default: break;
+      }
+    } else if (g.a_mn && g.b_mn) {
+      switch (epi) {
+        case EPI_F32: return launch_t<BN, true, true, EPI_F32, PAIR>(ma, mb, md, md2, mr, a, s);
+        case EPI_F32_ATOMIC:
+          return launch_t<BN, true, true, EPI_F32_ATOMIC, PAIR>(ma, mb, md, md2, mr, a, s);
+        default: break;
+      }
     }
   }
   return QAT_ERR_ARG;  // combination not instantiated

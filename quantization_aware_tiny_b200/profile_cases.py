@@ -45,6 +45,27 @@ def head_dx(T):
         qat.qat_linear_bwd(None, dL, 8, qw=q, dX=dX)
 
 
+def mlp_step(T):
+    """The int6 ReLU^2 MLP 512-2048-512 forward and backward (6 GEMMs per pass)."""
+    c = sy.head_mlp_case(T=1, seed=0)
+    d, H = 512, 2048
+    qf = qat.quantize_weight(torch.from_numpy(c["Wfc"]).cuda(), 6)
+    qp = qat.quantize_weight(torch.from_numpy(c["Wproj"]).cuda(), 6)
+    X = sy.act_bf16(np.random.default_rng(1), T, d).cuda()
+    dY = sy.act_bf16(np.random.default_rng(2), T, d, std=0.01).cuda()
+    bf = torch.bfloat16
+    Y, dX = (torch.empty((T, d), dtype=bf, device="cuda") for _ in range(2))
+    pre, h = (torch.empty((T, H), dtype=bf, device="cuda") for _ in range(2))
+    dWfc = torch.empty((H, d), dtype=torch.float32, device="cuda")
+    dWproj = torch.empty((d, H), dtype=torch.float32, device="cuda")
+    ws = torch.empty(qat.workspace_size(qat.QAT_OP_MLP_BWD, d, H, T, False), dtype=torch.uint8,
+                     device="cuda")
+    for _ in range(3):
+        qat.qat_mlp_fwd(X, Y, 6, d, H, qfc=qf, qproj=qp, pre_save=pre, h_save=h)
+        qat.qat_mlp_bwd(X, pre, h, dY, 6, d, H, qfc=qf, qproj=qp, dX=dX, dWfc=dWfc,
+                        dWproj=dWproj, workspace=ws)
+
+
 def export_state_dict(_T):
     sd = {k: torch.from_numpy(v).cuda() for k, v in sy.state_dict_case().items()}
     for _ in range(3):
@@ -52,7 +73,7 @@ def export_state_dict(_T):
 
 
 CASES = {"logits_fwd": logits_fwd, "head_dw": head_dw, "head_dx": head_dx,
-         "export_state_dict": export_state_dict}
+         "mlp_step": mlp_step, "export_state_dict": export_state_dict}
 
 
 def main(argv=None):
