@@ -36,9 +36,9 @@ VOCAB, D, H = 8192, 512, 2048
 # each at 16,384 tokens, scaled by 4 to the 65,536-token launch (the traffic
 # grows with the token count), with the hash of the GEMM sources the captures
 # were taken on: reported only while the sources still match.
-NCU_TRAFFIC = {"kernel_hash": "2c05f7b683b6a621",
-               "bytes_per_launch": {"logits_fwd": 4 * (25.281024e6 + 215.121664e6),
-                                    "head_dW": 4 * (303.659520e6 + 9.542912e6)}}
+NCU_TRAFFIC = {"kernel_hash": "501b0cf04b046d22",
+               "bytes_per_launch": {"logits_fwd": 4 * (25.227776e6 + 215.858176e6),
+                                    "head_dW": 4 * (303.518976e6 + 9.555712e6)}}
 
 
 def gemm_source_hash():
@@ -255,6 +255,7 @@ def run_ours(args):
             out["export_pack6"] = measure_export(dev, stream, pk, pack6=True)
             out["export_clip_search"] = measure_export(dev, stream, pk, clip_search=True)
             out["recurrent_core"] = measure_core(dev, stream, pk)
+            out["fused_producer"] = measure_fused_producer(dev, stream, pk)
             out["cpu_baseline"] = cpu_baseline()
         print(json.dumps(out), flush=True)
     if pg is not None:
@@ -360,6 +361,53 @@ def measure_export(dev, stream, pk, pack6=False, clip_search=False):
                         "+ small tensors fp16 passthrough; L2 flushed (256 MB written, 256 MB read) "
                         "before each launch" % ((" 6-bit packed" if pack6 else "") +
                                                 (" clip search" if clip_search else ""))}
+
+
+def measure_fused_producer(dev, stream, pk):
+    """The QAT linear forward from fp32 weights two ways: the GEMM that
+    quantizes W in its own producer (what qat_linear_fwd does when given no
+    workspace: the operand never reaches global memory, one launch) against
+    quantizing into a workspace first and then running the GEMM on the
+    materialised operand (the default).  Cases: the single int6 CastedLinear
+    512->512 at 256 tokens and the int8 tied head 8192x512 at 65,536 tokens.
+    Each timed call runs from the host: per-call times include the launch
+    path a caller sees."""
+    from quantization_aware_tiny_b200 import qat
+    g = torch.Generator(device="cpu").manual_seed(7)
+    out = {}
+    for name, (T, N, K, bits) in (("linear_512x512_T256_int6", (256, 512, 512, 6)),
+                                  ("head_8192x512_T65536_int8", (65536, 8192, 512, 8))):
+        W = (torch.randn(N, K, generator=g) * 0.02).to(dev)
+        X = torch.randn(T, K, generator=g).to(torch.bfloat16).to(dev)
+        Y = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(N * K * 2 + N * 4 + 4096, dtype=torch.uint8, device=dev)
+        q = qat.quantize_weight(W, bits)
+
+        def fused():
+            qat.qat_linear_fwd(X, Y, bits, W=W, stream=stream)  # no workspace: fused producer
+
+        def materialised():
+            qat.qat_quantize_weights(W, bits, q.scales, None, q.operand, stream=stream)
+            qat.qat_linear_fwd(X, Y, bits, qw=q, stream=stream)
+
+        res = {}
+        for label, fn in (("fused_us", fused), ("materialised_us", materialised)):
+            for _ in range(3):
+                fn()
+            reps = 50 if T <= 4096 else 10
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(reps):
+                fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            res[label] = round(a.elapsed_time(b) * 1000 / reps, 2)
+        flops = 2.0 * T * N * K
+        res["fused_tflops"] = round(flops / (res["fused_us"] * 1e-6) / 1e12, 1)
+        res["materialised_tflops"] = round(flops / (res["materialised_us"] * 1e-6) / 1e12, 1)
+        out[name] = res
+    out["device_error"] = qat.device_error()
+    return out
 
 
 def measure_core(dev, stream, pk):

@@ -119,9 +119,18 @@ size_t qat_workspace_size(int32_t op, int32_t N_or_d, int32_t K_or_H, int64_t T,
 
 /* [P5] CastedLinear forward with QAT: Y[T,N] = bf16( X[T,K] . Wq^T (+ residual) ),
  * fp32 accumulation on the tensor cores.  Weights: either W (fp32 [N,K],
- * quantized inside the call into the workspace) or qw (pre-quantized; W must
- * then be NULL).  ldx = row stride of X in elements (0 -> K); residual
- * (nullable) is [T,N] bf16 and may alias Y exactly. */
+ * quantized inside the call) or qw (pre-quantized; W must then be NULL).
+ * ldx = row stride of X in elements (0 -> K); residual (nullable) is [T,N]
+ * bf16 and may alias Y exactly.
+ * With W, one of two paths, both giving bf16(fl32(c * s)) as the operand:
+ *   - with a workspace (qat_workspace_size() bytes), the weight is quantized
+ *     into it first and the GEMM reads the bf16 operand from there -- the
+ *     faster path on B200 at every measured size;
+ *   - with workspace == NULL, the fused quantizing producer: the GEMM itself
+ *     computes each row's amax, scale, codes and bf16 operand in shared
+ *     memory, so the quantized weight never reaches global memory and no
+ *     scratch is needed.  Needs T >= 256 and K <= 1024 (a CTA pair holds the
+ *     whole B_ROWS x K slice of its N block); otherwise QAT_ERR_WORKSPACE. */
 int qat_linear_fwd(const float* W, const qat_qweight* qw, int32_t N, int32_t K, int32_t bits,
                    const qat_bf16* X, int64_t ldx, int64_t T, const qat_bf16* residual,
                    qat_bf16* Y, void* workspace, size_t ws_bytes, qat_stream_t stream);
@@ -140,7 +149,9 @@ int qat_linear_bwd(const float* W, const qat_qweight* qw, int32_t N, int32_t K, 
  * negative result #9 "LeakyReLU(0.5)²"; [P4] leaderboard entries use it). */
 enum { QAT_ACT_RELU2 = 0, QAT_ACT_LEAKY_RELU2 = 1 };
 
-/* [P5] "架构" ReLU^2 MLP forward, both linears int5/int6/int8 QAT:
+/* [P5] "架构" ReLU^2 MLP forward, both linears int5/int6/int8 QAT
+ * (given Wfc and workspace == NULL, the fc GEMM quantizes Wfc in its own
+ * producer as qat_linear_fwd does; proj then needs qproj and h_save):
  *   pre = X . Wfc_q^T  [T,H];  h = act(pre) (fused in the fc epilogue, from the
  *   fp32 accumulator: relu(pre)^2, or for QAT_ACT_LEAKY_RELU2 t^2 with t = pre
  *   (pre > 0) else pre/2);  Y = bf16(h . Wproj_q^T (+ residual))  [T,d].
@@ -172,7 +183,8 @@ int qat_mlp_bwd(const float* Wfc, const float* Wproj, const qat_qweight* qfc,
  * through its own pool, a fixed-budget service that allocates only at
  * start-up, latency-critical code that cannot afford the synchronization
  * cudaMalloc / cudaFree may cause).
- *   Computes exactly what qat_linear_fwd computes when given W (same kernels):
+ *   Computes what qat_linear_fwd computes when given W, always by quantizing
+ *   into the array first and then running the GEMM:
  *   Y[T,N] = bf16( X[T,K] . bf16(fl32(c*s))^T (+ residual) ).
  *   Scratch: a fixed device array inside the library holds the bf16 operand and
  *   the scales -- at most QAT_NOALLOC_MAX_ELEMS weights (N*K) and

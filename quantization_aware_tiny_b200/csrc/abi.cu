@@ -161,17 +161,24 @@ int qat_linear_fwd(const float* W, const qat_qweight* qw, int32_t N, int32_t K, 
   if (ldx == 0) ldx = K;
   if (ldx < K || (ldx & 7)) return QAT_ERR_SHAPE;
   if (T == 0) return ((W == nullptr) != (qw == nullptr)) ? QAT_OK : QAT_ERR_ARG;
-  Carver ws(workspace, ws_bytes);
-  const __nv_bfloat16* op = nullptr;
-  int rc = get_operand(W, qw, N, K, bits, ws, stream, &op);
-  if (rc) return rc;
   GemmDesc g;
   g.A = X; g.lda = ldx;
-  g.B = op; g.ldb = K;
   g.M = T; g.N = N; g.K = K;
   g.epi = residual ? EPI_BF16_RESID : EPI_BF16;
   g.D = Y; g.ldd = N;
   g.R = residual; g.ldr = N;
+  if (W && !qw && workspace == nullptr && fused_b_supported(T, N, K, g.epi)) {
+    // no workspace: the GEMM quantizes W itself, the operand never reaches global memory
+    if (!aligned16(W)) return QAT_ERR_ALIGN;
+    g.Wraw = W;
+    g.bits = bits;
+    return launch_gemm(g, stream);
+  }
+  Carver ws(workspace, ws_bytes);
+  const __nv_bfloat16* op = nullptr;
+  int rc = get_operand(W, qw, N, K, bits, ws, stream, &op);
+  if (rc) return rc;
+  g.B = op; g.ldb = K;
   return launch_gemm(g, stream);
 }
 
@@ -224,8 +231,16 @@ int qat_mlp_fwd(const float* Wfc, const float* Wproj, const qat_qweight* qfc,
   if ((pre_save && !aligned16(pre_save)) || (h_save && !aligned16(h_save))) return QAT_ERR_ALIGN;
   Carver ws(workspace, ws_bytes);
   const __nv_bfloat16 *op_fc = nullptr, *op_proj = nullptr;
-  int rc = get_operand(Wfc, qfc, H, d, bits, ws, stream, &op_fc);
-  if (rc) return rc;
+  const int fc_epi = act == QAT_ACT_RELU2 ? EPI_RELU2 : EPI_LRELU2;
+  // fc from fp32 weights and no workspace: the fc GEMM quantizes Wfc itself
+  const bool fc_fused = Wfc && !qfc && !workspace && T > 0 && fused_b_supported(T, H, d, fc_epi);
+  int rc = QAT_OK;
+  if (fc_fused) {
+    if (!aligned16(Wfc)) return QAT_ERR_ALIGN;
+  } else {
+    rc = get_operand(Wfc, qfc, H, d, bits, ws, stream, &op_fc);
+    if (rc) return rc;
+  }
   rc = get_operand(Wproj, qproj, d, H, bits, ws, stream, &op_proj);
   if (rc) return rc;
   if (T == 0) return QAT_OK;
@@ -237,8 +252,12 @@ int qat_mlp_fwd(const float* Wfc, const float* Wproj, const qat_qweight* qfc,
   GemmDesc g1;  // pre = X . Wfc^T ; h = act(pre)
   g1.A = X; g1.lda = d;
   g1.B = op_fc; g1.ldb = d;
+  if (fc_fused) {
+    g1.Wraw = Wfc;
+    g1.bits = bits;
+  }
   g1.M = T; g1.N = H; g1.K = d;
-  g1.epi = act == QAT_ACT_RELU2 ? EPI_RELU2 : EPI_LRELU2;
+  g1.epi = fc_epi;
   g1.D = pre_save; g1.ldd = H;
   g1.D2 = h; g1.ldd2 = H;
   rc = launch_gemm(g1, stream);

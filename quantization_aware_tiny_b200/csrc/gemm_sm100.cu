@@ -33,32 +33,46 @@ constexpr int BK = 64;
 // pre-activation) bring it in by TMA ahead of use (R).  bf16-output epilogues
 // run 8 warps (their HBM traffic per FLOP is high: a lone warp per lane
 // quarter left the tensor pipe idle), the fp32 split-K ones 4.
-template <int BN, bool PAIR, int EPI>
+// FB (fused quantizing B producer): B is not loaded by TMA.  Each CTA keeps
+// the B_ROWS x K slice of the current N block resident in shared memory as a
+// panel of KBP k-blocks, written by the epilogue warps straight from the fp32
+// weight (row amax, scale, codes, dequantized value, bf16) whenever the CTA's
+// run of tiles enters a new N block; only A streams through the ring.
+template <int BN, bool PAIR, int EPI, bool FB = false>
 struct Cfg {
   static constexpr bool F32 = (EPI == EPI_F32 || EPI == EPI_F32_ATOMIC);
   static constexpr bool HAS_R = epi_reads_r(EPI);
-  static constexpr int EW = F32 ? 4 : 8;              // epilogue warps
+  static constexpr bool ACT = epi_act_fwd(EPI);
+  static constexpr int EW = F32 ? 4 : (FB && (ACT || HAS_R)) ? 4 : 8;  // epilogue warps
   static constexpr int THREADS = 64 + 32 * EW;
   static constexpr int B_ROWS = PAIR ? BN / 2 : BN;  // B rows staged by one CTA
   static constexpr int TILE_M = PAIR ? 2 * BM : BM;
   static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = B_ROWS * BK * 2;
+  static constexpr int B_BYTES = FB ? 0 : B_ROWS * BK * 2;  // B bytes per ring stage
+  // FB panel: KBP k-blocks of B_ROWS rows x 128 bytes (K <= 64 * KBP)
+  static constexpr int KBP = !FB ? 0 : B_ROWS >= 128 ? 8 : B_ROWS >= 80 ? 10 : 16;
+  static constexpr int KB_BYTES = B_ROWS * 128;
+  static constexpr int PANEL_BYTES = KBP * KB_BYTES;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TMEM_COLS = (2 * BN <= 256) ? 256 : 512;  // a power of two >= 2*BN
   // per epilogue warp: two buffers of one or two 32x32 output chunks
-  static constexpr int WBUF = (F32 || epi_act_fwd(EPI)) ? 8192 : 4096;
+  static constexpr int WBUF = (F32 || ACT) ? 8192 : 4096;
   static constexpr int STAGING_BYTES = EW * WBUF;
-  static constexpr int R_BUFS = EW == 8 ? 2 : 4;  // R chunks in flight per epilogue warp
+  static constexpr int R_BUFS = (EW == 8 || FB) ? 2 : 4;  // R chunks in flight per epilogue warp
   static constexpr int R_BYTES = HAS_R ? EW * R_BUFS * 2048 : 0;
   static constexpr int BAR_BYTES = 512;
-  static constexpr int FIXED = STAGING_BYTES + R_BYTES + BAR_BYTES + 1024;
+  static constexpr int FIXED = PANEL_BYTES + STAGING_BYTES + R_BYTES + BAR_BYTES + 1024;
   static constexpr int STAGES_FIT = (232448 - FIXED) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + FIXED;
   static_assert(STAGES >= 3, "pipeline too shallow");
-  // barriers (full/empty per stage, tfull/tempty x2, mma_done, R ring per
-  // epilogue warp) followed by tmem_slot, abort flag and two ring positions
-  static_assert((2 * STAGES + 5 + EW * R_BUFS) * 8 + 16 <= BAR_BYTES, "barrier block overflow");
+  static_assert(KB_BYTES % 1024 == 0, "panel k-blocks must keep the 1024-byte swizzle atoms aligned");
+  // barriers (full/empty per stage, tfull/tempty x2, mma_done, panel_full, R
+  // ring per epilogue warp) followed by tmem_slot, abort flag and two ring positions
+  static_assert((2 * STAGES + 6 + EW * R_BUFS) * 8 + 16 <= BAR_BYTES, "barrier block overflow");
+  // FB conversion: rows per pass (float4 loads in flight per lane: RP * KBP / 2)
+  static constexpr int RP = KBP > 10 ? 2 : 4;
+  static_assert(RP >= 1, "conversion rows per pass");
 };
 
 struct KArgs {
@@ -72,6 +86,9 @@ struct KArgs {
   int64_t ldr;
   int accumulate;
   int* err;
+  const float* W;  // FB: fp32 weight [N, K] row-major, quantized in the producer
+  int K;           // FB: reduction length
+  int bits;        // FB: grid (5, 6 or 8)
 };
 
 __device__ __forceinline__ float bf2f(__nv_bfloat16 x) { return __bfloat162float(x); }
@@ -140,25 +157,102 @@ __device__ __forceinline__ void stage_chunk(const KArgs& p, const uint32_t (&acc
   }
 }
 
-template <int BN, bool A_MN, bool B_MN, int EPI, bool PAIR>
-__global__ void __launch_bounds__(Cfg<BN, PAIR, EPI>::THREADS, 1)
+__device__ __forceinline__ float absmax4(float4 v) {
+  return fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+}
+
+// FB producer: fill this CTA's panel with the STE operand of weight rows
+// n_base .. n_base + B_ROWS - 1, the training quantizer's arithmetic exactly:
+//   amax = max(max_j |W_nj|, 1e-12), s = fl32(amax / L) (L = 127, or 15 for
+//   int5), c = the grid's code of fl32(w / s), operand = bf16_rne(fl32(c * s)).
+// Row r of k-block kb lands at kb * KB_BYTES + r * 128, its 16-byte group g
+// (8 consecutive k) at g ^ (r & 7): the 128-byte-swizzled K-major layout a TMA
+// load of the same tile would write.  Rows >= N and columns >= K are zero.
+// Warp ew takes rows ew, ew + EW, ...; RP rows per pass keep RP * KBP / 2
+// 16-byte loads in flight per lane.
+template <class C>
+__device__ __forceinline__ void convert_panel(const KArgs& p, uint8_t* panel, int n_base, int ew,
+                                              int lane) {
+  constexpr int V = C::KBP / 2;  // float4 per lane per row (32 lanes x 4 floats per 128 columns)
+  const int K4 = p.K >> 2;
+  const int slots = p.kblk_total * 16;  // float4 slots of a panel row
+  const float levels = grid_levels(p.bits);
+  const uint32_t pbase = smem_u32(panel);
+#pragma unroll 1
+  for (int r0 = ew; r0 < C::B_ROWS; r0 += C::RP * C::EW) {
+    float4 v[C::RP][V];
+    float amax[C::RP];
+#pragma unroll
+    for (int h = 0; h < C::RP; ++h) {
+      const int r = r0 + h * C::EW;
+      const int n = n_base + r;
+      const bool valid = r < C::B_ROWS && n < p.N;
+      const float4* row = reinterpret_cast<const float4*>(p.W + static_cast<int64_t>(valid ? n : 0) * p.K);
+      amax[h] = 0.0f;
+#pragma unroll
+      for (int i = 0; i < V; ++i) {
+        const int j = lane + 32 * i;
+        v[h][i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (valid && j < K4) {
+          v[h][i] = __ldg(row + j);
+          amax[h] = fmaxf(amax[h], absmax4(v[h][i]));
+        }
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < C::RP; ++h) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+        amax[h] = fmaxf(amax[h], __shfl_xor_sync(0xffffffffu, amax[h], o));
+    }
+#pragma unroll
+    for (int h = 0; h < C::RP; ++h) {
+      const int r = r0 + h * C::EW;
+      if (r >= C::B_ROWS) break;  // warp-uniform
+      const float sc = div_rn(fmaxf(amax[h], 1e-12f), levels);
+      const float rs = __frcp_rn(sc);
+      const uint32_t rbase = pbase + static_cast<uint32_t>(r) * 128u;
+      const uint32_t sw = static_cast<uint32_t>(r & 7);
+#pragma unroll
+      for (int i = 0; i < V; ++i) {
+        const int j = lane + 32 * i;
+        if (j < slots) {
+          const float4 w = v[h][i];
+          const int c0 = quant_code(w.x, sc, rs, p.bits), c1 = quant_code(w.y, sc, rs, p.bits);
+          const int c2 = quant_code(w.z, sc, rs, p.bits), c3 = quant_code(w.w, sc, rs, p.bits);
+          const uint32_t lo = pack_bf16(mul_rn(static_cast<float>(c0), sc), mul_rn(static_cast<float>(c1), sc));
+          const uint32_t hi = pack_bf16(mul_rn(static_cast<float>(c2), sc), mul_rn(static_cast<float>(c3), sc));
+          const uint32_t kb = static_cast<uint32_t>(j >> 4), g = static_cast<uint32_t>((j & 15) >> 1);
+          st_shared_v2(rbase + kb * C::KB_BYTES + ((g ^ sw) << 4) + static_cast<uint32_t>(j & 1) * 8u,
+                       lo, hi);
+        }
+      }
+    }
+  }
+}
+
+template <int BN, bool A_MN, bool B_MN, int EPI, bool PAIR, bool FB>
+__global__ void __launch_bounds__(Cfg<BN, PAIR, EPI, FB>::THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmD, const __grid_constant__ CUtensorMap tmD2,
                 const __grid_constant__ CUtensorMap tmR, const KArgs p) {
-  using C = Cfg<BN, PAIR, EPI>;
+  using C = Cfg<BN, PAIR, EPI, FB>;
+  static_assert(!FB || (!A_MN && !B_MN && !C::F32), "fused B: forward GEMMs only");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sA = smem;
-  uint8_t* sB = smem + C::STAGES * C::A_BYTES;
-  uint8_t* staging = smem + C::STAGES * C::STAGE_BYTES;  // 1024-aligned
+  uint8_t* panel = smem;  // FB: resident B panel (PANEL_BYTES; 0 otherwise)
+  uint8_t* sA = smem + C::PANEL_BYTES;
+  uint8_t* sB = sA + C::STAGES * C::A_BYTES;
+  uint8_t* staging = sA + C::STAGES * C::STAGE_BYTES;  // 1024-aligned
   uint8_t* rstage = staging + C::STAGING_BYTES;          // R chunks (HAS_R)
   uint64_t* full = reinterpret_cast<uint64_t*>(rstage + C::R_BYTES);
   uint64_t* empty = full + C::STAGES;
   uint64_t* tfull = empty + C::STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* mma_done = tempty + 2;
-  uint64_t* rbar = mma_done + 1;  // EW epilogue warps x R_BUFS
+  uint64_t* panel_full = mma_done + 1;  // FB: the panel of the next N block is written
+  uint64_t* rbar = panel_full + 1;      // EW epilogue warps x R_BUFS
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rbar + C::EW * C::R_BUFS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* prod_pos = const_cast<int*>(abort_flag) + 1;  // producer ring position at exit
@@ -170,8 +264,19 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR, EPI>::THREADS, 1)
   // and owns the full / tmem-empty barriers both CTAs signal.
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
   const bool leader = (rank == 0);
-  const int tile0 = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
-  const int tile_step = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int units = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  // Tiles of this CTA (pair): every units-th tile, N block fastest; FB: one
+  // contiguous run in N-block-major order, so the B panel changes rarely.
+  int t_begin = unit, t_end = p.num_tiles, t_step = units;
+  if constexpr (FB) {
+    t_begin = static_cast<int>(static_cast<int64_t>(unit) * p.num_tiles / units);
+    t_end = static_cast<int>(static_cast<int64_t>(unit + 1) * p.num_tiles / units);
+    t_step = 1;
+  }
+  auto tile_nb = [&](int t) { return FB ? t / p.num_m_blk : t % p.num_n_blk; };
+  auto tile_mb = [&](int t) { return FB ? t % p.num_m_blk : (t / p.num_n_blk) % p.num_m_blk; };
+  auto tile_sp = [&](int t) { return FB ? 0 : t / (p.num_n_blk * p.num_m_blk); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -183,13 +288,14 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR, EPI>::THREADS, 1)
       mbar_init(&tempty[b], PAIR ? 2 * C::EW : C::EW);
     }
     mbar_init(mma_done, 1);
+    mbar_init(panel_full, PAIR ? 2 * C::EW : C::EW);
     for (int i = 0; i < C::EW * C::R_BUFS; ++i) mbar_init(&rbar[i], 1);
     *abort_flag = 0;
     *prod_pos = 0;
     *mma_pos = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
+    if constexpr (!FB) tma_prefetch_desc(&tmB);
     tma_prefetch_desc(&tmD);
     if constexpr (epi_reads_r(EPI)) tma_prefetch_desc(&tmR);
   }
@@ -213,10 +319,10 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR, EPI>::THREADS, 1)
       int stage = 0, pos = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int tile = tile0; ok && tile < p.num_tiles; tile += tile_step) {
-        const int nb = tile % p.num_n_blk;
-        const int mb = (tile / p.num_n_blk) % p.num_m_blk;
-        const int sp = tile / (p.num_n_blk * p.num_m_blk);
+      for (int tile = t_begin; ok && tile < t_end; tile += t_step) {
+        const int nb = tile_nb(tile);
+        const int mb = tile_mb(tile);
+        const int sp = tile_sp(tile);
         const int kb0 = sp * p.kblk_per_split;
         const int kb1 = min(kb0 + p.kblk_per_split, p.kblk_total);
         const int m0 = mb * C::TILE_M + static_cast<int>(rank) * BM;
@@ -236,7 +342,9 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR, EPI>::THREADS, 1)
               tma_load_2d_pair(&tmA, bar, a_dst, m0, k0);
               tma_load_2d_pair(&tmA, bar, a_dst + 64 * 128, m0 + 64, k0);
             }
-            if constexpr (!B_MN) {
+            if constexpr (FB) {
+              // B comes from the resident panel
+            } else if constexpr (!B_MN) {
               tma_load_2d_pair(&tmB, bar, b_dst, k0, n0);
             } else {
 #pragma unroll
@@ -251,7 +359,9 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR, EPI>::THREADS, 1)
               tma_load_2d(&tmA, &full[stage], a_dst, m0, k0);
               tma_load_2d(&tmA, &full[stage], a_dst + 64 * 128, m0 + 64, k0);
             }
-            if constexpr (!B_MN) {
+            if constexpr (FB) {
+              // B comes from the resident panel
+            } else if constexpr (!B_MN) {
               tma_load_2d(&tmB, &full[stage], b_dst, k0, n0);
             } else {
 #pragma unroll
@@ -283,10 +393,20 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR, EPI>::THREADS, 1)
           umma_commit(bar);
         }
       };
-      for (int tile = tile0; ok && tile < p.num_tiles; tile += tile_step) {
-        const int sp = tile / (p.num_n_blk * p.num_m_blk);
+      int panel_nb = -1;  // FB: N block whose panel the MMAs read
+      uint32_t panel_phase = 0;
+      for (int tile = t_begin; ok && tile < t_end; tile += t_step) {
+        const int sp = tile_sp(tile);
         const int kb0 = sp * p.kblk_per_split;
         const int kb1 = min(kb0 + p.kblk_per_split, p.kblk_total);
+        if constexpr (FB) {
+          if (tile_nb(tile) != panel_nb) {  // both CTAs' epilogue warps wrote the new panel
+            if (!mbar_wait(panel_full, panel_phase, abort_flag, p.err)) break;
+            panel_phase ^= 1u;
+            panel_nb = tile_nb(tile);
+            tc_fence_after();
+          }
+        }
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, p.err)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
@@ -294,7 +414,8 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR, EPI>::THREADS, 1)
           if (!mbar_wait(&full[stage], phase, abort_flag, p.err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_base = smem_u32(sA + stage * C::A_BYTES);
-          const uint32_t b_base = smem_u32(sB + stage * C::B_BYTES);
+          const uint32_t b_base = FB ? smem_u32(panel + kb * C::KB_BYTES)
+                                     : smem_u32(sB + stage * C::B_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t ad = A_MN ? sw128_desc(a_base + kk * 2048, 64 * 128, 1024)
@@ -337,9 +458,41 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR, EPI>::THREADS, 1)
     uint32_t r_issued = 0, r_used = 0;  // R ring: chunks requested / consumed
     // the leader's tmem-empty barrier, which both CTAs' epilogues release
     const uint32_t tempty_leader = PAIR ? mapa_shared(smem_u32(tempty), 0) : smem_u32(tempty);
-    for (int tile = tile0; tile < p.num_tiles; tile += tile_step) {
-      const int nb = tile % p.num_n_blk;
-      const int mb = (tile / p.num_n_blk) % p.num_m_blk;
+    // FB: write the panel of N block nb (this CTA's B_ROWS rows) and tell the MMA.
+    auto produce_panel = [&](int nb) {
+      if constexpr (FB) {
+        convert_panel<C>(p, panel, nb * BN + static_cast<int>(rank) * C::B_ROWS, ew, lane);
+        fence_proxy_async_smem();  // generic-proxy writes visible to the tensor cores
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(panel_full), 0));
+          else mbar_arrive(panel_full);
+        }
+      }
+    };
+    if constexpr (FB) {
+      if (ew == 0 && lane == 0) {
+        // L2 prefetch of the weight rows of the first few panels this CTA converts
+        int last = -1, count = 0;
+        for (int t = t_begin; t < t_end && count < 4; ++t) {
+          const int nb = tile_nb(t);
+          if (nb == last) continue;
+          last = nb;
+          ++count;
+          const int n0 = nb * BN + static_cast<int>(rank) * C::B_ROWS;
+          const int rows = min(C::B_ROWS, p.N - n0);
+          if (rows <= 0) continue;
+          const char* src = reinterpret_cast<const char*>(p.W + static_cast<int64_t>(n0) * p.K);
+          int64_t bytes = static_cast<int64_t>(rows) * p.K * 4;
+          for (; bytes > 0; bytes -= 65536, src += 65536)
+            bulk_prefetch_l2(src, static_cast<uint32_t>(bytes < 65536 ? bytes : 65536));
+        }
+      }
+      if (t_begin < t_end) produce_panel(tile_nb(t_begin));
+    }
+    for (int tile = t_begin; tile < t_end; tile += t_step) {
+      const int nb = tile_nb(tile);
+      const int mb = tile_mb(tile);
       const int row0 = mb * C::TILE_M + static_cast<int>(rank) * BM + q * 32;
       const int ncols = min(BN, p.N - nb * BN);
       const int nchunks = (ncols + 31) / 32;
@@ -358,6 +511,12 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR, EPI>::THREADS, 1)
       }
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err)) break;
       tc_fence_after();
+      if constexpr (FB) {
+        // Every MMA of this tile has completed, so the old panel is free: write
+        // the next N block's panel first (the MMA waits on it), then drain this
+        // tile's accumulator while the next tile runs.
+        if (tile + 1 < t_end && tile_nb(tile + 1) != nb) produce_panel(tile_nb(tile + 1));
+      }
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
       auto release_acc = [&]() {  // this warp's part of the accumulator is read
@@ -502,11 +661,11 @@ int make_out_map(CUtensorMap* m, const void* base, int64_t inner, int64_t outer,
   return r == CUDA_SUCCESS ? QAT_OK : QAT_ERR_ARG;
 }
 
-template <int BN, bool A_MN, bool B_MN, int EPI, bool PAIR>
+template <int BN, bool A_MN, bool B_MN, int EPI, bool PAIR, bool FB = false>
 int launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& md,
              const CUtensorMap& md2, const CUtensorMap& mr, const KArgs& a, cudaStream_t s) {
-  using C = Cfg<BN, PAIR, EPI>;
-  auto kern = gemm_kernel<BN, A_MN, B_MN, EPI, PAIR>;
+  using C = Cfg<BN, PAIR, EPI, FB>;
+  auto kern = gemm_kernel<BN, A_MN, B_MN, EPI, PAIR, FB>;
   static bool attr_done = false;  // per instantiation; set before first launch
   if (!attr_done) {
     cudaError_t e =
@@ -579,6 +738,37 @@ int dispatch_bn(const GemmDesc& g, const CUtensorMap& ma, const CUtensorMap& mb,
   return QAT_ERR_ARG;  // combination not instantiated
 }
 
+// Fused-B forward GEMMs (paired CTAs, K-major operands).
+template <int BN>
+int dispatch_fb(const CUtensorMap& ma, const CUtensorMap& md, const CUtensorMap& md2,
+                const CUtensorMap& mr, const KArgs& a, int epi, cudaStream_t s) {
+  switch (epi) {
+    case EPI_BF16: return launch_t<BN, false, false, EPI_BF16, true, true>(ma, ma, md, md2, mr, a, s);
+    case EPI_BF16_RESID:
+      return launch_t<BN, false, false, EPI_BF16_RESID, true, true>(ma, ma, md, md2, mr, a, s);
+    case EPI_RELU2: return launch_t<BN, false, false, EPI_RELU2, true, true>(ma, ma, md, md2, mr, a, s);
+    case EPI_LRELU2:
+      return launch_t<BN, false, false, EPI_LRELU2, true, true>(ma, ma, md, md2, mr, a, s);
+    default: return QAT_ERR_ARG;
+  }
+}
+
+// N tile of the fused-B GEMM: the panel (BN/2 rows x K bf16 per CTA) must fit
+// its KBP k-blocks; widest tile that divides N first.  0 = not supported.
+int fused_b_bn(int64_t N, int64_t K) {
+  const int64_t kblk = (K + BK - 1) / BK;
+  const bool k256 = kblk <= Cfg<256, true, EPI_BF16, true>::KBP;
+  const bool k192 = kblk <= Cfg<192, true, EPI_BF16, true>::KBP;
+  const bool k160 = kblk <= Cfg<160, true, EPI_BF16, true>::KBP;
+  const bool k128 = kblk <= Cfg<128, true, EPI_BF16, true>::KBP;
+  if (k256 && N % 256 == 0) return 256;
+  if (k192 && N % 192 == 0) return 192;
+  if (k160 && N % 160 == 0) return 160;
+  if (k256) return 256;
+  if (k128) return 128;
+  return 0;
+}
+
 // Split count for the fp32 weight-gradient GEMMs: minimise the makespan
 // ceil(tiles*s / SMs) * ceil(kblk / s), preferring fewer splits.
 int choose_splits(int tiles, int kblk, int sms) {
@@ -597,13 +787,22 @@ int choose_splits(int tiles, int kblk, int sms) {
 
 }  // namespace
 
+bool fused_b_supported(int64_t M, int64_t N, int64_t K, int epi) {
+  const bool fwd_epi = epi == EPI_BF16 || epi == EPI_BF16_RESID || epi == EPI_RELU2 || epi == EPI_LRELU2;
+  return fwd_epi && M >= 256 && N > 0 && K > 0 && (K & 7) == 0 && fused_b_bn(N, K) != 0;
+}
+
 int launch_gemm(const GemmDesc& g, cudaStream_t stream) {
   if (g.M < 0 || g.N <= 0 || g.K <= 0) return QAT_ERR_ARG;
   if (g.M == 0) return QAT_OK;
-  if (!g.A || !g.B || (!g.D && !epi_act_fwd(g.epi))) return QAT_ERR_ARG;
+  if (!g.A || (!g.B && !g.Wraw) || (!g.D && !epi_act_fwd(g.epi))) return QAT_ERR_ARG;
+  if (g.Wraw && (!fused_b_supported(g.M, g.N, g.K, g.epi) || g.a_mn || g.b_mn))
+    return QAT_ERR_UNSUPPORTED;
+  if (g.Wraw && (!aligned16(g.Wraw) || (g.bits != 5 && g.bits != 6 && g.bits != 8)))
+    return g.bits == 5 || g.bits == 6 || g.bits == 8 ? QAT_ERR_ALIGN : QAT_ERR_ARG;
   if (epi_act_fwd(g.epi) && !g.D2) return QAT_ERR_ARG;
   if (epi_reads_r(g.epi) && !g.R) return QAT_ERR_ARG;
-  if (!aligned16(g.A) || !aligned16(g.B) || (g.D && !aligned16(g.D)) || (g.D2 && !aligned16(g.D2)) ||
+  if (!aligned16(g.A) || (g.B && !aligned16(g.B)) || (g.D && !aligned16(g.D)) || (g.D2 && !aligned16(g.D2)) ||
       (g.R && !aligned16(g.R)))
     return QAT_ERR_ALIGN;
   if ((g.N & 7) || (g.lda & 7) || (g.ldb & 7) || (g.ldd & 7) || (g.D2 && (g.ldd2 & 7)) ||
@@ -617,7 +816,10 @@ int launch_gemm(const GemmDesc& g, cudaStream_t stream) {
   int BN;
   bool pair;
   const bool kmajor_fwd = !g.a_mn && !g.b_mn && g.epi != EPI_F32 && g.epi != EPI_F32_ATOMIC;
-  if (kmajor_fwd && g.M >= 256 && g.N >= 160) {
+  if (g.Wraw) {
+    pair = true;
+    BN = fused_b_bn(g.N, g.K);
+  } else if (kmajor_fwd && g.M >= 256 && g.N >= 160) {
     pair = true;
     BN = (g.N % 256 == 0) ? 256 : (g.N % 192 == 0) ? 192 : (g.N % 160 == 0) ? 160 : 256;
   } else {
@@ -643,6 +845,9 @@ int launch_gemm(const GemmDesc& g, cudaStream_t stream) {
   a.ldr = g.ldr;
   a.accumulate = g.accumulate ? 1 : 0;
   a.err = device_error_ptr();
+  a.W = g.Wraw;
+  a.K = static_cast<int>(g.K);
+  a.bits = g.bits;
 
   int epi = g.epi;
   if (epi == EPI_F32 || epi == EPI_F32_ATOMIC) {
@@ -676,9 +881,13 @@ int launch_gemm(const GemmDesc& g, cudaStream_t stream) {
   int rc = g.a_mn ? make_map(&ma, g.A, g.M, g.K, g.lda, 64)
                   : make_map(&ma, g.A, g.K, g.M, g.lda, BM);
   if (rc) return rc;
-  rc = g.b_mn ? make_map(&mb, g.B, g.N, g.K, g.ldb, 64)
-              : make_map(&mb, g.B, g.K, g.N, g.ldb, b_rows);
-  if (rc) return rc;
+  if (g.Wraw) {
+    mb = ma;  // unused: B is quantized from Wraw inside the kernel
+  } else {
+    rc = g.b_mn ? make_map(&mb, g.B, g.N, g.K, g.ldb, 64)
+                : make_map(&mb, g.B, g.K, g.N, g.ldb, b_rows);
+    if (rc) return rc;
+  }
   // Output maps: 32x32 boxes, bf16 with 64-byte swizzle or fp32 with 128-byte swizzle.
   CUtensorMap md, md2;
   const bool f32 = (epi == EPI_F32 || epi == EPI_F32_ATOMIC);
@@ -692,6 +901,14 @@ int launch_gemm(const GemmDesc& g, cudaStream_t stream) {
   if (epi_reads_r(g.epi)) {
     rc = make_out_map(&mr, g.R, g.N, g.M, g.ldr, false);
     if (rc) return rc;
+  }
+  if (g.Wraw) {
+    switch (BN) {
+      case 128: return dispatch_fb<128>(ma, md, md2, mr, a, epi, stream);
+      case 160: return dispatch_fb<160>(ma, md, md2, mr, a, epi, stream);
+      case 192: return dispatch_fb<192>(ma, md, md2, mr, a, epi, stream);
+      default: return dispatch_fb<256>(ma, md, md2, mr, a, epi, stream);
+    }
   }
   if (pair) {
     switch (BN) {

@@ -43,7 +43,18 @@ struct GemmDesc {
   const void* R = nullptr;
   int64_t ldr = 0;
   bool accumulate = false;  // fp32 epilogues: add into D instead of overwriting
+  // Fused quantizing B producer: when set, B / ldb are ignored and the kernel
+  // builds the bf16 operand bf16(fl32(c * s)) of this fp32 weight [N,K]
+  // (row-major, ld = K) on the grid `bits` in shared memory -- the quantized
+  // weight never reaches global memory.  Forward epilogues, M >= 256 and
+  // fused_b_supported() only.
+  const float* Wraw = nullptr;
+  int bits = 0;
 };
+
+// Whether launch_gemm can quantize B inside the GEMM for this shape / epilogue.
+bool fused_b_supported(int64_t M, int64_t N, int64_t K, int epi);
+
 
 // Validates, encodes the tensor maps and launches.  Returns a QAT_* code.
 int launch_gemm(const GemmDesc& g, cudaStream_t stream);

@@ -26,6 +26,17 @@ def logits_fwd(T):
         qat.qat_linear_fwd(Z, Y, 8, qw=q)
 
 
+def logits_fwd_fused(T):
+    """The same logits GEMM from the fp32 tied head: the GEMM quantizes it in
+    its producer (no workspace is passed, so the fused path is taken)."""
+    c = sy.head_mlp_case(T=1, seed=0)
+    W = torch.from_numpy(c["Wemb"]).cuda()
+    Z = sy.act_bf16(np.random.default_rng(1), T, 512, std=0.25).cuda()
+    Y = torch.empty((T, 8192), dtype=torch.bfloat16, device="cuda")
+    for _ in range(3):
+        qat.qat_linear_fwd(Z, Y, 8, W=W)
+
+
 def head_dw(T):
     c = sy.head_mlp_case(T=1, seed=0)
     Z = sy.act_bf16(np.random.default_rng(1), T, 512, std=0.25).cuda()
@@ -72,7 +83,7 @@ def export_state_dict(_T):
         qexport.export_state_dict(sd)
 
 
-CASES = {"logits_fwd": logits_fwd, "head_dw": head_dw, "head_dx": head_dx,
+CASES = {"logits_fwd": logits_fwd, "logits_fwd_fused": logits_fwd_fused, "head_dw": head_dw, "head_dx": head_dx,
          "mlp_step": mlp_step, "export_state_dict": export_state_dict}
 
 

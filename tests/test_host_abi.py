@@ -42,7 +42,12 @@ def test_strerror_and_workspace_sizes(L):
     assert "aligned" in qat.strerror(qat.QAT_ERR_ALIGN)
     assert qat.strerror(99) == "unknown error"
     # raw weights: bf16 operand + fp32 scales, each rounded up to 256 bytes
+    # raw weights: the operand and scales (a NULL workspace instead selects the
+    # fused quantizing producer where it applies)
     assert qat.workspace_size(qat.QAT_OP_LINEAR_FWD, 512, 512, 256, True) == 512 * 512 * 2 + 2048
+    assert qat.workspace_size(qat.QAT_OP_LINEAR_BWD, 512, 512, 256, True) == 512 * 512 * 2 + 2048
+    assert qat.workspace_size(qat.QAT_OP_MLP_FWD, 512, 1536, 100, True) == (
+        100 * 1536 * 2 + 2 * (512 * 1536 * 2) + 2048 + 6144)
     assert qat.workspace_size(qat.QAT_OP_LINEAR_FWD, 512, 512, 256, False) == 0
     assert qat.workspace_size(qat.QAT_OP_MLP_BWD, 512, 1536, 8192, False) == 8192 * 1536 * 2
     assert qat.workspace_size(qat.QAT_OP_MLP_FWD, 0, 1536, 8192, False) == 0
@@ -68,6 +73,11 @@ def test_argument_validation_before_launch(L):
     assert L.qat_quantize_weights(A_BAD, 512, 512, 6, None, A16, None, None) == qat.QAT_ERR_ALIGN
     # workspace too small for raw weights
     assert L.qat_linear_fwd(A16, None, 512, 512, 6, A16, 0, 256, None, A16, A16, 1024, None) == qat.QAT_ERR_WORKSPACE
+    # no workspace and no fused path (fewer than 256 tokens, or K > 1024)
+    assert L.qat_linear_fwd(A16, None, 512, 512, 6, A16, 0, 255, None, A16, None, 0, None) == qat.QAT_ERR_WORKSPACE
+    assert L.qat_linear_fwd(A16, None, 512, 2048, 6, A16, 0, 4096, None, A16, None, 0, None) == qat.QAT_ERR_WORKSPACE
+    # fused path: misaligned fp32 weights
+    assert L.qat_linear_fwd(A_BAD, None, 512, 512, 6, A16, 0, 256, None, A16, None, 0, None) == qat.QAT_ERR_ALIGN
     # export: longer rows than the top-2 quantile covers, bad mode, too many descs
     assert L.quantize_rows_export(A16, 4, 1 << 21, 6, A16, A16, None) == qat.QAT_ERR_SHAPE
     assert L.quantize_rows_export(A16, 4, 700000, 6, A16, A16, None) == qat.QAT_ERR_SHAPE
