@@ -233,57 +233,99 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
   return u2f(d);
 }
 
-// Codes of two weights on the row's grid, the same arithmetic as quant_code
-// (common.cuh) done pairwise: the Markstein-corrected quotient, then the
-// rounding offset 1.5 * 2^23 (see code_from_quotient).  For int6 the second
-// rounding rne(k / 4) is the same trick on k / 4, which
-// fma(k + offset, 1/4, -offset/4) produces exactly; 4 * (bits - offset bits)
-// is formed modulo 2^32.
-//
-// CLIP = false skips clamping w to [-clip, clip].  That is exact when
-// clip >= v_hi / 2 (always so for rows up to 32,768 columns, where the
-// interpolation fraction exceeds 0.947): only entries with |w| > clip differ,
-// their quotient |w / s| then lies in (L, 2L] (L = 127, or 15 for int5), and
-// after the grid's clamp their code equals the code of +-clip itself (+124 /
-// -128 for int6, +-127 for int8, +-15 for int5); the offset trick stays exact
-// for |x| < 2^22.
-template <int BITS, bool CLIP>
-__device__ __forceinline__ void codes2(const RowQuant& q, float a, float b, int& ca, int& cb) {
-  constexpr float kOff = 12582912.0f;  // 1.5 * 2^23
-  const float2 w = CLIP ? make_float2(fminf(fmaxf(a, -q.clip), q.clip),
-                                      fminf(fmaxf(b, -q.clip), q.clip))
-                        : make_float2(a, b);
+// Which clamps a row's codes need (chosen per row from its largest |w| a1 and
+// its clip; see row_range):
+//   kClampW    -- clamp w to [-clip, clip], then the grid's clamp;
+//   kClampGrid -- the grid's clamp only.  Exact when a1 <= 2 clip: only entries
+//                 with |w| > clip differ, their quotient |w / s| then lies in
+//                 (L, 2L] (L = 127, or 15 for int5), and after the grid's clamp
+//                 their code equals the code of +-clip itself (+124 / -128 for
+//                 int6, +-127 for int8, +-15 for int5);
+//   kNarrow    -- no clamp can bind except int6's top: when a1 <= fl32(1.0039 *
+//                 clip), every |fl32(w / s)| < L + 1/2 (s = fl32(clip / L) is
+//                 within 2^-24 of clip / L and the quotient adds one more
+//                 rounding: |w / s| < 1.0039003 L, i.e. 127.4953 or 15.0585),
+//                 so rne(w / s) is already in [-L, L]; int6's second rounding
+//                 can still give 4 * 32 = 128 (-> 124), never below -128.
+// The row clips of the pages' quantile sit within 0.3 % of the row maximum for
+// rows of up to 1536 columns, so nearly every row is kNarrow.
+constexpr int kClampW = 0, kClampGrid = 1, kNarrow = 2;
+constexpr float kNarrowRatio = 1.0039f;
+
+__device__ __forceinline__ int row_range(float a1, const RowQuant& q) {
+  if (a1 > 2.0f * q.clip) return kClampW;
+  return a1 <= __fmul_rn(kNarrowRatio, q.clip) ? kNarrow : kClampGrid;
+}
+
+constexpr float kOff = 12582912.0f;  // 1.5 * 2^23
+
+// kOff + rne(fl32(w / s)) for two weights: the Markstein-corrected quotient
+// (see div_by_scale) done pairwise, then the rounding offset 1.5 * 2^23 (see
+// code_from_quotient); the float's bit pattern is 0x4B400000 + rne(w / s).
+template <int R>
+__device__ __forceinline__ float2 rne_quot2(const RowQuant& q, float a, float b) {
+  const float2 w = R == kClampW ? make_float2(fminf(fmaxf(a, -q.clip), q.clip),
+                                              fminf(fmaxf(b, -q.clip), q.clip))
+                                : make_float2(a, b);
   const float2 s2 = make_float2(-q.s, -q.s), r2 = make_float2(q.rs, q.rs);
   const float2 q0 = mul2(w, r2);
   const float2 rem = fma2(q0, s2, w);
   const float2 x = fma2(rem, r2, q0);
-  const float2 t = add2(x, make_float2(kOff, kOff));  // kOff + rne(x)
+  return add2(x, make_float2(kOff, kOff));
+}
+
+// int6: kOff + rne(k / 4) from t = kOff + k; the fma forms k / 4 exactly.
+__device__ __forceinline__ float2 rne_quarter2(float2 t) {
+  const float2 y = fma2(t, make_float2(0.25f, 0.25f), make_float2(-kOff / 4, -kOff / 4));
+  return add2(y, make_float2(kOff, kOff));
+}
+
+// Codes of two weights on the row's grid, the same arithmetic as quant_code
+// (common.cuh) done pairwise; for int6 4 * (bits - offset bits) is formed
+// modulo 2^32.
+template <int BITS, int R>
+__device__ __forceinline__ void codes2(const RowQuant& q, float a, float b, int& ca, int& cb) {
+  const float2 t = rne_quot2<R>(q, a, b);
   if constexpr (BITS == 6) {
-    // k = rne(x) >= -254 gives 4 rne(k / 4) >= -256: both clamps can bind
-    const float2 y = fma2(t, make_float2(0.25f, 0.25f), make_float2(-kOff / 4, -kOff / 4));
-    const float2 u = add2(y, make_float2(kOff, kOff));  // kOff + rne(k / 4)
-    ca = min(max(static_cast<int>(__float_as_uint(u.x) * 4u - 0x2D000000u), -128), 124);
-    cb = min(max(static_cast<int>(__float_as_uint(u.y) * 4u - 0x2D000000u), -128), 124);
+    const float2 u = rne_quarter2(t);
+    ca = static_cast<int>(__float_as_uint(u.x) * 4u - 0x2D000000u);
+    cb = static_cast<int>(__float_as_uint(u.y) * 4u - 0x2D000000u);
+    if constexpr (R == kNarrow) {
+      ca = min(ca, 124);
+      cb = min(cb, 124);
+    } else {  // k = rne(x) >= -254 gives 4 rne(k / 4) >= -256: both clamps can bind
+      ca = min(max(ca, -128), 124);
+      cb = min(max(cb, -128), 124);
+    }
   } else {
     constexpr int L = BITS == 5 ? 15 : 127;
-    ca = min(max(__float_as_int(t.x) - 0x4B400000, -L), L);
-    cb = min(max(__float_as_int(t.y) - 0x4B400000, -L), L);
+    ca = __float_as_int(t.x) - 0x4B400000;
+    cb = __float_as_int(t.y) - 0x4B400000;
+    if constexpr (R != kNarrow) {
+      ca = min(max(ca, -L), L);
+      cb = min(max(cb, -L), L);
+    }
   }
 }
 
-// Calls f(integral_constant<int, bits>, bool_constant<clip>) for a row's grid.
+// Calls f(integral_constant<int, bits>, integral_constant<int, range>) for a
+// row's grid and clamp range.
 template <typename F>
-__device__ __forceinline__ void with_grid(int bits, bool clip, F&& f) {
+__device__ __forceinline__ void with_grid(int bits, int range, F&& f) {
   using T5 = std::integral_constant<int, 5>;
   using T6 = std::integral_constant<int, 6>;
   using T8 = std::integral_constant<int, 8>;
-  if (bits == 6) {
-    if (clip) f(T6{}, std::true_type{}); else f(T6{}, std::false_type{});
-  } else if (bits == 5) {
-    if (clip) f(T5{}, std::true_type{}); else f(T5{}, std::false_type{});
-  } else {
-    if (clip) f(T8{}, std::true_type{}); else f(T8{}, std::false_type{});
-  }
+  using R0 = std::integral_constant<int, kClampW>;
+  using R1 = std::integral_constant<int, kClampGrid>;
+  using R2 = std::integral_constant<int, kNarrow>;
+  auto by_range = [&](auto bt) {
+    if (range == kNarrow) f(bt, R2{});
+    else if (range == kClampGrid) f(bt, R1{});
+    else f(bt, R0{});
+  };
+  if (bits == 6) by_range(T6{});
+  else if (bits == 5) by_range(T5{});
+  else by_range(T8{});
 }
 
 // Four codes packed little-endian into a word (byte permutes).
@@ -293,17 +335,20 @@ __device__ __forceinline__ uint32_t pack4(int c0, int c1, int c2, int c3) {
   return __byte_perm(lo, hi, 0x5410);
 }
 
-template <int BITS, bool CLIP>
+template <int BITS, int R>
 __device__ __forceinline__ uint32_t codes4_t(const RowQuant& q, float4 v) {
-  int c0, c1, c2, c3;
-  codes2<BITS, CLIP>(q, v.x, v.y, c0, c1);
-  codes2<BITS, CLIP>(q, v.z, v.w, c2, c3);
-  return pack4(c0, c1, c2, c3);
-}
-
-__device__ __forceinline__ uint32_t codes4(const RowQuant& q, float4 v) {
-  if (q.bits == 6) return codes4_t<6, true>(q, v);
-  return q.bits == 5 ? codes4_t<5, true>(q, v) : codes4_t<8, true>(q, v);
+  if constexpr (R == kNarrow && BITS != 6) {
+    // no clamp binds: the code's byte is the low byte of kOff + rne(w / s)
+    // (0x4B400000 has a zero low byte), so the offset need not be removed
+    const float2 t0 = rne_quot2<R>(q, v.x, v.y), t1 = rne_quot2<R>(q, v.z, v.w);
+    return pack4(__float_as_int(t0.x), __float_as_int(t0.y), __float_as_int(t1.x),
+                 __float_as_int(t1.y));
+  } else {
+    int c0, c1, c2, c3;
+    codes2<BITS, R>(q, v.x, v.y, c0, c1);
+    codes2<BITS, R>(q, v.z, v.w, c2, c3);
+    return pack4(c0, c1, c2, c3);
+  }
 }
 
 // ---- 6-bit packing of int6 / int5 codes: one 6-bit two's-complement field per
@@ -350,7 +395,7 @@ __device__ __forceinline__ void store_pack6_chunk(uint8_t* dst, uint32_t p, int 
 // independent dependency chains per warp.
 constexpr int kUnroll = 4;
 
-template <int BITS, bool CLIP>
+template <int BITS, int R>
 __device__ __forceinline__ void quantize_smem_row(const RowQuant& q, const float4* buf, int K4,
                                                   uint32_t* out, int lane) {
   int j = lane;
@@ -360,11 +405,11 @@ __device__ __forceinline__ void quantize_smem_row(const RowQuant& q, const float
     for (int u = 0; u < kUnroll; ++u) v[u] = buf[j + 32 * u];
     uint32_t c[kUnroll];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) c[u] = codes4_t<BITS, CLIP>(q, v[u]);
+    for (int u = 0; u < kUnroll; ++u) c[u] = codes4_t<BITS, R>(q, v[u]);
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) out[j + 32 * u] = c[u];
   }
-  for (; j < K4; j += 32) out[j] = codes4_t<BITS, CLIP>(q, buf[j]);
+  for (; j < K4; j += 32) out[j] = codes4_t<BITS, R>(q, buf[j]);
 }
 
 // The same codes stored 6-bit packed: NR rows of K4 float4 groups (K4 even),
@@ -372,7 +417,7 @@ __device__ __forceinline__ void quantize_smem_row(const RowQuant& q, const float
 // aligned).  The rows are interleaved, 4 / NR chunks of 32 groups each per
 // iteration, so every lane has four independent groups in flight; chunks are
 // warp-uniform, so the packing shuffles see every lane.
-template <int BITS, bool CLIP, int NR, typename Src>
+template <int BITS, int R, int NR, typename Src>
 __device__ __forceinline__ void quantize_rows_pack6(const RowQuant (&q)[NR], Src src, int K4,
                                                     uint8_t* const (&out)[NR], int lane) {
   constexpr int U = 4 / NR;
@@ -383,7 +428,7 @@ __device__ __forceinline__ void quantize_rows_pack6(const RowQuant (&q)[NR], Src
       const int j = base + 32 * u + lane;
 #pragma unroll
       for (int k = 0; k < NR; ++k)
-        p[k][u] = j < K4 ? pack24<BITS>(codes4_t<BITS, CLIP>(q[k], src(k, j))) : 0u;
+        p[k][u] = j < K4 ? pack24<BITS>(codes4_t<BITS, R>(q[k], src(k, j))) : 0u;
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -398,6 +443,8 @@ __device__ __forceinline__ void quantize_rows_pack6(const RowQuant (&q)[NR], Src
 }
 
 // A quantized row staged in shared memory (cols <= the batch's buffer).
+// PACK: the kernel also serves 6-bit packed descriptors.
+template <bool PACK>
 __device__ __forceinline__ void export_row_smem(const ExportDescDev& d, int64_t row,
                                                 const float4* buf, int lane) {
   const int K4 = static_cast<int>(d.cols >> 2);
@@ -421,93 +468,105 @@ __device__ __forceinline__ void export_row_smem(const ExportDescDev& d, int64_t 
   top2_warp(a1, a2);
   const RowQuant q = row_params(d, a1, a2);
   if (lane == 0) d.scales[row] = __float2half_rn(q.s);
-  const bool clip = a1 > 2.0f * q.clip;  // see codes2: clamping needed only then
-  if (d.pack6) {
+  const int range = row_range(a1, q);
+  if (PACK && d.pack6) {
     const RowQuant qs[1] = {q};
     uint8_t* const out[1] = {reinterpret_cast<uint8_t*>(d.dst) + row * 3 * K4};
-    with_grid(q.bits, clip, [&](auto bits_tag, auto clip_tag) {
+    with_grid(q.bits, range, [&](auto bits_tag, auto range_tag) {
       constexpr int B = decltype(bits_tag)::value;
       if constexpr (B != 8)
-        quantize_rows_pack6<B, decltype(clip_tag)::value, 1>(
+        quantize_rows_pack6<B, decltype(range_tag)::value, 1>(
             qs, [&](int, int j) { return buf[j]; }, K4, out, lane);
     });
     return;
   }
   uint32_t* out = reinterpret_cast<uint32_t*>(reinterpret_cast<int8_t*>(d.dst) + row * d.cols);
-  with_grid(q.bits, clip, [&](auto bits_tag, auto clip_tag) {
-    quantize_smem_row<decltype(bits_tag)::value, decltype(clip_tag)::value>(q, buf, K4, out, lane);
+  with_grid(q.bits, range, [&](auto bits_tag, auto range_tag) {
+    quantize_smem_row<decltype(bits_tag)::value, decltype(range_tag)::value>(q, buf, K4, out, lane);
   });
 }
 
-// Two rows of the same tensor staged in shared memory, processed together so
-// their top-2 passes, warp merges, scale computations and quantization passes
-// interleave (two independent dependency chains through every phase).
-__device__ __forceinline__ void export_two_rows_smem(const ExportDescDev& d, int64_t row,
-                                                     const float4* bufA, const float4* bufB,
-                                                     int lane) {
+// NR rows of the same tensor staged in shared memory (consecutive rows of one
+// work unit), processed together so their top-2 passes, warp merges, scale
+// computations and quantization passes interleave (NR independent dependency
+// chains through every phase).  The rows share the strictest clamp range.
+template <bool PACK, int NR>
+__device__ __forceinline__ void export_rows_smem(const ExportDescDev& d, int64_t row,
+                                                 const float4* buf, int lane) {
   const int K4 = static_cast<int>(d.cols >> 2);
-  float a1 = 0.0f, a2 = 0.0f, b1 = 0.0f, b2 = 0.0f, c1 = 0.0f, c2 = 0.0f, e1 = 0.0f, e2 = 0.0f;
+  float t1[NR], t2[NR], u1[NR], u2[NR];
+#pragma unroll
+  for (int k = 0; k < NR; ++k) t1[k] = t2[k] = u1[k] = u2[k] = 0.0f;
   int j = lane;
   for (; j + 32 < K4; j += 64) {
-    top2_push4(bufA[j], a1, a2);
-    top2_push4(bufB[j], b1, b2);
-    top2_push4(bufA[j + 32], c1, c2);
-    top2_push4(bufB[j + 32], e1, e2);
+#pragma unroll
+    for (int k = 0; k < NR; ++k) {
+      top2_push4(buf[k * K4 + j], t1[k], t2[k]);
+      top2_push4(buf[k * K4 + j + 32], u1[k], u2[k]);
+    }
   }
   if (j < K4) {
-    top2_push4(bufA[j], a1, a2);
-    top2_push4(bufB[j], b1, b2);
+#pragma unroll
+    for (int k = 0; k < NR; ++k) top2_push4(buf[k * K4 + j], t1[k], t2[k]);
   }
-  {
-    const float n2 = fmaxf(fminf(a1, c1), fmaxf(a2, c2));
-    a1 = fmaxf(a1, c1);
-    a2 = n2;
-    const float m2 = fmaxf(fminf(b1, e1), fmaxf(b2, e2));
-    b1 = fmaxf(b1, e1);
-    b2 = m2;
+  RowQuant q[NR];
+  int range = kNarrow;
+#pragma unroll
+  for (int k = 0; k < NR; ++k) {
+    const float n2 = fmaxf(fminf(t1[k], u1[k]), fmaxf(t2[k], u2[k]));
+    t1[k] = fmaxf(t1[k], u1[k]);
+    t2[k] = n2;
+    top2_warp(t1[k], t2[k]);
+    q[k] = row_params(d, t1[k], t2[k]);
+    range = min(range, row_range(t1[k], q[k]));
   }
-  top2_warp(a1, a2);
-  top2_warp(b1, b2);
-  const RowQuant qa = row_params(d, a1, a2);
-  const RowQuant qb = row_params(d, b1, b2);
   if (lane == 0) {
-    d.scales[row] = __float2half_rn(qa.s);
-    d.scales[row + 1] = __float2half_rn(qb.s);
+#pragma unroll
+    for (int k = 0; k < NR; ++k) d.scales[row + k] = __float2half_rn(q[k].s);
   }
-  const bool clip = (a1 > 2.0f * qa.clip) || (b1 > 2.0f * qb.clip);
-  if (d.pack6) {
-    const RowQuant qs[2] = {qa, qb};
-    uint8_t* const outA = reinterpret_cast<uint8_t*>(d.dst) + row * 3 * K4;
-    uint8_t* const out[2] = {outA, outA + 3 * K4};
-    with_grid(qa.bits, clip, [&](auto bits_tag, auto clip_tag) {
+  if (PACK && d.pack6) {
+    uint8_t* const out0 = reinterpret_cast<uint8_t*>(d.dst) + row * 3 * K4;
+    uint8_t* out[NR];
+#pragma unroll
+    for (int k = 0; k < NR; ++k) out[k] = out0 + k * 3 * K4;
+    with_grid(q[0].bits, range, [&](auto bits_tag, auto range_tag) {
       constexpr int B = decltype(bits_tag)::value;
       if constexpr (B != 8)
-        quantize_rows_pack6<B, decltype(clip_tag)::value, 2>(
-            qs, [&](int k, int j) { return k == 0 ? bufA[j] : bufB[j]; }, K4, out, lane);
+        quantize_rows_pack6<B, decltype(range_tag)::value, NR>(
+            q, [&](int k, int jj) { return buf[k * K4 + jj]; }, K4, out, lane);
     });
     return;
   }
-  uint32_t* outA = reinterpret_cast<uint32_t*>(reinterpret_cast<int8_t*>(d.dst) + row * d.cols);
-  uint32_t* outB = outA + K4;
-  auto run = [&](auto bits_tag, auto clip_tag) {
+  uint32_t* out = reinterpret_cast<uint32_t*>(reinterpret_cast<int8_t*>(d.dst) + row * d.cols);
+  auto run = [&](auto bits_tag, auto range_tag) {
     constexpr int BITS = decltype(bits_tag)::value;
-    constexpr bool CLIP = decltype(clip_tag)::value;
-    int k = lane;
-    for (; k + 32 < K4; k += 64) {
-      const float4 v0 = bufA[k], v1 = bufB[k], v2 = bufA[k + 32], v3 = bufB[k + 32];
-      const uint32_t c0 = codes4_t<BITS, CLIP>(qa, v0), c1v = codes4_t<BITS, CLIP>(qb, v1);
-      const uint32_t c2v = codes4_t<BITS, CLIP>(qa, v2), c3 = codes4_t<BITS, CLIP>(qb, v3);
-      outA[k] = c0;
-      outB[k] = c1v;
-      outA[k + 32] = c2v;
-      outB[k + 32] = c3;
+    constexpr int R = decltype(range_tag)::value;
+    int jj = lane;
+    for (; jj + 32 < K4; jj += 64) {
+      float4 v[NR][2];
+#pragma unroll
+      for (int k = 0; k < NR; ++k) {
+        v[k][0] = buf[k * K4 + jj];
+        v[k][1] = buf[k * K4 + jj + 32];
+      }
+      uint32_t c[NR][2];
+#pragma unroll
+      for (int k = 0; k < NR; ++k) {
+        c[k][0] = codes4_t<BITS, R>(q[k], v[k][0]);
+        c[k][1] = codes4_t<BITS, R>(q[k], v[k][1]);
+      }
+#pragma unroll
+      for (int k = 0; k < NR; ++k) {
+        out[k * K4 + jj] = c[k][0];
+        out[k * K4 + jj + 32] = c[k][1];
+      }
     }
-    if (k < K4) {
-      outA[k] = codes4_t<BITS, CLIP>(qa, bufA[k]);
-      outB[k] = codes4_t<BITS, CLIP>(qb, bufB[k]);
+    if (jj < K4) {
+#pragma unroll
+      for (int k = 0; k < NR; ++k) out[k * K4 + jj] = codes4_t<BITS, R>(q[k], buf[k * K4 + jj]);
     }
   };
-  with_grid(qa.bits, clip, run);
+  with_grid(q[0].bits, range, run);
 }
 
 // ---- clip search (the leaderboard's "GPTQ-lite" clip search, read as: per row,
@@ -582,8 +641,8 @@ __device__ __forceinline__ RowQuant candidate_params(const float (&top)[kClipSea
 template <int BITS>
 __device__ __forceinline__ float sq_err4(const RowQuant& q, float sh, float4 v, float e) {
   int c0, c1, c2, c3;
-  codes2<BITS, true>(q, v.x, v.y, c0, c1);
-  codes2<BITS, true>(q, v.z, v.w, c2, c3);
+  codes2<BITS, kClampW>(q, v.x, v.y, c0, c1);
+  codes2<BITS, kClampW>(q, v.z, v.w, c2, c3);
   const float d0 = __fmaf_rn(-static_cast<float>(c0), sh, v.x);
   const float d1 = __fmaf_rn(-static_cast<float>(c1), sh, v.y);
   const float d2 = __fmaf_rn(-static_cast<float>(c2), sh, v.z);
@@ -642,12 +701,12 @@ __device__ __forceinline__ void export_row_search_t(const ExportDescDev& d, int6
     if constexpr (BITS != 8) {
       const RowQuant qs[1] = {qb};
       uint8_t* const out[1] = {reinterpret_cast<uint8_t*>(d.dst) + row * 3 * K4};
-      quantize_rows_pack6<BITS, true, 1>(qs, [&](int, int j) { return buf[j]; }, K4, out, lane);
+      quantize_rows_pack6<BITS, kClampW, 1>(qs, [&](int, int j) { return buf[j]; }, K4, out, lane);
     }
     return;
   }
   uint32_t* out = reinterpret_cast<uint32_t*>(reinterpret_cast<int8_t*>(d.dst) + row * d.cols);
-  quantize_smem_row<BITS, true>(qb, buf, K4, out, lane);
+  quantize_smem_row<BITS, kClampW>(qb, buf, K4, out, lane);
 }
 
 __device__ __forceinline__ void export_row_search(const ExportDescDev& d, int64_t row,
@@ -658,6 +717,7 @@ __device__ __forceinline__ void export_row_search(const ExportDescDev& d, int64_
 }
 
 // A quantized row read from global memory (rows longer than the staging buffer).
+template <bool PACK>
 __device__ __forceinline__ void export_row_global(const ExportDescDev& d, int64_t row, int lane) {
   const int K4 = static_cast<int>(d.cols >> 2);
   const float4* r = reinterpret_cast<const float4*>(d.src + row * d.cols);
@@ -666,19 +726,23 @@ __device__ __forceinline__ void export_row_global(const ExportDescDev& d, int64_
   top2_warp(t1, t2);
   const RowQuant q = row_params(d, t1, t2);
   if (lane == 0) d.scales[row] = __float2half_rn(q.s);
-  if (d.pack6) {
+  if (PACK && d.pack6) {
     const RowQuant qs[1] = {q};
     uint8_t* const out[1] = {reinterpret_cast<uint8_t*>(d.dst) + row * 3 * K4};
-    with_grid(q.bits, true, [&](auto bits_tag, auto clip_tag) {
+    with_grid(q.bits, kClampW, [&](auto bits_tag, auto range_tag) {
       constexpr int B = decltype(bits_tag)::value;
       if constexpr (B != 8)
-        quantize_rows_pack6<B, decltype(clip_tag)::value, 1>(
+        quantize_rows_pack6<B, decltype(range_tag)::value, 1>(
             qs, [&](int, int j) { return __ldg(r + j); }, K4, out, lane);
     });
     return;
   }
   uint32_t* out = reinterpret_cast<uint32_t*>(reinterpret_cast<int8_t*>(d.dst) + row * d.cols);
-  for (int j = lane; j < K4; j += 32) out[j] = codes4(q, __ldg(r + j));
+  with_grid(q.bits, row_range(t1, q), [&](auto bits_tag, auto range_tag) {
+    constexpr int B = decltype(bits_tag)::value;
+    constexpr int R = decltype(range_tag)::value;
+    for (int j = lane; j < K4; j += 32) out[j] = codes4_t<B, R>(q, __ldg(r + j));
+  });
 }
 
 // fp16 passthrough of one chunk ("row") of a flat tensor.
@@ -768,7 +832,12 @@ __device__ __forceinline__ UnitPos unit_at(const ExportBatch& b, int64_t u) {
 // arrives in one bulk copy into one of the warp's kExportBufs buffers while
 // the warp quantizes the previous one.  Units that are not staged still arrive once on their buffer's
 // mbarrier so every buffer's phases stay in step with the unit count.
-template <bool SEARCH>
+// KIND selects the code a batch needs, so a plain export carries neither the
+// packing nor the search code (registers, instruction cache): kExportPlain,
+// kExportPacked (some descriptors 6-bit packed), kExportSearch (some with the
+// clip search; packing included).
+constexpr int kExportPlain = 0, kExportPacked = 1, kExportSearch = 2;
+template <int KIND>
 __global__ void __launch_bounds__(kExportMaxWarps * 32, 1)
     export_batch_kernel(const __grid_constant__ ExportBatch b, int* err) {
   extern __shared__ __align__(128) uint8_t xsmem[];
@@ -822,15 +891,20 @@ __global__ void __launch_bounds__(kExportMaxWarps * 32, 1)
       const int K4 = static_cast<int>(d.cols >> 2);
       const float4* ub = bufs + slot * stride;
       int r = 0;
-      if (SEARCH && d.search) {
+      constexpr bool PACK = KIND != kExportPlain;
+      if (KIND == kExportSearch && d.search) {
         for (; r < pos[0].nrows; ++r) export_row_search(d, pos[0].row0 + r, ub + r * K4, lane);
       } else {
-        for (; r + 1 < pos[0].nrows; r += 2)
-          export_two_rows_smem(d, pos[0].row0 + r, ub + r * K4, ub + (r + 1) * K4, lane);
-        if (r < pos[0].nrows) export_row_smem(d, pos[0].row0 + r, ub + r * K4, lane);
+        for (; r + 2 < pos[0].nrows; r += 3)
+          export_rows_smem<PACK, 3>(d, pos[0].row0 + r, ub + r * K4, lane);
+        if (r + 1 < pos[0].nrows) {
+          export_rows_smem<PACK, 2>(d, pos[0].row0 + r, ub + r * K4, lane);
+          r += 2;
+        }
+        if (r < pos[0].nrows) export_row_smem<PACK>(d, pos[0].row0 + r, ub + r * K4, lane);
       }
     } else {
-      export_row_global(d, pos[0].row0, lane);
+      export_row_global<KIND != kExportPlain>(d, pos[0].row0, lane);
     }
     // the buffer is read; order those reads before the copy engine refills it
     fence_proxy_async_smem();
@@ -960,10 +1034,13 @@ int launch_export_batch(ExportBatch& b, cudaStream_t s) {
   if (b.total_units == 0) return QAT_OK;
   static bool attr_done = false;
   if (!attr_done) {
-    if (cudaFuncSetAttribute(export_batch_kernel<false>,
+    if (cudaFuncSetAttribute(export_batch_kernel<kExportPlain>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kExportSmemBudget) != cudaSuccess ||
-        cudaFuncSetAttribute(export_batch_kernel<true>,
+        cudaFuncSetAttribute(export_batch_kernel<kExportPacked>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kExportSmemBudget) != cudaSuccess ||
+        cudaFuncSetAttribute(export_batch_kernel<kExportSearch>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kExportSmemBudget) != cudaSuccess)
       return QAT_ERR_CUDA;
@@ -979,13 +1056,17 @@ int launch_export_batch(ExportBatch& b, cudaStream_t s) {
   const int smem = warps * per_warp;
   const int64_t want = (b.total_units + warps - 1) / warps;
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, sm_count())));
-  bool search = false;
-  for (int i = 0; i < b.n; ++i) search = search || b.d[i].search;
-  // the search's registers stay out of the plain export kernel
+  bool search = false, packed = false;
+  for (int i = 0; i < b.n; ++i) {
+    search = search || b.d[i].search;
+    packed = packed || b.d[i].pack6;
+  }
   if (search)
-    export_batch_kernel<true><<<grid, warps * 32, smem, s>>>(b, device_error_ptr());
+    export_batch_kernel<kExportSearch><<<grid, warps * 32, smem, s>>>(b, device_error_ptr());
+  else if (packed)
+    export_batch_kernel<kExportPacked><<<grid, warps * 32, smem, s>>>(b, device_error_ptr());
   else
-    export_batch_kernel<false><<<grid, warps * 32, smem, s>>>(b, device_error_ptr());
+    export_batch_kernel<kExportPlain><<<grid, warps * 32, smem, s>>>(b, device_error_ptr());
   count_launch();
   return cuda_status(cudaGetLastError());
 }
