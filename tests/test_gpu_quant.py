@@ -35,6 +35,20 @@ def _weights():
     z[2] = 0.5
     z[3, ::2] = -7.0
     cases["degenerate_8x64"] = z
+    # rows longer than one staged unit are exported as two half-row units by a
+    # warp pair: ragged halves (1040), halves of 1024 (2048), a width that is
+    # not split (1032, not a multiple of 16), and rows whose top two |w| tie
+    # across the halves, inside one half, or sit in different halves
+    cases["split_37x1040"] = (rng.standard_normal((37, 1040)) * 0.02).astype(np.float32)
+    cases["split_9x2048"] = (rng.standard_normal((9, 2048)) * 0.02).astype(np.float32)
+    cases["whole_11x1032"] = (rng.standard_normal((11, 1032)) * 0.02).astype(np.float32)
+    t = (rng.standard_normal((5, 1536)) * 0.02).astype(np.float32)
+    t[0, 100], t[0, 1200] = 0.5, -0.5  # max once in each half
+    t[1, 10], t[1, 20] = 0.5, 0.5      # max twice in the first half
+    t[2, 800], t[2, 1500] = 0.5, 0.25  # top two in the second half
+    t[3, 767], t[3, 768] = -0.4, 0.3   # top two on either side of the split
+    t[4] = 0.125                       # a constant row
+    cases["split_ties_5x1536"] = t
     return cases
 
 
