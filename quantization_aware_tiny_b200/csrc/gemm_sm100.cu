@@ -312,6 +312,12 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR, EPI, FB>::THREADS, 1)
   if constexpr (PAIR) cluster_sync(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Launched as a programmatic dependent of the previous kernel in the stream:
+  // everything above (barriers, TMEM, descriptor prefetch) overlapped its tail;
+  // no global memory is touched before the previous grid has completed.  Then
+  // let the next GEMM's CTAs launch onto SMs as this grid's CTAs retire.
+  grid_dependency_wait();
+  grid_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -680,13 +686,16 @@ int launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& md
   cfg.blockDim = dim3(C::THREADS);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = PAIR ? 2 : 1;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // programmatic dependent launch (the kernel waits with griddepcontrol.wait)
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ma, mb, md, md2, mr, a);
   count_launch();
   return cuda_status(e == cudaSuccess ? cudaGetLastError() : e);
