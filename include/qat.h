@@ -94,6 +94,23 @@ typedef struct qat_qweight {
 int qat_quantize_weights(const float* W, int32_t N, int32_t K, int32_t bits, int8_t* codes,
                          float* scales, qat_bf16* operand, qat_stream_t stream);
 
+/* The same quantization for several weights in one launch (all of a training
+ * step's weights, each on its own grid): descs[i] holds W [N,K] fp32, bits,
+ * scales [N] (required), codes [N,K] and operand [N,K] (nullable) exactly as
+ * qat_quantize_weights takes them.  1 <= n <= QAT_QUANT_MAX_DESCS; the
+ * descriptor array is read on the host during the call.  Each weight's
+ * outputs are bit-identical to a qat_quantize_weights call on it; outputs
+ * must not overlap one another or any W. */
+#define QAT_QUANT_MAX_DESCS 16
+typedef struct qat_quant_desc {
+  const float* W;
+  int8_t* codes;
+  float* scales;
+  qat_bf16* operand;
+  int32_t N, K, bits, pad;
+} qat_quant_desc;
+int qat_quantize_weights_batch(const qat_quant_desc* descs, int32_t n, qat_stream_t stream);
+
 /* Noisy QAT for the shared blocks of a depth-recurrent core ([P1] "幸存发现 1
  * Noisy QAT"): instead of the STE fake quantization, the forward weight is
  *   w' = fl32(w + fl32(fl32(u - 1/2) * s)),  s = fl32(max(amax_row, 1e-12) / L),

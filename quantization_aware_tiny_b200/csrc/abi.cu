@@ -153,6 +153,24 @@ int qat_quantize_weights(const float* W, int32_t N, int32_t K, int32_t bits, int
                                  reinterpret_cast<__nv_bfloat16*>(operand), stream);
 }
 
+int qat_quantize_weights_batch(const qat_quant_desc* descs, int32_t n, qat_stream_t stream) {
+  if (!descs || n <= 0 || n > QAT_QUANT_MAX_DESCS) return QAT_ERR_ARG;
+  QuantBatch b;
+  b.n = n;
+  b.row_begin[0] = 0;
+  for (int i = 0; i < n; ++i) {
+    const qat_quant_desc& s = descs[i];
+    if (!s.W || !s.scales || s.N <= 0 || !bits_ok(s.bits)) return QAT_ERR_ARG;
+    if (!dim_ok(s.K)) return QAT_ERR_SHAPE;
+    if (!aligned16(s.W) || (s.codes && !aligned16(s.codes)) || (s.operand && !aligned16(s.operand)))
+      return QAT_ERR_ALIGN;
+    b.d[i] = QuantDescDev{s.W, s.codes, s.scales, reinterpret_cast<__nv_bfloat16*>(s.operand),
+                          s.N, s.K, s.bits, 0};
+    b.row_begin[i + 1] = b.row_begin[i] + s.N;
+  }
+  return launch_quantize_batch(b, stream);
+}
+
 int qat_linear_fwd(const float* W, const qat_qweight* qw, int32_t N, int32_t K, int32_t bits,
                    const qat_bf16* X, int64_t ldx, int64_t T, const qat_bf16* residual,
                    qat_bf16* Y, void* workspace, size_t ws_bytes, qat_stream_t stream) {

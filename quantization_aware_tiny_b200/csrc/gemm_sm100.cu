@@ -830,6 +830,9 @@ int launch_gemm(const GemmDesc& g, cudaStream_t stream) {
     BN = fused_b_bn(g.N, g.K);
   } else if (kmajor_fwd && g.M >= 256 && g.N >= 160) {
     pair = true;
+    // (a wave-count rule -- the width of fewest ceil(tiles / pairs) * BN -- was
+    // slower: 160-wide tiles for the d = 640 core's N = 1280 filled the waves
+    // better but cost more operand traffic per FLOP, core 0.42 -> 0.44 ms)
     BN = (g.N % 256 == 0) ? 256 : (g.N % 192 == 0) ? 192 : (g.N % 160 == 0) ? 160 : 256;
   } else {
     const int64_t pad256 = (g.N + 255) / 256 * 256 - g.N;

@@ -43,46 +43,56 @@ __device__ __forceinline__ uint2 operand4(int c0, int c1, int c2, int c3, float 
 }
 
 // ------------------------------------------------------------------ QAT quantize
-__global__ void __launch_bounds__(kQThreads)
-    quantize_weights_kernel(const float* __restrict__ W, int N, int K, int bits,
-                            int8_t* __restrict__ codes, float* __restrict__ scales,
-                            __nv_bfloat16* __restrict__ operand) {
-  const int lane = threadIdx.x & 31;
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+// One row of one weight: amax over the row (cached in registers up to 2048
+// columns), the IEEE scale, codes and the bf16 operand.
+__device__ __forceinline__ void quantize_row(const QuantDescDev& d, int row, int lane) {
+  const int K = d.K, bits = d.bits;
   const int K4 = K >> 2;
-  for (int row = warp; row < N; row += nwarps) {
-    const float4* r = reinterpret_cast<const float4*>(W + static_cast<int64_t>(row) * K);
-    float4 cache[kRegV4];
-    float amax = 0.0f;
+  const float4* r = reinterpret_cast<const float4*>(d.W + static_cast<int64_t>(row) * K);
+  float4 cache[kRegV4];
+  float amax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < kRegV4; ++i) {
-      const int j = lane + 32 * i;
-      if (j < K4) {
-        cache[i] = __ldg(r + j);
-        amax = fmaxf(amax, amax4(cache[i]));
-      }
+  for (int i = 0; i < kRegV4; ++i) {
+    const int j = lane + 32 * i;
+    if (j < K4) {
+      cache[i] = __ldg(r + j);
+      amax = fmaxf(amax, amax4(cache[i]));
     }
-    for (int j = lane + 32 * kRegV4; j < K4; j += 32) amax = fmaxf(amax, amax4(__ldg(r + j)));
+  }
+  for (int j = lane + 32 * kRegV4; j < K4; j += 32) amax = fmaxf(amax, amax4(__ldg(r + j)));
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    amax = fmaxf(amax, 1e-12f);
-    const float s = div_rn(amax, grid_levels(bits));
-    const float rs = __frcp_rn(s);
-    if (lane == 0) scales[row] = s;
-    auto emit = [&](int j, float4 v) {
-      const int c0 = quant_code(v.x, s, rs, bits), c1 = quant_code(v.y, s, rs, bits);
-      const int c2 = quant_code(v.z, s, rs, bits), c3 = quant_code(v.w, s, rs, bits);
-      const int64_t e = static_cast<int64_t>(row) * K + 4 * j;
-      if (codes) *reinterpret_cast<uint32_t*>(codes + e) = pack_codes(c0, c1, c2, c3);
-      if (operand) *reinterpret_cast<uint2*>(operand + e) = operand4(c0, c1, c2, c3, s);
-    };
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  amax = fmaxf(amax, 1e-12f);
+  const float s = div_rn(amax, grid_levels(bits));
+  const float rs = __frcp_rn(s);
+  if (lane == 0) d.scales[row] = s;
+  auto emit = [&](int j, float4 v) {
+    const int c0 = quant_code(v.x, s, rs, bits), c1 = quant_code(v.y, s, rs, bits);
+    const int c2 = quant_code(v.z, s, rs, bits), c3 = quant_code(v.w, s, rs, bits);
+    const int64_t e = static_cast<int64_t>(row) * K + 4 * j;
+    if (d.codes) *reinterpret_cast<uint32_t*>(d.codes + e) = pack_codes(c0, c1, c2, c3);
+    if (d.operand) *reinterpret_cast<uint2*>(d.operand + e) = operand4(c0, c1, c2, c3, s);
+  };
 #pragma unroll
-    for (int i = 0; i < kRegV4; ++i) {
-      const int j = lane + 32 * i;
-      if (j < K4) emit(j, cache[i]);
-    }
-    for (int j = lane + 32 * kRegV4; j < K4; j += 32) emit(j, __ldg(r + j));
+  for (int i = 0; i < kRegV4; ++i) {
+    const int j = lane + 32 * i;
+    if (j < K4) emit(j, cache[i]);
+  }
+  for (int j = lane + 32 * kRegV4; j < K4; j += 32) emit(j, __ldg(r + j));
+}
+
+// All rows of all the batch's weights, a warp per row (grid-stride over the
+// concatenated rows), so small weights share the launch and the SMs.
+__global__ void __launch_bounds__(kQThreads)
+    quantize_batch_kernel(const __grid_constant__ QuantBatch b) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int64_t total = b.row_begin[b.n];
+  int k = 0;
+  for (int64_t g = warp; g < total; g += nwarps) {
+    while (k + 1 < b.n && b.row_begin[k + 1] <= g) ++k;  // rows are visited in increasing order
+    quantize_row(b.d[k], static_cast<int>(g - b.row_begin[k]), lane);
   }
 }
 
@@ -987,12 +997,22 @@ int grid_for_rows(int64_t rows_or_items, int items_per_block) {
 
 }  // namespace
 
-int launch_quantize_weights(const float* W, int N, int K, int bits, int8_t* codes, float* scales,
-                            __nv_bfloat16* operand, cudaStream_t s) {
-  quantize_weights_kernel<<<grid_for_rows(N, kQThreads / 32), kQThreads, 0, s>>>(
-      W, N, K, bits, codes, scales, operand);
+int launch_quantize_batch(const QuantBatch& b, cudaStream_t s) {
+  const int64_t total = b.row_begin[b.n];
+  if (total == 0) return QAT_OK;
+  quantize_batch_kernel<<<grid_for_rows(total, kQThreads / 32), kQThreads, 0, s>>>(b);
   count_launch();
   return cuda_status(cudaGetLastError());
+}
+
+int launch_quantize_weights(const float* W, int N, int K, int bits, int8_t* codes, float* scales,
+                            __nv_bfloat16* operand, cudaStream_t s) {
+  QuantBatch b;
+  b.n = 1;
+  b.row_begin[0] = 0;
+  b.row_begin[1] = N;
+  b.d[0] = QuantDescDev{W, codes, scales, operand, N, K, bits, 0};
+  return launch_quantize_batch(b, s);
 }
 
 int launch_noisy_operand(const float* W, int N, int K, int bits, uint64_t seed, uint64_t offset,

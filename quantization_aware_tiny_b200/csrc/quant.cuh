@@ -55,6 +55,22 @@ constexpr int64_t kExportMaxStagedCols = 2048;
 constexpr int kExportSmemBudget = 224 * 1024;
 constexpr int kExportMaxWarps = 16;
 
+// Training-time quantization of several weights in one launch (a warp per row
+// over the rows of all of them).
+constexpr int kQuantMaxDescs = QAT_QUANT_MAX_DESCS;
+struct QuantDescDev {
+  const float* W;
+  int8_t* codes;
+  float* scales;
+  __nv_bfloat16* operand;
+  int N, K, bits, pad;
+};
+struct QuantBatch {
+  int n;
+  int64_t row_begin[kQuantMaxDescs + 1];  // first global row of each weight; [n] = total
+  QuantDescDev d[kQuantMaxDescs];
+};
+int launch_quantize_batch(const QuantBatch& b, cudaStream_t s);
 int launch_quantize_weights(const float* W, int N, int K, int bits, int8_t* codes, float* scales,
                             __nv_bfloat16* operand, cudaStream_t s);
 int launch_noisy_operand(const float* W, int N, int K, int bits, uint64_t seed, uint64_t offset,

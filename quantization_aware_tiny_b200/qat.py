@@ -26,7 +26,8 @@ QAT_DTYPE_F32, QAT_DTYPE_BF16 = 0, 1
 EXPORTED = ("qat_strerror", "qat_launch_count", "qat_device_error", "qat_quantize_weights",
             "qat_workspace_size", "qat_linear_fwd", "qat_linear_bwd", "qat_mlp_fwd",
             "qat_mlp_bwd", "quantize_rows_export", "quantize_export_batch", "dequantize_rows",
-            "qat_linear_fwd_noalloc", "qat_noisy_operand", "unpack_codes6")
+            "qat_linear_fwd_noalloc", "qat_noisy_operand", "unpack_codes6",
+            "qat_quantize_weights_batch")
 QAT_EXPORT_PACK6 = 1
 QAT_EXPORT_CLIP_SEARCH = 2
 QAT_ACT_RELU2 = 0
@@ -46,6 +47,12 @@ class _QWeight(ctypes.Structure):
     _fields_ = [("operand", ctypes.c_void_p), ("scales", ctypes.c_void_p),
                 ("codes", ctypes.c_void_p), ("N", ctypes.c_int32), ("K", ctypes.c_int32),
                 ("bits", ctypes.c_int32)]
+
+
+class _QuantDesc(ctypes.Structure):
+    _fields_ = [("W", ctypes.c_void_p), ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("operand", ctypes.c_void_p), ("N", ctypes.c_int32), ("K", ctypes.c_int32),
+                ("bits", ctypes.c_int32), ("pad", ctypes.c_int32)]
 
 
 class _ExportDesc(ctypes.Structure):
@@ -72,6 +79,7 @@ def lib():
         L.qat_launch_count.restype = I64
         L.qat_device_error.argtypes = [P]
         L.qat_quantize_weights.argtypes = [P, I32, I32, I32, P, P, P, P]
+        L.qat_quantize_weights_batch.argtypes = [P, I32, P]
         L.qat_workspace_size.argtypes = [I32, I32, I32, I64, I32]
         L.qat_workspace_size.restype = SZ
         L.qat_linear_fwd.argtypes = [P, P, I32, I32, I32, P, I64, I64, P, P, P, SZ, P]
@@ -155,6 +163,36 @@ def qat_quantize_weights(W, bits, scales, codes=None, operand=None, stream=None)
     N, K = W.shape
     _check(lib().qat_quantize_weights(_p(W), N, K, bits, _p(codes), _p(scales), _p(operand),
                                       _stream(stream)), "qat_quantize_weights")
+
+
+QAT_QUANT_MAX_DESCS = 16
+
+
+def qat_quantize_weights_batch(items, stream=None):
+    """items: (W, bits, scales, codes, operand) per weight (codes / operand may
+    be None); one launch for all of them."""
+    arr = (_QuantDesc * len(items))()
+    for i, (W, bits, scales, codes, operand) in enumerate(items):
+        N, K = W.shape
+        arr[i] = _QuantDesc(W.data_ptr(), _p(codes), _p(scales), _p(operand), N, K, bits, 0)
+    _check(lib().qat_quantize_weights_batch(ctypes.cast(arr, ctypes.c_void_p), len(items),
+                                            _stream(stream)), "qat_quantize_weights_batch")
+
+
+def quantize_weights(Ws, bits, keep_codes=False, stream=None):
+    """Quantize several weights (bits: one per weight, or one for all) in one
+    launch into new QWeights."""
+    bits = list(bits) if isinstance(bits, (list, tuple)) else [bits] * len(Ws)
+    out = []
+    for W, b in zip(Ws, bits):
+        N, K = W.shape
+        out.append(QWeight(torch.empty((N, K), dtype=torch.bfloat16, device=W.device),
+                           torch.empty(N, dtype=torch.float32, device=W.device),
+                           torch.empty((N, K), dtype=torch.int8, device=W.device) if keep_codes else None,
+                           b))
+    qat_quantize_weights_batch([(W, q.bits, q.scales, q.codes, q.operand) for W, q in zip(Ws, out)],
+                               stream)
+    return out
 
 
 def quantize_weight(W, bits, keep_codes=False, stream=None):

@@ -29,8 +29,8 @@ class RecurrentCore:
         self.act = act
         Wqkv = torch.cat([Wq, Wk, Wv], dim=0).contiguous()
         self.W = (Wqkv, Wo.contiguous(), Wfc.contiguous(), Wproj.contiguous())
-        self.q_qkv, self.q_o, self.q_fc, self.q_proj = (
-            qat.quantize_weight(w, bits, stream=stream) for w in self.W)
+        self.q_qkv, self.q_o, self.q_fc, self.q_proj = qat.quantize_weights(self.W, bits,
+                                                                             stream=stream)
         self.nqkv = Wqkv.shape[0]
         self._buf = None
 
@@ -102,8 +102,9 @@ class HeadMlpStep:
         self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
 
     def quantize(self, stream=None):
-        for w, q in zip(self.W, self.q):
-            qat.qat_quantize_weights(w, q.bits, q.scales, None, q.operand, stream)
+        """All three weights' operands in one launch."""
+        qat.qat_quantize_weights_batch([(w, q.bits, q.scales, None, q.operand)
+                                        for w, q in zip(self.W, self.q)], stream)
 
     def forward(self, X, stream=None):
         qe, qf, qp = self.q

@@ -273,3 +273,23 @@ def test_near_tie_quotients_bit_exact(bits):
     c_ref, s_ref, _ = o.export_rows(W, bits)
     assert np.array_equal(codes.cpu().numpy(), c_ref)
     assert np.array_equal(bits16(s16), s_ref)
+
+
+def test_quantize_weights_batch_one_launch():
+    """Several weights (mixed grids and widths) quantized in one launch equal
+    the oracle bit for bit, as one call per weight does."""
+    ws = _weights()
+    names = ["head_8192x512", "fc_1536x512_heavy", "proj_512x1536_heavy", "ragged_200x136",
+             "longrow_64x4104", "degenerate_8x64"]
+    bits = [8, 6, 6, 5, 6, 8]
+    Ws = [_dev(ws[n]) for n in names]
+    n0 = qat.launch_count()
+    qs = qat.quantize_weights(Ws, bits, keep_codes=True)
+    torch.cuda.synchronize()
+    assert qat.launch_count() - n0 == 1
+    for n, b, q in zip(names, bits, qs):
+        ref = o.quantize_weight(ws[n], b)
+        assert np.array_equal(q.codes.cpu().numpy(), ref["codes"]), n
+        assert np.array_equal(q.scales.cpu().numpy().view(np.uint32), ref["scales"].view(np.uint32)), n
+        assert np.array_equal(bits16(q.operand), o.operand_bf16_bits(ref["codes"], ref["scales"])), n
+    assert qat.device_error() == 0

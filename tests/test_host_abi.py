@@ -71,6 +71,19 @@ def test_argument_validation_before_launch(L):
     assert L.qat_linear_fwd(None, None, 512, 512, 6, A16, 0, 256, None, A16, None, 0, None) == qat.QAT_ERR_ARG
     # misaligned weights
     assert L.qat_quantize_weights(A_BAD, 512, 512, 6, None, A16, None, None) == qat.QAT_ERR_ALIGN
+    # batched quantize: descriptor count, null pointers, bits, shape, alignment
+    Q = qat._QuantDesc
+    ok = Q(0x10000, None, 0x10000, 0x10000, 512, 512, 6, 0)
+    arr = (Q * 17)(*([ok] * 17))
+    assert L.qat_quantize_weights_batch(None, 1, None) == qat.QAT_ERR_ARG
+    assert L.qat_quantize_weights_batch(ctypes.cast(arr, ctypes.c_void_p), 0, None) == qat.QAT_ERR_ARG
+    assert L.qat_quantize_weights_batch(ctypes.cast(arr, ctypes.c_void_p), 17, None) == qat.QAT_ERR_ARG
+    for bad, rc in ((Q(0x10000, None, None, 0x10000, 512, 512, 6, 0), qat.QAT_ERR_ARG),
+                    (Q(0x10000, None, 0x10000, 0x10000, 512, 512, 7, 0), qat.QAT_ERR_ARG),
+                    (Q(0x10000, None, 0x10000, 0x10000, 512, 500, 6, 0), qat.QAT_ERR_SHAPE),
+                    (Q(0x10004, None, 0x10000, 0x10000, 512, 512, 6, 0), qat.QAT_ERR_ALIGN)):
+        two = (Q * 2)(ok, bad)  # the bad descriptor second: nothing launches for the first either
+        assert L.qat_quantize_weights_batch(ctypes.cast(two, ctypes.c_void_p), 2, None) == rc
     # workspace too small for raw weights
     assert L.qat_linear_fwd(A16, None, 512, 512, 6, A16, 0, 256, None, A16, A16, 1024, None) == qat.QAT_ERR_WORKSPACE
     # no workspace and no fused path (fewer than 256 tokens, or K > 1024)
