@@ -132,9 +132,10 @@ def make_inputs(seed, device):
     return {k: (torch.from_numpy(v) if isinstance(v, np.ndarray) else v) for k, v in c.items()}
 
 
-def timed_calls(step, X, dL, ev_pairs, stream):
+def timed_calls(step, X, dL, ev_pairs, stream, on_head_grad=None):
     """One step with CUDA events around each call (the head GEMM calls are
-    single kernels; quantize and the MLP calls are the step's other launches)."""
+    single kernels; quantize and the MLP calls are the step's other launches).
+    on_head_grad() runs between the head's backward and the MLP backward."""
     from quantization_aware_tiny_b200 import qat
     qe, qf, qp = step.q
 
@@ -150,6 +151,8 @@ def timed_calls(step, X, dL, ev_pairs, stream):
     timed("head_dX", lambda: qat.qat_linear_bwd(step.Z, dL, 8, qw=qe, dX=step.dZ, stream=stream))
     timed("head_dW", lambda: qat.qat_linear_bwd(step.Z, dL, 8, dW=step.dWemb, N=VOCAB, K=D,
                                                 stream=stream))
+    if on_head_grad is not None:
+        on_head_grad()
     timed("mlp_bwd", lambda: qat.qat_mlp_bwd(X, step.pre, step.h, step.dZ, 6, D, H, qfc=qf,
                                              qproj=qp, dX=step.dX, dWfc=step.dWfc,
                                              dWproj=step.dWproj, workspace=step.ws,
@@ -181,16 +184,22 @@ def run_ours(args):
     names = CALLS
     per_step_events = []
 
+    sync = dp.GradSync(pg) if pg is not None else None
+    # with N > 1 the tied head's gradient is summed while the MLP backward runs;
+    # the MLP's gradients follow, and every sum completes within the step
+    head_hook = (lambda: sync.start([step.dWemb], stream)) if sync is not None else None
+
     def one(i, timed):
         if timed:
             ev = {n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                   for n in names}
             per_step_events.append(ev)
-            timed_calls(step, X, dL, ev, stream)
+            timed_calls(step, X, dL, ev, stream, head_hook)
         else:
-            step.step(X, dL, stream)
-        if pg is not None:
-            dp.allreduce_grads(step.grads(), pg)
+            step.step(X, dL, stream, head_hook)
+        if sync is not None:
+            sync.start([step.dWfc, step.dWproj], stream)
+            sync.wait(stream)
 
     for i in range(args.warmup):
         one(i, False)
@@ -274,12 +283,16 @@ def measure_e2e(step, inp, dev, stream, args, pg, flops_step, world):
     hg = [torch.empty(g.shape, dtype=g.dtype, pin_memory=True) for g in step.grads()]
     steps_e2e = max(3, min(args.steps, 10))
 
+    sync = dp.GradSync(pg) if pg is not None else None
+    head_hook = (lambda: sync.start([step.dWemb], stream)) if sync is not None else None
+
     def one():
         X.copy_(hX, non_blocking=True)
         dL.copy_(hdL, non_blocking=True)
-        step.step(X, dL, stream)
-        if pg is not None:
-            dp.allreduce_grads(step.grads(), pg)
+        step.step(X, dL, stream, head_hook)
+        if sync is not None:
+            sync.start([step.dWfc, step.dWproj], stream)
+            sync.wait(stream)
         for h, g in zip(hg, step.grads()):
             h.copy_(g, non_blocking=True)
 

@@ -112,18 +112,22 @@ class HeadMlpStep:
                         pre_save=self.pre, h_save=self.h, stream=stream, act=self.act)
         qat.qat_linear_fwd(self.Z, self.logits, self.head_bits, qw=qe, stream=stream)
 
-    def backward(self, X, dLogits, stream=None):
+    def backward(self, X, dLogits, stream=None, on_head_grad=None):
+        """on_head_grad(): called once the head's backward is queued (its dWemb
+        is then complete in stream order), before the MLP backward."""
         qe, qf, qp = self.q
         qat.qat_linear_bwd(self.Z, dLogits, self.head_bits, qw=qe, dX=self.dZ, dW=self.dWemb,
                            stream=stream)
+        if on_head_grad is not None:
+            on_head_grad()
         qat.qat_mlp_bwd(X, self.pre, self.h, self.dZ, self.mlp_bits, self.d, self.H, qfc=qf,
                         qproj=qp, dX=self.dX, dWfc=self.dWfc, dWproj=self.dWproj,
                         workspace=self.ws, stream=stream, act=self.act)
 
-    def step(self, X, dLogits, stream=None):
+    def step(self, X, dLogits, stream=None, on_head_grad=None):
         self.quantize(stream)
         self.forward(X, stream)
-        self.backward(X, dLogits, stream)
+        self.backward(X, dLogits, stream, on_head_grad)
 
     def grads(self):
         return [self.dWemb, self.dWfc, self.dWproj]

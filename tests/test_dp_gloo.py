@@ -65,3 +65,46 @@ def test_dp_allreduce_equals_full_batch_gradient():
     for g, k in zip(grads, ("dWemb", "dWfc", "dWproj")):
         assert np.allclose(g, full[k], rtol=1e-12, atol=1e-12), k
     assert mx == 11.0
+
+
+def _sync_worker(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from quantization_aware_tiny_b200 import dp
+        g = torch.Generator().manual_seed(100 + rank)
+        head = torch.randn(64, 32, generator=g)
+        fc, proj = torch.randn(16, 32, generator=g), torch.randn(32, 16, generator=g)
+        mine = [head.clone(), fc.clone(), proj.clone()]
+        sync = dp.GradSync(dist)
+        sync.start([head])           # as soon as the head's backward is queued
+        busy = torch.randn(256, 256, generator=g) @ torch.randn(256, 256, generator=g)  # "MLP backward"
+        sync.start([fc, proj])       # the MLP's gradients at the end of the step
+        sync.wait()
+        if rank == 0:
+            out.put(([t.numpy() for t in (head, fc, proj)], [t.numpy() for t in mine], float(busy.sum())))
+        else:
+            out.put(([t.numpy() for t in mine], None, None))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_grad_sync_overlapped_sums_equal_plain_sums():
+    """GradSync (the head gradient's sum started before the MLP backward, the
+    MLP's after it, one wait) gives every rank the plain sum of all ranks'
+    gradients, as the serial all-reduce did."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_sync_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = [q.get(timeout=120) for _ in range(2)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    summed = next(g for g in got if g[1] is not None)
+    other = next(g for g in got if g[1] is None)[0]
+    for s, a, b in zip(summed[0], summed[1], other):
+        assert np.allclose(s, a + b, rtol=0, atol=1e-5)
