@@ -105,6 +105,38 @@ def test_head_mlp_step_small():
         assert_close(g, ref[name], name)
 
 
+def test_head_mlp_step_4096_tokens_every_output():
+    """The throughput configuration at its smallest token count (4,096): every
+    output and every gradient entry against the oracle."""
+    c = sy.head_mlp_case(T=4096, seed=3)
+    s = _head_step(c)
+    qe, qf, qp = _head_q(c)
+    ref = o.head_mlp_step(qe, qf, qp, c["X"].float().numpy(), c["dLogits"].float().numpy())
+    for name, g in (("Z", s.Z), ("logits", s.logits), ("dZ", s.dZ), ("dX", s.dX),
+                    ("dWemb", s.dWemb), ("dWfc", s.dWfc), ("dWproj", s.dWproj)):
+        assert_close(g, ref[name], name)
+    assert qat.device_error() == 0
+
+
+def test_head_mlp_step_16384_tokens_sampled():
+    """16,384 tokens: per-token outputs on sampled rows; weight-gradient entries
+    on sampled rows and columns, each summed over all tokens by the oracle."""
+    T = 16384
+    c = sy.head_mlp_case(T=T, seed=4)
+    s = _head_step(c)
+    qe, qf, qp = _head_q(c)
+    rows = np.concatenate([np.random.default_rng(2).choice(T, 40, replace=False), [0, T - 1]])
+    Xall, dLall = c["X"].float().numpy(), c["dLogits"].float().numpy()
+    ref = o.head_mlp_step(qe, qf, qp, Xall[rows], dLall[rows])
+    for name, g in (("Z", s.Z), ("logits", s.logits), ("dZ", s.dZ), ("dX", s.dX)):
+        assert_close(to_np(g)[rows], ref[name], name)
+    # dWemb[v, k] = sum_t dL[t, v] Z[t, k], with Z the MLP output of every token
+    Z = o.linear_fwd(qp["operand"], o.relu2(o.linear_fwd(qf["operand"], Xall)))
+    vs, ks = [0, 4095, 8191], [0, 255, 511]
+    assert_close(to_np(s.dWemb)[np.ix_(vs, ks)], dLall[:, vs].T @ Z[:, ks], "dWemb sampled")
+    assert qat.device_error() == 0
+
+
 @pytest.fixture(scope="module")
 def full_head():
     c = sy.head_mlp_case(T=65536)
