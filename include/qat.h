@@ -94,8 +94,9 @@ typedef struct qat_qweight {
 int qat_quantize_weights(const float* W, int32_t N, int32_t K, int32_t bits, int8_t* codes,
                          float* scales, qat_bf16* operand, qat_stream_t stream);
 
-/* The same quantization for several weights in one launch (all of a training
- * step's weights, each on its own grid): descs[i] holds W [N,K] fp32, bits,
+/* [P5] "训练时的模拟量化", as qat_quantize_weights, for several weights in one
+ * launch (all of a training step's weights, each on its own grid; the pages
+ * quantize every CastedLinear weight at every step): descs[i] holds W [N,K] fp32, bits,
  * scales [N] (required), codes [N,K] and operand [N,K] (nullable) exactly as
  * qat_quantize_weights takes them.  1 <= n <= QAT_QUANT_MAX_DESCS; the
  * descriptor array is read on the host during the call.  Each weight's
