@@ -193,6 +193,15 @@ int qat_mlp_bwd(const float* Wfc, const float* Wproj, const qat_qweight* qfc,
                 int64_t T, qat_bf16* dX, float* dWfc, float* dWproj, int32_t accumulate_dW,
                 void* workspace, size_t ws_bytes, qat_stream_t stream);
 
+/* Diagnostic (the pages have no counterpart): runs the library's bounded
+ * device wait on a barrier that nothing arrives on, with a limit of limit_ns
+ * (1 us .. 10 s, else QAT_ERR_ARG).  The wait gives up, records
+ * QAT_ERR_TIMEOUT in the device error flag and the kernel returns: the next
+ * qat_device_error() returns QAT_ERR_TIMEOUT (and clears the flag) and the
+ * context stays usable.  Lets a caller check its failure handling without a
+ * GPU fault. */
+int qat_selftest_wait_timeout(int64_t limit_ns, qat_stream_t stream);
+
 /* ---------------------------------------------------------------------------
  * qat_linear_fwd_noalloc -- the QAT linear forward from fp32 weights that
  * allocates nothing and takes no workspace.  The pages have no counterpart:

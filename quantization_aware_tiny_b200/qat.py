@@ -27,7 +27,7 @@ EXPORTED = ("qat_strerror", "qat_launch_count", "qat_device_error", "qat_quantiz
             "qat_workspace_size", "qat_linear_fwd", "qat_linear_bwd", "qat_mlp_fwd",
             "qat_mlp_bwd", "quantize_rows_export", "quantize_export_batch", "dequantize_rows",
             "qat_linear_fwd_noalloc", "qat_noisy_operand", "unpack_codes6",
-            "qat_quantize_weights_batch")
+            "qat_quantize_weights_batch", "qat_selftest_wait_timeout")
 QAT_EXPORT_PACK6 = 1
 QAT_EXPORT_CLIP_SEARCH = 2
 QAT_ACT_RELU2 = 0
@@ -80,6 +80,7 @@ def lib():
         L.qat_device_error.argtypes = [P]
         L.qat_quantize_weights.argtypes = [P, I32, I32, I32, P, P, P, P]
         L.qat_quantize_weights_batch.argtypes = [P, I32, P]
+        L.qat_selftest_wait_timeout.argtypes = [I64, P]
         L.qat_workspace_size.argtypes = [I32, I32, I32, I64, I32]
         L.qat_workspace_size.restype = SZ
         L.qat_linear_fwd.argtypes = [P, P, I32, I32, I32, P, I64, I64, P, P, P, SZ, P]
@@ -155,6 +156,13 @@ def device_error(stream=None):
 
 def workspace_size(op, a, b, T, raw_weights):
     return int(lib().qat_workspace_size(op, a, b, T, int(bool(raw_weights))))
+
+
+def qat_selftest_wait_timeout(limit_ns, stream=None):
+    """Diagnostic: a bounded device wait that runs out after limit_ns and
+    records QAT_ERR_TIMEOUT for the next device_error()."""
+    _check(lib().qat_selftest_wait_timeout(int(limit_ns), _stream(stream)),
+           "qat_selftest_wait_timeout")
 
 
 def qat_quantize_weights(W, bits, scales, codes=None, operand=None, stream=None):

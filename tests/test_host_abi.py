@@ -71,6 +71,9 @@ def test_argument_validation_before_launch(L):
     assert L.qat_linear_fwd(None, None, 512, 512, 6, A16, 0, 256, None, A16, None, 0, None) == qat.QAT_ERR_ARG
     # misaligned weights
     assert L.qat_quantize_weights(A_BAD, 512, 512, 6, None, A16, None, None) == qat.QAT_ERR_ALIGN
+    # the wait-timeout diagnostic: limit outside 1 us .. 10 s
+    assert L.qat_selftest_wait_timeout(999, None) == qat.QAT_ERR_ARG
+    assert L.qat_selftest_wait_timeout(10000000001, None) == qat.QAT_ERR_ARG
     # batched quantize: descriptor count, null pointers, bits, shape, alignment
     Q = qat._QuantDesc
     ok = Q(0x10000, None, 0x10000, 0x10000, 512, 512, 6, 0)
