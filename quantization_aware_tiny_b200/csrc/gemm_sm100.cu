@@ -20,6 +20,7 @@
 #include "gemm_sm100.cuh"
 #include "sm100_ptx.cuh"
 
+
 namespace qat {
 
 namespace {
@@ -705,8 +706,7 @@ template <int BN, bool PAIR>
 int dispatch_bn(const GemmDesc& g, const CUtensorMap& ma, const CUtensorMap& mb,
                 const CUtensorMap& md, const CUtensorMap& md2, const CUtensorMap& mr,
                 const KArgs& a, int epi, cudaStream_t s) {
-  if constexpr (BN % 128 != 0) {  // 160 / 192: forward (K-major B) epilogues only
-    if (g.a_mn || g.b_mn) return QAT_ERR_ARG;
+  if (!g.a_mn && !g.b_mn) {
     switch (epi) {
       case EPI_BF16: return launch_t<BN, false, false, EPI_BF16, PAIR>(ma, mb, md, md2, mr, a, s);
       case EPI_BF16_RESID:
@@ -714,34 +714,22 @@ int dispatch_bn(const GemmDesc& g, const CUtensorMap& ma, const CUtensorMap& mb,
       case EPI_RELU2: return launch_t<BN, false, false, EPI_RELU2, PAIR>(ma, mb, md, md2, mr, a, s);
       case EPI_LRELU2:
         return launch_t<BN, false, false, EPI_LRELU2, PAIR>(ma, mb, md, md2, mr, a, s);
-      default: return QAT_ERR_ARG;
+      default: break;
     }
-  } else {
-    if (!g.a_mn && !g.b_mn) {
-      switch (epi) {
-        case EPI_BF16: return launch_t<BN, false, false, EPI_BF16, PAIR>(ma, mb, md, md2, mr, a, s);
-        case EPI_BF16_RESID:
-          return launch_t<BN, false, false, EPI_BF16_RESID, PAIR>(ma, mb, md, md2, mr, a, s);
-        case EPI_RELU2: return launch_t<BN, false, false, EPI_RELU2, PAIR>(ma, mb, md, md2, mr, a, s);
-        case EPI_LRELU2:
-          return launch_t<BN, false, false, EPI_LRELU2, PAIR>(ma, mb, md, md2, mr, a, s);
-        default: break;
-      }
-    } else if (!g.a_mn && g.b_mn) {
-      switch (epi) {
-        case EPI_BF16: return launch_t<BN, false, true, EPI_BF16, PAIR>(ma, mb, md, md2, mr, a, s);
-        case EPI_DRELU2: return launch_t<BN, false, true, EPI_DRELU2, PAIR>(ma, mb, md, md2, mr, a, s);
-        case EPI_DLRELU2:
-          return launch_t<BN, false, true, EPI_DLRELU2, PAIR>(ma, mb, md, md2, mr, a, s);
-        default: break;
-      }
-    } else if (g.a_mn && g.b_mn) {
-      switch (epi) {
-        case EPI_F32: return launch_t<BN, true, true, EPI_F32, PAIR>(ma, mb, md, md2, mr, a, s);
-        case EPI_F32_ATOMIC:
-          return launch_t<BN, true, true, EPI_F32_ATOMIC, PAIR>(ma, mb, md, md2, mr, a, s);
-        default: break;
-      }
+  } else if (!g.a_mn && g.b_mn) {
+    switch (epi) {
+      case EPI_BF16: return launch_t<BN, false, true, EPI_BF16, PAIR>(ma, mb, md, md2, mr, a, s);
+      case EPI_DRELU2: return launch_t<BN, false, true, EPI_DRELU2, PAIR>(ma, mb, md, md2, mr, a, s);
+      case EPI_DLRELU2:
+        return launch_t<BN, false, true, EPI_DLRELU2, PAIR>(ma, mb, md, md2, mr, a, s);
+      default: break;
+    }
+  } else if (g.a_mn && g.b_mn) {
+    switch (epi) {
+      case EPI_F32: return launch_t<BN, true, true, EPI_F32, PAIR>(ma, mb, md, md2, mr, a, s);
+      case EPI_F32_ATOMIC:
+        return launch_t<BN, true, true, EPI_F32_ATOMIC, PAIR>(ma, mb, md, md2, mr, a, s);
+      default: break;
     }
   }
   return QAT_ERR_ARG;  // combination not instantiated
@@ -820,8 +808,8 @@ int launch_gemm(const GemmDesc& g, cudaStream_t stream) {
   if (g.M > (1ll << 31) - 256 || g.N > (1 << 30) || g.K > (1ll << 31) - 256) return QAT_ERR_SHAPE;
 
   // N tile.  Forward GEMMs (K-major B) with at least 256 rows run on CTA pairs
-  // with the widest of 256 / 192 / 160 that divides N, else 256; the other
-  // GEMMs take 256 (paired when M >= 256) unless 128 wastes fewer columns.
+  // 256 columns wide; the other GEMMs take 256 (paired when M >= 256) unless
+  // 128 wastes fewer columns.
   int BN;
   bool pair;
   const bool kmajor_fwd = !g.a_mn && !g.b_mn && g.epi != EPI_F32 && g.epi != EPI_F32_ATOMIC;
@@ -833,7 +821,12 @@ int launch_gemm(const GemmDesc& g, cudaStream_t stream) {
     // (a wave-count rule -- the width of fewest ceil(tiles / pairs) * BN -- was
     // slower: 160-wide tiles for the d = 640 core's N = 1280 filled the waves
     // better but cost more operand traffic per FLOP, core 0.42 -> 0.44 ms)
-    BN = (g.N % 256 == 0) ? 256 : (g.N % 192 == 0) ? 192 : (g.N % 160 == 0) ? 160 : 256;
+    // 256 wide even when it does not divide N (the last N block is partial):
+    // narrower tiles re-read A once more per FLOP, and with K this short the
+    // operand stream from L2 then sets the pace (d = 640 core: 160-wide tiles
+    // for N = 640, 192-wide for N = 1920 took 0.417 ms per R = 3 forward,
+    // 256-wide everywhere 0.365 ms)
+    BN = 256;
   } else {
     const int64_t pad256 = (g.N + 255) / 256 * 256 - g.N;
     const int64_t pad128 = (g.N + 127) / 128 * 128 - g.N;
@@ -922,13 +915,7 @@ int launch_gemm(const GemmDesc& g, cudaStream_t stream) {
       default: return dispatch_fb<256>(ma, md, md2, mr, a, epi, stream);
     }
   }
-  if (pair) {
-    switch (BN) {
-      case 160: return dispatch_bn<160, true>(g, ma, mb, md, md2, mr, a, epi, stream);
-      case 192: return dispatch_bn<192, true>(g, ma, mb, md, md2, mr, a, epi, stream);
-      default: return dispatch_bn<256, true>(g, ma, mb, md, md2, mr, a, epi, stream);
-    }
-  }
+  if (pair) return dispatch_bn<256, true>(g, ma, mb, md, md2, mr, a, epi, stream);
   return BN == 256 ? dispatch_bn<256, false>(g, ma, mb, md, md2, mr, a, epi, stream)
                    : dispatch_bn<128, false>(g, ma, mb, md, md2, mr, a, epi, stream);
 }
