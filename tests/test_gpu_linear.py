@@ -36,10 +36,13 @@ def test_linear_fwd_cfg1(raw):
     assert qat.device_error() == 0
 
 
-@pytest.mark.parametrize("shape", [(333, 136, 200), (1, 8, 8), (129, 264, 72), (700, 512, 1536)])
+@pytest.mark.parametrize("shape", [(333, 136, 200), (1, 8, 8), (129, 264, 72), (700, 512, 1536),
+                                   (600, 200, 136), (520, 264, 512), (1024, 640, 640)])
 @pytest.mark.parametrize("bits", [6, 8])
 def test_linear_fwd_ragged_and_residual(shape, bits):
-    """Ragged T (M tail), N not a multiple of the tile, K not a multiple of 64."""
+    """Ragged T (M tail), N not a multiple of the tile, K not a multiple of 64;
+    with at least 256 rows the forward runs on CTA pairs 256 columns wide, so
+    N = 200, 264 (a second block of 8 columns) and 640 end in a partial block."""
     T, N, K = shape
     rng = np.random.default_rng(T + N + K)
     W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
