@@ -275,8 +275,26 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR, EPI, FB>::THREADS, 1)
     t_end = static_cast<int>(static_cast<int64_t>(unit + 1) * p.num_tiles / units);
     t_step = 1;
   }
+  // FB: within N block nb the M blocks are rotated so that the run starting
+  // inside nb (at position base) begins at M block 0.  Every run then walks the
+  // M blocks in step with the runs of the other N blocks, and the concurrent
+  // pairs read a handful of A tiles (shared through L2) instead of one each.
+  auto fb_base = [&](int nb) {
+    const int64_t x = static_cast<int64_t>(nb) * p.num_m_blk;
+    const int64_t q = (x * units + p.num_tiles - 1) / p.num_tiles;  // first run starting at or after x
+    if (q >= units) return 0;
+    const int64_t s = q * p.num_tiles / units;
+    return s < x + p.num_m_blk ? static_cast<int>(s - x) : 0;
+  };
   auto tile_nb = [&](int t) { return FB ? t / p.num_m_blk : t % p.num_n_blk; };
-  auto tile_mb = [&](int t) { return FB ? t % p.num_m_blk : (t / p.num_n_blk) % p.num_m_blk; };
+  auto tile_mb = [&](int t) {
+    if constexpr (FB) {
+      const int nb = t / p.num_m_blk;
+      const int r = t - nb * p.num_m_blk - fb_base(nb);
+      return r < 0 ? r + p.num_m_blk : r;
+    }
+    return (t / p.num_n_blk) % p.num_m_blk;
+  };
   auto tile_sp = [&](int t) { return FB ? 0 : t / (p.num_n_blk * p.num_m_blk); };
 
   if (threadIdx.x == 0) {
