@@ -20,6 +20,7 @@ namespace {
 
 constexpr int kQThreads = 256;  // 8 warps per block
 constexpr int kRegV4 = 16;      // float4 per lane kept in registers (2048 columns)
+constexpr int kQuantV4 = 4;     // the training quantizer's cached float4 per lane (512 columns)
 
 __device__ __forceinline__ float amax4(float4 v) {
   return fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
@@ -30,70 +31,10 @@ __device__ __forceinline__ uint32_t pack_codes(int a, int b, int c, int d) {
          ((static_cast<uint32_t>(c) & 0xffu) << 16) | ((static_cast<uint32_t>(d) & 0xffu) << 24);
 }
 
-__device__ __forceinline__ uint2 operand4(int c0, int c1, int c2, int c3, float s) {
-  // bf16_rne(fl32(c * s)) for four codes
-  __nv_bfloat162 lo = __floats2bfloat162_rn(mul_rn(static_cast<float>(c0), s),
-                                            mul_rn(static_cast<float>(c1), s));
-  __nv_bfloat162 hi = __floats2bfloat162_rn(mul_rn(static_cast<float>(c2), s),
-                                            mul_rn(static_cast<float>(c3), s));
-  uint2 r;
-  r.x = *reinterpret_cast<uint32_t*>(&lo);
-  r.y = *reinterpret_cast<uint32_t*>(&hi);
-  return r;
-}
-
-// ------------------------------------------------------------------ QAT quantize
-// One row of one weight: amax over the row (cached in registers up to 2048
-// columns), the IEEE scale, codes and the bf16 operand.
-__device__ __forceinline__ void quantize_row(const QuantDescDev& d, int row, int lane) {
-  const int K = d.K, bits = d.bits;
-  const int K4 = K >> 2;
-  const float4* r = reinterpret_cast<const float4*>(d.W + static_cast<int64_t>(row) * K);
-  float4 cache[kRegV4];
-  float amax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < kRegV4; ++i) {
-    const int j = lane + 32 * i;
-    if (j < K4) {
-      cache[i] = __ldg(r + j);
-      amax = fmaxf(amax, amax4(cache[i]));
-    }
-  }
-  for (int j = lane + 32 * kRegV4; j < K4; j += 32) amax = fmaxf(amax, amax4(__ldg(r + j)));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  amax = fmaxf(amax, 1e-12f);
-  const float s = div_rn(amax, grid_levels(bits));
-  const float rs = __frcp_rn(s);
-  if (lane == 0) d.scales[row] = s;
-  auto emit = [&](int j, float4 v) {
-    const int c0 = quant_code(v.x, s, rs, bits), c1 = quant_code(v.y, s, rs, bits);
-    const int c2 = quant_code(v.z, s, rs, bits), c3 = quant_code(v.w, s, rs, bits);
-    const int64_t e = static_cast<int64_t>(row) * K + 4 * j;
-    if (d.codes) *reinterpret_cast<uint32_t*>(d.codes + e) = pack_codes(c0, c1, c2, c3);
-    if (d.operand) *reinterpret_cast<uint2*>(d.operand + e) = operand4(c0, c1, c2, c3, s);
-  };
-#pragma unroll
-  for (int i = 0; i < kRegV4; ++i) {
-    const int j = lane + 32 * i;
-    if (j < K4) emit(j, cache[i]);
-  }
-  for (int j = lane + 32 * kRegV4; j < K4; j += 32) emit(j, __ldg(r + j));
-}
-
-// All rows of all the batch's weights, a warp per row (grid-stride over the
-// concatenated rows), so small weights share the launch and the SMs.
-__global__ void __launch_bounds__(kQThreads)
-    quantize_batch_kernel(const __grid_constant__ QuantBatch b) {
-  const int lane = threadIdx.x & 31;
-  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  const int64_t total = b.row_begin[b.n];
-  int k = 0;
-  for (int64_t g = warp; g < total; g += nwarps) {
-    while (k + 1 < b.n && b.row_begin[k + 1] <= g) ++k;  // rows are visited in increasing order
-    quantize_row(b.d[k], static_cast<int>(g - b.row_begin[k]), lane);
-  }
+// Two floats as one word of bf16 (round to nearest even), the first in the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
 }
 
 // ------------------------------------------------------------------ Noisy QAT
@@ -358,6 +299,100 @@ __device__ __forceinline__ uint32_t codes4_t(const RowQuant& q, float4 v) {
     codes2<BITS, R>(q, v.x, v.y, c0, c1);
     codes2<BITS, R>(q, v.z, v.w, c2, c3);
     return pack4(c0, c1, c2, c3);
+  }
+}
+
+// ------------------------------------------------------------------ QAT quantize
+// Codes of two weights as exact float values, for the training quantizer's
+// row scale s = fl32(amax / L) (L = 127, or 15 for int5): every
+// |fl32(w / s)| <= amax / s < L + 1/2, so rne(w / s) is already in [-L, L]
+// and only int6's second rounding can leave the grid (4 * rne(127 / 4) = 128
+// -> 124).  The paired arithmetic of codes2: kOff + rne(w / s), then for int6
+// kOff + rne(k / 4); 4 * (that - kOff) is formed exactly by one fma.
+template <int BITS>
+__device__ __forceinline__ float2 code_values2(const RowQuant& q, float a, float b) {
+  const float2 t = rne_quot2<kNarrow>(q, a, b);
+  if constexpr (BITS == 6) {
+    const float2 u = rne_quarter2(t);
+    const float2 c = fma2(u, make_float2(4.0f, 4.0f), make_float2(-4.0f * kOff, -4.0f * kOff));
+    return make_float2(fminf(c.x, 124.0f), fminf(c.y, 124.0f));
+  } else {
+    return add2(t, make_float2(-kOff, -kOff));
+  }
+}
+
+// One row of one weight: amax over the row (the first 512 columns cached in
+// registers, the rest read again from L2), the IEEE scale, codes and the bf16
+// operand bf16(fl32(c * s)).
+template <int BITS>
+__device__ __forceinline__ void quantize_row_t(const QuantDescDev& d, int row, int lane) {
+  const int K = d.K;
+  const int K4 = K >> 2;
+  const float4* r = reinterpret_cast<const float4*>(d.W + static_cast<int64_t>(row) * K);
+  float4 cache[kQuantV4];
+  float amax = 0.0f, amax2 = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kQuantV4; ++i) {
+    const int j = lane + 32 * i;
+    if (j < K4) {
+      cache[i] = __ldg(r + j);
+      if (i & 1) amax2 = fmaxf(amax2, amax4(cache[i]));
+      else amax = fmaxf(amax, amax4(cache[i]));
+    }
+  }
+  for (int j = lane + 32 * kQuantV4; j < K4; j += 64) {
+    amax = fmaxf(amax, amax4(__ldg(r + j)));
+    if (j + 32 < K4) amax2 = fmaxf(amax2, amax4(__ldg(r + j + 32)));
+  }
+  amax = fmaxf(amax, amax2);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  RowQuant q;
+  q.clip = fmaxf(amax, 1e-12f);
+  q.s = div_rn(q.clip, grid_levels(BITS));
+  q.rs = __frcp_rn(q.s);
+  q.bits = BITS;
+  if (lane == 0) d.scales[row] = q.s;
+  const float2 s2 = make_float2(q.s, q.s);
+  auto emit = [&](int j, float4 v) {
+    const float2 c01 = code_values2<BITS>(q, v.x, v.y), c23 = code_values2<BITS>(q, v.z, v.w);
+    const int64_t e = static_cast<int64_t>(row) * K + 4 * j;
+    if (d.codes)
+      *reinterpret_cast<uint32_t*>(d.codes + e) =
+          pack_codes(__float2int_rn(c01.x), __float2int_rn(c01.y), __float2int_rn(c23.x),
+                     __float2int_rn(c23.y));
+    if (d.operand) {
+      const float2 w01 = mul2(c01, s2), w23 = mul2(c23, s2);
+      uint2 o;
+      o.x = pack_bf16x2(w01.x, w01.y);
+      o.y = pack_bf16x2(w23.x, w23.y);
+      *reinterpret_cast<uint2*>(d.operand + e) = o;
+    }
+  };
+#pragma unroll
+  for (int i = 0; i < kQuantV4; ++i) {
+    const int j = lane + 32 * i;
+    if (j < K4) emit(j, cache[i]);
+  }
+  for (int j = lane + 32 * kQuantV4; j < K4; j += 32) emit(j, __ldg(r + j));
+}
+
+// All rows of all the batch's weights, a warp per row (grid-stride over the
+// concatenated rows), so small weights share the launch and the SMs.
+__global__ void __launch_bounds__(kQThreads, 3)
+    quantize_batch_kernel(const __grid_constant__ QuantBatch b) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int64_t total = b.row_begin[b.n];
+  int k = 0;
+  for (int64_t g = warp; g < total; g += nwarps) {
+    while (k + 1 < b.n && b.row_begin[k + 1] <= g) ++k;  // rows are visited in increasing order
+    const QuantDescDev& d = b.d[k];
+    const int row = static_cast<int>(g - b.row_begin[k]);
+    if (d.bits == 6) quantize_row_t<6>(d, row, lane);
+    else if (d.bits == 5) quantize_row_t<5>(d, row, lane);
+    else quantize_row_t<8>(d, row, lane);
   }
 }
 
