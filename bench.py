@@ -300,6 +300,7 @@ def run_ours(args):
             out["export"] = measure_export(dev, stream, pk)
             out["export_pack6"] = measure_export(dev, stream, pk, pack6=True)
             out["export_clip_search"] = measure_export(dev, stream, pk, clip_search=True)
+            out["dequantize"] = measure_dequant(dev, stream, pk)
             out["recurrent_core"] = measure_core(dev, stream, pk)
             out["fused_producer"] = measure_fused_producer(dev, stream, pk)
             out["cpu_baseline"] = cpu_baseline()
@@ -458,6 +459,69 @@ def measure_export(dev, stream, pk, pack6=False, clip_search=False):
                         "+ small tensors fp16 passthrough; L2 flushed (256 MB written, 256 MB read) "
                         "before each launch" % ((" 6-bit packed" if pack6 else "") +
                                                 (" clip search" if clip_search else ""))}
+
+
+def measure_dequant(dev, stream, pk):
+    """The roundtrip dequantize of the exported 11-layer d=512 state dict (66
+    int6 tensors: codes + fp16 row scales -> fp32) in one dequantize_rows_batch
+    launch, L2 flushed before each; beside it the same work as 66 per-tensor
+    dequantize_rows calls replayed from a CUDA graph.  Algorithmic bytes: 1 B
+    code read + 4 B written per element, 2 B per row scale."""
+    from quantization_aware_tiny_b200 import export as qexport
+    from quantization_aware_tiny_b200 import qat
+    from quantization_aware_tiny_b200 import synthetic as sy
+    sd = {k: torch.from_numpy(v).to(dev) for k, v in sy.state_dict_case().items()}
+    ex = qexport.export_state_dict(sd)
+    items = []
+    algo = 0
+    for name, e in ex.items():
+        if "codes" in e:
+            c = e["codes"]
+            items.append((c, e["scale16"], torch.empty(c.shape, dtype=torch.float32, device=dev)))
+            algo += c.numel() * 5 + c.shape[0] * 2
+    arr = qat.dequant_descs(items)  # marshalled once
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+    clean = torch.zeros(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+
+    def per_tensor(st):
+        for c, s16, o in items:
+            qat.dequantize_rows(c, s16, o, stream=st)
+
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        per_tensor(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            per_tensor(side)
+    stream.wait_stream(side)
+
+    def timed(fn):
+        events = []
+        for i in range(60):
+            flush_l2(flush, clean)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            events.append((a, b))
+        torch.cuda.synchronize()
+        return statistics.median(a.elapsed_time(b) for a, b in events[10:])
+
+    ms = timed(lambda: qat.dequantize_rows_batch(arr, stream=stream))
+    with torch.cuda.stream(stream):
+        ms_graph = timed(graph.replay)
+    del graph
+    gbs = algo / (ms * 1e-3) / 1e9
+    return {"value": round(gbs, 1), "unit": "GB/s", "ms": round(ms, 4), "launches": 1,
+            "per_tensor_graph": {"ms": round(ms_graph, 4), "launches": len(items),
+                                 "value": round(algo / (ms_graph * 1e-3) / 1e9, 1)},
+            "algorithmic_bytes": algo,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(gbs / pk["hbm_gbs"], 4),
+                         "peak_kind": "copy bandwidth (%s)" % pk["source"]},
+            "workload": "66 int6 tensors of the exported 11-layer d=512 state dict -> fp32 in one "
+                        "grouped launch; L2 flushed before each"}
 
 
 def measure_fused_producer(dev, stream, pk):

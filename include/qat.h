@@ -287,10 +287,31 @@ int unpack_codes6(const uint8_t* packed, int64_t n, int32_t bits, int8_t* codes,
                   qat_stream_t stream);
 
 /* Roundtrip dequantize ([P5] "后训练量化导出", roundtrip re-evaluation):
- *   out = fl32(c * fp32(scale_fp16))  as fp32 (out_dtype 0) or bf16_rne of it (1). */
+ *   out = fl32(c * fp32(scale_fp16))  as fp32 (out_dtype 0) or bf16_rne of it (1).
+ * codes int8 [rows, cols] row-major, scales fp16 [rows] (one per row, as
+ * quantize_rows_export writes them), out [rows, cols] row-major; all device
+ * pointers, caller-owned.  cols a positive multiple of 8 (QAT_ERR_SHAPE), codes
+ * and out 16-byte aligned (QAT_ERR_ALIGN), a null pointer, rows < 0 or another
+ * out_dtype QAT_ERR_ARG.  Bit-exact with the oracle. */
 enum { QAT_DTYPE_F32 = 0, QAT_DTYPE_BF16 = 1 };
 int dequantize_rows(const int8_t* codes, const qat_fp16* scales, int64_t rows, int64_t cols,
                     int32_t out_dtype, void* out, qat_stream_t stream);
+
+/* Grouped dequantize_rows: the rows of up to QAT_DEQUANT_MAX_DESCS tensors in
+ * one launch (a state dict's roundtrip), each descriptor the arguments of one
+ * dequantize_rows call.  Every descriptor is checked as dequantize_rows checks
+ * its arguments before anything launches; the first failing one decides the
+ * error.  n outside 1 .. QAT_DEQUANT_MAX_DESCS or a null array: QAT_ERR_ARG. */
+#define QAT_DEQUANT_MAX_DESCS 256
+typedef struct qat_dequant_desc {
+  const int8_t* codes;
+  const qat_fp16* scales;
+  int64_t rows, cols;
+  int32_t out_dtype;
+  int32_t reserved; /* 0 */
+  void* out;
+} qat_dequant_desc;
+int dequantize_rows_batch(const qat_dequant_desc* descs, int32_t n, qat_stream_t stream);
 
 #ifdef __cplusplus
 }

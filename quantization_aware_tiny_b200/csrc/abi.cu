@@ -442,4 +442,27 @@ int dequantize_rows(const int8_t* codes, const qat_fp16* scales, int64_t rows, i
                         out_dtype == QAT_DTYPE_BF16, out, stream);
 }
 
+int dequantize_rows_batch(const qat_dequant_desc* descs, int32_t n, qat_stream_t stream) {
+  if (!descs || n <= 0 || n > QAT_DEQUANT_MAX_DESCS) return QAT_ERR_ARG;
+  static thread_local DequantBatch b;  // ~14 KB: kept off the stack
+  b.n = n;
+  b.item_begin[0] = 0;
+  for (int i = 0; i < n; ++i) {
+    const qat_dequant_desc& s = descs[i];
+    if (!s.codes || !s.scales || !s.out || s.rows < 0) return QAT_ERR_ARG;
+    if (s.out_dtype != QAT_DTYPE_F32 && s.out_dtype != QAT_DTYPE_BF16) return QAT_ERR_ARG;
+    if (!dim_ok(s.cols)) return QAT_ERR_SHAPE;
+    if (!aligned16(s.codes) || !aligned16(s.out)) return QAT_ERR_ALIGN;
+    DequantDescDev& d = b.d[i];
+    d.codes = s.codes;
+    d.scales = reinterpret_cast<const __half*>(s.scales);
+    d.out = s.out;
+    d.cols = s.cols;
+    d.out_bf16 = s.out_dtype == QAT_DTYPE_BF16;
+    d.pad = 0;
+    b.item_begin[i + 1] = b.item_begin[i] + s.rows * (s.cols >> 3);
+  }
+  return launch_dequant_batch(b, stream);
+}
+
 }  // extern "C"

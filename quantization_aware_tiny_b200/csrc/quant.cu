@@ -971,35 +971,54 @@ __global__ void __launch_bounds__(kExportMaxWarps * 32, 1)
 }
 
 // ------------------------------------------------------------------ dequantize
+// Eight consecutive codes of a row (item i: elements 8i .. 8i + 7; cols a
+// multiple of 8, so they share the row's scale): fl32(c * fp32(scale_fp16)),
+// stored as fp32 or rounded to bf16.
+__device__ __forceinline__ void dequant8(const int8_t* __restrict__ codes,
+                                         const __half* __restrict__ scales, int64_t cols,
+                                         int64_t i, int out_bf16, void* __restrict__ out) {
+  const int64_t row = i / (cols >> 3);
+  const int64_t e = i * 8;
+  const float s = __half2float(scales[row]);
+  const uint2 cc = *reinterpret_cast<const uint2*>(codes + e);
+  const int8_t* c = reinterpret_cast<const int8_t*>(&cc);
+  float v[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) v[k] = mul_rn(static_cast<float>(c[k]), s);
+  if (out_bf16) {
+    uint4 w;
+    w.x = pack_bf16x2(v[0], v[1]);
+    w.y = pack_bf16x2(v[2], v[3]);
+    w.z = pack_bf16x2(v[4], v[5]);
+    w.w = pack_bf16x2(v[6], v[7]);
+    *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(out) + e) = w;
+  } else {
+    float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + e);
+    o[0] = make_float4(v[0], v[1], v[2], v[3]);
+    o[1] = make_float4(v[4], v[5], v[6], v[7]);
+  }
+}
+
 __global__ void __launch_bounds__(kQThreads)
     dequant_kernel(const int8_t* __restrict__ codes, const __half* __restrict__ scales,
                    int64_t rows, int64_t cols, int out_bf16, void* __restrict__ out) {
-  const int64_t n8_row = cols >> 3;
-  const int64_t total = rows * n8_row;
+  const int64_t total = rows * (cols >> 3);
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    dequant8(codes, scales, cols, i, out_bf16, out);
+}
+
+// All descriptors' items in one grid-stride loop; a thread's items increase,
+// so its descriptor index only moves forward.
+__global__ void __launch_bounds__(kQThreads)
+    dequant_batch_kernel(const __grid_constant__ DequantBatch b) {
+  const int64_t total = b.item_begin[b.n];
+  int k = 0;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t row = i / n8_row;
-    const int64_t e = i * 8;
-    const float s = __half2float(scales[row]);
-    const uint2 cc = *reinterpret_cast<const uint2*>(codes + e);
-    const int8_t* c = reinterpret_cast<const int8_t*>(&cc);
-    float v[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) v[k] = mul_rn(static_cast<float>(c[k]), s);
-    if (out_bf16) {
-      __nv_bfloat162 p0 = __floats2bfloat162_rn(v[0], v[1]), p1 = __floats2bfloat162_rn(v[2], v[3]);
-      __nv_bfloat162 p2 = __floats2bfloat162_rn(v[4], v[5]), p3 = __floats2bfloat162_rn(v[6], v[7]);
-      uint4 w;
-      w.x = *reinterpret_cast<uint32_t*>(&p0);
-      w.y = *reinterpret_cast<uint32_t*>(&p1);
-      w.z = *reinterpret_cast<uint32_t*>(&p2);
-      w.w = *reinterpret_cast<uint32_t*>(&p3);
-      *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(out) + e) = w;
-    } else {
-      float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + e);
-      o[0] = make_float4(v[0], v[1], v[2], v[3]);
-      o[1] = make_float4(v[4], v[5], v[6], v[7]);
-    }
+    while (k + 1 < b.n && b.item_begin[k + 1] <= i) ++k;
+    const DequantDescDev& d = b.d[k];
+    dequant8(d.codes, d.scales, d.cols, i - b.item_begin[k], d.out_bf16, d.out);
   }
 }
 
@@ -1132,6 +1151,14 @@ int launch_dequant(const int8_t* codes, const __half* scales, int64_t rows, int6
   if (items == 0) return QAT_OK;
   dequant_kernel<<<grid_for_rows(items, kQThreads), kQThreads, 0, s>>>(codes, scales, rows, cols,
                                                                        out_bf16, out);
+  count_launch();
+  return cuda_status(cudaGetLastError());
+}
+
+int launch_dequant_batch(const DequantBatch& b, cudaStream_t s) {
+  const int64_t items = b.item_begin[b.n];
+  if (items == 0) return QAT_OK;
+  dequant_batch_kernel<<<grid_for_rows(items, kQThreads), kQThreads, 0, s>>>(b);
   count_launch();
   return cuda_status(cudaGetLastError());
 }

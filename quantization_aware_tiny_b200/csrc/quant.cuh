@@ -80,6 +80,23 @@ int clip_search_supported(int64_t cols);
 int launch_export_batch(ExportBatch& b, cudaStream_t s);
 int launch_dequant(const int8_t* codes, const __half* scales, int64_t rows, int64_t cols,
                    int out_bf16, void* out, cudaStream_t s);
+
+// Grouped dequantize: descriptor k covers the 8-element groups
+// [item_begin[k], item_begin[k + 1]) of the concatenation.
+struct DequantDescDev {
+  const int8_t* codes;
+  const __half* scales;
+  void* out;
+  int64_t cols;
+  int out_bf16, pad;
+};
+constexpr int kDequantMaxDescs = QAT_DEQUANT_MAX_DESCS;
+struct DequantBatch {
+  int n;
+  int64_t item_begin[kDequantMaxDescs + 1];
+  DequantDescDev d[kDequantMaxDescs];
+};
+int launch_dequant_batch(const DequantBatch& b, cudaStream_t s);
 int launch_unpack6(const uint8_t* packed, int64_t n, int bits, int8_t* codes, cudaStream_t s);
 
 }  // namespace qat

@@ -27,7 +27,7 @@ EXPORTED = ("qat_strerror", "qat_launch_count", "qat_device_error", "qat_quantiz
             "qat_workspace_size", "qat_linear_fwd", "qat_linear_bwd", "qat_mlp_fwd",
             "qat_mlp_bwd", "quantize_rows_export", "quantize_export_batch", "dequantize_rows",
             "qat_linear_fwd_noalloc", "qat_noisy_operand", "unpack_codes6",
-            "qat_quantize_weights_batch", "qat_selftest_wait_timeout")
+            "qat_quantize_weights_batch", "qat_selftest_wait_timeout", "dequantize_rows_batch")
 QAT_EXPORT_PACK6 = 1
 QAT_EXPORT_CLIP_SEARCH = 2
 QAT_ACT_RELU2 = 0
@@ -53,6 +53,15 @@ class _QuantDesc(ctypes.Structure):
     _fields_ = [("W", ctypes.c_void_p), ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
                 ("operand", ctypes.c_void_p), ("N", ctypes.c_int32), ("K", ctypes.c_int32),
                 ("bits", ctypes.c_int32), ("pad", ctypes.c_int32)]
+
+
+class _DequantDesc(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("rows", ctypes.c_int64),
+                ("cols", ctypes.c_int64), ("out_dtype", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("out", ctypes.c_void_p)]
+
+
+QAT_DEQUANT_MAX_DESCS = 256
 
 
 class _ExportDesc(ctypes.Structure):
@@ -91,6 +100,7 @@ def lib():
         L.quantize_rows_export.argtypes = [P, I64, I64, I32, P, P, P]
         L.quantize_export_batch.argtypes = [P, I32, P]
         L.dequantize_rows.argtypes = [P, P, I64, I64, I32, P, P]
+        L.dequantize_rows_batch.argtypes = [P, I32, P]
         L.unpack_codes6.argtypes = [P, I64, I32, P, P]
         L.qat_linear_fwd_noalloc.argtypes = [P, I32, I32, I32, P, I64, I64, P, P, P]
         L.qat_noisy_operand.argtypes = [P, I32, I32, I32, ctypes.c_uint64, ctypes.c_uint64, P, P,
@@ -310,6 +320,23 @@ def dequantize_rows(codes, scales16, out, stream=None):
     dt = QAT_DTYPE_BF16 if out.dtype == torch.bfloat16 else QAT_DTYPE_F32
     _check(lib().dequantize_rows(_p(codes), _p(scales16), rows, cols, dt, _p(out),
                                  _stream(stream)), "dequantize_rows")
+
+
+def dequantize_rows_batch(items, stream=None):
+    """items: list of (codes int8 [rows, cols], scales16 fp16 [rows], out fp32 or
+    bf16 [rows, cols]) device tensors -- or an array from dequant_descs()."""
+    arr = items if isinstance(items, ctypes.Array) else dequant_descs(items)
+    _check(lib().dequantize_rows_batch(arr, len(arr), _stream(stream)), "dequantize_rows_batch")
+
+
+def dequant_descs(items):
+    """Marshal (codes, scales16, out) tuples into the C descriptor array once."""
+    arr = (_DequantDesc * len(items))()
+    for i, (codes, scales16, out) in enumerate(items):
+        rows, cols = codes.shape
+        dt = QAT_DTYPE_BF16 if out.dtype == torch.bfloat16 else QAT_DTYPE_F32
+        arr[i] = _DequantDesc(codes.data_ptr(), scales16.data_ptr(), rows, cols, dt, 0, out.data_ptr())
+    return arr
 
 
 def qat_linear_fwd_noalloc(W, X, Y, bits, residual=None, ldx=0, T=None, stream=None):

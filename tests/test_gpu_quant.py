@@ -234,6 +234,32 @@ def test_dequantize_rows_bit_exact():
         assert np.array_equal(bits16(out16), o.bf16_bits(ref)), name
 
 
+def test_dequantize_rows_batch_one_launch():
+    """The roundtrip of a whole exported state dict (3 layers: 18 int6 tensors
+    of 256-1536 columns, plus a ragged 200 x 136 int8 tensor) in one grouped
+    launch, fp32 and bf16 outputs mixed: bit-exact with the oracle."""
+    sd = sy.state_dict_case(n_layers=3, seed=6)
+    rng = np.random.default_rng(6)
+    W = {k: v for k, v in sd.items() if v.ndim == 2 and v.size > 65536 and "tok_emb" not in k}
+    W["ragged"] = (rng.standard_normal((200, 136)) * 0.02).astype(np.float32)
+    items, refs = [], []
+    for i, (name, w) in enumerate(sorted(W.items())):
+        c, s16, _ = o.export_rows(w, 8 if name == "ragged" else 6)
+        out = torch.full(w.shape, float("nan"), device="cuda",
+                         dtype=torch.bfloat16 if i % 2 else torch.float32)
+        items.append((_dev(c), _dev(s16.view(np.float16)), out))
+        refs.append((name, o.dequant_export(c, s16)))
+    n0 = qat.launch_count()
+    qat.dequantize_rows_batch(items)
+    torch.cuda.synchronize()
+    assert qat.launch_count() - n0 == 1
+    for (name, ref), (_, _, out) in zip(refs, items):
+        if out.dtype == torch.float32:
+            assert np.array_equal(out.cpu().numpy().view(np.uint32), ref.view(np.uint32)), name
+        else:
+            assert np.array_equal(bits16(out), o.bf16_bits(ref)), name
+
+
 def _near_tie_rows(n_rows=256, cols=512, seed=21, levels=127):
     """Rows whose entries sit within a few ulps of (k + 1/2) * s: the code then
     depends on the correctly rounded quotient w / s (and on ties going to

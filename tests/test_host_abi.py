@@ -119,6 +119,20 @@ def test_argument_validation_before_launch(L):
     assert L.unpack_codes6(A16, 16, 8, A16, None) == qat.QAT_ERR_ARG
     assert L.unpack_codes6(A_BAD, 16, 6, A16, None) == qat.QAT_ERR_ALIGN
     assert L.dequantize_rows(A16, A16, 4, 16, 3, A16, None) == qat.QAT_ERR_ARG
+    # grouped dequantize: count, null array, then a bad descriptor after a good one
+    D = qat._DequantDesc
+    good = D(0x10000, 0x10000, 4, 16, qat.QAT_DTYPE_F32, 0, 0x10000)
+    assert L.dequantize_rows_batch(None, 1, None) == qat.QAT_ERR_ARG
+    many = (D * 257)(*([good] * 257))
+    assert L.dequantize_rows_batch(ctypes.cast(many, ctypes.c_void_p), 0, None) == qat.QAT_ERR_ARG
+    assert L.dequantize_rows_batch(ctypes.cast(many, ctypes.c_void_p), 257, None) == qat.QAT_ERR_ARG
+    for bad, rc in ((D(0x10000, None, 4, 16, 0, 0, 0x10000), qat.QAT_ERR_ARG),
+                    (D(0x10000, 0x10000, 4, 16, 2, 0, 0x10000), qat.QAT_ERR_ARG),
+                    (D(0x10000, 0x10000, -1, 16, 0, 0, 0x10000), qat.QAT_ERR_ARG),
+                    (D(0x10000, 0x10000, 4, 12, 0, 0, 0x10000), qat.QAT_ERR_SHAPE),
+                    (D(0x10000, 0x10000, 4, 16, 0, 0, 0x10008), qat.QAT_ERR_ALIGN)):
+        two = (D * 2)(good, bad)
+        assert L.dequantize_rows_batch(ctypes.cast(two, ctypes.c_void_p), 2, None) == rc
     assert L.qat_mlp_bwd(None, None, None, None, 512, 1536, 6, 0, A16, A16, None, A16, 8, None,
                          None, None, 0, None, 0, None) == qat.QAT_ERR_ARG
     # activation outside {relu^2, leaky^2}; bits 7
