@@ -83,8 +83,22 @@ def export_state_dict(_T):
         qexport.export_state_dict(sd)
 
 
+def dequant_state_dict(_T):
+    """The exported 11-layer state dict's int6 tensors back to fp32, one
+    dequantize_rows_batch launch (after an export launch and an L2-sized
+    write, so the codes start in DRAM)."""
+    sd = {k: torch.from_numpy(v).cuda() for k, v in sy.state_dict_case().items()}
+    ex = qexport.export_state_dict(sd)
+    items = [(e["codes"], e["scale16"], torch.empty(e["codes"].shape, dtype=torch.float32, device="cuda"))
+             for e in ex.values() if "codes" in e]
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
+    for _ in range(3):
+        flush.add_(1)
+        qat.dequantize_rows_batch(items)
+
+
 CASES = {"logits_fwd": logits_fwd, "logits_fwd_fused": logits_fwd_fused, "head_dw": head_dw, "head_dx": head_dx,
-         "mlp_step": mlp_step, "export_state_dict": export_state_dict}
+         "mlp_step": mlp_step, "export_state_dict": export_state_dict, "dequant_state_dict": dequant_state_dict}
 
 
 def main(argv=None):
