@@ -62,11 +62,13 @@ def peaks():
 
 
 class ClockSampler:
-    """SM clock and throttle-reason samples while the timed region runs: NVML
+    """SM clock and throttle-reason samples, each with a host timestamp: NVML
     queries (read-only) from a thread every few milliseconds, else
-    nvidia-smi's own loop."""
+    nvidia-smi's own loop.  Started before the warm-up (nvidia-smi needs a
+    moment to start); summary() keeps the samples inside the window marked
+    by begin() / end() around the timed region."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
     REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
@@ -74,7 +76,9 @@ class ClockSampler:
     def __init__(self, index, period_s=0.004):
         self.index, self.period = index, period_s
         self.proc, self.thread = None, None
-        self.sm, self.mx, self.reasons = [], [], set()
+        self.samples = []  # (host time, sm MHz, max MHz, reasons)
+        self.t0 = self.t1 = None
+        self.nvml_error = None
 
     def _nvml_handle(self):
         import pynvml
@@ -86,37 +90,51 @@ class ClockSampler:
         except Exception:
             return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.index)
 
-    def _nvml_loop(self, nv, h):
+    def _nvml_loop(self, nv, h, mx):
         bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
                 "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
                 "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
                 "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
-        mx = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
         while not self.stop.is_set():
-            self.sm.append(float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)))
-            self.mx.append(mx)
-            r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
-            self.reasons.update(n for n, b in bits.items() if r & b)
+            try:
+                sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                try:
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                except Exception:
+                    r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+                self.samples.append((time.monotonic(), sm, mx,
+                                     tuple(n for n, bit in bits.items() if r & bit)))
+            except Exception as e:  # keep sampling; report the last failure
+                self.nvml_error = "%s: %s" % (type(e).__name__, e)
             self.stop.wait(self.period)
 
     def __enter__(self):
         import threading
         try:
             nv, h = self._nvml_handle()
+            mx = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
             self.stop = threading.Event()
-            self.thread = threading.Thread(target=self._nvml_loop, args=(nv, h), daemon=True)
+            self.thread = threading.Thread(target=self._nvml_loop, args=(nv, h, mx), daemon=True)
             self.thread.start()
             return self
-        except Exception:
+        except Exception as e:
+            self.nvml_error = "%s: %s" % (type(e).__name__, e)
             self.thread = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
                  "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.smi_t0 = (time.time(), time.monotonic())
         except OSError:
             self.proc = None
         return self
+
+    def begin(self):
+        self.t0 = time.monotonic()
+
+    def end(self):
+        self.t1 = time.monotonic()
 
     def __exit__(self, *a):
         if self.thread is not None:
@@ -131,25 +149,37 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
                 out, _ = self.proc.communicate()
+        import datetime
         for line in out.strip().splitlines():
             parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 7:
+            if len(parts) < 8:
                 continue
-            try:
-                sm, mx = float(parts[0]), float(parts[1])
+            try:  # nvidia-smi's wall-clock timestamp mapped onto time.monotonic()
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                sm, mx = float(parts[1]), float(parts[2])
             except ValueError:
                 continue
-            self.sm.append(sm)
-            self.mx.append(mx)
-            self.reasons.update(n for n, v in zip(self.REASONS, parts[3:7]) if v.lower() == "active")
+            t = ts - self.smi_t0[0] + self.smi_t0[1]
+            self.samples.append((t, sm, mx, tuple(n for n, v in zip(self.REASONS, parts[4:8])
+                                                 if v.lower() == "active")))
 
     def summary(self):
-        if not self.sm:
-            return None
-        loaded = [s for s in self.sm if s > 0.5 * max(self.sm)] or self.sm
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(self.mx),
-                "samples": len(self.sm), "source": "nvml" if self.thread is not None else "nvidia-smi",
-                "reasons": sorted(self.reasons)}
+        inside = [x for x in self.samples
+                  if self.t0 is not None and self.t1 is not None and self.t0 <= x[0] <= self.t1]
+        source = "nvml" if self.thread is not None else "nvidia-smi"
+        if not inside:
+            out = {"samples": 0, "samples_outside_window": len(self.samples), "source": source}
+            if self.nvml_error:
+                out["nvml_error"] = self.nvml_error
+            return out
+        sm = [x[1] for x in inside]
+        loaded = [v for v in sm if v > 0.5 * max(sm)] or sm
+        reasons = sorted({r for x in inside for r in x[3]})
+        out = {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(x[2] for x in inside),
+               "samples": len(inside), "source": source, "reasons": reasons}
+        if self.nvml_error:
+            out["nvml_error"] = self.nvml_error
+        return out
 
 
 def dist_env():
@@ -238,19 +268,21 @@ def run_ours(args):
             sync.start([step.dWfc, step.dWproj], stream)
             sync.wait(stream)
 
-    for i in range(args.warmup):
-        one(i, False)
-    if pg is not None:
-        pg.barrier()
-    torch.cuda.synchronize()
-    n0 = qat.launch_count()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
+    with ClockSampler(local) as clk:  # started before the warm-up, read over the timed window
+        for i in range(args.warmup):
+            one(i, False)
+        if pg is not None:
+            pg.barrier()
+        torch.cuda.synchronize()
+        n0 = qat.launch_count()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        clk.begin()
         start.record(stream)
         for i in range(args.steps):
             one(i, True)
         end.record(stream)
         torch.cuda.synchronize()
+        clk.end()
     if pg is not None:
         pg.barrier()
     launches = qat.launch_count() - n0
