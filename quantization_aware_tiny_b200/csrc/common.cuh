@@ -78,6 +78,50 @@ __device__ __forceinline__ int code_from_quotient(float x, int bits) {
 // int8 (the int6 grid is every fourth int8 level).
 __device__ __forceinline__ float grid_levels(int bits) { return bits == 5 ? 15.0f : 127.0f; }
 
+// ---- paired fp32 arithmetic (two IEEE round-to-nearest operations per instruction)
+__device__ __forceinline__ uint64_t f2u(float2 v) { return *reinterpret_cast<uint64_t*>(&v); }
+__device__ __forceinline__ float2 u2f(uint64_t v) { return *reinterpret_cast<float2*>(&v); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2u(a)), "l"(f2u(b)));
+  return u2f(d);
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2u(a)), "l"(f2u(b)));
+  return u2f(d);
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f2u(a)), "l"(f2u(b)), "l"(f2u(c)));
+  return u2f(d);
+}
+
+constexpr float kOff = 12582912.0f;  // 1.5 * 2^23: x + kOff rounds x to an integer (|x| < 2^22)
+
+// Codes of two weights as exact float values, for a row scale s = fl32(amax / L)
+// (L = 127, or 15 for int5) and r = fl32(1 / s): kOff + rne(fl32(w / s)) from
+// the Markstein-corrected quotient (see div_by_scale), done pairwise; for int6
+// kOff + rne(k / 4) (the fma forms k / 4 exactly) and 4 * (that - kOff) by one
+// exact fma.  With that scale every |fl32(w / s)| < L + 1/2, so rne(w / s) is
+// already in [-L, L] and only int6's second rounding can leave the grid
+// (4 * rne(127 / 4) = 128 -> 124).
+template <int BITS>
+__device__ __forceinline__ float2 grid_code_values2(float a, float b, float s, float r) {
+  const float2 w = make_float2(a, b), r2 = make_float2(r, r);
+  const float2 q0 = mul2(w, r2);
+  const float2 rem = fma2(q0, make_float2(-s, -s), w);
+  const float2 t = add2(fma2(rem, r2, q0), make_float2(kOff, kOff));
+  if constexpr (BITS == 6) {
+    const float2 y = fma2(t, make_float2(0.25f, 0.25f), make_float2(-kOff / 4, -kOff / 4));
+    const float2 u = add2(y, make_float2(kOff, kOff));
+    const float2 c = fma2(u, make_float2(4.0f, 4.0f), make_float2(-4.0f * kOff, -4.0f * kOff));
+    return make_float2(fminf(c.x, 124.0f), fminf(c.y, 124.0f));
+  } else {
+    return add2(t, make_float2(-kOff, -kOff));
+  }
+}
+
 // Code of one weight on the int5 / int6 / int8 grid; r = fl32(1 / s).
 __device__ __forceinline__ int quant_code(float w, float s, float r, int bits) {
   return code_from_quotient(div_by_scale(w, s, r), bits);

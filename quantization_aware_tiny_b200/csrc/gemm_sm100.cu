@@ -171,13 +171,13 @@ __device__ __forceinline__ float absmax4(float4 v) {
 // load of the same tile would write.  Rows >= N and columns >= K are zero.
 // Warp ew takes rows ew, ew + EW, ...; RP rows per pass keep RP * KBP / 2
 // 16-byte loads in flight per lane.
-template <class C>
+template <class C, int BITS>
 __device__ __forceinline__ void convert_panel(const KArgs& p, uint8_t* panel, int n_base, int ew,
                                               int lane) {
   constexpr int V = C::KBP / 2;  // float4 per lane per row (32 lanes x 4 floats per 128 columns)
   const int K4 = p.K >> 2;
   const int slots = p.kblk_total * 16;  // float4 slots of a panel row
-  const float levels = grid_levels(p.bits);
+  const float levels = grid_levels(BITS);
   const uint32_t pbase = smem_u32(panel);
 #pragma unroll 1
   for (int r0 = ew; r0 < C::B_ROWS; r0 += C::RP * C::EW) {
@@ -219,10 +219,12 @@ __device__ __forceinline__ void convert_panel(const KArgs& p, uint8_t* panel, in
         const int j = lane + 32 * i;
         if (j < slots) {
           const float4 w = v[h][i];
-          const int c0 = quant_code(w.x, sc, rs, p.bits), c1 = quant_code(w.y, sc, rs, p.bits);
-          const int c2 = quant_code(w.z, sc, rs, p.bits), c3 = quant_code(w.w, sc, rs, p.bits);
-          const uint32_t lo = pack_bf16(mul_rn(static_cast<float>(c0), sc), mul_rn(static_cast<float>(c1), sc));
-          const uint32_t hi = pack_bf16(mul_rn(static_cast<float>(c2), sc), mul_rn(static_cast<float>(c3), sc));
+          // the training quantizer's codes (exact float values) and fl32(c * s)
+          const float2 s2 = make_float2(sc, sc);
+          const float2 w01 = mul2(grid_code_values2<BITS>(w.x, w.y, sc, rs), s2);
+          const float2 w23 = mul2(grid_code_values2<BITS>(w.z, w.w, sc, rs), s2);
+          const uint32_t lo = pack_bf16(w01.x, w01.y);
+          const uint32_t hi = pack_bf16(w23.x, w23.y);
           const uint32_t kb = static_cast<uint32_t>(j >> 4), g = static_cast<uint32_t>((j & 15) >> 1);
           st_shared_v2(rbase + kb * C::KB_BYTES + ((g ^ sw) << 4) + static_cast<uint32_t>(j & 1) * 8u,
                        lo, hi);
@@ -483,10 +485,23 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR, EPI, FB>::THREADS, 1)
     uint32_t r_issued = 0, r_used = 0;  // R ring: chunks requested / consumed
     // the leader's tmem-empty barrier, which both CTAs' epilogues release
     const uint32_t tempty_leader = PAIR ? mapa_shared(smem_u32(tempty), 0) : smem_u32(tempty);
+    // FB: L2 prefetch of this CTA's weight rows of N block nb (one thread).
+    auto prefetch_panel = [&](int nb) {
+      const int n0 = nb * BN + static_cast<int>(rank) * C::B_ROWS;
+      const int rows = min(C::B_ROWS, p.N - n0);
+      if (rows <= 0) return;
+      const char* src = reinterpret_cast<const char*>(p.W + static_cast<int64_t>(n0) * p.K);
+      int64_t bytes = static_cast<int64_t>(rows) * p.K * 4;
+      for (; bytes > 0; bytes -= 65536, src += 65536)
+        bulk_prefetch_l2(src, static_cast<uint32_t>(bytes < 65536 ? bytes : 65536));
+    };
     // FB: write the panel of N block nb (this CTA's B_ROWS rows) and tell the MMA.
     auto produce_panel = [&](int nb) {
       if constexpr (FB) {
-        convert_panel<C>(p, panel, nb * BN + static_cast<int>(rank) * C::B_ROWS, ew, lane);
+        const int n_base = nb * BN + static_cast<int>(rank) * C::B_ROWS;
+        if (p.bits == 6) convert_panel<C, 6>(p, panel, n_base, ew, lane);
+        else if (p.bits == 5) convert_panel<C, 5>(p, panel, n_base, ew, lane);
+        else convert_panel<C, 8>(p, panel, n_base, ew, lane);
         fence_proxy_async_smem();  // generic-proxy writes visible to the tensor cores
         __syncwarp();
         if (lane == 0) {
@@ -504,13 +519,7 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR, EPI, FB>::THREADS, 1)
           if (nb == last) continue;
           last = nb;
           ++count;
-          const int n0 = nb * BN + static_cast<int>(rank) * C::B_ROWS;
-          const int rows = min(C::B_ROWS, p.N - n0);
-          if (rows <= 0) continue;
-          const char* src = reinterpret_cast<const char*>(p.W + static_cast<int64_t>(n0) * p.K);
-          int64_t bytes = static_cast<int64_t>(rows) * p.K * 4;
-          for (; bytes > 0; bytes -= 65536, src += 65536)
-            bulk_prefetch_l2(src, static_cast<uint32_t>(bytes < 65536 ? bytes : 65536));
+          prefetch_panel(nb);
         }
       }
       if (t_begin < t_end) produce_panel(tile_nb(t_begin));
@@ -518,6 +527,14 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR, EPI, FB>::THREADS, 1)
     for (int tile = t_begin; tile < t_end; tile += t_step) {
       const int nb = tile_nb(tile);
       const int mb = tile_mb(tile);
+      if constexpr (FB) {
+        // refresh the L2 copy of the next panel's rows a few tiles before it is
+        // built (the start-of-kernel prefetch is long evicted by then)
+        constexpr int kAhead = 3;
+        if (ew == 0 && lane == 0 && tile + kAhead < t_end &&
+            tile_nb(tile + kAhead) != tile_nb(tile + kAhead - 1))
+          prefetch_panel(tile_nb(tile + kAhead));
+      }
       const int row0 = mb * C::TILE_M + static_cast<int>(rank) * BM + q * 32;
       const int ncols = min(BN, p.N - nb * BN);
       const int nchunks = (ncols + 31) / 32;

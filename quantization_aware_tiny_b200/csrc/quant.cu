@@ -165,25 +165,6 @@ __device__ __forceinline__ RowQuant row_params(const ExportDescDev& d, float t1,
   return q;
 }
 
-// ---- paired fp32 arithmetic (two IEEE round-to-nearest operations per instruction)
-__device__ __forceinline__ uint64_t f2u(float2 v) { return *reinterpret_cast<uint64_t*>(&v); }
-__device__ __forceinline__ float2 u2f(uint64_t v) { return *reinterpret_cast<float2*>(&v); }
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
-  uint64_t d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2u(a)), "l"(f2u(b)));
-  return u2f(d);
-}
-__device__ __forceinline__ float2 add2(float2 a, float2 b) {
-  uint64_t d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2u(a)), "l"(f2u(b)));
-  return u2f(d);
-}
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f2u(a)), "l"(f2u(b)), "l"(f2u(c)));
-  return u2f(d);
-}
-
 // Which clamps a row's codes need (chosen per row from its largest |w| a1 and
 // its clip; see row_range):
 //   kClampW    -- clamp w to [-clip, clip], then the grid's clamp;
@@ -208,7 +189,6 @@ __device__ __forceinline__ int row_range(float a1, const RowQuant& q) {
   return a1 <= __fmul_rn(kNarrowRatio, q.clip) ? kNarrow : kClampGrid;
 }
 
-constexpr float kOff = 12582912.0f;  // 1.5 * 2^23
 
 // kOff + rne(fl32(w / s)) for two weights: the Markstein-corrected quotient
 // (see div_by_scale) done pairwise, then the rounding offset 1.5 * 2^23 (see
@@ -303,24 +283,6 @@ __device__ __forceinline__ uint32_t codes4_t(const RowQuant& q, float4 v) {
 }
 
 // ------------------------------------------------------------------ QAT quantize
-// Codes of two weights as exact float values, for the training quantizer's
-// row scale s = fl32(amax / L) (L = 127, or 15 for int5): every
-// |fl32(w / s)| <= amax / s < L + 1/2, so rne(w / s) is already in [-L, L]
-// and only int6's second rounding can leave the grid (4 * rne(127 / 4) = 128
-// -> 124).  The paired arithmetic of codes2: kOff + rne(w / s), then for int6
-// kOff + rne(k / 4); 4 * (that - kOff) is formed exactly by one fma.
-template <int BITS>
-__device__ __forceinline__ float2 code_values2(const RowQuant& q, float a, float b) {
-  const float2 t = rne_quot2<kNarrow>(q, a, b);
-  if constexpr (BITS == 6) {
-    const float2 u = rne_quarter2(t);
-    const float2 c = fma2(u, make_float2(4.0f, 4.0f), make_float2(-4.0f * kOff, -4.0f * kOff));
-    return make_float2(fminf(c.x, 124.0f), fminf(c.y, 124.0f));
-  } else {
-    return add2(t, make_float2(-kOff, -kOff));
-  }
-}
-
 // One row of one weight: amax over the row (the first 512 columns cached in
 // registers, the rest read again from L2), the IEEE scale, codes and the bf16
 // operand bf16(fl32(c * s)).
@@ -355,7 +317,8 @@ __device__ __forceinline__ void quantize_row_t(const QuantDescDev& d, int row, i
   if (lane == 0) d.scales[row] = q.s;
   const float2 s2 = make_float2(q.s, q.s);
   auto emit = [&](int j, float4 v) {
-    const float2 c01 = code_values2<BITS>(q, v.x, v.y), c23 = code_values2<BITS>(q, v.z, v.w);
+    const float2 c01 = grid_code_values2<BITS>(v.x, v.y, q.s, q.rs);
+    const float2 c23 = grid_code_values2<BITS>(v.z, v.w, q.s, q.rs);
     const int64_t e = static_cast<int64_t>(row) * K + 4 * j;
     if (d.codes)
       *reinterpret_cast<uint32_t*>(d.codes + e) =
