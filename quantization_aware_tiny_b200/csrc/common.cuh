@@ -54,26 +54,6 @@ __device__ __forceinline__ float div_by_scale(float w, float s, float r) {
   return __fmaf_rn(rem, r, q0);
 }
 
-// Code from the quotient x = fl32(w / s) (see qat_quantize_weights):
-//   k = rne(x) (round half to even; |x| <= 128 here);
-//   int6: 4 * rne(k / 4) in integers -- with k = 4m + f, f in 0..3, the result
-//         is 4m for f <= 1, 4m + 4 for f = 3 and the even one of 4m, 4m + 4 for
-//         f = 2, i.e. (k + 1 + (m & 1)) & ~3 -- then clamped to [-128, 124];
-//   int8: k clamped to [-127, 127];
-//   int5: k clamped to [-15, 15] (the scale is then amax / 15).
-__device__ __forceinline__ int code_from_quotient(float x, int bits) {
-  // rne(x) for |x| < 2^22: adding 1.5 * 2^23 gives a float whose ulp is 1, so
-  // the sum is rounded to an integer -- ties to even, as the offset is even --
-  // and its bit pattern minus the offset's is that integer.
-  int k = __float_as_int(__fadd_rn(x, 12582912.0f)) - 0x4B400000;
-  if (bits == 6) {
-    k = (k + 1 + ((k >> 2) & 1)) & ~3;
-    return min(max(k, -128), 124);
-  }
-  if (bits == 5) return min(max(k, -15), 15);
-  return min(max(k, -127), 127);
-}
-
 // Levels of a grid's scale, s = amax / levels: 15 for int5, 127 for int6 and
 // int8 (the int6 grid is every fourth int8 level).
 __device__ __forceinline__ float grid_levels(int bits) { return bits == 5 ? 15.0f : 127.0f; }
@@ -97,7 +77,9 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
   return u2f(d);
 }
 
-constexpr float kOff = 12582912.0f;  // 1.5 * 2^23: x + kOff rounds x to an integer (|x| < 2^22)
+// 1.5 * 2^23: for |x| < 2^22, fl32(x + kOff) = kOff + rne(x) (the sum's ulp is 1,
+// and ties go to even since kOff is even), whose bit pattern is 0x4B400000 + rne(x).
+constexpr float kOff = 12582912.0f;
 
 // Codes of two weights as exact float values, for a row scale s = fl32(amax / L)
 // (L = 127, or 15 for int5) and r = fl32(1 / s): kOff + rne(fl32(w / s)) from
@@ -120,11 +102,6 @@ __device__ __forceinline__ float2 grid_code_values2(float a, float b, float s, f
   } else {
     return add2(t, make_float2(-kOff, -kOff));
   }
-}
-
-// Code of one weight on the int5 / int6 / int8 grid; r = fl32(1 / s).
-__device__ __forceinline__ int quant_code(float w, float s, float r, int bits) {
-  return code_from_quotient(div_by_scale(w, s, r), bits);
 }
 
 }  // namespace qat

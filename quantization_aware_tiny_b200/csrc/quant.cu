@@ -191,8 +191,8 @@ __device__ __forceinline__ int row_range(float a1, const RowQuant& q) {
 
 
 // kOff + rne(fl32(w / s)) for two weights: the Markstein-corrected quotient
-// (see div_by_scale) done pairwise, then the rounding offset 1.5 * 2^23 (see
-// code_from_quotient); the float's bit pattern is 0x4B400000 + rne(w / s).
+// (see div_by_scale) done pairwise, then the rounding offset kOff = 1.5 * 2^23
+// (common.cuh); the float's bit pattern is 0x4B400000 + rne(w / s).
 template <int R>
 __device__ __forceinline__ float2 rne_quot2(const RowQuant& q, float a, float b) {
   const float2 w = R == kClampW ? make_float2(fminf(fmaxf(a, -q.clip), q.clip),
@@ -211,9 +211,10 @@ __device__ __forceinline__ float2 rne_quarter2(float2 t) {
   return add2(y, make_float2(kOff, kOff));
 }
 
-// Codes of two weights on the row's grid, the same arithmetic as quant_code
-// (common.cuh) done pairwise; for int6 4 * (bits - offset bits) is formed
-// modulo 2^32.
+// Integer codes of two weights on the row's grid, with the clamps the row's
+// range needs: k = rne(fl32(w / s)); int6: 4 * rne(k / 4) clamped to
+// [-128, 124], formed as 4 * (bits of kOff + rne(k / 4)) minus 4 * (bits of
+// kOff) modulo 2^32; int8 / int5: k clamped to [-L, L].
 template <int BITS, int R>
 __device__ __forceinline__ void codes2(const RowQuant& q, float a, float b, int& ca, int& cb) {
   const float2 t = rne_quot2<R>(q, a, b);
