@@ -97,8 +97,25 @@ def dequant_state_dict(_T):
         qat.dequantize_rows_batch(items)
 
 
+def quantize_step_weights(_T):
+    """The training step's three weights (tied head 8192 x 512 int8, MLP fc
+    2048 x 512 and proj 512 x 2048 int6) quantized to their bf16 operands in
+    one qat_quantize_weights_batch launch, after a 256 MB write so the fp32
+    weights start in DRAM."""
+    c = sy.head_mlp_case(T=8)
+    W = [torch.from_numpy(c[k]).cuda() for k in ("Wemb", "Wfc", "Wproj")]
+    bits = (8, 6, 6)
+    items = [(w, b, torch.empty(w.shape[0], dtype=torch.float32, device="cuda"), None,
+              torch.empty(w.shape, dtype=torch.bfloat16, device="cuda")) for w, b in zip(W, bits)]
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
+    for _ in range(3):
+        flush.add_(1)
+        qat.qat_quantize_weights_batch(items)
+
+
 CASES = {"logits_fwd": logits_fwd, "logits_fwd_fused": logits_fwd_fused, "head_dw": head_dw, "head_dx": head_dx,
-         "mlp_step": mlp_step, "export_state_dict": export_state_dict, "dequant_state_dict": dequant_state_dict}
+         "mlp_step": mlp_step, "export_state_dict": export_state_dict, "dequant_state_dict": dequant_state_dict,
+         "quantize_step_weights": quantize_step_weights}
 
 
 def main(argv=None):
