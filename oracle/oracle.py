@@ -232,38 +232,139 @@ def mlp_bwd(Wfc_op, Wproj_op, X, pre, h, dY, act="relu2"):
     return dX, dWfc, dWproj
 
 
-def recurrent_core_fwd(q_qkv, q_o, q_fc, q_proj, X, R, d, act="relu2"):
+def _bf16_or_exact(exact):
+    """The rounding applied where the core materialises an activation or a
+    gradient tensor: bf16 round-to-nearest-even (the pages train in bf16), or
+    none at all (exact=True: the plain fp64 composition, which the
+    finite-difference pins differentiate)."""
+    if exact:
+        return lambda a: _f64(a)
+    return lambda a: bf16_round(_f64(a).astype(np.float32)).astype(np.float64)
+
+
+def core_application_fwd(ops, x, d, act="relu2", exact=False):
+    """One application of the depth-recurrent core block (P1 "Stem / Core /
+    Tail"; attention left out, so the O projection reads the query slice of
+    QKV -- a reading stated in the design notes).  ops = (qkv, o, fc, proj),
+    each a dict with the bf16 "operand" of that weight; x [T,d] is the state.
+        qkv = x Wqkv^T ; x1 = x + q Wo^T ; pre = x1 Wfc^T ; h = act(pre)
+        out = x1 + h Wproj^T
+    Each tensor handed from one GEMM to the next (qkv, x1, pre, h, out) is
+    rounded to bf16 once where it is materialised (exact=False); every sum and
+    product in between is exact fp64.  Returns the saved activations
+    {x, qkv, x1, pre, h, out} and the unrounded residual sums u1 (of x1) and
+    u2 (of out)."""
+    b = _bf16_or_exact(exact)
+    q_qkv, q_o, q_fc, q_proj = ops
+    x = _f64(x)
+    qkv = b(x @ q_qkv["operand"].T)
+    u1 = x + qkv[:, :d] @ q_o["operand"].T
+    x1 = b(u1)
+    pre_exact = x1 @ q_fc["operand"].T
+    h = b(relu2(pre_exact) if act == "relu2" else leaky2(pre_exact))
+    u2 = x1 + h @ q_proj["operand"].T
+    return {"x": x, "qkv": qkv, "x1": x1, "pre": b(pre_exact), "h": h, "out": b(u2),
+            "u1": u1, "u2": u2}
+
+
+def core_fwd_apps(apps_ops, X, d, act="relu2", exact=False):
+    """The core applied once per entry of apps_ops (application r uses
+    apps_ops[r]); returns the final state and the list of saved activations."""
+    x = _bf16_or_exact(exact)(_f64(X))
+    saved = []
+    for ops in apps_ops:
+        s = core_application_fwd(ops, x, d, act, exact)
+        saved.append(s)
+        x = s["out"]
+    return x, saved
+
+
+def recurrent_core_fwd(q_qkv, q_o, q_fc, q_proj, X, R, d, act="relu2", exact=False):
     """Depth-recurrent core (P1 "Stem / Core / Tail", "税 1"): the block's
-    linears, quantized once, applied R times.  Attention is left out, so the
-    O projection reads the query slice of QKV (reading stated in the design
-    notes).  Per application:
-        qkv = x Wqkv^T ; x1 = x + q Wo^T ; h = relu(x1 Wfc^T)^2 ; x = x1 + h Wproj^T
-    The activations handed from one GEMM to the next (qkv, x1, h and x) are
-    bf16 tensors, as in the bf16 training the pages describe: each is rounded
-    to bf16 once where it is materialised; every sum and product in between
-    is exact (fp64)."""
-    x = bf16_round(_f64(X).astype(np.float32)).astype(np.float64)
-    b = lambda a: bf16_round(a.astype(np.float32)).astype(np.float64)
-    for _ in range(R):
-        qkv = b(x @ q_qkv["operand"].T)
-        x1 = b(x + qkv[:, :d] @ q_o["operand"].T)
-        pre = x1 @ q_fc["operand"].T
-        h = b(relu2(pre) if act == "relu2" else leaky2(pre))
-        x = b(x1 + h @ q_proj["operand"].T)
-    return x
+    linears, quantized once, applied R times (see core_application_fwd)."""
+    return core_fwd_apps([(q_qkv, q_o, q_fc, q_proj)] * R, X, d, act, exact)[0]
+
+
+def core_application_bwd(ops, s, g, d, act="relu2", exact=False):
+    """Backward of one core application (chain rule through
+    core_application_fwd, STE: the quantized weights' gradients are the fp32
+    weights' gradients).  s = that application's saved activations, g = dL/d out.
+        dWproj = g^T h ; dpre = (g Wproj) * act'(pre) ; dWfc = dpre^T x1
+        dx1 = g + dpre Wfc            (residual of out = x1 + ...)
+        dWo = dx1^T q ; dq = dx1 Wo
+        dWqkv[:d] = dq^T x ; dWqkv[d:] = 0   (k and v do not reach the output
+                                               with attention left out)
+        dx = dx1 + dq Wq              (residual of x1 = x + ...)
+    The gradient tensors handed between GEMMs (dpre, dx1, dq, dx) are rounded
+    to bf16 where materialised (exact=False), as the forward's activations.
+    Returns dx and the four weight gradients {qkv, o, fc, proj}."""
+    b = _bf16_or_exact(exact)
+    q_qkv, q_o, q_fc, q_proj = ops
+    g = _f64(g)
+    dWproj = g.T @ s["h"]
+    dpre = b((g @ q_proj["operand"]) * act_grad(s["pre"], act))
+    dWfc = dpre.T @ s["x1"]
+    dx1 = b(g + dpre @ q_fc["operand"])
+    q = s["qkv"][:, :d]
+    dWo = dx1.T @ q
+    dq = b(dx1 @ q_o["operand"])
+    dWqkv = np.zeros(q_qkv["operand"].shape)
+    dWqkv[:d] = dq.T @ s["x"]
+    dx = b(dx1 + dq @ q_qkv["operand"][:d])
+    return dx, {"qkv": dWqkv, "o": dWo, "fc": dWfc, "proj": dWproj}
+
+
+def core_bwd_apps(apps_ops, saved, dY, d, act="relu2", exact=False):
+    """Backward through the applications in reverse order; each shared weight's
+    gradient is the sum of its gradients over the applications that used it
+    (P1 "税 1": one stored weight, R uses).  Returns dX, the four summed weight
+    gradients and the incoming gradient of every application (grads[r] =
+    dL/d out of application r)."""
+    g = _bf16_or_exact(exact)(_f64(dY))
+    tot = None
+    grads = [None] * len(saved)
+    for r in reversed(range(len(saved))):
+        grads[r] = g
+        g, dW = core_application_bwd(apps_ops[r], saved[r], g, d, act, exact)
+        tot = dW if tot is None else {k: tot[k] + dW[k] for k in tot}
+    return g, tot, grads
+
+
+def recurrent_core_bwd(q_qkv, q_o, q_fc, q_proj, X, dY, R, d, act="relu2", exact=False):
+    """Forward and STE backward of the recurrent core (quantized once, applied
+    R times in the forward and R times, in reverse, in the backward, dW summed
+    over the R uses).  dY = dL/d x_R.  Returns {out, dX, dWqkv, dWo, dWfc,
+    dWproj, saved, grads}."""
+    ops = [(q_qkv, q_o, q_fc, q_proj)] * R
+    out, saved = core_fwd_apps(ops, X, d, act, exact)
+    dX, dW, grads = core_bwd_apps(ops, saved, dY, d, act, exact)
+    return {"out": out, "dX": dX, "dWqkv": dW["qkv"], "dWo": dW["o"], "dWfc": dW["fc"],
+            "dWproj": dW["proj"], "saved": saved, "grads": grads}
+
+
+def noisy_core_ops(Ws, R, seed, offset, bits=6):
+    """Noisy QAT operands of the core (P1 "幸存发现 1"): application r draws the
+    four weights (qkv, o, fc, proj -> k = 0..3) at Philox offset
+    offset + 4*r + k (noise at the int8 step, or the int5 step for bits = 5)."""
+    return [tuple({"operand": noisy_weight(w, seed, offset + 4 * r + k, bits)["operand"]}
+                  for k, w in enumerate(Ws)) for r in range(R)]
 
 
 def recurrent_core_fwd_noisy(Ws, X, R, d, seed, offset, bits=6, act="relu2"):
-    """The recurrent core under Noisy QAT (P1 "幸存发现 1"): application r uses
-    the noisy operands of the four weights (qkv, o, fc, proj -> k = 0..3) drawn
-    at Philox offset offset + 4*r + k (noise at the int8 step, or at the int5
-    step for bits = 5), composed exactly as recurrent_core_fwd."""
-    x = X
-    for r in range(R):
-        q = [{"operand": noisy_weight(w, seed, offset + 4 * r + k, bits)["operand"]}
-             for k, w in enumerate(Ws)]
-        x = recurrent_core_fwd(q[0], q[1], q[2], q[3], x, 1, d, act)
-    return x
+    """The recurrent core under Noisy QAT: application r uses its own noisy
+    operands (noisy_core_ops), composed exactly as recurrent_core_fwd."""
+    return core_fwd_apps(noisy_core_ops(Ws, R, seed, offset, bits), X, d, act)[0]
+
+
+def recurrent_core_bwd_noisy(Ws, X, dY, R, d, seed, offset, bits=6, act="relu2"):
+    """Forward and backward of the Noisy-QAT core: the backward of application
+    r uses that application's noisy operands (the noise carries no gradient,
+    so the weight gradient is the operand's)."""
+    ops = noisy_core_ops(Ws, R, seed, offset, bits)
+    out, saved = core_fwd_apps(ops, X, d, act)
+    dX, dW, grads = core_bwd_apps(ops, saved, dY, d, act)
+    return {"out": out, "dX": dX, "dWqkv": dW["qkv"], "dWo": dW["o"], "dWfc": dW["fc"],
+            "dWproj": dW["proj"], "saved": saved, "grads": grads}
 
 
 def head_mlp_step(q_emb, q_fc, q_proj, X, dLogits, act="relu2"):

@@ -503,6 +503,90 @@ def test_recurrent_core_is_r_applications():
     assert np.array_equal(one, ref)
 
 
+def _tiny_core(rng, d, H, scale):
+    nqkv = 2 * d
+    ops = tuple({"operand": rng.standard_normal(shp) * scale}
+                for shp in ((nqkv, d), (d, d), (H, d), (d, H)))
+    return ops
+
+
+@pytest.mark.parametrize("act", ["relu2", "leaky2"])
+def test_recurrent_core_bwd_finite_differences(act):
+    """The core's backward through R = 3 applications (exact composition, no
+    bf16 rounding) matches central differences of L = sum(dY * x_R) for the
+    input and for all four shared weights -- each weight's gradient is the
+    sum over the three uses (P1 "税 1")."""
+    rng = np.random.default_rng(21)
+    d, H, T, R = 8, 24, 3, 3
+    ops = _tiny_core(rng, d, H, 0.35)
+    X, dY = rng.standard_normal((T, d)), rng.standard_normal((T, d))
+    out = o.recurrent_core_bwd(*ops, X, dY, R, d, act=act, exact=True)
+    assert min(np.abs(s["pre"]).min() for s in out["saved"]) > 1e-3  # off the kink
+    L = lambda: float(np.sum(dY * o.recurrent_core_fwd(*ops, X, R, d, act=act, exact=True)))
+    assert np.allclose(out["dX"], _fd(L, X), atol=1e-5, rtol=1e-6)
+    for name, k in (("dWqkv", 0), ("dWo", 1), ("dWfc", 2), ("dWproj", 3)):
+        assert np.allclose(out[name], _fd(L, ops[k]["operand"]), atol=1e-5, rtol=1e-6), name
+    # k and v do not reach the output when attention is left out
+    assert np.all(out["dWqkv"][d:] == 0)
+
+
+def test_recurrent_core_bwd_against_torch_autograd():
+    """The same composition written with torch ops in float64 and
+    differentiated by torch.autograd, at the small core shape d = 64."""
+    rng = np.random.default_rng(22)
+    d, H, T, R = 64, 192, 16, 3
+    ops = _tiny_core(rng, d, H, 0.05)
+    X, dY = rng.standard_normal((T, d)), rng.standard_normal((T, d))
+    out = o.recurrent_core_bwd(*ops, X, dY, R, d, exact=True)
+    W = [torch.tensor(op["operand"], requires_grad=True) for op in ops]
+    x = torch.tensor(X, requires_grad=True)
+    s = x
+    for _ in range(R):
+        q = (s @ W[0].T)[:, :d]
+        x1 = s + q @ W[1].T
+        s = x1 + torch.relu(x1 @ W[2].T) ** 2 @ W[3].T
+    (s * torch.tensor(dY)).sum().backward()
+    assert np.allclose(out["out"], s.detach().numpy(), rtol=1e-12, atol=1e-12)
+    assert np.allclose(out["dX"], x.grad.numpy(), rtol=1e-10, atol=1e-12)
+    for name, w in zip(("dWqkv", "dWo", "dWfc", "dWproj"), W):
+        assert np.allclose(out[name], w.grad.numpy(), rtol=1e-10, atol=1e-12), name
+
+
+def test_recurrent_core_bwd_bf16_application_by_hand():
+    """One application's backward with the bf16 rounding of each materialised
+    gradient (dpre, dx1, dq, dx) done by torch; the summed weight gradient over
+    R = 3 equals the sum of the per-application gradients at the saved states."""
+    c = sy.recurrent_core_case(d=64, H=192, T=16)
+    ops = tuple(o.quantize_weight(w, 6) for w in
+                (np.concatenate([c["Wq"], c["Wk"], c["Wv"]]), c["Wo"], c["Wfc"], c["Wproj"]))
+    X = c["X"].float().numpy()
+    dY = sy.act_bf16(np.random.default_rng(5), 16, 64, std=0.01).float().numpy()
+    out = o.recurrent_core_bwd(*ops, X, dY, 3, 64)
+    b = lambda a: torch.from_numpy(np.asarray(a, np.float32)).to(torch.bfloat16).double().numpy()
+    s, g = out["saved"][2], out["grads"][2]
+    assert np.array_equal(g, b(dY))
+    Wqkv, Wo, Wfc, Wproj = (op["operand"] for op in ops)
+    dpre = b((g @ Wproj) * 2.0 * np.maximum(s["pre"], 0.0))
+    dx1 = b(g + dpre @ Wfc)
+    dq = b(dx1 @ Wo)
+    dx = b(dx1 + dq @ Wqkv[:64])
+    assert np.array_equal(out["grads"][1], dx)
+    tot = {"qkv": 0.0, "o": 0.0, "fc": 0.0, "proj": 0.0}
+    for r in range(3):
+        s, g = out["saved"][r], out["grads"][r]
+        dpre = b((g @ Wproj) * 2.0 * np.maximum(s["pre"], 0.0))
+        dx1 = b(g + dpre @ Wfc)
+        dq = b(dx1 @ Wo)
+        tot["proj"] = tot["proj"] + g.T @ s["h"]
+        tot["fc"] = tot["fc"] + dpre.T @ s["x1"]
+        tot["o"] = tot["o"] + dx1.T @ s["qkv"][:, :64]
+        tot["qkv"] = tot["qkv"] + np.vstack([dq.T @ s["x"], np.zeros((64, 64))])
+    for k in tot:
+        assert np.allclose(out["dW" + k], tot[k], rtol=1e-12, atol=1e-15), k
+    for k in ("dX",):
+        assert np.array_equal(out[k], b(out[k]))
+
+
 # ------------------------------------------------------------- Noisy QAT
 
 def test_philox_known_answers():
