@@ -155,13 +155,20 @@ int qat_linear_fwd(const float* W, const qat_qweight* qw, int32_t N, int32_t K, 
 
 /* STE backward of qat_linear_fwd ([P5]: the forward uses the quantized weight,
  * the gradient flows to the fp32 weight unchanged):
- *   dX[T,K] = bf16( dY[T,N] . Wq )            (nullable)
- *   dW[N,K] (+)= dY^T . X   in fp32            (nullable; accumulate_dW != 0 adds
- *                                               into dW, e.g. over R recurrent uses)
- * dX needs W or qw; dW needs neither. */
+ *   dX[T,K] = bf16( dY[T,N] . Wq (+ dX_residual) )   (nullable)
+ *   dW[N,K] (+)= dY^T . X   in fp32                   (nullable; accumulate_dW != 0
+ *                                                      adds into dW, e.g. over the
+ *                                                      R uses of a recurrent weight)
+ * dX needs W or qw; dW needs neither.  ldx = row stride of X in elements
+ * (0 -> K; a multiple of 8, >= K), so X may be a column slice of a wider
+ * activation.  dX_residual (nullable, [T,K] bf16, needs dX) is added to the
+ * fp32 product before the bf16 rounding -- the gradient of a residual
+ * connection around the linear -- and may alias dX exactly.  With T = 0, dW
+ * is zeroed unless accumulate_dW. */
 int qat_linear_bwd(const float* W, const qat_qweight* qw, int32_t N, int32_t K, int32_t bits,
-                   const qat_bf16* X, const qat_bf16* dY, int64_t T, qat_bf16* dX, float* dW,
-                   int32_t accumulate_dW, void* workspace, size_t ws_bytes, qat_stream_t stream);
+                   const qat_bf16* X, int64_t ldx, const qat_bf16* dY, int64_t T,
+                   const qat_bf16* dX_residual, qat_bf16* dX, float* dW, int32_t accumulate_dW,
+                   void* workspace, size_t ws_bytes, qat_stream_t stream);
 
 /* MLP activations: [P5] "架构" relu(x)^2, and leaky_relu(x, 0.5)^2 ([P1]
  * negative result #9 "LeakyReLU(0.5)²"; [P4] leaderboard entries use it). */
@@ -185,13 +192,17 @@ int qat_mlp_fwd(const float* Wfc, const float* Wproj, const qat_qweight* qfc,
 /* STE backward of qat_mlp_fwd from the saved pre and h:
  *   dh = dY . Wproj_q;  dpre = dh * act'(pre) (fused in the dh epilogue:
  *   2*relu(pre), or for QAT_ACT_LEAKY_RELU2 2*pre (pre > 0) else pre/2);
- *   dWproj (+)= dY^T . h;  dWfc (+)= dpre^T . X;  dX = dpre . Wfc_q.
- * dX, dWfc, dWproj may each be NULL.  The workspace holds dpre [T,H] bf16. */
+ *   dWproj (+)= dY^T . h;  dWfc (+)= dpre^T . X;
+ *   dX = bf16( dpre . Wfc_q (+ dX_residual) ).
+ * dX, dWfc, dWproj may each be NULL.  dX_residual (nullable, [T,d] bf16,
+ * needs dX; may alias dX exactly) adds the gradient that bypasses the MLP
+ * through a residual connection.  The workspace holds dpre [T,H] bf16. */
 int qat_mlp_bwd(const float* Wfc, const float* Wproj, const qat_qweight* qfc,
                 const qat_qweight* qproj, int32_t d, int32_t H, int32_t bits, int32_t act,
                 const qat_bf16* X, const qat_bf16* pre, const qat_bf16* h, const qat_bf16* dY,
-                int64_t T, qat_bf16* dX, float* dWfc, float* dWproj, int32_t accumulate_dW,
-                void* workspace, size_t ws_bytes, qat_stream_t stream);
+                int64_t T, const qat_bf16* dX_residual, qat_bf16* dX, float* dWfc,
+                float* dWproj, int32_t accumulate_dW, void* workspace, size_t ws_bytes,
+                qat_stream_t stream);
 
 /* Diagnostic (the pages have no counterpart): runs the library's bounded
  * device wait on a barrier that nothing arrives on, with a limit of limit_ns
@@ -219,7 +230,9 @@ int qat_selftest_wait_timeout(int64_t limit_ns, qat_stream_t stream);
  *   that loads the library holds this array (8 MiB + 64 KiB) until exit.
  *   The first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress, with that device current); make that first call
- *   before any stream capture.
+ *   before any stream capture.  The address is cached per process and per
+ *   device's primary context: after cudaDeviceReset on a device, the cached
+ *   address is stale and this entry point must not be called there again.
  *   All calls share the array and each rewrites what it reads, so nothing
  *   must start at zero; calls whose kernels overlap on the GPU (other streams
  *   or host threads on the same device) race on it -- serialize them.

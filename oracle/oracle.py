@@ -297,7 +297,8 @@ def core_application_bwd(ops, s, g, d, act="relu2", exact=False):
         dx = dx1 + dq Wq              (residual of x1 = x + ...)
     The gradient tensors handed between GEMMs (dpre, dx1, dq, dx) are rounded
     to bf16 where materialised (exact=False), as the forward's activations.
-    Returns dx and the four weight gradients {qkv, o, fc, proj}."""
+    Returns dx, the four weight gradients {qkv, o, fc, proj} and the
+    intermediate gradients {dpre, dx1, dq}."""
     b = _bf16_or_exact(exact)
     q_qkv, q_o, q_fc, q_proj = ops
     g = _f64(g)
@@ -311,23 +312,26 @@ def core_application_bwd(ops, s, g, d, act="relu2", exact=False):
     dWqkv = np.zeros(q_qkv["operand"].shape)
     dWqkv[:d] = dq.T @ s["x"]
     dx = b(dx1 + dq @ q_qkv["operand"][:d])
-    return dx, {"qkv": dWqkv, "o": dWo, "fc": dWfc, "proj": dWproj}
+    return dx, {"qkv": dWqkv, "o": dWo, "fc": dWfc, "proj": dWproj}, \
+        {"dpre": dpre, "dx1": dx1, "dq": dq}
 
 
 def core_bwd_apps(apps_ops, saved, dY, d, act="relu2", exact=False):
     """Backward through the applications in reverse order; each shared weight's
     gradient is the sum of its gradients over the applications that used it
     (P1 "税 1": one stored weight, R uses).  Returns dX, the four summed weight
-    gradients and the incoming gradient of every application (grads[r] =
-    dL/d out of application r)."""
+    gradients, the incoming gradient of every application (grads[r] =
+    dL/d out of application r) and each application's intermediate
+    gradients."""
     g = _bf16_or_exact(exact)(_f64(dY))
     tot = None
     grads = [None] * len(saved)
+    inter = [None] * len(saved)
     for r in reversed(range(len(saved))):
         grads[r] = g
-        g, dW = core_application_bwd(apps_ops[r], saved[r], g, d, act, exact)
+        g, dW, inter[r] = core_application_bwd(apps_ops[r], saved[r], g, d, act, exact)
         tot = dW if tot is None else {k: tot[k] + dW[k] for k in tot}
-    return g, tot, grads
+    return g, tot, grads, inter
 
 
 def recurrent_core_bwd(q_qkv, q_o, q_fc, q_proj, X, dY, R, d, act="relu2", exact=False):
@@ -337,9 +341,9 @@ def recurrent_core_bwd(q_qkv, q_o, q_fc, q_proj, X, dY, R, d, act="relu2", exact
     dWproj, saved, grads}."""
     ops = [(q_qkv, q_o, q_fc, q_proj)] * R
     out, saved = core_fwd_apps(ops, X, d, act, exact)
-    dX, dW, grads = core_bwd_apps(ops, saved, dY, d, act, exact)
+    dX, dW, grads, inter = core_bwd_apps(ops, saved, dY, d, act, exact)
     return {"out": out, "dX": dX, "dWqkv": dW["qkv"], "dWo": dW["o"], "dWfc": dW["fc"],
-            "dWproj": dW["proj"], "saved": saved, "grads": grads}
+            "dWproj": dW["proj"], "saved": saved, "grads": grads, "inter": inter}
 
 
 def noisy_core_ops(Ws, R, seed, offset, bits=6):
@@ -362,9 +366,9 @@ def recurrent_core_bwd_noisy(Ws, X, dY, R, d, seed, offset, bits=6, act="relu2")
     so the weight gradient is the operand's)."""
     ops = noisy_core_ops(Ws, R, seed, offset, bits)
     out, saved = core_fwd_apps(ops, X, d, act)
-    dX, dW, grads = core_bwd_apps(ops, saved, dY, d, act)
+    dX, dW, grads, inter = core_bwd_apps(ops, saved, dY, d, act)
     return {"out": out, "dX": dX, "dWqkv": dW["qkv"], "dWo": dW["o"], "dWfc": dW["fc"],
-            "dWproj": dW["proj"], "saved": saved, "grads": grads}
+            "dWproj": dW["proj"], "saved": saved, "grads": grads, "inter": inter}
 
 
 def head_mlp_step(q_emb, q_fc, q_proj, X, dLogits, act="relu2"):

@@ -1,6 +1,7 @@
-"""Small single-kernel cases for profiler captures (ncu -k ... -c ...).
+"""Small single-kernel cases for profiler captures (ncu -k ... -c ...), next to
+the benchmark that times the same kernels at full size.
 
-    python -m quantization_aware_tiny_b200.profile_cases <case> [--T tokens]
+    python profile_cases.py <case> [--T tokens]
 
 Each case sets up its inputs, launches the named kernel a few times and exits.
 Cases are sized so one capture stays small (a few hundred MB on the device)
@@ -12,9 +13,10 @@ import sys
 import numpy as np
 import torch
 
-from . import export as qexport
-from . import qat
-from . import synthetic as sy
+from quantization_aware_tiny_b200 import export as qexport
+from quantization_aware_tiny_b200 import qat
+from quantization_aware_tiny_b200 import steps
+from quantization_aware_tiny_b200 import synthetic as sy
 
 
 def logits_fwd(T):
@@ -113,7 +115,20 @@ def quantize_step_weights(_T):
         qat.qat_quantize_weights_batch(items)
 
 
-CASES = {"logits_fwd": logits_fwd, "logits_fwd_fused": logits_fwd_fused, "head_dw": head_dw, "head_dx": head_dx,
+def core_train(T):
+    """The d=640 recurrent core (R=3): forward keeping activations and the
+    backward over the three applications (8 backward GEMMs per application)."""
+    c = sy.recurrent_core_case(T=T)
+    w = {k: torch.from_numpy(c[k]).cuda() for k in ("Wq", "Wk", "Wv", "Wo", "Wfc", "Wproj")}
+    core = steps.RecurrentCore(w["Wq"], w["Wk"], w["Wv"], w["Wo"], w["Wfc"], w["Wproj"], 6)
+    x = c["X"].cuda()
+    dY = sy.act_bf16(np.random.default_rng(3), T, 640, std=0.01).cuda()
+    for _ in range(2):
+        core.forward_train(x, 3)
+        core.backward(dY)
+
+
+CASES = {"core_train": core_train, "logits_fwd": logits_fwd, "logits_fwd_fused": logits_fwd_fused, "head_dw": head_dw, "head_dx": head_dx,
          "mlp_step": mlp_step, "export_state_dict": export_state_dict, "dequant_state_dict": dequant_state_dict,
          "quantize_step_weights": quantize_step_weights}
 

@@ -12,32 +12,48 @@ namespace qat {
 // The one device-side error flag (per device, zero-initialised at load).
 __device__ int g_device_error = 0;
 
+// Per-device caches below are filled on first use with the device current;
+// concurrent first calls from several host threads store the same value.
 int* device_error_ptr() {
-  static int* cached[64] = {nullptr};
+  static std::atomic<int*> cached[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!cached[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
-    cached[dev] = static_cast<int*>(p);
+  int* p = cached[dev].load(std::memory_order_acquire);
+  if (!p) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_device_error) != cudaSuccess) return nullptr;
+    p = static_cast<int*>(a);
+    cached[dev].store(p, std::memory_order_release);
   }
-  return cached[dev];
+  return p;
 }
 
 static std::atomic<int64_t> g_launches{0};
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 int sm_count() {
-  static int cached[64] = {0};
+  static std::atomic<int> cached[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (cached[dev] == 0) {
-    int n = 0;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
       n = 148;
-    cached[dev] = n;
+    cached[dev].store(n, std::memory_order_relaxed);
   }
-  return cached[dev];
+  return n;
+}
+
+bool device_flag_once(std::atomic<uint64_t>& done, int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  if (dev_out) *dev_out = dev;
+  if (dev < 0 || dev >= 64) return false;
+  return (done.load(std::memory_order_acquire) >> dev) & 1u;
+}
+
+void device_flag_set(std::atomic<uint64_t>& done, int dev) {
+  if (dev >= 0 && dev < 64) done.fetch_or(uint64_t{1} << dev, std::memory_order_acq_rel);
 }
 
 namespace {
@@ -201,23 +217,28 @@ int qat_linear_fwd(const float* W, const qat_qweight* qw, int32_t N, int32_t K, 
 }
 
 int qat_linear_bwd(const float* W, const qat_qweight* qw, int32_t N, int32_t K, int32_t bits,
-                   const qat_bf16* X, const qat_bf16* dY, int64_t T, qat_bf16* dX, float* dW,
-                   int32_t accumulate_dW, void* workspace, size_t ws_bytes, qat_stream_t stream) {
+                   const qat_bf16* X, int64_t ldx, const qat_bf16* dY, int64_t T,
+                   const qat_bf16* dX_residual, qat_bf16* dX, float* dW, int32_t accumulate_dW,
+                   void* workspace, size_t ws_bytes, qat_stream_t stream) {
   if ((T > 0 && !dY) || T < 0 || !bits_ok(bits)) return QAT_ERR_ARG;
   if (!dim_ok(N) || !dim_ok(K)) return QAT_ERR_SHAPE;
   if (T > 0 && dW && !X) return QAT_ERR_ARG;
+  if (dX_residual && !dX) return QAT_ERR_ARG;
+  if (ldx == 0) ldx = K;
+  if (ldx < K || (ldx & 7)) return QAT_ERR_SHAPE;
   Carver ws(workspace, ws_bytes);
   if (dX) {
     const __nv_bfloat16* op = nullptr;
     int rc = get_operand(W, qw, N, K, bits, ws, stream, &op);
     if (rc) return rc;
     if (T > 0) {
-      GemmDesc g;  // dX[T,K] = dY[T,N] . Wq[N,K]: B = Wq read N-major along K
+      GemmDesc g;  // dX[T,K] = dY[T,N] . Wq[N,K] (+ residual): B = Wq read N-major along K
       g.A = dY; g.lda = N;
       g.B = op; g.ldb = K; g.b_mn = true;
       g.M = T; g.N = K; g.K = N;
-      g.epi = EPI_BF16;
+      g.epi = dX_residual ? EPI_BF16_RESID : EPI_BF16;
       g.D = dX; g.ldd = K;
+      g.R = dX_residual; g.ldr = K;
       rc = launch_gemm(g, stream);
       if (rc) return rc;
     }
@@ -229,7 +250,7 @@ int qat_linear_bwd(const float* W, const qat_qweight* qw, int32_t N, int32_t K, 
     }
     GemmDesc g;  // dW[N,K] = dY^T . X : both operands read along T
     g.A = dY; g.lda = N; g.a_mn = true;
-    g.B = X; g.ldb = K; g.b_mn = true;
+    g.B = X; g.ldb = ldx; g.b_mn = true;
     g.M = N; g.N = K; g.K = T;
     g.epi = EPI_F32;
     g.D = dW; g.ldd = K;
@@ -293,10 +314,11 @@ int qat_mlp_fwd(const float* Wfc, const float* Wproj, const qat_qweight* qfc,
 int qat_mlp_bwd(const float* Wfc, const float* Wproj, const qat_qweight* qfc,
                 const qat_qweight* qproj, int32_t d, int32_t H, int32_t bits, int32_t act,
                 const qat_bf16* X, const qat_bf16* pre, const qat_bf16* h, const qat_bf16* dY,
-                int64_t T, qat_bf16* dX, float* dWfc, float* dWproj, int32_t accumulate_dW,
-                void* workspace, size_t ws_bytes, qat_stream_t stream) {
+                int64_t T, const qat_bf16* dX_residual, qat_bf16* dX, float* dWfc, float* dWproj,
+                int32_t accumulate_dW, void* workspace, size_t ws_bytes, qat_stream_t stream) {
   if ((T > 0 && (!X || !pre || !h || !dY)) || T < 0 || !bits_ok(bits) || !act_ok(act))
     return QAT_ERR_ARG;
+  if (dX_residual && !dX) return QAT_ERR_ARG;
   if (!dim_ok(d) || !dim_ok(H)) return QAT_ERR_SHAPE;
   Carver ws(workspace, ws_bytes);
   const __nv_bfloat16 *op_fc = nullptr, *op_proj = nullptr;
@@ -348,13 +370,14 @@ int qat_mlp_bwd(const float* Wfc, const float* Wproj, const qat_qweight* qfc,
     rc = launch_gemm(g, stream);
     if (rc) return rc;
   }
-  if (dX) {  // dX[T,d] = dpre . Wfc_q
+  if (dX) {  // dX[T,d] = dpre . Wfc_q (+ residual)
     GemmDesc g;
     g.A = dpre; g.lda = H;
     g.B = op_fc; g.ldb = d; g.b_mn = true;
     g.M = T; g.N = d; g.K = H;
-    g.epi = EPI_BF16;
+    g.epi = dX_residual ? EPI_BF16_RESID : EPI_BF16;
     g.D = dX; g.ldd = d;
+    g.R = dX_residual; g.ldr = d;
     rc = launch_gemm(g, stream);
     if (rc) return rc;
   }

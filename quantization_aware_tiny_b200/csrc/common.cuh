@@ -7,6 +7,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/qat.h"
 
 namespace qat {
@@ -24,7 +26,13 @@ inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? QAT_OK : QAT_E
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int sm_count();
+int sm_count();  // SMs of the current device (cached per device)
+
+// One bit per device of a once-per-device flag (e.g. a kernel attribute, which
+// belongs to each device's context).  device_flag_once returns whether the
+// current device's bit is set and reports the device; device_flag_set sets it.
+bool device_flag_once(std::atomic<uint64_t>& done, int* dev_out);
+void device_flag_set(std::atomic<uint64_t>& done, int dev);
 
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
   unsigned long long t;

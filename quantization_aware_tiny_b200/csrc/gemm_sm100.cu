@@ -15,6 +15,7 @@
 // overlap the main loop of tile i+1.  Tiles are 128 x BN x 64; split-K (for
 // the long-K weight-gradient GEMMs) adds fp32 partial sums with TMA reduce-add.
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "gemm_sm100.cuh"
@@ -708,12 +709,15 @@ int launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& md
              const CUtensorMap& md2, const CUtensorMap& mr, const KArgs& a, cudaStream_t s) {
   using C = Cfg<BN, PAIR, EPI, FB>;
   auto kern = gemm_kernel<BN, A_MN, B_MN, EPI, PAIR, FB>;
-  static bool attr_done = false;  // per instantiation; set before first launch
-  if (!attr_done) {
+  // the shared-memory attribute belongs to each device's context: set it once
+  // per instantiation and device, before the first launch there
+  static std::atomic<uint64_t> attr_done{0};
+  int dev = 0;
+  if (!device_flag_once(attr_done, &dev)) {
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return QAT_ERR_CUDA;
-    attr_done = true;
+    device_flag_set(attr_done, dev);
   }
   const int units = PAIR ? sm_count() / 2 : sm_count();
   const int grid = std::max(1, std::min(a.num_tiles, units)) * (PAIR ? 2 : 1);
@@ -754,6 +758,8 @@ int dispatch_bn(const GemmDesc& g, const CUtensorMap& ma, const CUtensorMap& mb,
   } else if (!g.a_mn && g.b_mn) {
     switch (epi) {
       case EPI_BF16: return launch_t<BN, false, true, EPI_BF16, PAIR>(ma, mb, md, md2, mr, a, s);
+      case EPI_BF16_RESID:
+        return launch_t<BN, false, true, EPI_BF16_RESID, PAIR>(ma, mb, md, md2, mr, a, s);
       case EPI_DRELU2: return launch_t<BN, false, true, EPI_DRELU2, PAIR>(ma, mb, md, md2, mr, a, s);
       case EPI_DLRELU2:
         return launch_t<BN, false, true, EPI_DLRELU2, PAIR>(ma, mb, md, md2, mr, a, s);

@@ -61,10 +61,9 @@ extern "C" int qat_linear_fwd_noalloc(const float* W, int32_t N, int32_t K, int3
     return QAT_ERR_SHAPE;
   if (ldx == 0) ldx = K;
   if (ldx < K || (ldx & 7)) return QAT_ERR_SHAPE;
-  if (!aligned16(W) || (X && !aligned16(X)) || (Y && !aligned16(Y)) ||
-      (residual && !aligned16(residual)))
+  if (T == 0) return QAT_OK;  // as qat_linear_fwd: no tokens, nothing checked further
+  if (!aligned16(W) || !aligned16(X) || !aligned16(Y) || (residual && !aligned16(residual)))
     return QAT_ERR_ALIGN;
-  if (T == 0) return QAT_OK;
   unsigned char* scratch = nullptr;
   int rc = scratch_on_current_device(&scratch);
   if (rc) return rc;

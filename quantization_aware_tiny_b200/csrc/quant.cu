@@ -8,6 +8,7 @@
 // SM; the training-time kernel caches the row in registers between its
 // reduction and quantization passes.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <type_traits>
 
@@ -1070,8 +1071,9 @@ int clip_search_supported(int64_t cols) {
 
 int launch_export_batch(ExportBatch& b, cudaStream_t s) {
   if (b.total_units == 0) return QAT_OK;
-  static bool attr_done = false;
-  if (!attr_done) {
+  static std::atomic<uint64_t> attr_done{0};  // per device: attributes live in its context
+  int dev = 0;
+  if (!device_flag_once(attr_done, &dev)) {
     if (cudaFuncSetAttribute(export_batch_kernel<kExportPlain>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kExportSmemBudget) != cudaSuccess ||
@@ -1082,7 +1084,7 @@ int launch_export_batch(ExportBatch& b, cudaStream_t s) {
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kExportSmemBudget) != cudaSuccess)
       return QAT_ERR_CUDA;
-    attr_done = true;
+    device_flag_set(attr_done, dev);
   }
   int64_t longest = 16;  // bytes of the longest staged unit
   for (int i = 0; i < b.n; ++i)

@@ -93,10 +93,10 @@ def lib():
         L.qat_workspace_size.argtypes = [I32, I32, I32, I64, I32]
         L.qat_workspace_size.restype = SZ
         L.qat_linear_fwd.argtypes = [P, P, I32, I32, I32, P, I64, I64, P, P, P, SZ, P]
-        L.qat_linear_bwd.argtypes = [P, P, I32, I32, I32, P, P, I64, P, P, I32, P, SZ, P]
+        L.qat_linear_bwd.argtypes = [P, P, I32, I32, I32, P, I64, P, I64, P, P, P, I32, P, SZ, P]
         L.qat_mlp_fwd.argtypes = [P, P, P, P, I32, I32, I32, I32, P, I64, P, P, P, P, P, SZ, P]
-        L.qat_mlp_bwd.argtypes = [P, P, P, P, I32, I32, I32, I32, P, P, P, P, I64, P, P, P, I32, P,
-                                  SZ, P]
+        L.qat_mlp_bwd.argtypes = [P, P, P, P, I32, I32, I32, I32, P, P, P, P, I64, P, P, P, P, I32,
+                                  P, SZ, P]
         L.quantize_rows_export.argtypes = [P, I64, I64, I32, P, P, P]
         L.quantize_export_batch.argtypes = [P, I32, P]
         L.dequantize_rows.argtypes = [P, P, I64, I64, I32, P, P]
@@ -252,13 +252,14 @@ def qat_linear_fwd(X, Y, bits, W=None, qw=None, residual=None, workspace=None, N
 
 
 def qat_linear_bwd(X, dY, bits, W=None, qw=None, dX=None, dW=None, accumulate_dW=False,
-                   workspace=None, N=None, K=None, stream=None):
+                   workspace=None, N=None, K=None, ldx=0, dX_residual=None, stream=None):
+    """dX = bf16(dY . Wq (+ dX_residual)); dW (+)= dY^T . X (X rows ldx apart)."""
     if N is None:
         N, K = (qw.N, qw.K) if qw is not None else ((W.shape) if W is not None else dW.shape)
     ws, wsb = _ws(workspace)
-    _check(lib().qat_linear_bwd(_p(W), _qref(qw), N, K, bits, _p(X), _p(dY), dY.shape[0], _p(dX),
-                                _p(dW), int(bool(accumulate_dW)), ws, wsb, _stream(stream)),
-           "qat_linear_bwd")
+    _check(lib().qat_linear_bwd(_p(W), _qref(qw), N, K, bits, _p(X), ldx, _p(dY), dY.shape[0],
+                                _p(dX_residual), _p(dX), _p(dW), int(bool(accumulate_dW)), ws, wsb,
+                                _stream(stream)), "qat_linear_bwd")
 
 
 def qat_mlp_fwd(X, Y, bits, d, H, Wfc=None, Wproj=None, qfc=None, qproj=None, residual=None,
@@ -273,12 +274,13 @@ def qat_mlp_fwd(X, Y, bits, d, H, Wfc=None, Wproj=None, qfc=None, qproj=None, re
 
 def qat_mlp_bwd(X, pre, h, dY, bits, d, H, Wfc=None, Wproj=None, qfc=None, qproj=None, dX=None,
                 dWfc=None, dWproj=None, accumulate_dW=False, workspace=None, stream=None,
-                act="relu2"):
+                act="relu2", dX_residual=None):
     ws, wsb = _ws(workspace)
     _check(lib().qat_mlp_bwd(_p(Wfc), _p(Wproj), _qref(qfc), _qref(qproj), d, H, bits,
                              _ACTS[act], _p(X),
-                             _p(pre), _p(h), _p(dY), X.shape[0], _p(dX), _p(dWfc), _p(dWproj),
-                             int(bool(accumulate_dW)), ws, wsb, _stream(stream)), "qat_mlp_bwd")
+                             _p(pre), _p(h), _p(dY), X.shape[0], _p(dX_residual), _p(dX),
+                             _p(dWfc), _p(dWproj), int(bool(accumulate_dW)), ws, wsb,
+                             _stream(stream)), "qat_mlp_bwd")
 
 
 def quantize_rows_export(W, bits, codes, scales, stream=None):

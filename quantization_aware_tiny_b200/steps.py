@@ -70,8 +70,109 @@ class RecurrentCore:
                             h_save=h, stream=stream, act=self.act)
         return x
 
+    # ------------------------------------------------------------- training
+
+    def _ops_for_noise(self, noise, R, stream):
+        """Noisy QAT operands of every application (kept for the backward):
+        application r draws weight k at Philox offset offset + 4*r + k."""
+        seed, offset = noise
+        apps = []
+        for r in range(R):
+            ops = tuple(qat.QWeight(torch.empty_like(q.operand), None, None, 0)
+                        for q in (self.q_qkv, self.q_o, self.q_fc, self.q_proj))
+            for k, (w, q) in enumerate(zip(self.W, ops)):
+                qat.qat_noisy_operand(w, seed, offset + 4 * r + k, q.operand, stream=stream,
+                                      bits=self.bits)
+            apps.append(ops)
+        return apps
+
+    def forward_train(self, x, R, stream=None, noise=None):
+        """The forward of forward() for training: x [T,d] bf16 is left as it is
+        and every application's activations are kept for backward() -- its
+        input state, qkv, x1, pre, h and output state.  Returns the output
+        state of the last application (a buffer the core owns)."""
+        T, dev, bf = x.shape[0], x.device, torch.bfloat16
+        e = lambda n: torch.empty((T, n), dtype=bf, device=dev)
+        apps = self._ops_for_noise(noise, R, stream) if noise is not None else \
+            [(self.q_qkv, self.q_o, self.q_fc, self.q_proj)] * R
+        saved = []
+        xin = x
+        for r in range(R):
+            s = {"x": xin, "qkv": e(self.nqkv), "x1": e(self.d), "pre": e(self.H),
+                 "h": e(self.H), "out": e(self.d), "ops": apps[r]}
+            q_qkv, q_o, q_fc, q_proj = apps[r]
+            qat.qat_linear_fwd(xin, s["qkv"], self.bits, qw=q_qkv, stream=stream)
+            qat.qat_linear_fwd(s["qkv"], s["x1"], self.bits, qw=q_o, ldx=self.nqkv, T=T,
+                               residual=xin, stream=stream)
+            qat.qat_mlp_fwd(s["x1"], s["out"], self.bits, self.d, self.H, qfc=q_fc, qproj=q_proj,
+                            residual=s["x1"], pre_save=s["pre"], h_save=s["h"], stream=stream,
+                            act=self.act)
+            saved.append(s)
+            xin = s["out"]
+        self._saved = saved
+        return xin
+
+    def _grad_buffers(self, T, device):
+        if getattr(self, "_gbuf", None) is None or self._gbuf["dx1"].shape[0] != T:
+            bf, f32 = torch.bfloat16, torch.float32
+            e = lambda *sh, dt=bf: torch.empty(sh, dtype=dt, device=device)
+            self._gbuf = {"dx1": e(T, self.d), "dq": e(T, self.d), "g": (e(T, self.d), e(T, self.d)),
+                          "ws": e(qat.workspace_size(qat.QAT_OP_MLP_BWD, self.d, self.H, T, False),
+                                  dt=torch.uint8)}
+            self.dWqkv = e(self.nqkv, self.d, dt=f32)
+            self.dWo = e(self.d, self.d, dt=f32)
+            self.dWfc = e(self.H, self.d, dt=f32)
+            self.dWproj = e(self.d, self.H, dt=f32)
+        return self._gbuf
+
+    def backward_application(self, s, g, dx, accumulate, stream=None):
+        """STE backward of one application from its saved activations s (x,
+        qkv, x1, pre, h and its operands) and g = dL/d out; writes dL/dx into
+        dx and adds (accumulate) or writes the application's weight gradients
+        into dWqkv, dWo, dWfc, dWproj:
+            dx1 = g + dpre Wfc      (qat_mlp_bwd, residual fused; dWfc, dWproj)
+            dq  = dx1 Wo            (qat_linear_bwd on the query slice of qkv; dWo)
+            dx  = dx1 + dq Wq       (qat_linear_bwd, residual fused; dWq)
+        K and V do not reach the output with attention left out: their rows of
+        dWqkv are zeroed when not accumulating and otherwise left as they are."""
+        T = g.shape[0]
+        gb = self._grad_buffers(T, g.device)
+        q_qkv, q_o, q_fc, q_proj = s["ops"]
+        d = self.d
+        qat.qat_mlp_bwd(s["x1"], s["pre"], s["h"], g, self.bits, d, self.H, qfc=q_fc,
+                        qproj=q_proj, dX=gb["dx1"], dX_residual=g, dWfc=self.dWfc,
+                        dWproj=self.dWproj, accumulate_dW=accumulate, workspace=gb["ws"],
+                        stream=stream, act=self.act)
+        qat.qat_linear_bwd(s["qkv"], gb["dx1"], self.bits, qw=q_o, dX=gb["dq"], dW=self.dWo,
+                           accumulate_dW=accumulate, ldx=self.nqkv, stream=stream)
+        q_q = qat.QWeight(q_qkv.operand[:d], None, None, self.bits)
+        qat.qat_linear_bwd(s["x"], gb["dq"], self.bits, qw=q_q, dX=dx, dX_residual=gb["dx1"],
+                           dW=self.dWqkv[:d], accumulate_dW=accumulate, stream=stream)
+        if not accumulate:  # T = 0 call: zeroes the k|v rows of dWqkv
+            qat.qat_linear_bwd(None, gb["dq"][:0], self.bits, dW=self.dWqkv[d:],
+                               N=self.nqkv - d, K=d, stream=stream)
+
+    def backward(self, dY, stream=None, accumulate=False):
+        """Backward through the applications of the last forward_train, in
+        reverse (P1 "税 1": the shared weights' gradients are summed over the R
+        uses).  dY = dL/d(output state) [T,d] bf16.  Returns dL/dx (a buffer
+        the core owns); weight gradients in dWqkv, dWo, dWfc, dWproj (fp32,
+        overwritten, or added to with accumulate=True)."""
+        gb = self._grad_buffers(dY.shape[0], dY.device)
+        g = dY
+        for i, r in enumerate(reversed(range(len(self._saved)))):
+            dx = gb["g"][i % 2]
+            self.backward_application(self._saved[r], g, dx, accumulate or i > 0, stream)
+            g = dx
+        return g
+
     def flops(self, T, R):
         return 2.0 * T * self.d * (self.nqkv + self.d + 2 * self.H) * R
+
+    def flops_bwd(self, T, R):
+        """Contractions of backward(): per application the MLP's four GEMMs
+        (2*T*d*H each) and the O and Q projections' two each (2*T*d*d)."""
+        return (8.0 * T * self.d * self.H + 8.0 * T * self.d * self.d) * R
 
 
 class HeadMlpStep:

@@ -101,6 +101,33 @@ def test_linear_bwd_and_dw_accumulation(shape):
     assert qat.device_error() == 0
 
 
+@pytest.mark.parametrize("shape", [(333, 136, 200), (1000, 640, 640), (4096, 640, 640)])
+@pytest.mark.parametrize("alias", [False, True])
+def test_linear_bwd_strided_input_and_dx_residual(shape, alias):
+    """The backward given X as a column slice of a wider activation (row
+    stride ldx) and a dX residual, added before the bf16 rounding -- also
+    when the residual is dX itself (in place)."""
+    T, N, K = shape
+    rng = np.random.default_rng(T + N + K)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    wide = torch.from_numpy(rng.standard_normal((T, 2 * K + 8)).astype(np.float32)).to(torch.bfloat16)
+    X = wide[:, 8:8 + K]
+    dY = torch.from_numpy((rng.standard_normal((T, N)) * 0.01).astype(np.float32)).to(torch.bfloat16)
+    Rs = torch.from_numpy((rng.standard_normal((T, K)) * 0.01).astype(np.float32)).to(torch.bfloat16)
+    q = qat.quantize_weight(torch.from_numpy(W).cuda(), 6)
+    wd = wide.cuda()
+    Rd = Rs.cuda()
+    dX = Rd if alias else torch.empty((T, K), dtype=torch.bfloat16, device="cuda")
+    dW = torch.empty((N, K), dtype=torch.float32, device="cuda")
+    qat.qat_linear_bwd(wd[:, 8:], dY.cuda(), 6, qw=q, dX=dX, dW=dW, ldx=2 * K + 8, dX_residual=Rd)
+    torch.cuda.synchronize()
+    op = o.quantize_weight(W, 6)["operand"]
+    rdX, rdW = o.linear_bwd(op, _x(X), _x(dY))
+    assert_close(dX, rdX + _x(Rs), "dX + residual")
+    assert_close(dW, rdW, "dW from the strided X")
+    assert qat.device_error() == 0
+
+
 def test_zero_tokens_is_a_noop():
     q = qat.quantize_weight(torch.zeros((64, 64), device="cuda"), 6)
     X = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")

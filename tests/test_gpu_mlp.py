@@ -80,3 +80,30 @@ def test_mlp_leaky2_full_size():
     c = sy.mlp_case(T=8192, seed=8)
     _check(c, _run(c, 512, 1536, bits=5, act="leaky2"), bits=5, act="leaky2")
     assert qat.device_error() == 0
+
+
+@pytest.mark.parametrize("alias", [False, True])
+def test_mlp_bwd_dx_residual(alias):
+    """dX = dpre . Wfc_q + residual (the gradient around a residual MLP), the
+    residual added before the bf16 rounding, also in place in dX."""
+    d, H, T = 640, 1920, 700
+    c = sy.mlp_case(d=d, H=H, T=T, seed=9)
+    Rs = sy.act_bf16(np.random.default_rng(9), T, d, std=0.01)
+    qf = qat.quantize_weight(torch.from_numpy(c["Wfc"]).cuda(), 6)
+    qp = qat.quantize_weight(torch.from_numpy(c["Wproj"]).cuda(), 6)
+    bf = torch.bfloat16
+    X, dY = c["X"].cuda(), c["dY"].cuda()
+    Y, pre, h = (torch.empty((T, n), dtype=bf, device="cuda") for n in (d, H, H))
+    Rd = Rs.cuda()
+    dX = Rd if alias else torch.empty((T, d), dtype=bf, device="cuda")
+    ws = torch.empty(qat.workspace_size(qat.QAT_OP_MLP_BWD, d, H, T, False), dtype=torch.uint8,
+                     device="cuda")
+    qat.qat_mlp_fwd(X, Y, 6, d, H, qfc=qf, qproj=qp, pre_save=pre, h_save=h)
+    qat.qat_mlp_bwd(X, pre, h, dY, 6, d, H, qfc=qf, qproj=qp, dX=dX, dX_residual=Rd, workspace=ws)
+    torch.cuda.synchronize()
+    rf, rp = o.quantize_weight(c["Wfc"], 6), o.quantize_weight(c["Wproj"], 6)
+    Xn = c["X"].float().numpy()
+    p_, h_, _ = o.mlp_fwd(rf["operand"], rp["operand"], Xn)
+    rdX = o.mlp_bwd(rf["operand"], rp["operand"], Xn, p_, h_, c["dY"].float().numpy())[0]
+    assert_close(dX, rdX + Rs.float().numpy(), "dX + residual")
+    assert qat.device_error() == 0

@@ -9,7 +9,8 @@ import torch
 import oracle as o
 from quantization_aware_tiny_b200 import qat, steps
 from quantization_aware_tiny_b200 import synthetic as sy
-from parity import assert_close, assert_close_chain, bits16
+from parity import (assert_close, assert_close_chain, bits16, chain_allowance, core_sums,
+                    rounding_noise_allowance)
 
 pytestmark = pytest.mark.gpu
 
@@ -50,16 +51,37 @@ def test_noisy_linear_fwd_bwd():
     assert_close(dW, rdW, "dW")
 
 
+def _noisy_core(c, bits=6, act="relu2"):
+    dev = {k: torch.from_numpy(c[k]).cuda() for k in ("Wq", "Wk", "Wv", "Wo", "Wfc", "Wproj")}
+    core = steps.RecurrentCore(dev["Wq"], dev["Wk"], dev["Wv"], dev["Wo"], dev["Wfc"], dev["Wproj"],
+                               bits=bits, act=act)
+    Ws = [np.concatenate([c["Wq"], c["Wk"], c["Wv"]]), c["Wo"], c["Wfc"], c["Wproj"]]
+    return core, Ws
+
+
 def test_noisy_recurrent_core():
     c = sy.recurrent_core_case(T=300)
-    dev = {k: torch.from_numpy(c[k]).cuda() for k in ("Wq", "Wk", "Wv", "Wo", "Wfc", "Wproj")}
-    core = steps.RecurrentCore(dev["Wq"], dev["Wk"], dev["Wv"], dev["Wo"], dev["Wfc"], dev["Wproj"])
+    core, Ws = _noisy_core(c)
     x = c["X"].cuda()
     core.forward(x, 3, noise=(2024, 100))
     torch.cuda.synchronize()
-    Ws = [np.concatenate([c["Wq"], c["Wk"], c["Wv"]]), c["Wo"], c["Wfc"], c["Wproj"]]
-    ref = o.recurrent_core_fwd_noisy(Ws, c["X"].float().numpy(), 3, 640, 2024, 100)
-    assert_close_chain(x, ref, 6, "noisy core, 3 applications")
+    ref, saved = o.core_fwd_apps(o.noisy_core_ops(Ws, 3, 2024, 100), c["X"].float().numpy(), 640)
+    assert_close_chain(x, ref, chain_allowance(core_sums(saved)), "noisy core, 3 applications")
+    assert qat.device_error() == 0
+
+
+def test_noisy_recurrent_core_per_application():
+    """Each Noisy-QAT application from the oracle's state before it, at the
+    single-op tolerance: application r draws at offsets offset + 4*r + k."""
+    c = sy.recurrent_core_case(T=300, seed=6)
+    core, Ws = _noisy_core(c)
+    apps = o.noisy_core_ops(Ws, 3, 31, 8)
+    _, saved = o.core_fwd_apps(apps, c["X"].float().numpy(), 640)
+    for r, s in enumerate(saved):
+        x = torch.from_numpy(s["x"].astype(np.float32)).to(torch.bfloat16).cuda()
+        out = core.forward_train(x, 1, noise=(31, 8 + 4 * r))
+        torch.cuda.synchronize()
+        assert_close(out, s["out"], "noisy application %d" % r)
     assert qat.device_error() == 0
 
 
@@ -67,14 +89,35 @@ def test_noisy_recurrent_core_int5_leaky2():
     """An all-int5 core (noise at the int5 step, as the write-up proposes for an
     int5 export) with the LeakyReLU(0.5)^2 MLP."""
     c = sy.recurrent_core_case(T=300, seed=3)
-    dev = {k: torch.from_numpy(c[k]).cuda() for k in ("Wq", "Wk", "Wv", "Wo", "Wfc", "Wproj")}
-    core = steps.RecurrentCore(dev["Wq"], dev["Wk"], dev["Wv"], dev["Wo"], dev["Wfc"], dev["Wproj"],
-                               bits=5, act="leaky2")
+    core, Ws = _noisy_core(c, bits=5, act="leaky2")
     x = c["X"].cuda()
     core.forward(x, 2, noise=(77, 4))
     torch.cuda.synchronize()
-    Ws = [np.concatenate([c["Wq"], c["Wk"], c["Wv"]]), c["Wo"], c["Wfc"], c["Wproj"]]
-    ref = o.recurrent_core_fwd_noisy(Ws, c["X"].float().numpy(), 2, 640, 77, 4, bits=5,
-                                     act="leaky2")
-    assert_close_chain(x, ref, 6, "noisy int5 leaky core, 2 applications")
+    ref, saved = o.core_fwd_apps(o.noisy_core_ops(Ws, 2, 77, 4, bits=5), c["X"].float().numpy(),
+                                 640, act="leaky2")
+    assert_close_chain(x, ref, chain_allowance(core_sums(saved)),
+                       "noisy int5 leaky core, 2 applications")
+    assert qat.device_error() == 0
+
+
+def test_noisy_recurrent_core_bwd():
+    """Noisy-QAT core forward and backward through R = 3 applications: the
+    backward of application r uses that application's noisy operands (the
+    noise carries no gradient)."""
+    T = 300
+    c = sy.recurrent_core_case(T=T, seed=4)
+    core, Ws = _noisy_core(c)
+    dY = sy.act_bf16(np.random.default_rng(14), T, 640, std=sy.DY_STD)
+    out = core.forward_train(c["X"].cuda(), 3, noise=(5, 40))
+    dX = core.backward(dY.cuda())
+    torch.cuda.synchronize()
+    ref = o.recurrent_core_bwd_noisy(Ws, c["X"].float().numpy(), dY.float().numpy(), 3, 640, 5, 40)
+    ops = o.noisy_core_ops(Ws, 3, 5, 40)
+    _, sx = o.core_fwd_apps(ops, c["X"].float().numpy(), 640, exact=True)
+    ex = o.core_bwd_apps(ops, sx, dY.float().numpy(), 640, exact=True)[1]
+    assert_close_chain(out, ref["out"], chain_allowance(core_sums(ref["saved"])), "noisy core: out")
+    assert_close(dX, ref["dX"], "noisy core: dX")
+    for k in ("qkv", "o", "fc", "proj"):
+        assert_close_chain(getattr(core, "dW" + k), ref["dW" + k],
+                           rounding_noise_allowance(ref["dW" + k], ex[k]), "noisy core: dW" + k)
     assert qat.device_error() == 0

@@ -10,7 +10,8 @@ import oracle as o
 from quantization_aware_tiny_b200 import qat
 from quantization_aware_tiny_b200 import steps
 from quantization_aware_tiny_b200 import synthetic as sy
-from parity import assert_close, assert_close_chain, to_np
+from parity import (assert_close, assert_close_chain, chain_allowance, core_sums,
+                    rounding_noise_allowance, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -28,6 +29,10 @@ def _core_oracle(c, bits=6):
     return q
 
 
+def _core_ops(q):
+    return (q["qkv"], q["o"], q["fc"], q["proj"])
+
+
 def test_recurrent_core_small():
     c = sy.recurrent_core_case(T=300)
     core = _core(c)
@@ -37,8 +42,30 @@ def test_recurrent_core_small():
     torch.cuda.synchronize()
     assert qat.launch_count() - n0 == 3 * 4  # no re-quantization inside the loop
     q = _core_oracle(c)
-    ref = o.recurrent_core_fwd(q["qkv"], q["o"], q["fc"], q["proj"], c["X"].float().numpy(), 3, 640)
-    assert_close_chain(x, ref, 6, "x after 3 applications")
+    ref, saved = o.core_fwd_apps([_core_ops(q)] * 3, c["X"].float().numpy(), 640)
+    assert_close_chain(x, ref, chain_allowance(core_sums(saved)), "x after 3 applications")
+
+
+@pytest.mark.parametrize("bits,act", [(6, "relu2"), (5, "leaky2")])
+def test_recurrent_core_per_application(bits, act):
+    """Each application on its own, from the oracle's bf16 state before it:
+    the output state and the kept activations (qkv, x1, pre, h) at the
+    single-op tolerance, with no allowance for a chain."""
+    c = sy.recurrent_core_case(T=300, seed=2)
+    core = _core(c, bits, act)
+    q = _core_oracle(c, bits)
+    _, saved = o.core_fwd_apps([_core_ops(q)] * 3, c["X"].float().numpy(), 640, act)
+    for r, s in enumerate(saved):
+        x = torch.from_numpy(s["x"].astype(np.float32)).to(torch.bfloat16).cuda()
+        out = core.forward_train(x, 1)
+        torch.cuda.synchronize()
+        assert_close(out, s["out"], "application %d: out" % r)
+        for k in ("qkv", "x1", "pre", "h"):
+            assert_close(core._saved[0][k], s[k], "application %d: %s" % (r, k))
+        x1 = x.clone()
+        core.forward(x1, 1)  # the inference forward, in place
+        assert_close(x1, s["out"], "application %d: in-place forward" % r)
+    assert qat.device_error() == 0
 
 
 @pytest.mark.parametrize("bits,act", [(5, "relu2"), (5, "leaky2"), (6, "leaky2")])
@@ -50,9 +77,8 @@ def test_recurrent_core_int5_and_leaky2(bits, act):
     core.forward(x, 3)
     torch.cuda.synchronize()
     q = _core_oracle(c, bits)
-    ref = o.recurrent_core_fwd(q["qkv"], q["o"], q["fc"], q["proj"], c["X"].float().numpy(), 3, 640,
-                               act)
-    assert_close_chain(x, ref, 6, "x after 3 applications")
+    ref, saved = o.core_fwd_apps([_core_ops(q)] * 3, c["X"].float().numpy(), 640, act)
+    assert_close_chain(x, ref, chain_allowance(core_sums(saved)), "x after 3 applications")
 
 
 def test_recurrent_cache_matches_fresh_quantization():
@@ -77,8 +103,141 @@ def test_recurrent_core_full_size_sampled_rows():
     rows = np.random.default_rng(0).choice(16384, 64, replace=False)
     rows = np.concatenate([rows, [0, 16383]])
     q = _core_oracle(c)
-    ref = o.recurrent_core_fwd(q["qkv"], q["o"], q["fc"], q["proj"], c["X"].float().numpy()[rows], 3, 640)
-    assert_close_chain(to_np(x)[rows], ref, 6, "sampled rows")
+    ref, saved = o.core_fwd_apps([_core_ops(q)] * 3, c["X"].float().numpy()[rows], 640)
+    assert_close_chain(to_np(x)[rows], ref, chain_allowance(core_sums(saved)), "sampled rows")
+    assert qat.device_error() == 0
+
+
+# ------------------------------------------------- recurrent core backward
+
+def _core_bwd_check(core, ref, exact, x_out, dX, what, rows=None):
+    """The chained forward + backward: the output state within the chain
+    allowance, dX at the single-op tolerance, the summed weight gradients
+    within the chain's bf16 rounding noise (measured by the oracle as its
+    rounded run against its exact run); relative Frobenius <= 5e-3 for all."""
+    sel = (lambda a: a) if rows is None else (lambda a: np.asarray(a)[rows])
+    assert_close_chain(sel(to_np(x_out)), sel(ref["out"]),
+                       chain_allowance([sel(u) for u in core_sums(ref["saved"])]), what + ": out")
+    assert_close(sel(to_np(dX)), sel(ref["dX"]), what + ": dX")
+    for k in ("dWqkv", "dWo", "dWfc", "dWproj"):
+        assert_close_chain(getattr(core, k), ref[k], rounding_noise_allowance(ref[k], exact[k]),
+                           what + ": " + k)
+    d = core.d
+    assert torch.count_nonzero(core.dWqkv[d:]).item() == 0  # k, v: no gradient
+
+
+@pytest.mark.parametrize("bits,act", [(6, "relu2"), (5, "leaky2")])
+def test_recurrent_core_bwd_small(bits, act):
+    """Forward (activations kept) and backward through R = 3 applications in
+    reverse, the shared weights' gradients summed over the three uses."""
+    T = 300
+    c = sy.recurrent_core_case(T=T, seed=1)
+    dY = sy.act_bf16(np.random.default_rng(11), T, 640, std=sy.DY_STD)
+    core = _core(c, bits, act)
+    x = c["X"].cuda()
+    n0 = qat.launch_count()
+    out = core.forward_train(x, 3)
+    dX = core.backward(dY.cuda())
+    torch.cuda.synchronize()
+    # 4 GEMMs per application forward; 8 per application backward (the MLP's
+    # four, two each for O and Q)
+    assert qat.launch_count() - n0 == 3 * 4 + 3 * 8
+    assert torch.equal(x, c["X"].cuda())  # the input state is left as it is
+    q = _core_oracle(c, bits)
+    args = (*_core_ops(q), c["X"].float().numpy(), dY.float().numpy(), 3, 640, act)
+    ref = o.recurrent_core_bwd(*args)
+    exact = o.recurrent_core_bwd(*args, exact=True)
+    _core_bwd_check(core, ref, exact, out, dX, "R=3")
+    assert qat.device_error() == 0
+
+
+def test_recurrent_core_bwd_per_application():
+    """Each application's backward on its own, from the oracle's saved bf16
+    activations and incoming gradient: dx and the application's weight
+    gradients at the single-op tolerance."""
+    T = 300
+    c = sy.recurrent_core_case(T=T, seed=3)
+    dY = sy.act_bf16(np.random.default_rng(12), T, 640, std=sy.DY_STD)
+    core = _core(c)
+    q = _core_oracle(c)
+    ops = _core_ops(q)
+    ref = o.recurrent_core_bwd(*ops, c["X"].float().numpy(), dY.float().numpy(), 3, 640)
+    bf = lambda a: torch.from_numpy(np.asarray(a, np.float32)).to(torch.bfloat16).cuda()
+    dx = torch.empty((T, 640), dtype=torch.bfloat16, device="cuda")
+    for r, s in enumerate(ref["saved"]):
+        sd = {k: bf(s[k]) for k in ("x", "qkv", "x1", "pre", "h")}
+        sd["ops"] = (core.q_qkv, core.q_o, core.q_fc, core.q_proj)
+        core.backward_application(sd, bf(ref["grads"][r]), dx, accumulate=False)
+        torch.cuda.synchronize()
+        gx, dW, _ = o.core_application_bwd(ops, s, ref["grads"][r], 640)
+        assert_close(dx, gx, "application %d: dx" % r)
+        for k, name in (("qkv", "dWqkv"), ("o", "dWo"), ("fc", "dWfc"), ("proj", "dWproj")):
+            assert_close(getattr(core, name), dW[k], "application %d: %s" % (r, name))
+    # accumulate over the three applications into the same gradients
+    for r, s in enumerate(ref["saved"]):
+        sd = {k: bf(s[k]) for k in ("x", "qkv", "x1", "pre", "h")}
+        sd["ops"] = (core.q_qkv, core.q_o, core.q_fc, core.q_proj)
+        core.backward_application(sd, bf(ref["grads"][r]), dx, accumulate=r > 0)
+    torch.cuda.synchronize()
+    for k in ("dWqkv", "dWo", "dWfc", "dWproj"):
+        assert_close(getattr(core, k), ref[k], "summed over applications: " + k)
+    assert qat.device_error() == 0
+
+
+@pytest.fixture(scope="module")
+def full_core():
+    """The 3x3 core at d=640, 16x1024 tokens, R=3, forward (activations kept)
+    and backward as the benchmark launches them, and the oracle's rounded
+    run of the same."""
+    T = 16384
+    c = sy.recurrent_core_case(T=T)
+    dY = sy.act_bf16(np.random.default_rng(13), T, 640, std=sy.DY_STD)
+    core = _core(c)
+    out = core.forward_train(c["X"].cuda(), 3)
+    dX = core.backward(dY.cuda())
+    torch.cuda.synchronize()
+    q = _core_oracle(c)
+    args = (*_core_ops(q), c["X"].float().numpy(), dY.float().numpy(), 3, 640)
+    ref = o.recurrent_core_bwd(*args)
+    return c, core, q, args, ref, out, dX
+
+
+def test_recurrent_core_bwd_full_size_chained(full_core):
+    """Chained at full size: the output state and dX on sampled rows (rows
+    are independent without attention), every entry of the four summed
+    weight gradients within the chain's rounding noise."""
+    c, core, q, args, ref, out, dX = full_core
+    exact = o.recurrent_core_bwd(*args, exact=True)
+    rows = np.concatenate([np.random.default_rng(4).choice(16384, 64, replace=False), [0, 16383]])
+    _core_bwd_check(core, ref, exact, out, dX, "R=3 full size", rows=rows)
+    assert qat.device_error() == 0
+
+
+def test_recurrent_core_per_application_full_size(full_core):
+    """Each application at full size on its own, from the oracle's bf16
+    inputs, at the single-op tolerance: the forward's output state on sampled
+    rows, the backward's dx on sampled rows and every entry of that
+    application's four weight gradients."""
+    c, core, q, args, ref, out, dX = full_core
+    ops = _core_ops(q)
+    T = 16384
+    rows = np.concatenate([np.random.default_rng(5).choice(T, 64, replace=False), [0, T - 1]])
+    bf = lambda a: torch.from_numpy(np.asarray(a, np.float32)).to(torch.bfloat16).cuda()
+    dx = torch.empty((T, 640), dtype=torch.bfloat16, device="cuda")
+    for r, s in enumerate(ref["saved"]):
+        x = bf(s["x"])
+        y = core.forward_train(x, 1)
+        torch.cuda.synchronize()
+        assert_close(to_np(y)[rows], s["out"][rows], "application %d: out" % r)
+        sd = {k: bf(s[k]) for k in ("x", "qkv", "x1", "pre", "h")}
+        sd["ops"] = (core.q_qkv, core.q_o, core.q_fc, core.q_proj)
+        core.backward_application(sd, bf(ref["grads"][r]), dx, accumulate=False)
+        torch.cuda.synchronize()
+        gx, dW, _ = o.core_application_bwd(ops, s, ref["grads"][r], 640)
+        assert_close(to_np(dx)[rows], gx[rows], "application %d: dx" % r)
+        for k, name in (("qkv", "dWqkv"), ("o", "dWo"), ("fc", "dWfc"), ("proj", "dWproj")):
+            assert_close(getattr(core, name), dW[k], "application %d: %s" % (r, name))
+        del sd
     assert qat.device_error() == 0
 
 
