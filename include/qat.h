@@ -196,13 +196,15 @@ int qat_mlp_fwd(const float* Wfc, const float* Wproj, const qat_qweight* qfc,
  *   dX = bf16( dpre . Wfc_q (+ dX_residual) ).
  * dX, dWfc, dWproj may each be NULL.  dX_residual (nullable, [T,d] bf16,
  * needs dX; may alias dX exactly) adds the gradient that bypasses the MLP
- * through a residual connection.  The workspace holds dpre [T,H] bf16. */
+ * through a residual connection.  dpre_save (nullable, [T,H] bf16) receives
+ * dpre -- e.g. to form dWfc later over several token batches in one call --
+ * else the workspace holds it (qat_workspace_size counts it either way). */
 int qat_mlp_bwd(const float* Wfc, const float* Wproj, const qat_qweight* qfc,
                 const qat_qweight* qproj, int32_t d, int32_t H, int32_t bits, int32_t act,
                 const qat_bf16* X, const qat_bf16* pre, const qat_bf16* h, const qat_bf16* dY,
-                int64_t T, const qat_bf16* dX_residual, qat_bf16* dX, float* dWfc,
-                float* dWproj, int32_t accumulate_dW, void* workspace, size_t ws_bytes,
-                qat_stream_t stream);
+                int64_t T, const qat_bf16* dX_residual, qat_bf16* dX, qat_bf16* dpre_save,
+                float* dWfc, float* dWproj, int32_t accumulate_dW, void* workspace,
+                size_t ws_bytes, qat_stream_t stream);
 
 /* Diagnostic (the pages have no counterpart): runs the library's bounded
  * device wait on a barrier that nothing arrives on, with a limit of limit_ns

@@ -314,8 +314,9 @@ int qat_mlp_fwd(const float* Wfc, const float* Wproj, const qat_qweight* qfc,
 int qat_mlp_bwd(const float* Wfc, const float* Wproj, const qat_qweight* qfc,
                 const qat_qweight* qproj, int32_t d, int32_t H, int32_t bits, int32_t act,
                 const qat_bf16* X, const qat_bf16* pre, const qat_bf16* h, const qat_bf16* dY,
-                int64_t T, const qat_bf16* dX_residual, qat_bf16* dX, float* dWfc, float* dWproj,
-                int32_t accumulate_dW, void* workspace, size_t ws_bytes, qat_stream_t stream) {
+                int64_t T, const qat_bf16* dX_residual, qat_bf16* dX, qat_bf16* dpre_save,
+                float* dWfc, float* dWproj, int32_t accumulate_dW, void* workspace,
+                size_t ws_bytes, qat_stream_t stream) {
   if ((T > 0 && (!X || !pre || !h || !dY)) || T < 0 || !bits_ok(bits) || !act_ok(act))
     return QAT_ERR_ARG;
   if (dX_residual && !dX) return QAT_ERR_ARG;
@@ -335,7 +336,8 @@ int qat_mlp_bwd(const float* Wfc, const float* Wproj, const qat_qweight* qfc,
     }
     return QAT_OK;
   }
-  void* dpre = ws.take(static_cast<size_t>(T) * H * 2);
+  if (dpre_save && !aligned16(dpre_save)) return QAT_ERR_ALIGN;
+  void* dpre = dpre_save ? static_cast<void*>(dpre_save) : ws.take(static_cast<size_t>(T) * H * 2);
   if (!dpre) return QAT_ERR_WORKSPACE;
   if (dWproj) {  // dWproj[d,H] = dY^T . h
     GemmDesc g;

@@ -848,12 +848,18 @@ int launch_gemm(const GemmDesc& g, cudaStream_t stream) {
     return QAT_ERR_SHAPE;
   if (g.M > (1ll << 31) - 256 || g.N > (1 << 30) || g.K > (1ll << 31) - 256) return QAT_ERR_SHAPE;
 
-  // N tile.  Forward GEMMs (K-major B) with at least 256 rows run on CTA pairs
-  // 256 columns wide; the other GEMMs take 256 (paired when M >= 256) unless
-  // 128 wastes fewer columns.
+  // N tile.  GEMMs with at least 256 rows run on CTA pairs 256 columns wide,
+  // the last N block partial where 256 does not divide N: the forward and dX
+  // GEMMs (bf16 output) when N >= 160, and the weight-gradient GEMMs (both
+  // operands MN-major).  The rest take 256 (paired when M >= 256) unless 128
+  // wastes fewer columns.  (For the d = 640 core's backward, 256-wide pairs
+  // against 128-wide single-CTA tiles: dX GEMMs 57 -> 44 us (N = 640,
+  // K = 1920) and 58 -> 50 us (N = 1920, K = 640), weight gradients 33 -> 25 us
+  // (640 x 640) and 70 -> 64 us (1920 x 640), per 16,384 tokens.)
   int BN;
   bool pair;
-  const bool kmajor_fwd = !g.a_mn && !g.b_mn && g.epi != EPI_F32 && g.epi != EPI_F32_ATOMIC;
+  const bool kmajor_fwd = (!g.a_mn && g.epi != EPI_F32 && g.epi != EPI_F32_ATOMIC) ||
+                          (g.a_mn && g.M >= 256);
   if (g.Wraw) {
     pair = true;
     BN = fused_b_bn(g.N, g.K);

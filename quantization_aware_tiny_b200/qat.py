@@ -95,8 +95,8 @@ def lib():
         L.qat_linear_fwd.argtypes = [P, P, I32, I32, I32, P, I64, I64, P, P, P, SZ, P]
         L.qat_linear_bwd.argtypes = [P, P, I32, I32, I32, P, I64, P, I64, P, P, P, I32, P, SZ, P]
         L.qat_mlp_fwd.argtypes = [P, P, P, P, I32, I32, I32, I32, P, I64, P, P, P, P, P, SZ, P]
-        L.qat_mlp_bwd.argtypes = [P, P, P, P, I32, I32, I32, I32, P, P, P, P, I64, P, P, P, P, I32,
-                                  P, SZ, P]
+        L.qat_mlp_bwd.argtypes = [P, P, P, P, I32, I32, I32, I32, P, P, P, P, I64, P, P, P, P, P,
+                                  I32, P, SZ, P]
         L.quantize_rows_export.argtypes = [P, I64, I64, I32, P, P, P]
         L.quantize_export_batch.argtypes = [P, I32, P]
         L.dequantize_rows.argtypes = [P, P, I64, I64, I32, P, P]
@@ -274,13 +274,13 @@ def qat_mlp_fwd(X, Y, bits, d, H, Wfc=None, Wproj=None, qfc=None, qproj=None, re
 
 def qat_mlp_bwd(X, pre, h, dY, bits, d, H, Wfc=None, Wproj=None, qfc=None, qproj=None, dX=None,
                 dWfc=None, dWproj=None, accumulate_dW=False, workspace=None, stream=None,
-                act="relu2", dX_residual=None):
+                act="relu2", dX_residual=None, dpre_save=None):
     ws, wsb = _ws(workspace)
     _check(lib().qat_mlp_bwd(_p(Wfc), _p(Wproj), _qref(qfc), _qref(qproj), d, H, bits,
                              _ACTS[act], _p(X),
                              _p(pre), _p(h), _p(dY), X.shape[0], _p(dX_residual), _p(dX),
-                             _p(dWfc), _p(dWproj), int(bool(accumulate_dW)), ws, wsb,
-                             _stream(stream)), "qat_mlp_bwd")
+                             _p(dpre_save), _p(dWfc), _p(dWproj), int(bool(accumulate_dW)), ws,
+                             wsb, _stream(stream)), "qat_mlp_bwd")
 
 
 def quantize_rows_export(W, bits, codes, scales, stream=None):

@@ -86,85 +86,125 @@ class RecurrentCore:
             apps.append(ops)
         return apps
 
-    def forward_train(self, x, R, stream=None, noise=None):
-        """The forward of forward() for training: x [T,d] bf16 is left as it is
-        and every application's activations are kept for backward() -- its
-        input state, qkv, x1, pre, h and output state.  Returns the output
-        state of the last application (a buffer the core owns)."""
-        T, dev, bf = x.shape[0], x.device, torch.bfloat16
-        e = lambda n: torch.empty((T, n), dtype=bf, device=dev)
-        apps = self._ops_for_noise(noise, R, stream) if noise is not None else \
-            [(self.q_qkv, self.q_o, self.q_fc, self.q_proj)] * R
-        saved = []
-        xin = x
-        for r in range(R):
-            s = {"x": xin, "qkv": e(self.nqkv), "x1": e(self.d), "pre": e(self.H),
-                 "h": e(self.H), "out": e(self.d), "ops": apps[r]}
-            q_qkv, q_o, q_fc, q_proj = apps[r]
-            qat.qat_linear_fwd(xin, s["qkv"], self.bits, qw=q_qkv, stream=stream)
-            qat.qat_linear_fwd(s["qkv"], s["x1"], self.bits, qw=q_o, ldx=self.nqkv, T=T,
-                               residual=xin, stream=stream)
-            qat.qat_mlp_fwd(s["x1"], s["out"], self.bits, self.d, self.H, qfc=q_fc, qproj=q_proj,
-                            residual=s["x1"], pre_save=s["pre"], h_save=s["h"], stream=stream,
-                            act=self.act)
-            saved.append(s)
-            xin = s["out"]
-        self._saved = saved
-        return xin
-
-    def _grad_buffers(self, T, device):
-        if getattr(self, "_gbuf", None) is None or self._gbuf["dx1"].shape[0] != T:
+    def _train_buffers(self, T, R, device):
+        """Activations and gradients of every application, stacked [R, T, .]
+        so that each weight gradient is one GEMM over all R * T token uses:
+        states [R+1, T, d] (state 0 is the input, state r+1 the output of
+        application r), qkv, x1, pre, h; the gradient's g [R, T, d] (g[r] =
+        dL/d output of application r), dx1, dq [R, T, d], dpre [R, T, H]."""
+        key = (T, R)
+        if getattr(self, "_tkey", None) != key:
             bf, f32 = torch.bfloat16, torch.float32
             e = lambda *sh, dt=bf: torch.empty(sh, dtype=dt, device=device)
-            self._gbuf = {"dx1": e(T, self.d), "dq": e(T, self.d), "g": (e(T, self.d), e(T, self.d)),
-                          "ws": e(qat.workspace_size(qat.QAT_OP_MLP_BWD, self.d, self.H, T, False),
-                                  dt=torch.uint8)}
-            self.dWqkv = e(self.nqkv, self.d, dt=f32)
-            self.dWo = e(self.d, self.d, dt=f32)
-            self.dWfc = e(self.H, self.d, dt=f32)
-            self.dWproj = e(self.d, self.H, dt=f32)
-        return self._gbuf
+            d, H = self.d, self.H
+            self._tb = {"states": e(R + 1, T, d), "qkv": e(R, T, self.nqkv), "x1": e(R, T, d),
+                        "pre": e(R, T, H), "h": e(R, T, H), "g": e(R, T, d), "dx1": e(R, T, d),
+                        "dq": e(R, T, d), "dpre": e(R, T, H), "dX": e(T, d)}
+            self.dWqkv = e(self.nqkv, d, dt=f32)
+            self.dWo = e(d, d, dt=f32)
+            self.dWfc = e(H, d, dt=f32)
+            self.dWproj = e(d, H, dt=f32)
+            self._tkey = key
+        return self._tb
 
-    def backward_application(self, s, g, dx, accumulate, stream=None):
-        """STE backward of one application from its saved activations s (x,
-        qkv, x1, pre, h and its operands) and g = dL/d out; writes dL/dx into
-        dx and adds (accumulate) or writes the application's weight gradients
-        into dWqkv, dWo, dWfc, dWproj:
-            dx1 = g + dpre Wfc      (qat_mlp_bwd, residual fused; dWfc, dWproj)
-            dq  = dx1 Wo            (qat_linear_bwd on the query slice of qkv; dWo)
-            dx  = dx1 + dq Wq       (qat_linear_bwd, residual fused; dWq)
-        K and V do not reach the output with attention left out: their rows of
-        dWqkv are zeroed when not accumulating and otherwise left as they are."""
-        T = g.shape[0]
-        gb = self._grad_buffers(T, g.device)
+    def forward_train(self, x, R, stream=None, noise=None):
+        """The forward of forward() for training: x [T,d] bf16 is left as it is
+        (copied in as state 0) and every application's activations are kept
+        for backward().  Returns the output state of the last application (a
+        buffer the core owns)."""
+        T = x.shape[0]
+        tb = self._train_buffers(T, R, x.device)
+        apps = self._ops_for_noise(noise, R, stream) if noise is not None else \
+            [(self.q_qkv, self.q_o, self.q_fc, self.q_proj)] * R
+        st = tb["states"]
+        with torch.cuda.stream(stream if stream is not None else torch.cuda.current_stream()):
+            st[0].copy_(x)
+        for r in range(R):
+            q_qkv, q_o, q_fc, q_proj = apps[r]
+            qat.qat_linear_fwd(st[r], tb["qkv"][r], self.bits, qw=q_qkv, stream=stream)
+            qat.qat_linear_fwd(tb["qkv"][r], tb["x1"][r], self.bits, qw=q_o, ldx=self.nqkv, T=T,
+                               residual=st[r], stream=stream)
+            qat.qat_mlp_fwd(tb["x1"][r], st[r + 1], self.bits, self.d, self.H, qfc=q_fc,
+                            qproj=q_proj, residual=tb["x1"][r], pre_save=tb["pre"][r],
+                            h_save=tb["h"][r], stream=stream, act=self.act)
+        self._apps, self._R = apps, R
+        return st[R]
+
+    def _saved(self, r):
+        """Application r's kept activations and operands (for backward_application)."""
+        tb = self._tb
+        return {"x": tb["states"][r], "qkv": tb["qkv"][r], "x1": tb["x1"][r], "pre": tb["pre"][r],
+                "h": tb["h"][r], "ops": self._apps[r]}
+
+    def _dx_chain(self, s, g, dx1, dq, dpre, dx, stream):
+        """The gradient's chain through one application (no weight gradients):
+            dpre = (g Wproj) * act'(pre) ; dx1 = g + dpre Wfc   (qat_mlp_bwd)
+            dq   = dx1 Wo                                       (qat_linear_bwd)
+            dx   = dx1 + dq Wq                                  (qat_linear_bwd)"""
         q_qkv, q_o, q_fc, q_proj = s["ops"]
         d = self.d
         qat.qat_mlp_bwd(s["x1"], s["pre"], s["h"], g, self.bits, d, self.H, qfc=q_fc,
-                        qproj=q_proj, dX=gb["dx1"], dX_residual=g, dWfc=self.dWfc,
-                        dWproj=self.dWproj, accumulate_dW=accumulate, workspace=gb["ws"],
-                        stream=stream, act=self.act)
-        qat.qat_linear_bwd(s["qkv"], gb["dx1"], self.bits, qw=q_o, dX=gb["dq"], dW=self.dWo,
-                           accumulate_dW=accumulate, ldx=self.nqkv, stream=stream)
+                        qproj=q_proj, dX=dx1, dX_residual=g, dpre_save=dpre, stream=stream,
+                        act=self.act)
+        qat.qat_linear_bwd(None, dx1, self.bits, qw=q_o, dX=dq, stream=stream)
         q_q = qat.QWeight(q_qkv.operand[:d], None, None, self.bits)
-        qat.qat_linear_bwd(s["x"], gb["dq"], self.bits, qw=q_q, dX=dx, dX_residual=gb["dx1"],
-                           dW=self.dWqkv[:d], accumulate_dW=accumulate, stream=stream)
+        qat.qat_linear_bwd(None, dq, self.bits, qw=q_q, dX=dx, dX_residual=dx1, stream=stream)
+
+    def _weight_grads(self, x, qkv, x1, h, g, dx1, dq, dpre, accumulate, stream):
+        """The four weight gradients from token-stacked operands (one GEMM each,
+        the reduction over every token of every application given):
+            dWproj (+)= g^T h ; dWfc (+)= dpre^T x1 ; dWo (+)= dx1^T q ;
+            dWqkv[:d] (+)= dq^T x ; dWqkv[d:] = 0 unless accumulating
+        (k and v do not reach the output with attention left out)."""
+        d, H = self.d, self.H
+        qat.qat_linear_bwd(h, g, self.bits, dW=self.dWproj, N=d, K=H,
+                           accumulate_dW=accumulate, stream=stream)
+        qat.qat_linear_bwd(x1, dpre, self.bits, dW=self.dWfc, N=H, K=d,
+                           accumulate_dW=accumulate, stream=stream)
+        qat.qat_linear_bwd(qkv, dx1, self.bits, dW=self.dWo, N=d, K=d, ldx=self.nqkv,
+                           accumulate_dW=accumulate, stream=stream)
+        qat.qat_linear_bwd(x, dq, self.bits, dW=self.dWqkv[:d], N=d, K=d,
+                           accumulate_dW=accumulate, stream=stream)
         if not accumulate:  # T = 0 call: zeroes the k|v rows of dWqkv
-            qat.qat_linear_bwd(None, gb["dq"][:0], self.bits, dW=self.dWqkv[d:],
+            qat.qat_linear_bwd(None, dq[:0], self.bits, dW=self.dWqkv[d:],
                                N=self.nqkv - d, K=d, stream=stream)
+
+    def backward_application(self, s, g, dx, accumulate, stream=None):
+        """STE backward of one application from its activations s (x, qkv, x1,
+        pre, h and its operands) and g = dL/d out: dL/dx into dx, and that
+        application's weight gradients written into (or, accumulate, added to)
+        dWqkv, dWo, dWfc, dWproj."""
+        T = g.shape[0]
+        if getattr(self, "_tkey", None) is None or self._tkey[0] != T:
+            self._train_buffers(T, 1, g.device)
+        tb = self._tb
+        dx1, dq, dpre = tb["dx1"][0], tb["dq"][0], tb["dpre"][0]
+        self._dx_chain(s, g, dx1, dq, dpre, dx, stream)
+        self._weight_grads(s["x"], s["qkv"], s["x1"], s["h"], g, dx1, dq, dpre, accumulate, stream)
 
     def backward(self, dY, stream=None, accumulate=False):
         """Backward through the applications of the last forward_train, in
-        reverse (P1 "税 1": the shared weights' gradients are summed over the R
-        uses).  dY = dL/d(output state) [T,d] bf16.  Returns dL/dx (a buffer
+        reverse, the shared weights' gradients summed over the R uses (P1
+        "税 1").  The gradient's chain runs application by application (4
+        GEMMs each, the per-application gradients kept); then each weight's
+        gradient is ONE GEMM whose reduction runs over the R * T token uses
+        (the stacked activations and gradients), instead of R accumulating
+        ones.  dY = dL/d(output state) [T,d] bf16.  Returns dL/dx (a buffer
         the core owns); weight gradients in dWqkv, dWo, dWfc, dWproj (fp32,
         overwritten, or added to with accumulate=True)."""
-        gb = self._grad_buffers(dY.shape[0], dY.device)
-        g = dY
-        for i, r in enumerate(reversed(range(len(self._saved)))):
-            dx = gb["g"][i % 2]
-            self.backward_application(self._saved[r], g, dx, accumulate or i > 0, stream)
-            g = dx
-        return g
+        R, tb = self._R, self._tb
+        T = dY.shape[0]
+        with torch.cuda.stream(stream if stream is not None else torch.cuda.current_stream()):
+            tb["g"][R - 1].copy_(dY)
+        for r in reversed(range(R)):
+            dx = tb["g"][r - 1] if r > 0 else tb["dX"]
+            self._dx_chain(self._saved(r), tb["g"][r], tb["dx1"][r], tb["dq"][r], tb["dpre"][r],
+                           dx, stream)
+        flat = lambda a: a.reshape(R * T, a.shape[-1])
+        self._weight_grads(flat(tb["states"][:R]), flat(tb["qkv"]), flat(tb["x1"]), flat(tb["h"]),
+                           flat(tb["g"]), flat(tb["dx1"]), flat(tb["dq"]), flat(tb["dpre"]),
+                           accumulate, stream)
+        return tb["dX"]
 
     def flops(self, T, R):
         return 2.0 * T * self.d * (self.nqkv + self.d + 2 * self.H) * R

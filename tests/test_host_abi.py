@@ -134,10 +134,10 @@ def test_argument_validation_before_launch(L):
         two = (D * 2)(good, bad)
         assert L.dequantize_rows_batch(ctypes.cast(two, ctypes.c_void_p), 2, None) == rc
     assert L.qat_mlp_bwd(None, None, None, None, 512, 1536, 6, 0, A16, A16, None, A16, 8, None,
-                         None, None, None, 0, None, 0, None) == qat.QAT_ERR_ARG
+                         None, None, None, None, 0, None, 0, None) == qat.QAT_ERR_ARG
     # a dX residual needs dX; the X row stride is at least K and a multiple of 8
     assert L.qat_mlp_bwd(None, None, None, None, 512, 1536, 6, 0, A16, A16, A16, A16, 8, A16,
-                         None, None, None, 0, None, 0, None) == qat.QAT_ERR_ARG
+                         None, None, None, None, 0, None, 0, None) == qat.QAT_ERR_ARG
     assert L.qat_linear_bwd(None, None, 512, 512, 6, A16, 0, A16, 8, A16, None, A16, 0, None, 0,
                             None) == qat.QAT_ERR_ARG
     assert L.qat_linear_bwd(None, None, 512, 512, 6, A16, 256, A16, 8, None, None, A16, 0, None, 0,
