@@ -107,3 +107,32 @@ def test_mlp_bwd_dx_residual(alias):
     rdX = o.mlp_bwd(rf["operand"], rp["operand"], Xn, p_, h_, c["dY"].float().numpy())[0]
     assert_close(dX, rdX + Rs.float().numpy(), "dX + residual")
     assert qat.device_error() == 0
+
+
+def test_mlp_bwd_dpre_save():
+    """dpre written to the caller's buffer (no workspace): dh * act'(pre) at the
+    single-op tolerance, and dX / dWfc / dWproj as with the workspace."""
+    d, H, T = 512, 2048, 1000
+    c = sy.mlp_case(d=d, H=H, T=T, seed=10)
+    qf = qat.quantize_weight(torch.from_numpy(c["Wfc"]).cuda(), 6)
+    qp = qat.quantize_weight(torch.from_numpy(c["Wproj"]).cuda(), 6)
+    bf = torch.bfloat16
+    X, dY = c["X"].cuda(), c["dY"].cuda()
+    Y, pre, h, dpre = (torch.empty((T, n), dtype=bf, device="cuda") for n in (d, H, H, H))
+    dX = torch.empty((T, d), dtype=bf, device="cuda")
+    dWfc = torch.empty((H, d), dtype=torch.float32, device="cuda")
+    dWproj = torch.empty((d, H), dtype=torch.float32, device="cuda")
+    qat.qat_mlp_fwd(X, Y, 6, d, H, qfc=qf, qproj=qp, pre_save=pre, h_save=h)
+    qat.qat_mlp_bwd(X, pre, h, dY, 6, d, H, qfc=qf, qproj=qp, dX=dX, dWfc=dWfc, dWproj=dWproj,
+                    dpre_save=dpre)
+    torch.cuda.synchronize()
+    rf, rp = o.quantize_weight(c["Wfc"], 6), o.quantize_weight(c["Wproj"], 6)
+    Xn, dYn = c["X"].float().numpy(), c["dY"].float().numpy()
+    p_, h_, _ = o.mlp_fwd(rf["operand"], rp["operand"], Xn)
+    rdpre = (dYn.astype(np.float64) @ rp["operand"]) * o.act_grad(p_)
+    assert_close(dpre, rdpre, "dpre")
+    rdX, rdWfc, rdWproj = o.mlp_bwd(rf["operand"], rp["operand"], Xn, p_, h_, dYn)
+    assert_close(dX, rdX, "dX")
+    assert_close(dWfc, rdWfc, "dWfc")
+    assert_close(dWproj, rdWproj, "dWproj")
+    assert qat.device_error() == 0
