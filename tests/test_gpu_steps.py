@@ -156,6 +156,67 @@ def test_recurrent_core_bwd_small(bits, act):
     assert qat.device_error() == 0
 
 
+@pytest.mark.parametrize("T,R,d,H,bits,act", [(257, 1, 640, 1920, 6, "relu2"),
+                                               (1000, 2, 512, 1536, 8, "relu2"),
+                                               (513, 3, 512, 2048, 5, "leaky2")])
+def test_recurrent_core_bwd_shapes(T, R, d, H, bits, act):
+    """Forward + backward at other shapes: ragged token counts (not multiples
+    of the 256-row tiles), R = 1 and 2, the d = 512 core (8 query / 4 KV heads
+    of dim 64) with 3x and 4x MLPs, the int8 and int5 grids, LeakyReLU(0.5)^2."""
+    c = sy.recurrent_core_case(d=d, H=H, T=T, seed=T)
+    dY = sy.act_bf16(np.random.default_rng(T), T, d, std=sy.DY_STD)
+    core = _core(c, bits, act)
+    out = core.forward_train(c["X"].cuda(), R)
+    dX = core.backward(dY.cuda())
+    torch.cuda.synchronize()
+    q = _core_oracle(c, bits)
+    args = (*_core_ops(q), c["X"].float().numpy(), dY.float().numpy(), R, d, act)
+    ref = o.recurrent_core_bwd(*args)
+    exact = o.recurrent_core_bwd(*args, exact=True)
+    _core_bwd_check(_grads(core), ref, exact, out, dX, "T=%d R=%d d=%d" % (T, R, d))
+    assert qat.device_error() == 0
+
+
+def test_recurrent_core_bwd_accumulates_across_calls():
+    """backward(accumulate=True) adds this call's summed gradients to the
+    held ones (gradient accumulation over micro-batches): two micro-batches
+    give the sum of their oracle gradients."""
+    T = 300
+    cs = [sy.recurrent_core_case(T=T, seed=s) for s in (21, 22)]
+    core = _core(cs[0])
+    dYs = [sy.act_bf16(np.random.default_rng(30 + i), T, 640, std=sy.DY_STD) for i in range(2)]
+    for i, c in enumerate(cs):
+        core.forward_train(c["X"].cuda(), 2)
+        core.backward(dYs[i].cuda(), accumulate=i > 0)
+    torch.cuda.synchronize()
+    q = _core_oracle(cs[0])
+    refs = [o.recurrent_core_bwd(*_core_ops(q), c["X"].float().numpy(), dY.float().numpy(), 2, 640)
+            for c, dY in zip(cs, dYs)]
+    exs = [o.recurrent_core_bwd(*_core_ops(q), c["X"].float().numpy(), dY.float().numpy(), 2, 640,
+                                exact=True) for c, dY in zip(cs, dYs)]
+    for k in ("dWqkv", "dWo", "dWfc", "dWproj"):
+        ref = refs[0][k] + refs[1][k]
+        noise = np.hypot(rounding_noise_allowance(refs[0][k], exs[0][k]),
+                         rounding_noise_allowance(refs[1][k], exs[1][k]))
+        assert_close_chain(getattr(core, k), ref, noise, "accumulated " + k)
+    assert qat.device_error() == 0
+
+
+def test_recurrent_core_bwd_zero_tokens():
+    """No tokens: the forward returns an empty state, dX is empty and every
+    weight gradient is zero (no token uses to sum)."""
+    c = sy.recurrent_core_case(T=8)
+    core = _core(c)
+    x = torch.empty((0, 640), dtype=torch.bfloat16, device="cuda")
+    out = core.forward_train(x, 3)
+    dX = core.backward(torch.empty((0, 640), dtype=torch.bfloat16, device="cuda"))
+    torch.cuda.synchronize()
+    assert out.shape == (0, 640) and dX.shape == (0, 640)
+    for k in ("dWqkv", "dWo", "dWfc", "dWproj"):
+        assert torch.count_nonzero(getattr(core, k)).item() == 0, k
+    assert qat.device_error() == 0
+
+
 def test_recurrent_core_bwd_per_application():
     """Each application's backward on its own, from the oracle's saved bf16
     activations and incoming gradient: dx and the application's weight
