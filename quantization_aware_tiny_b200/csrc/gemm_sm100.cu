@@ -904,7 +904,13 @@ int launch_gemm(const GemmDesc& g, cudaStream_t stream) {
   int epi = g.epi;
   if (epi == EPI_F32 || epi == EPI_F32_ATOMIC) {
     const int tiles = a.num_m_blk * a.num_n_blk;
-    int s = choose_splits(tiles, a.kblk_total, pair ? sm_count() / 2 : sm_count());
+    // Split K only while the output tiles occupy fewer than half the CTAs
+    // (pairs): with more tiles, a wave of whole tiles already keeps at least
+    // half of them busy, and the split's zero-fill and fp32 reduce-adds cost
+    // more than the better wave fill returns (head dW 8192 x 512 over 65,536
+    // tokens: 64 tiles on 74 pairs, 447-461 us split 8 ways, 424-426 us whole).
+    const int cunits = pair ? sm_count() / 2 : sm_count();
+    int s = (2 * tiles >= cunits) ? 1 : choose_splits(tiles, a.kblk_total, cunits);
     a.kblk_per_split = (a.kblk_total + s - 1) / s;
     s = (a.kblk_total + a.kblk_per_split - 1) / a.kblk_per_split;  // no empty split
     a.splits = s;
