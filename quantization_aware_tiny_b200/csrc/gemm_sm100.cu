@@ -808,13 +808,18 @@ int fused_b_bn(int64_t N, int64_t K) {
 }
 
 // Split count for the fp32 weight-gradient GEMMs: minimise the makespan
-// ceil(tiles*s / SMs) * ceil(kblk / s), preferring fewer splits.
+// ceil(tiles*s / SMs) * (ceil(kblk / s) + E), preferring fewer splits, where
+// E = kSplitCost k-blocks charges each split work unit for its partial tile's
+// fp32 reduce-add and the zero-fill.  (Measured, 16 against 0, 28 and 48: the
+// MLP's 512 x 2048 weight gradients at 65,536 tokens 109 -> 103 us -- 9 splits
+// instead of 32 -- and the d = 640 core's training step 1.106 -> 1.064 ms.)
+constexpr int kSplitCost = 16;
 int choose_splits(int tiles, int kblk, int sms) {
   int best_s = 1;
   long long best = -1;
   for (int s = 1; s <= std::min(kblk, 64); ++s) {
     const long long waves = (static_cast<long long>(tiles) * s + sms - 1) / sms;
-    const long long cost = waves * ((kblk + s - 1) / s);
+    const long long cost = waves * ((kblk + s - 1) / s + (s > 1 ? kSplitCost : 0));
     if (best < 0 || cost < best) {
       best = cost;
       best_s = s;
