@@ -91,7 +91,10 @@ class RecurrentCore:
         so that each weight gradient is one GEMM over all R * T token uses:
         states [R+1, T, d] (state 0 is the input, state r+1 the output of
         application r), qkv, x1, pre, h; the gradient's g [R, T, d] (g[r] =
-        dL/d output of application r), dx1, dq [R, T, d], dpre [R, T, H]."""
+        dL/d output of application r), dx1, dq [R, T, d], dpre [R, T, H].
+        They, and the weight gradients dWqkv, dWo, dWfc, dWproj, are allocated
+        again when T or R changes: accumulate=True carries gradients across
+        calls of the same T and R only."""
         key = (T, R)
         if getattr(self, "_tkey", None) != key:
             bf, f32 = torch.bfloat16, torch.float32
