@@ -268,6 +268,22 @@ __device__ __forceinline__ uint32_t pack4(int c0, int c1, int c2, int c3) {
   return __byte_perm(lo, hi, 0x5410);
 }
 
+// The codes c_i = MUL (x_i - B) of four words x_i (int6: x_i the bit pattern
+// of kOff + rne(k / 4), B = 0x4B400000, MUL = 4), each in [-128, 127], as one
+// word of their two's-complement bytes.  sum_i (c_i + 128) 2^(8i) has no
+// carries between bytes, so four multiply-adds form it (modulo 2^32, B's
+// share folded into the constant), and flipping each byte's top bit turns
+// c + 128 into c's byte: no per-code byte permutes.
+template <uint32_t MUL, uint32_t B>
+__device__ __forceinline__ uint32_t pack_offset4(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3) {
+  constexpr uint32_t kC = (128u - MUL * B) * 0x01010101u;  // modulo 2^32
+  uint32_t acc = x3 * (MUL << 24) + kC;
+  acc = x2 * (MUL << 16) + acc;
+  acc = x1 * (MUL << 8) + acc;
+  acc = x0 * MUL + acc;
+  return acc ^ 0x80808080u;
+}
+
 template <int BITS, int R>
 __device__ __forceinline__ uint32_t codes4_t(const RowQuant& q, float4 v) {
   if constexpr (R == kNarrow && BITS != 6) {
@@ -276,6 +292,14 @@ __device__ __forceinline__ uint32_t codes4_t(const RowQuant& q, float4 v) {
     const float2 t0 = rne_quot2<R>(q, v.x, v.y), t1 = rne_quot2<R>(q, v.z, v.w);
     return pack4(__float_as_int(t0.x), __float_as_int(t0.y), __float_as_int(t1.x),
                  __float_as_int(t1.y));
+  } else if constexpr (R == kNarrow) {
+    // int6: only the top clamp can bind, 4 rne(k / 4) <= 124, i.e. the
+    // pattern kOff + rne(k / 4) at most 0x4B40001F; then the bytes 4 rne(k / 4)
+    const float2 u0 = rne_quarter2(rne_quot2<R>(q, v.x, v.y));
+    const float2 u1 = rne_quarter2(rne_quot2<R>(q, v.z, v.w));
+    return pack_offset4<4u, 0x4B400000u>(
+        min(__float_as_uint(u0.x), 0x4B40001Fu), min(__float_as_uint(u0.y), 0x4B40001Fu),
+        min(__float_as_uint(u1.x), 0x4B40001Fu), min(__float_as_uint(u1.y), 0x4B40001Fu));
   } else {
     int c0, c1, c2, c3;
     codes2<BITS, R>(q, v.x, v.y, c0, c1);
@@ -579,6 +603,109 @@ __device__ __forceinline__ void export_rows_smem(const ExportDescDev& d, int64_t
   with_grid(q[0].bits, range, run);
 }
 
+// ---- full units of the common widths, specialised: 384 float4 groups, as
+// three rows of 512 columns or one of 1,536 -- nearly every unit of the
+// 11-layer d = 512 state dict.  Every offset is a compile-time constant, so
+// the per-element work is the arithmetic alone (the generic path spends about
+// as many instructions again on loop control and addresses).
+
+// Three-input max (sm_100): max(a, b, c) in one instruction.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Running top-2 of |w| (with multiplicity) over four more weights, by sorted
+// pairs: (h, l) = sorted |v.x|, |v.y| and |v.z|, |v.w|; the four's largest is
+// max(h_xy, h_zw) and their second max(min(h_xy, h_zw), l_xy, l_zw); merging
+// two sorted pairs (t1, t2), (X1, X2) gives max(t1, X1) and
+// max(t2, X2, min(t1, X1)).  Ten min / max operations for four weights.
+__device__ __forceinline__ void top2_push4_pairs(float4 v, float& t1, float& t2) {
+  const float a = fabsf(v.x), b = fabsf(v.y), c = fabsf(v.z), e = fabsf(v.w);
+  const float hab = fmaxf(a, b), lab = fminf(a, b);
+  const float hce = fmaxf(c, e), lce = fminf(c, e);
+  const float x1 = fmaxf(hab, hce);
+  const float x2 = fmax3(fminf(hab, hce), lab, lce);
+  const float y = fminf(t1, x1);
+  t1 = fmaxf(t1, x1);
+  t2 = fmax3(t2, y, x2);
+}
+
+// Merge of two top-2 lists (t1 >= t2, u1 >= u2) into (t1, t2).
+__device__ __forceinline__ void top2_merge(float& t1, float& t2, float u1, float u2) {
+  const float y = fminf(t1, u1);
+  t1 = fmaxf(t1, u1);
+  t2 = fmax3(t2, u2, y);
+}
+
+// A full unit of NR rows (NR = 3: K4 = 128; NR = 1: K4 = 384) staged at buf:
+// lane holds groups lane + 32 i, i < 12; row k owns i in [12k / NR, 12(k+1) / NR).
+template <int NR>
+__device__ __forceinline__ void export_unit384(const ExportDescDev& d, int64_t row0,
+                                               const float4* __restrict__ buf, int lane) {
+  constexpr int K4 = 384 / NR;
+  // three chains of four groups: chain c = row c (NR = 3) or a third of the row
+  float t1[3], t2[3];
+#pragma unroll
+  for (int c = 0; c < 3; ++c) t1[c] = t2[c] = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int c = 0; c < 3; ++c) top2_push4_pairs(buf[lane + 32 * (4 * c + i)], t1[c], t2[c]);
+  }
+  if constexpr (NR == 1) {
+    top2_merge(t1[0], t2[0], t1[1], t2[1]);
+    top2_merge(t1[0], t2[0], t1[2], t2[2]);
+  }
+#pragma unroll
+  for (int k = 0; k < NR; ++k) top2_warp(t1[k], t2[k]);
+  // lane k works out row k's clip, scales and clamp range once for the warp
+  float m1 = t1[0], m2 = t2[0];
+#pragma unroll
+  for (int k = 1; k < NR; ++k) {
+    if (lane == k) {
+      m1 = t1[k];
+      m2 = t2[k];
+    }
+  }
+  const RowQuant mine = row_params(d, m1, m2);
+  const int my_range = row_range(m1, mine);
+  if (lane < NR) d.scales[row0 + lane] = __float2half_rn(mine.s);
+  RowQuant q[NR];
+  int range = kNarrow;
+#pragma unroll
+  for (int k = 0; k < NR; ++k) {
+    q[k].clip = __shfl_sync(0xffffffffu, mine.clip, k);
+    q[k].s = __shfl_sync(0xffffffffu, mine.s, k);
+    q[k].rs = __shfl_sync(0xffffffffu, mine.rs, k);
+    q[k].bits = mine.bits;
+    range = min(range, __shfl_sync(0xffffffffu, my_range, k));
+  }
+  uint32_t* out = reinterpret_cast<uint32_t*>(reinterpret_cast<int8_t*>(d.dst) + row0 * d.cols) + lane;
+  const float4* src = buf + lane;
+  with_grid(q[0].bits, range, [&](auto bits_tag, auto range_tag) {
+    constexpr int BITS = decltype(bits_tag)::value;
+    constexpr int R = decltype(range_tag)::value;
+#pragma unroll 1
+    for (int c = 0; c < 3; ++c) {
+      RowQuant qc = q[0];  // selects, not an indexed (local-memory) array
+      if constexpr (NR == 3) {
+        if (c == 1) qc = q[1];
+        if (c == 2) qc = q[NR - 1];
+      }
+      const float4* sc = src + 128 * c;
+      uint32_t* oc = out + 128 * c;
+      float4 v[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[i] = sc[32 * i];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) oc[32 * i] = codes4_t<BITS, R>(qc, v[i]);
+    }
+  });
+  (void)K4;
+}
+
 // ---- clip search (the leaderboard's "GPTQ-lite" clip search, read as: per row,
 // export at each candidate quantile and keep the first candidate of least
 // squared error of the stored row, sum_j (w_j - c_j * fp16(s))^2).
@@ -817,28 +944,13 @@ struct UnitPos {
   int d;
 };
 
-// Unit u of the batch, or d < 0 past the last unit.
-__device__ __forceinline__ UnitPos unit_at(const ExportBatch& b, int64_t u) {
-  UnitPos p;
-  if (u >= b.total_units) {
-    p.d = -1;
-    p.row0 = 0;
-    p.nrows = 0;
-    return p;
-  }
-  p.d = find_desc(b, u);
-  const ExportDescDev& d = b.d[p.d];
-  p.row0 = (u - d.unit_begin) * d.unit_rows;
-  p.nrows = static_cast<int>(min(d.unit_rows, d.rows - p.row0));
-  return p;
-}
-
 // One launch over all descriptors.  Work units are runs of consecutive rows of
 // one tensor -- as many as fit kExportUnitBytes for rows staged in shared
 // memory, one row otherwise, one chunk of about the same bytes for fp16
-// passthrough -- so units cost about the same.  Warp w of the grid takes units
-// w, w + W, w + 2W, ... (W = warps in the grid; a static assignment: one
-// shared work counter would serialise the warps on its atomics); a staged unit
+// passthrough -- so units cost about the same.  Warp w of the grid takes the
+// w-th run of ceil(units / W) consecutive units (W = warps in the grid; a
+// static assignment: one shared work counter would serialise the warps on its
+// atomics); a staged unit
 // arrives in one bulk copy into one of the warp's kExportBufs buffers while
 // the warp quantizes the previous one.  Units that are not staged still arrive once on their buffer's
 // mbarrier so every buffer's phases stay in step with the unit count.
@@ -865,9 +977,30 @@ __global__ void __launch_bounds__(kExportMaxWarps * 32, 1)
   }
   __syncthreads();
 
+  // Warp gw takes the consecutive units [gw * per, (gw + 1) * per): units cost
+  // about the same, and consecutive units mostly share their descriptor, so
+  // a cursor replaces a search per unit.
   const int64_t W = static_cast<int64_t>(gridDim.x) * nw;
   const int64_t gw = static_cast<int64_t>(blockIdx.x) * nw + wib;
+  const int64_t per = (b.total_units + W - 1) / W;
+  const int64_t u_end = min(b.total_units, (gw + 1) * per);
   const int stride = b.buf_bytes / 16;
+  int dcur = find_desc(b, min(gw * per, b.total_units - 1));
+  auto next_unit = [&](int64_t u) {
+    UnitPos p;
+    if (u >= u_end) {
+      p.d = -1;
+      p.row0 = 0;
+      p.nrows = 0;
+      return p;
+    }
+    while (dcur + 1 < b.n && b.d[dcur + 1].unit_begin <= u) ++dcur;
+    p.d = dcur;
+    const ExportDescDev& d = b.d[dcur];
+    p.row0 = (u - d.unit_begin) * d.unit_rows;
+    p.nrows = static_cast<int>(min(d.unit_rows, d.rows - p.row0));
+    return p;
+  };
 
   auto issue = [&](const UnitPos& p, int slot) {
     if (p.d < 0 || lane != 0) return;
@@ -883,10 +1016,10 @@ __global__ void __launch_bounds__(kExportMaxWarps * 32, 1)
 
   // ring of kExportBufs units: pos[k] is the unit in buffer (i + k) % kExportBufs
   UnitPos pos[kExportBufs];
-  int64_t next_u = gw;
+  int64_t next_u = gw * per;
   for (int k = 0; k < kExportBufs; ++k) {
-    pos[k] = unit_at(b, next_u);
-    next_u += W;
+    pos[k] = next_unit(next_u);
+    ++next_u;
     issue(pos[k], k);
   }
   int i = 0;
@@ -904,6 +1037,9 @@ __global__ void __launch_bounds__(kExportMaxWarps * 32, 1)
       constexpr bool PACK = KIND != kExportPlain;
       if (KIND == kExportSearch && d.search) {
         for (; r < pos[0].nrows; ++r) export_row_search(d, pos[0].row0 + r, ub + r * K4, lane);
+      } else if (KIND == kExportPlain && pos[0].nrows * K4 == 384 && (K4 == 128 || K4 == 384)) {
+        if (K4 == 128) export_unit384<3>(d, pos[0].row0, ub, lane);
+        else export_unit384<1>(d, pos[0].row0, ub, lane);
       } else {
         for (; r + 2 < pos[0].nrows; r += 3)
           export_rows_smem<PACK, 3>(d, pos[0].row0 + r, ub + r * K4, lane);
@@ -919,8 +1055,8 @@ __global__ void __launch_bounds__(kExportMaxWarps * 32, 1)
     // the buffer is read; order those reads before the copy engine refills it
     fence_proxy_async_smem();
     __syncwarp();
-    const UnitPos nn = unit_at(b, next_u);
-    next_u += W;
+    const UnitPos nn = next_unit(next_u);
+    ++next_u;
     issue(nn, slot);
 #pragma unroll
     for (int k = 0; k + 1 < kExportBufs; ++k) pos[k] = pos[k + 1];

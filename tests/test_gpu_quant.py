@@ -35,20 +35,35 @@ def _weights():
     z[2] = 0.5
     z[3, ::2] = -7.0
     cases["degenerate_8x64"] = z
-    # rows longer than one staged unit are exported as two half-row units by a
-    # warp pair: ragged halves (1040), halves of 1024 (2048), a width that is
-    # not split (1032, not a multiple of 16), and rows whose top two |w| tie
-    # across the halves, inside one half, or sit in different halves
+    # long staged rows: ragged widths (1040), the longest staged row (2048), a
+    # width that is not a multiple of 16 (1032), and 1536-column rows whose
+    # top two |w| tie or sit in different thirds of the row (a lane reduces
+    # each third separately before merging) or on either side of a third
     cases["split_37x1040"] = (rng.standard_normal((37, 1040)) * 0.02).astype(np.float32)
     cases["split_9x2048"] = (rng.standard_normal((9, 2048)) * 0.02).astype(np.float32)
     cases["whole_11x1032"] = (rng.standard_normal((11, 1032)) * 0.02).astype(np.float32)
-    t = (rng.standard_normal((5, 1536)) * 0.02).astype(np.float32)
-    t[0, 100], t[0, 1200] = 0.5, -0.5  # max once in each half
-    t[1, 10], t[1, 20] = 0.5, 0.5      # max twice in the first half
-    t[2, 800], t[2, 1500] = 0.5, 0.25  # top two in the second half
-    t[3, 767], t[3, 768] = -0.4, 0.3   # top two on either side of the split
+    t = (rng.standard_normal((9, 1536)) * 0.02).astype(np.float32)
+    t[0, 100], t[0, 1200] = 0.5, -0.5  # max once in two thirds
+    t[1, 10], t[1, 20] = 0.5, 0.5      # max twice in the first third
+    t[2, 800], t[2, 1500] = 0.5, 0.25  # top two in the last two thirds
+    t[3, 511], t[3, 512] = -0.4, 0.3   # top two on either side of a third
     t[4] = 0.125                       # a constant row
-    cases["split_ties_5x1536"] = t
+    t[5, 4], t[5, 516] = 0.5, -0.5     # max twice in one lane, in two thirds
+    t[6, 8], t[6, 9] = 0.5, 0.5        # max twice in one group of four
+    t[7, 1028], t[7, 1029] = 0.5, 0.375  # top two in one group of four
+    t[8, 0], t[8, 128], t[8, 1024] = 0.25, 0.5, 0.5  # one lane holds all three
+    cases["ties_9x1536"] = t
+    # 512-column rows (exported three to a unit): ties and top two inside one
+    # group of four, in one lane's groups, a zero row, a constant row
+    t = (rng.standard_normal((7, 512)) * 0.02).astype(np.float32)
+    t[0, 4], t[0, 5] = 0.5, -0.5
+    t[1, 1], t[1, 129] = -0.5, 0.5
+    t[2, 200], t[2, 203] = 0.5, 0.4375
+    t[3] = -0.0625
+    t[4] = 0.0
+    t[5, 511], t[5, 0] = 0.5, 0.25
+    t[6, 3], t[6, 131], t[6, 259] = 0.5, 0.5, 0.5
+    cases["ties_7x512"] = t
     return cases
 
 
