@@ -4,7 +4,7 @@
 //
 // Quantization uses one warp per row.  The export kernel stages rows in shared
 // memory with 1-D bulk async copies (the copy engine, completing on an
-// mbarrier) one row ahead of the row being quantized, with up to 16 warps per
+// mbarrier) one work unit ahead of the unit being quantized, with up to 16 warps per
 // SM; the training-time kernel caches the row in registers between its
 // reduction and quantization passes.
 #include <algorithm>
