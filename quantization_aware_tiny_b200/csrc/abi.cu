@@ -483,9 +483,10 @@ int dequantize_rows_batch(const qat_dequant_desc* descs, int32_t n, qat_stream_t
     d.scales = reinterpret_cast<const __half*>(s.scales);
     d.out = s.out;
     d.cols = s.cols;
+    d.row_magic = dequant_row_magic(s.cols >> 2);
     d.out_bf16 = s.out_dtype == QAT_DTYPE_BF16;
     d.pad = 0;
-    b.item_begin[i + 1] = b.item_begin[i] + s.rows * (s.cols >> 3);
+    b.item_begin[i + 1] = b.item_begin[i] + s.rows * (s.cols >> 2);
   }
   return launch_dequant_batch(b, stream);
 }

@@ -1072,54 +1072,82 @@ __global__ void __launch_bounds__(kExportMaxWarps * 32, 1)
 }
 
 // ------------------------------------------------------------------ dequantize
-// Eight consecutive codes of a row (item i: elements 8i .. 8i + 7; cols a
-// multiple of 8, so they share the row's scale): fl32(c * fp32(scale_fp16)),
-// stored as fp32 or rounded to bf16.
-__device__ __forceinline__ void dequant8(const int8_t* __restrict__ codes,
-                                         const __half* __restrict__ scales, int64_t cols,
-                                         int64_t i, int out_bf16, void* __restrict__ out) {
-  const int64_t row = i / (cols >> 3);
-  const int64_t e = i * 8;
-  const float s = __half2float(scales[row]);
-  const uint2 cc = *reinterpret_cast<const uint2*>(codes + e);
-  const int8_t* c = reinterpret_cast<const int8_t*>(&cc);
-  float v[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) v[k] = mul_rn(static_cast<float>(c[k]), s);
+// Items of four consecutive codes of a row (item l of a tensor: elements
+// 4l .. 4l + 3; cols a multiple of 8, so the four share the row's scale): the
+// codes as one 32-bit load, fl32(c * fp32(scale_fp16)) stored as one 16-byte
+// fp32 word (or 8 bytes of bf16), so a warp's loads and stores are
+// contiguous.  Each thread takes two items a grid stride apart per iteration
+// and issues both items' loads before either item's stores, two loads in
+// flight per thread at full occupancy; the row index comes from a
+// multiply-high by row_magic instead of a 64-bit division.
+struct DequantItem {
+  uint32_t c;  // four codes, little-endian bytes
+  float s;     // the row's scale
+};
+
+__device__ __forceinline__ DequantItem dequant_load(const int8_t* __restrict__ codes,
+                                                    const __half* __restrict__ scales,
+                                                    uint64_t row_magic, int64_t l) {
+  DequantItem it;
+  it.c = __ldg(reinterpret_cast<const uint32_t*>(codes) + l);
+  it.s = __half2float(__ldg(scales + __umul64hi(static_cast<uint64_t>(l), row_magic)));
+  return it;
+}
+
+__device__ __forceinline__ void dequant_store(const DequantItem& it, int out_bf16,
+                                              void* __restrict__ out, int64_t l) {
+  const float v0 = mul_rn(static_cast<float>(static_cast<int8_t>(it.c & 0xFFu)), it.s);
+  const float v1 = mul_rn(static_cast<float>(static_cast<int8_t>((it.c >> 8) & 0xFFu)), it.s);
+  const float v2 = mul_rn(static_cast<float>(static_cast<int8_t>((it.c >> 16) & 0xFFu)), it.s);
+  const float v3 = mul_rn(static_cast<float>(static_cast<int8_t>(it.c >> 24)), it.s);
   if (out_bf16) {
-    uint4 w;
-    w.x = pack_bf16x2(v[0], v[1]);
-    w.y = pack_bf16x2(v[2], v[3]);
-    w.z = pack_bf16x2(v[4], v[5]);
-    w.w = pack_bf16x2(v[6], v[7]);
-    *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(out) + e) = w;
+    uint2 w;
+    w.x = pack_bf16x2(v0, v1);
+    w.y = pack_bf16x2(v2, v3);
+    reinterpret_cast<uint2*>(out)[l] = w;
   } else {
-    float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + e);
-    o[0] = make_float4(v[0], v[1], v[2], v[3]);
-    o[1] = make_float4(v[4], v[5], v[6], v[7]);
+    reinterpret_cast<float4*>(out)[l] = make_float4(v0, v1, v2, v3);
   }
 }
 
-__global__ void __launch_bounds__(kQThreads)
+__global__ void __launch_bounds__(kQThreads, 8)
     dequant_kernel(const int8_t* __restrict__ codes, const __half* __restrict__ scales,
-                   int64_t rows, int64_t cols, int out_bf16, void* __restrict__ out) {
-  const int64_t total = rows * (cols >> 3);
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    dequant8(codes, scales, cols, i, out_bf16, out);
+                   int64_t total, uint64_t row_magic, int out_bf16, void* __restrict__ out) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i0 < total;
+       i0 += 2 * stride) {
+    const int64_t i1 = i0 + stride;
+    const DequantItem a = dequant_load(codes, scales, row_magic, i0);
+    DequantItem b{0u, 0.0f};
+    if (i1 < total) b = dequant_load(codes, scales, row_magic, i1);
+    dequant_store(a, out_bf16, out, i0);
+    if (i1 < total) dequant_store(b, out_bf16, out, i1);
+  }
 }
 
-// All descriptors' items in one grid-stride loop; a thread's items increase,
-// so its descriptor index only moves forward.
-__global__ void __launch_bounds__(kQThreads)
+// All descriptors' items in one grid-stride loop.  The two items of an
+// iteration keep a descriptor cursor each; a thread's items increase, so the
+// cursors only move forward.
+__global__ void __launch_bounds__(kQThreads, 8)
     dequant_batch_kernel(const __grid_constant__ DequantBatch b) {
   const int64_t total = b.item_begin[b.n];
-  int k = 0;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    while (k + 1 < b.n && b.item_begin[k + 1] <= i) ++k;
-    const DequantDescDev& d = b.d[k];
-    dequant8(d.codes, d.scales, d.cols, i - b.item_begin[k], d.out_bf16, d.out);
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  int k0 = 0, k1 = 0;
+  for (int64_t i0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i0 < total;
+       i0 += 2 * stride) {
+    const int64_t i1 = i0 + stride;
+    while (k0 + 1 < b.n && b.item_begin[k0 + 1] <= i0) ++k0;
+    const int64_t l0 = i0 - b.item_begin[k0];
+    const DequantItem a = dequant_load(b.d[k0].codes, b.d[k0].scales, b.d[k0].row_magic, l0);
+    DequantItem c{0u, 0.0f};
+    int64_t l1 = 0;
+    if (i1 < total) {
+      while (k1 + 1 < b.n && b.item_begin[k1 + 1] <= i1) ++k1;
+      l1 = i1 - b.item_begin[k1];
+      c = dequant_load(b.d[k1].codes, b.d[k1].scales, b.d[k1].row_magic, l1);
+    }
+    dequant_store(a, b.d[k0].out_bf16, b.d[k0].out, l0);
+    if (i1 < total) dequant_store(c, b.d[k1].out_bf16, b.d[k1].out, l1);
   }
 }
 
@@ -1249,10 +1277,10 @@ int launch_export_batch(ExportBatch& b, cudaStream_t s) {
 
 int launch_dequant(const int8_t* codes, const __half* scales, int64_t rows, int64_t cols,
                    int out_bf16, void* out, cudaStream_t s) {
-  const int64_t items = rows * (cols >> 3);
+  const int64_t items = rows * (cols >> 2);
   if (items == 0) return QAT_OK;
-  dequant_kernel<<<grid_for_rows(items, kQThreads), kQThreads, 0, s>>>(codes, scales, rows, cols,
-                                                                       out_bf16, out);
+  dequant_kernel<<<grid_for_rows(items, kQThreads), kQThreads, 0, s>>>(
+      codes, scales, items, dequant_row_magic(cols >> 2), out_bf16, out);
   count_launch();
   return cuda_status(cudaGetLastError());
 }

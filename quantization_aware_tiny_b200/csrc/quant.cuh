@@ -81,15 +81,24 @@ int launch_export_batch(ExportBatch& b, cudaStream_t s);
 int launch_dequant(const int8_t* codes, const __half* scales, int64_t rows, int64_t cols,
                    int out_bf16, void* out, cudaStream_t s);
 
-// Grouped dequantize: descriptor k covers the 8-element groups
-// [item_begin[k], item_begin[k + 1]) of the concatenation.
+// Grouped dequantize: descriptor k covers the 4-element groups
+// [item_begin[k], item_begin[k + 1]) of the concatenation.  The row of group
+// l is l / (cols / 4) = the high 64 bits of l * row_magic, row_magic =
+// ceil(2^64 / (cols / 4)) (exact for l < 2^46: the product's error,
+// l (row_magic - 2^64 / (cols / 4)) / 2^64 < l / 2^64, stays below the gap
+// 1 / (cols / 4) between l / (cols / 4) and the next integer).
 struct DequantDescDev {
   const int8_t* codes;
   const __half* scales;
   void* out;
   int64_t cols;
+  uint64_t row_magic;
   int out_bf16, pad;
 };
+// ceil(2^64 / c4) for c4 >= 2.
+inline uint64_t dequant_row_magic(int64_t c4) {
+  return ~0ull / static_cast<uint64_t>(c4) + 1ull;
+}
 constexpr int kDequantMaxDescs = QAT_DEQUANT_MAX_DESCS;
 struct DequantBatch {
   int n;
