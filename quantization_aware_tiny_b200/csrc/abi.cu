@@ -471,7 +471,7 @@ int dequantize_rows_batch(const qat_dequant_desc* descs, int32_t n, qat_stream_t
   if (!descs || n <= 0 || n > QAT_DEQUANT_MAX_DESCS) return QAT_ERR_ARG;
   static thread_local DequantBatch b;  // ~14 KB: kept off the stack
   b.n = n;
-  b.item_begin[0] = 0;
+  b.tile_begin[0] = 0;
   for (int i = 0; i < n; ++i) {
     const qat_dequant_desc& s = descs[i];
     if (!s.codes || !s.scales || !s.out || s.rows < 0) return QAT_ERR_ARG;
@@ -482,11 +482,11 @@ int dequantize_rows_batch(const qat_dequant_desc* descs, int32_t n, qat_stream_t
     d.codes = s.codes;
     d.scales = reinterpret_cast<const __half*>(s.scales);
     d.out = s.out;
-    d.cols = s.cols;
+    d.items = s.rows * (s.cols >> 2);
     d.row_magic = dequant_row_magic(s.cols >> 2);
     d.out_bf16 = s.out_dtype == QAT_DTYPE_BF16;
     d.pad = 0;
-    b.item_begin[i + 1] = b.item_begin[i] + s.rows * (s.cols >> 2);
+    b.tile_begin[i + 1] = b.tile_begin[i] + (d.items + kDequantTile - 1) / kDequantTile;
   }
   return launch_dequant_batch(b, stream);
 }

@@ -1076,10 +1076,10 @@ __global__ void __launch_bounds__(kExportMaxWarps * 32, 1)
 // 4l .. 4l + 3; cols a multiple of 8, so the four share the row's scale): the
 // codes as one 32-bit load, fl32(c * fp32(scale_fp16)) stored as one 16-byte
 // fp32 word (or 8 bytes of bf16), so a warp's loads and stores are
-// contiguous.  Each thread takes two items a grid stride apart per iteration
-// and issues both items' loads before either item's stores, two loads in
-// flight per thread at full occupancy; the row index comes from a
-// multiply-high by row_magic instead of a 64-bit division.
+// contiguous.  A thread block takes one tile of kDequantTile items; each
+// thread issues its kDequantPerThread items' loads before any store.  The row
+// index comes from a multiply-high by row_magic instead of a 64-bit division,
+// and every descriptor field a tile needs is block-uniform.
 struct DequantItem {
   uint32_t c;  // four codes, little-endian bytes
   float s;     // the row's scale
@@ -1110,45 +1110,45 @@ __device__ __forceinline__ void dequant_store(const DequantItem& it, int out_bf1
   }
 }
 
-__global__ void __launch_bounds__(kQThreads, 8)
-    dequant_kernel(const int8_t* __restrict__ codes, const __half* __restrict__ scales,
-                   int64_t total, uint64_t row_magic, int out_bf16, void* __restrict__ out) {
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i0 < total;
-       i0 += 2 * stride) {
-    const int64_t i1 = i0 + stride;
-    const DequantItem a = dequant_load(codes, scales, row_magic, i0);
-    DequantItem b{0u, 0.0f};
-    if (i1 < total) b = dequant_load(codes, scales, row_magic, i1);
-    dequant_store(a, out_bf16, out, i0);
-    if (i1 < total) dequant_store(b, out_bf16, out, i1);
+static_assert(kDequantTile == kQThreads * kDequantPerThread, "one tile per block of kQThreads");
+
+// Tile `tile` of one tensor's items.
+__device__ __forceinline__ void dequant_tile(const int8_t* __restrict__ codes,
+                                             const __half* __restrict__ scales, int64_t items,
+                                             uint64_t row_magic, int out_bf16,
+                                             void* __restrict__ out, int64_t tile) {
+  const int64_t base = tile * kDequantTile + threadIdx.x;
+  DequantItem it[kDequantPerThread];
+#pragma unroll
+  for (int j = 0; j < kDequantPerThread; ++j) {
+    const int64_t l = base + j * kQThreads;
+    if (l < items) it[j] = dequant_load(codes, scales, row_magic, l);
+  }
+#pragma unroll
+  for (int j = 0; j < kDequantPerThread; ++j) {
+    const int64_t l = base + j * kQThreads;
+    if (l < items) dequant_store(it[j], out_bf16, out, l);
   }
 }
 
-// All descriptors' items in one grid-stride loop.  The two items of an
-// iteration keep a descriptor cursor each; a thread's items increase, so the
-// cursors only move forward.
-__global__ void __launch_bounds__(kQThreads, 8)
+__global__ void __launch_bounds__(kQThreads)
+    dequant_kernel(const int8_t* __restrict__ codes, const __half* __restrict__ scales,
+                   int64_t items, uint64_t row_magic, int out_bf16, void* __restrict__ out) {
+  dequant_tile(codes, scales, items, row_magic, out_bf16, out, blockIdx.x);
+}
+
+// One block per tile of the concatenation; its descriptor is the last k with
+// tile_begin[k] <= tile (tensors without items own no tile).
+__global__ void __launch_bounds__(kQThreads)
     dequant_batch_kernel(const __grid_constant__ DequantBatch b) {
-  const int64_t total = b.item_begin[b.n];
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  int k0 = 0, k1 = 0;
-  for (int64_t i0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i0 < total;
-       i0 += 2 * stride) {
-    const int64_t i1 = i0 + stride;
-    while (k0 + 1 < b.n && b.item_begin[k0 + 1] <= i0) ++k0;
-    const int64_t l0 = i0 - b.item_begin[k0];
-    const DequantItem a = dequant_load(b.d[k0].codes, b.d[k0].scales, b.d[k0].row_magic, l0);
-    DequantItem c{0u, 0.0f};
-    int64_t l1 = 0;
-    if (i1 < total) {
-      while (k1 + 1 < b.n && b.item_begin[k1 + 1] <= i1) ++k1;
-      l1 = i1 - b.item_begin[k1];
-      c = dequant_load(b.d[k1].codes, b.d[k1].scales, b.d[k1].row_magic, l1);
-    }
-    dequant_store(a, b.d[k0].out_bf16, b.d[k0].out, l0);
-    if (i1 < total) dequant_store(c, b.d[k1].out_bf16, b.d[k1].out, l1);
+  const int64_t t = blockIdx.x;
+  int lo = 0, hi = b.n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (b.tile_begin[mid] <= t) lo = mid; else hi = mid - 1;
   }
+  const DequantDescDev& d = b.d[lo];
+  dequant_tile(d.codes, d.scales, d.items, d.row_magic, d.out_bf16, d.out, t - b.tile_begin[lo]);
 }
 
 // 6-bit packed codes back to int8 codes: thread per 8 codes (6 bytes read as
@@ -1279,16 +1279,19 @@ int launch_dequant(const int8_t* codes, const __half* scales, int64_t rows, int6
                    int out_bf16, void* out, cudaStream_t s) {
   const int64_t items = rows * (cols >> 2);
   if (items == 0) return QAT_OK;
-  dequant_kernel<<<grid_for_rows(items, kQThreads), kQThreads, 0, s>>>(
+  const int64_t tiles = (items + kDequantTile - 1) / kDequantTile;
+  if (tiles > 0x7FFFFFFF) return QAT_ERR_SHAPE;
+  dequant_kernel<<<static_cast<unsigned>(tiles), kQThreads, 0, s>>>(
       codes, scales, items, dequant_row_magic(cols >> 2), out_bf16, out);
   count_launch();
   return cuda_status(cudaGetLastError());
 }
 
 int launch_dequant_batch(const DequantBatch& b, cudaStream_t s) {
-  const int64_t items = b.item_begin[b.n];
-  if (items == 0) return QAT_OK;
-  dequant_batch_kernel<<<grid_for_rows(items, kQThreads), kQThreads, 0, s>>>(b);
+  const int64_t tiles = b.tile_begin[b.n];
+  if (tiles == 0) return QAT_OK;
+  if (tiles > 0x7FFFFFFF) return QAT_ERR_SHAPE;
+  dequant_batch_kernel<<<static_cast<unsigned>(tiles), kQThreads, 0, s>>>(b);
   count_launch();
   return cuda_status(cudaGetLastError());
 }

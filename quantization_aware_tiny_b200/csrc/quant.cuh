@@ -81,8 +81,9 @@ int launch_export_batch(ExportBatch& b, cudaStream_t s);
 int launch_dequant(const int8_t* codes, const __half* scales, int64_t rows, int64_t cols,
                    int out_bf16, void* out, cudaStream_t s);
 
-// Grouped dequantize: descriptor k covers the 4-element groups
-// [item_begin[k], item_begin[k + 1]) of the concatenation.  The row of group
+// Grouped dequantize: descriptor k covers tiles [tile_begin[k],
+// tile_begin[k + 1]) of kDequantTile 4-element groups (items) each, the last
+// one partial; one thread block per tile.  The row of group
 // l is l / (cols / 4) = the high 64 bits of l * row_magic, row_magic =
 // ceil(2^64 / (cols / 4)) (exact for l < 2^46: the product's error,
 // l (row_magic - 2^64 / (cols / 4)) / 2^64 < l / 2^64, stays below the gap
@@ -91,10 +92,12 @@ struct DequantDescDev {
   const int8_t* codes;
   const __half* scales;
   void* out;
-  int64_t cols;
+  int64_t items;  // rows * cols / 4
   uint64_t row_magic;
   int out_bf16, pad;
 };
+constexpr int kDequantPerThread = 4;                 // items per thread
+constexpr int kDequantTile = 256 * kDequantPerThread;  // items per block
 // ceil(2^64 / c4) for c4 >= 2.
 inline uint64_t dequant_row_magic(int64_t c4) {
   return ~0ull / static_cast<uint64_t>(c4) + 1ull;
@@ -102,7 +105,7 @@ inline uint64_t dequant_row_magic(int64_t c4) {
 constexpr int kDequantMaxDescs = QAT_DEQUANT_MAX_DESCS;
 struct DequantBatch {
   int n;
-  int64_t item_begin[kDequantMaxDescs + 1];
+  int64_t tile_begin[kDequantMaxDescs + 1];
   DequantDescDev d[kDequantMaxDescs];
 };
 int launch_dequant_batch(const DequantBatch& b, cudaStream_t s);
