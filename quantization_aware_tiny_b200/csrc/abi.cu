@@ -173,7 +173,7 @@ int qat_quantize_weights_batch(const qat_quant_desc* descs, int32_t n, qat_strea
   if (!descs || n <= 0 || n > QAT_QUANT_MAX_DESCS) return QAT_ERR_ARG;
   QuantBatch b;
   b.n = n;
-  b.row_begin[0] = 0;
+  b.tile_begin[0] = 0;
   for (int i = 0; i < n; ++i) {
     const qat_quant_desc& s = descs[i];
     if (!s.W || !s.scales || s.N <= 0 || !bits_ok(s.bits)) return QAT_ERR_ARG;
@@ -182,7 +182,7 @@ int qat_quantize_weights_batch(const qat_quant_desc* descs, int32_t n, qat_strea
       return QAT_ERR_ALIGN;
     b.d[i] = QuantDescDev{s.W, s.codes, s.scales, reinterpret_cast<__nv_bfloat16*>(s.operand),
                           s.N, s.K, s.bits, 0};
-    b.row_begin[i + 1] = b.row_begin[i] + s.N;
+    b.tile_begin[i + 1] = b.tile_begin[i] + quant_tiles(s.N, s.K);
   }
   return launch_quantize_batch(b, stream);
 }

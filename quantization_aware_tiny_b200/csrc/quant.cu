@@ -21,7 +21,6 @@ namespace {
 
 constexpr int kQThreads = 256;  // 8 warps per block
 constexpr int kRegV4 = 16;      // float4 per lane kept in registers (2048 columns)
-constexpr int kQuantV4 = 4;     // the training quantizer's cached float4 per lane (512 columns)
 
 __device__ __forceinline__ float amax4(float4 v) {
   return fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
@@ -309,43 +308,56 @@ __device__ __forceinline__ uint32_t codes4_t(const RowQuant& q, float4 v) {
 }
 
 // ------------------------------------------------------------------ QAT quantize
-// One row of one weight: amax over the row (the first 512 columns cached in
-// registers, the rest read again from L2), the IEEE scale, codes and the bf16
-// operand bf16(fl32(c * s)).
+// Rows in segments of 512 columns (128 float4 groups, four per lane), a warp
+// per segment: a row of K columns takes S = ceil(K / 512) segments, and a
+// block of 8 warps takes 8 / min(S, 8) rows with min(S, 8) warps each, so
+// every warp issues its four loads at once whatever the row length (a warp
+// looping over a 2,048-column row waited on memory four times in a row).  The
+// warps of a row merge their amax through shared memory; each keeps its first
+// segment in registers for the code pass and reads any further segments (rows
+// over 4,096 columns) a second time.
 template <int BITS>
-__device__ __forceinline__ void quantize_row_t(const QuantDescDev& d, int row, int lane) {
-  const int K = d.K;
-  const int K4 = K >> 2;
-  const float4* r = reinterpret_cast<const float4*>(d.W + static_cast<int64_t>(row) * K);
-  float4 cache[kQuantV4];
-  float amax = 0.0f, amax2 = 0.0f;
+__device__ __forceinline__ void quantize_tile(const QuantDescDev& d, int64_t tile, float* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int K = d.K, K4 = K >> 2;
+  const int S = (K4 + 127) >> 7;
+  const int wpr = min(S, kQuantTileRows);  // warps per row
+  const int rpb = kQuantTileRows / wpr;    // rows per block
+  const int rib = warp / wpr, wir = warp - rib * wpr;
+  const int64_t row = tile * rpb + rib;
+  const bool active = rib < rpb && row < d.N;
+  const float4* r = reinterpret_cast<const float4*>(d.W + (active ? row : 0) * static_cast<int64_t>(K));
+  float4 v[4];
+  float amax = 0.0f;
+  if (active) {
 #pragma unroll
-  for (int i = 0; i < kQuantV4; ++i) {
-    const int j = lane + 32 * i;
-    if (j < K4) {
-      cache[i] = __ldg(r + j);
-      if (i & 1) amax2 = fmaxf(amax2, amax4(cache[i]));
-      else amax = fmaxf(amax, amax4(cache[i]));
+    for (int u = 0; u < 4; ++u) {
+      const int j = wir * 128 + lane + 32 * u;
+      v[u] = j < K4 ? __ldg(r + j) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    }
+    amax = fmaxf(fmaxf(amax4(v[0]), amax4(v[1])), fmaxf(amax4(v[2]), amax4(v[3])));
+    for (int sg = wir + wpr; sg < S; sg += wpr) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = sg * 128 + lane + 32 * u;
+        if (j < K4) amax = fmaxf(amax, amax4(__ldg(r + j)));
+      }
     }
   }
-  for (int j = lane + 32 * kQuantV4; j < K4; j += 64) {
-    amax = fmaxf(amax, amax4(__ldg(r + j)));
-    if (j + 32 < K4) amax2 = fmaxf(amax2, amax4(__ldg(r + j + 32)));
-  }
-  amax = fmaxf(amax, amax2);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  RowQuant q;
-  q.clip = fmaxf(amax, 1e-12f);
-  q.s = div_rn(q.clip, grid_levels(BITS));
-  q.rs = __frcp_rn(q.s);
-  q.bits = BITS;
-  if (lane == 0) d.scales[row] = q.s;
-  const float2 s2 = make_float2(q.s, q.s);
-  auto emit = [&](int j, float4 v) {
-    const float2 c01 = grid_code_values2<BITS>(v.x, v.y, q.s, q.rs);
-    const float2 c23 = grid_code_values2<BITS>(v.z, v.w, q.s, q.rs);
-    const int64_t e = static_cast<int64_t>(row) * K + 4 * j;
+  if (lane == 0) red[warp] = amax;
+  __syncthreads();
+  if (!active) return;
+  for (int w = rib * wpr; w < rib * wpr + wpr; ++w) amax = fmaxf(amax, red[w]);
+  const float s = div_rn(fmaxf(amax, 1e-12f), grid_levels(BITS));
+  const float rs = __frcp_rn(s);
+  if (wir == 0 && lane == 0) d.scales[row] = s;
+  const float2 s2 = make_float2(s, s);
+  auto emit = [&](int j, float4 x) {
+    const float2 c01 = grid_code_values2<BITS>(x.x, x.y, s, rs);
+    const float2 c23 = grid_code_values2<BITS>(x.z, x.w, s, rs);
+    const int64_t e = row * K + 4 * j;
     if (d.codes)
       *reinterpret_cast<uint32_t*>(d.codes + e) =
           pack_codes(__float2int_rn(c01.x), __float2int_rn(c01.y), __float2int_rn(c23.x),
@@ -359,30 +371,36 @@ __device__ __forceinline__ void quantize_row_t(const QuantDescDev& d, int row, i
     }
   };
 #pragma unroll
-  for (int i = 0; i < kQuantV4; ++i) {
-    const int j = lane + 32 * i;
-    if (j < K4) emit(j, cache[i]);
+  for (int u = 0; u < 4; ++u) {
+    const int j = wir * 128 + lane + 32 * u;
+    if (j < K4) emit(j, v[u]);
   }
-  for (int j = lane + 32 * kQuantV4; j < K4; j += 32) emit(j, __ldg(r + j));
+  for (int sg = wir + wpr; sg < S; sg += wpr) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = sg * 128 + lane + 32 * u;
+      if (j < K4) emit(j, __ldg(r + j));
+    }
+  }
 }
 
-// All rows of all the batch's weights, a warp per row (grid-stride over the
-// concatenated rows), so small weights share the launch and the SMs.
-__global__ void __launch_bounds__(kQThreads, 3)
+// The batch's weights in tiles (8 / min(S, 8) rows of one weight each), one
+// thread block per tile: the tile's descriptor is block-uniform, found by a
+// binary search on the tile index.
+__global__ void __launch_bounds__(kQThreads, 6)
     quantize_batch_kernel(const __grid_constant__ QuantBatch b) {
-  const int lane = threadIdx.x & 31;
-  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  const int64_t total = b.row_begin[b.n];
-  int k = 0;
-  for (int64_t g = warp; g < total; g += nwarps) {
-    while (k + 1 < b.n && b.row_begin[k + 1] <= g) ++k;  // rows are visited in increasing order
-    const QuantDescDev& d = b.d[k];
-    const int row = static_cast<int>(g - b.row_begin[k]);
-    if (d.bits == 6) quantize_row_t<6>(d, row, lane);
-    else if (d.bits == 5) quantize_row_t<5>(d, row, lane);
-    else quantize_row_t<8>(d, row, lane);
+  __shared__ float red[kQuantTileRows];
+  const int64_t t = blockIdx.x;
+  int lo = 0, hi = b.n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (b.tile_begin[mid] <= t) lo = mid; else hi = mid - 1;
   }
+  const QuantDescDev& d = b.d[lo];
+  const int64_t tile = t - b.tile_begin[lo];
+  if (d.bits == 6) quantize_tile<6>(d, tile, red);
+  else if (d.bits == 5) quantize_tile<5>(d, tile, red);
+  else quantize_tile<8>(d, tile, red);
 }
 
 // ---- 6-bit packing of int6 / int5 codes: one 6-bit two's-complement field per
@@ -1111,6 +1129,7 @@ __device__ __forceinline__ void dequant_store(const DequantItem& it, int out_bf1
 }
 
 static_assert(kDequantTile == kQThreads * kDequantPerThread, "one tile per block of kQThreads");
+static_assert(kQuantTileRows * 32 == kQThreads, "a warp per row of a quantize tile");
 
 // Tile `tile` of one tensor's items.
 __device__ __forceinline__ void dequant_tile(const int8_t* __restrict__ codes,
@@ -1181,9 +1200,10 @@ int grid_for_rows(int64_t rows_or_items, int items_per_block) {
 }  // namespace
 
 int launch_quantize_batch(const QuantBatch& b, cudaStream_t s) {
-  const int64_t total = b.row_begin[b.n];
-  if (total == 0) return QAT_OK;
-  quantize_batch_kernel<<<grid_for_rows(total, kQThreads / 32), kQThreads, 0, s>>>(b);
+  const int64_t tiles = b.tile_begin[b.n];
+  if (tiles == 0) return QAT_OK;
+  if (tiles > 0x7FFFFFFF) return QAT_ERR_SHAPE;
+  quantize_batch_kernel<<<static_cast<unsigned>(tiles), kQThreads, 0, s>>>(b);
   count_launch();
   return cuda_status(cudaGetLastError());
 }
@@ -1192,8 +1212,8 @@ int launch_quantize_weights(const float* W, int N, int K, int bits, int8_t* code
                             __nv_bfloat16* operand, cudaStream_t s) {
   QuantBatch b;
   b.n = 1;
-  b.row_begin[0] = 0;
-  b.row_begin[1] = N;
+  b.tile_begin[0] = 0;
+  b.tile_begin[1] = quant_tiles(N, K);
   b.d[0] = QuantDescDev{W, codes, scales, operand, N, K, bits, 0};
   return launch_quantize_batch(b, s);
 }

@@ -65,9 +65,17 @@ struct QuantDescDev {
   __nv_bfloat16* operand;
   int N, K, bits, pad;
 };
+constexpr int kQuantTileRows = 8;  // warps per thread block (rows of up to 512 columns)
+// Thread blocks for N rows of K columns: min(S, 8) warps per row, S = the
+// row's 512-column segments, 8 / min(S, 8) rows per block.
+inline int64_t quant_tiles(int64_t N, int64_t K) {
+  const int64_t S = ((K >> 2) + 127) >> 7;
+  const int64_t rpb = kQuantTileRows / (S < kQuantTileRows ? S : kQuantTileRows);
+  return (N + rpb - 1) / rpb;
+}
 struct QuantBatch {
   int n;
-  int64_t row_begin[kQuantMaxDescs + 1];  // first global row of each weight; [n] = total
+  int64_t tile_begin[kQuantMaxDescs + 1];  // first tile of each weight; [n] = total
   QuantDescDev d[kQuantMaxDescs];
 };
 int launch_quantize_batch(const QuantBatch& b, cudaStream_t s);
