@@ -133,6 +133,10 @@ def test_argument_validation_before_launch(L):
                     (D(0x10000, 0x10000, 4, 16, 0, 0, 0x10008), qat.QAT_ERR_ALIGN)):
         two = (D * 2)(good, bad)
         assert L.dequantize_rows_batch(ctypes.cast(two, ctypes.c_void_p), 2, None) == rc
+    # more 1,024-item tiles (one thread block each) than a grid can hold: 2^40 rows of 16
+    assert L.dequantize_rows(A16, A16, 1 << 40, 16, 0, A16, None) == qat.QAT_ERR_SHAPE
+    huge = (D * 2)(good, D(0x10000, 0x10000, 1 << 40, 16, 0, 0, 0x10000))
+    assert L.dequantize_rows_batch(ctypes.cast(huge, ctypes.c_void_p), 2, None) == qat.QAT_ERR_SHAPE
     assert L.qat_mlp_bwd(None, None, None, None, 512, 1536, 6, 0, A16, A16, None, A16, 8, None,
                          None, None, None, None, 0, None, 0, None) == qat.QAT_ERR_ARG
     # a dX residual needs dX; the X row stride is at least K and a multiple of 8
