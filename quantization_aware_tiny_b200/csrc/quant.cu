@@ -941,7 +941,8 @@ __device__ __forceinline__ void export_fp16_chunk(const ExportDescDev& d, int64_
 
 // Descriptor owning work unit u (unit_begin is non-decreasing; the last
 // descriptor with unit_begin <= u).
-__device__ __forceinline__ int find_desc(const ExportBatch& b, int64_t u) {
+template <class Batch>
+__device__ __forceinline__ int find_desc(const Batch& b, int64_t u) {
   int lo = 0, hi = b.n - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -977,9 +978,9 @@ struct UnitPos {
 // kExportPacked (some descriptors 6-bit packed), kExportSearch (some with the
 // clip search; packing included).
 constexpr int kExportPlain = 0, kExportPacked = 1, kExportSearch = 2;
-template <int KIND>
+template <int KIND, int CAP>
 __global__ void __launch_bounds__(kExportMaxWarps * 32, 1)
-    export_batch_kernel(const __grid_constant__ ExportBatch b, int* err) {
+    export_batch_kernel(const __grid_constant__ ExportBatchT<CAP> b, int* err) {
   extern __shared__ __align__(128) uint8_t xsmem[];
   const int lane = threadIdx.x & 31;
   const int wib = threadIdx.x >> 5;
@@ -1158,8 +1159,9 @@ __global__ void __launch_bounds__(kQThreads)
 
 // One block per tile of the concatenation; its descriptor is the last k with
 // tile_begin[k] <= tile (tensors without items own no tile).
+template <int CAP>
 __global__ void __launch_bounds__(kQThreads)
-    dequant_batch_kernel(const __grid_constant__ DequantBatch b) {
+    dequant_batch_kernel(const __grid_constant__ DequantBatchT<CAP> b) {
   const int64_t t = blockIdx.x;
   int lo = 0, hi = b.n - 1;
   while (lo < hi) {
@@ -1253,23 +1255,42 @@ int clip_search_supported(int64_t cols) {
   return 1;
 }
 
-int launch_export_batch(ExportBatch& b, cudaStream_t s) {
-  if (b.total_units == 0) return QAT_OK;
+// Descriptor capacities the batched kernels are built for, smallest first.
+constexpr int kBatchCapSmall = 24, kBatchCapMid = 96;
+
+// The export kernel of kind KIND at capacity CAP, its shared-memory limit
+// raised once per device.
+template <int KIND, int CAP>
+int export_launch_kind(const ExportBatchT<CAP>& t, int grid, int warps, int smem, cudaStream_t s) {
   static std::atomic<uint64_t> attr_done{0};  // per device: attributes live in its context
   int dev = 0;
   if (!device_flag_once(attr_done, &dev)) {
-    if (cudaFuncSetAttribute(export_batch_kernel<kExportPlain>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kExportSmemBudget) != cudaSuccess ||
-        cudaFuncSetAttribute(export_batch_kernel<kExportPacked>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kExportSmemBudget) != cudaSuccess ||
-        cudaFuncSetAttribute(export_batch_kernel<kExportSearch>,
+    if (cudaFuncSetAttribute(export_batch_kernel<KIND, CAP>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kExportSmemBudget) != cudaSuccess)
       return QAT_ERR_CUDA;
     device_flag_set(attr_done, dev);
   }
+  export_batch_kernel<KIND, CAP><<<grid, warps * 32, smem, s>>>(t, device_error_ptr());
+  return QAT_OK;
+}
+
+// The batch copied into a parameter block of capacity CAP (n <= CAP).
+template <int CAP>
+int export_launch_cap(const ExportBatch& b, int kind, int grid, int warps, int smem,
+                      cudaStream_t s) {
+  static thread_local ExportBatchT<CAP> t;
+  t.n = b.n;
+  t.buf_bytes = b.buf_bytes;
+  t.total_units = b.total_units;
+  std::copy(b.d, b.d + b.n, t.d);
+  if (kind == kExportSearch) return export_launch_kind<kExportSearch, CAP>(t, grid, warps, smem, s);
+  if (kind == kExportPacked) return export_launch_kind<kExportPacked, CAP>(t, grid, warps, smem, s);
+  return export_launch_kind<kExportPlain, CAP>(t, grid, warps, smem, s);
+}
+
+int launch_export_batch(ExportBatch& b, cudaStream_t s) {
+  if (b.total_units == 0) return QAT_OK;
   int64_t longest = 16;  // bytes of the longest staged unit
   for (int i = 0; i < b.n; ++i)
     if (b.d[i].mode != QAT_EXPORT_FP16 && b.d[i].cols <= kExportMaxStagedCols)
@@ -1285,12 +1306,12 @@ int launch_export_batch(ExportBatch& b, cudaStream_t s) {
     search = search || b.d[i].search;
     packed = packed || b.d[i].pack6;
   }
-  if (search)
-    export_batch_kernel<kExportSearch><<<grid, warps * 32, smem, s>>>(b, device_error_ptr());
-  else if (packed)
-    export_batch_kernel<kExportPacked><<<grid, warps * 32, smem, s>>>(b, device_error_ptr());
-  else
-    export_batch_kernel<kExportPlain><<<grid, warps * 32, smem, s>>>(b, device_error_ptr());
+  const int kind = search ? kExportSearch : packed ? kExportPacked : kExportPlain;
+  int rc;
+  if (b.n <= kBatchCapSmall) rc = export_launch_cap<kBatchCapSmall>(b, kind, grid, warps, smem, s);
+  else if (b.n <= kBatchCapMid) rc = export_launch_cap<kBatchCapMid>(b, kind, grid, warps, smem, s);
+  else rc = export_launch_cap<QAT_EXPORT_BATCH_CAP>(b, kind, grid, warps, smem, s);
+  if (rc != QAT_OK) return rc;
   count_launch();
   return cuda_status(cudaGetLastError());
 }
@@ -1307,11 +1328,24 @@ int launch_dequant(const int8_t* codes, const __half* scales, int64_t rows, int6
   return cuda_status(cudaGetLastError());
 }
 
+// The batch copied into a parameter block of capacity CAP (n <= CAP).
+template <int CAP>
+void dequant_launch_cap(const DequantBatch& b, unsigned grid, cudaStream_t s) {
+  static thread_local DequantBatchT<CAP> t;
+  t.n = b.n;
+  std::copy(b.tile_begin, b.tile_begin + b.n + 1, t.tile_begin);
+  std::copy(b.d, b.d + b.n, t.d);
+  dequant_batch_kernel<CAP><<<grid, kQThreads, 0, s>>>(t);
+}
+
 int launch_dequant_batch(const DequantBatch& b, cudaStream_t s) {
   const int64_t tiles = b.tile_begin[b.n];
   if (tiles == 0) return QAT_OK;
   if (tiles > 0x7FFFFFFF) return QAT_ERR_SHAPE;
-  dequant_batch_kernel<<<static_cast<unsigned>(tiles), kQThreads, 0, s>>>(b);
+  const unsigned grid = static_cast<unsigned>(tiles);
+  if (b.n <= kBatchCapSmall) dequant_launch_cap<kBatchCapSmall>(b, grid, s);
+  else if (b.n <= kBatchCapMid) dequant_launch_cap<kBatchCapMid>(b, grid, s);
+  else dequant_launch_cap<kDequantMaxDescs>(b, grid, s);
   count_launch();
   return cuda_status(cudaGetLastError());
 }

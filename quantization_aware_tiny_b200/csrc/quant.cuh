@@ -32,12 +32,17 @@ constexpr int kClipSearchTop = 4;
 #ifndef QAT_EXPORT_BATCH_CAP
 #define QAT_EXPORT_BATCH_CAP QAT_EXPORT_MAX_DESCS
 #endif
-struct ExportBatch {
+// A batch as the kernel receives it (a __grid_constant__ parameter).  The
+// launch passes the smallest capacity that holds the batch's descriptors: a
+// launch uploads its whole parameter block, and the largest one is 22 KB.
+template <int CAP>
+struct ExportBatchT {
   int n;
   int buf_bytes;  // bytes of one row buffer (longest staged row, rounded to 128)
   int64_t total_units;
-  ExportDescDev d[QAT_EXPORT_BATCH_CAP];
+  ExportDescDev d[CAP];
 };
+using ExportBatch = ExportBatchT<QAT_EXPORT_BATCH_CAP>;
 
 // Chunk length of the fp16 passthrough "rows" (6 KB of fp32, like a staged unit).
 constexpr int64_t kFp16Chunk = 1536;
@@ -111,11 +116,14 @@ inline uint64_t dequant_row_magic(int64_t c4) {
   return ~0ull / static_cast<uint64_t>(c4) + 1ull;
 }
 constexpr int kDequantMaxDescs = QAT_DEQUANT_MAX_DESCS;
-struct DequantBatch {
+// As ExportBatchT: the launch passes the smallest capacity that holds it.
+template <int CAP>
+struct DequantBatchT {
   int n;
-  int64_t tile_begin[kDequantMaxDescs + 1];
-  DequantDescDev d[kDequantMaxDescs];
+  int64_t tile_begin[CAP + 1];
+  DequantDescDev d[CAP];
 };
+using DequantBatch = DequantBatchT<kDequantMaxDescs>;
 int launch_dequant_batch(const DequantBatch& b, cudaStream_t s);
 int launch_unpack6(const uint8_t* packed, int64_t n, int bits, int8_t* codes, cudaStream_t s);
 
