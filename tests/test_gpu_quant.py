@@ -275,6 +275,52 @@ def test_dequantize_rows_batch_one_launch():
             assert np.array_equal(bits16(out), o.bf16_bits(ref)), name
 
 
+def test_export_and_dequantize_past_96_descriptors():
+    """More descriptors than the mid-size parameter block holds (100 small
+    weights of assorted shapes, int6 / int8 / int5, and two fp16 passthrough
+    tensors): one export launch and one grouped dequantize launch, both
+    bit-exact with the oracle."""
+    rng = np.random.default_rng(31)
+    shapes = [(8 + 8 * (i % 5), (16, 64, 136, 512)[i % 4]) for i in range(100)]
+    bits = [(6, 8, 5)[i % 3] for i in range(100)]
+    Ws = [(rng.standard_normal(sh) * 0.02).astype(np.float32) for sh in shapes]
+    descs, outs = [], []
+    for w, b in zip(Ws, bits):
+        codes = torch.empty(w.shape, dtype=torch.int8, device="cuda")
+        s16 = torch.empty(w.shape[0], dtype=torch.float16, device="cuda")
+        descs.append((_dev(w), b, codes, s16))
+        outs.append((codes, s16))
+    flat = [(rng.standard_normal(300) * 0.02).astype(np.float32) for _ in range(2)]
+    f16 = [torch.empty(300, dtype=torch.float16, device="cuda") for _ in flat]
+    for f, o16 in zip(flat, f16):
+        descs.append((_dev(f), qat.QAT_EXPORT_FP16, o16, None))
+    n0 = qat.launch_count()
+    qat.quantize_export_batch(descs)
+    torch.cuda.synchronize()
+    assert qat.launch_count() - n0 == 1
+    items, refs = [], []
+    for i, (w, b, (codes, s16)) in enumerate(zip(Ws, bits, outs)):
+        c_ref, s_ref, _ = o.export_rows(w, b)
+        assert np.array_equal(codes.cpu().numpy(), c_ref), i
+        assert np.array_equal(bits16(s16), s_ref), i
+        out = torch.full(w.shape, float("nan"), device="cuda",
+                         dtype=torch.bfloat16 if i % 2 else torch.float32)
+        items.append((codes, s16, out))
+        refs.append(o.dequant_export(c_ref, s_ref))
+    for f, o16 in zip(flat, f16):
+        assert np.array_equal(bits16(o16), f.astype(np.float16).view(np.uint16))
+    n0 = qat.launch_count()
+    qat.dequantize_rows_batch(items)
+    torch.cuda.synchronize()
+    assert qat.launch_count() - n0 == 1
+    for i, (ref, (_, _, out)) in enumerate(zip(refs, items)):
+        if out.dtype == torch.float32:
+            assert np.array_equal(out.cpu().numpy().view(np.uint32), ref.view(np.uint32)), i
+        else:
+            assert np.array_equal(bits16(out), o.bf16_bits(ref)), i
+    assert qat.device_error() == 0
+
+
 def _near_tie_rows(n_rows=256, cols=512, seed=21, levels=127):
     """Rows whose entries sit within a few ulps of (k + 1/2) * s: the code then
     depends on the correctly rounded quotient w / s (and on ties going to
