@@ -307,7 +307,9 @@ int unpack_codes6(const uint8_t* packed, int64_t n, int32_t bits, int8_t* codes,
  * quantize_rows_export writes them), out [rows, cols] row-major; all device
  * pointers, caller-owned.  cols a positive multiple of 8 (QAT_ERR_SHAPE), codes
  * and out 16-byte aligned (QAT_ERR_ALIGN), a null pointer, rows < 0 or another
- * out_dtype QAT_ERR_ARG.  Bit-exact with the oracle. */
+ * out_dtype QAT_ERR_ARG; more than 2^41 groups of four codes (rows * cols / 4:
+ * one thread block per 1,024 groups) QAT_ERR_SHAPE.  Bit-exact with the
+ * oracle. */
 enum { QAT_DTYPE_F32 = 0, QAT_DTYPE_BF16 = 1 };
 int dequantize_rows(const int8_t* codes, const qat_fp16* scales, int64_t rows, int64_t cols,
                     int32_t out_dtype, void* out, qat_stream_t stream);
@@ -316,7 +318,9 @@ int dequantize_rows(const int8_t* codes, const qat_fp16* scales, int64_t rows, i
  * one launch (a state dict's roundtrip), each descriptor the arguments of one
  * dequantize_rows call.  Every descriptor is checked as dequantize_rows checks
  * its arguments before anything launches; the first failing one decides the
- * error.  n outside 1 .. QAT_DEQUANT_MAX_DESCS or a null array: QAT_ERR_ARG. */
+ * error.  n outside 1 .. QAT_DEQUANT_MAX_DESCS or a null array: QAT_ERR_ARG;
+ * more than 2^31 - 1 thread blocks in all (one per 1,024 groups of four codes
+ * of a tensor, each tensor rounded up to whole blocks): QAT_ERR_SHAPE. */
 #define QAT_DEQUANT_MAX_DESCS 256
 typedef struct qat_dequant_desc {
   const int8_t* codes;
