@@ -351,6 +351,8 @@ def run_ours(args):
             out["recurrent_core"] = measure_core(dev, stream, pk)
             out["recurrent_core_fwd_bwd"] = measure_core_train(dev, stream, pk)
             out["fused_producer"] = measure_fused_producer(dev, stream, pk)
+            out["export_int5_mlp"] = auxiliary(lambda: measure_export(dev, stream, pk, mlp_int5=True))
+            out["noisy_operand"] = auxiliary(lambda: measure_noisy(dev, stream, pk))
             out["cpu_baseline"] = cpu_baseline()
         print(json.dumps(out), flush=True)
     if pg is not None:
@@ -440,7 +442,7 @@ def flush_l2(buf, clean):
     clean.sum()
 
 
-def measure_export(dev, stream, pk, pack6=False, clip_search=False):
+def measure_export(dev, stream, pk, pack6=False, clip_search=False, mlp_int5=False):
     """Export quantizer over the 11-layer d=512 state dict: one grouped launch,
     L2 flushed (256 MB write) before every timed launch.  pack6: the int6 codes
     are stored 6-bit packed (3 bytes per 4 codes); clip_search: each row keeps
@@ -450,11 +452,11 @@ def measure_export(dev, stream, pk, pack6=False, clip_search=False):
     from quantization_aware_tiny_b200 import qat
     from quantization_aware_tiny_b200 import synthetic as sy
     sd = {k: torch.from_numpy(v).to(dev) for k, v in sy.state_dict_case().items()}
-    out = qexport.export_state_dict(sd, pack6=pack6)  # allocates outputs once
+    out = qexport.export_state_dict(sd, pack6=pack6, mlp_int5=mlp_int5)  # allocates outputs once
     fl = qat.QAT_EXPORT_CLIP_SEARCH if clip_search else 0
     descs = []
     algo = 0
-    for name, mode in qexport.plan(sd):
+    for name, mode in qexport.plan(sd, mlp_int5=mlp_int5):
         t = sd[name]
         o = out[name]
         if mode == qat.QAT_EXPORT_FP16:
@@ -506,7 +508,60 @@ def measure_export(dev, stream, pk, pack6=False, clip_search=False):
             "workload": "11 blocks x (Q,K,V,O,fc,proj) d=512 MLP3x int6%s + tied emb 1024x512 "
                         "+ small tensors fp16 passthrough; L2 flushed (256 MB written, 256 MB read) "
                         "before each launch" % ((" 6-bit packed" if pack6 else "") +
-                                                (" clip search" if clip_search else ""))}
+                                                (" clip search" if clip_search else "") +
+                                                (", MLP weights int5" if mlp_int5 else ""))}
+
+
+def measure_noisy(dev, stream, pk):
+    """Noisy-QAT forward operands of the 3x3 core's shared weights at d=640
+    (Q, K, V, O, fc 1920x640, proj 640x1920: 3.69 M weights), one
+    qat_noisy_operand call each (six launches), int8 step amax/127, L2
+    flushed before each set.  Algorithmic bytes: 4 B read + 2 B bf16 written
+    per weight, 4 B per row scale."""
+    from quantization_aware_tiny_b200 import qat
+    from quantization_aware_tiny_b200 import synthetic as sy
+    c = sy.recurrent_core_case(T=8)
+    Ws = [torch.from_numpy(c[k]).to(dev) for k in ("Wq", "Wk", "Wv", "Wo", "Wfc", "Wproj")]
+    outs = [(torch.empty(w.shape, dtype=torch.bfloat16, device=dev),
+             torch.empty(w.shape[0], dtype=torch.float32, device=dev)) for w in Ws]
+    algo = sum(w.numel() * 6 + w.shape[0] * 4 for w in Ws)
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+    clean = torch.zeros(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+    n0 = qat.launch_count()
+
+    def run(step):
+        for i, (w, (op, sc)) in enumerate(zip(Ws, outs)):
+            qat.qat_noisy_operand(w, 1234, 6 * step + i, op, sc, stream=stream, bits=8)
+
+    events = []
+    for it in range(60):
+        flush_l2(flush, clean)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        run(it)
+        b.record(stream)
+        events.append((a, b))
+    torch.cuda.synchronize()
+    ms = statistics.median(a.elapsed_time(b) for a, b in events[10:])
+    gbs = algo / (ms * 1e-3) / 1e9
+    return {"value": round(gbs, 1), "unit": "GB/s", "ms": round(ms, 4), "algorithmic_bytes": algo,
+            "launches_per_set": (qat.launch_count() - n0) // 60,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(gbs / pk["hbm_gbs"], 4),
+                         "peak_kind": "copy bandwidth (%s)" % pk["source"]},
+            "device_error": qat.device_error(),
+            "workload": "Noisy-QAT bf16 operands (Philox-4x32-10 noise, int8 step) of the 3x3 "
+                        "core's six shared weights at d=640, one call per weight; L2 flushed "
+                        "(256 MB written, 256 MB read) before each set"}
+
+
+def auxiliary(fn):
+    """A sub-measurement that must not cost the benchmark line: an exception is
+    recorded in its place in the line, with nothing else skipped."""
+    try:
+        return fn()
+    except Exception as e:  # recorded, not hidden
+        return {"error": "%s: %s" % (type(e).__name__, e)}
 
 
 def measure_dequant(dev, stream, pk):
