@@ -623,9 +623,10 @@ __device__ __forceinline__ void export_rows_smem(const ExportDescDev& d, int64_t
 
 // ---- full units of the common widths, specialised: 384 float4 groups, as
 // three rows of 512 columns or one of 1,536 -- nearly every unit of the
-// 11-layer d = 512 state dict.  Every offset is a compile-time constant, so
-// the per-element work is the arithmetic alone (the generic path spends about
-// as many instructions again on loop control and addresses).
+// 11-layer d = 512 state dict.  Every offset is a compile-time constant,
+// which takes the generic loops' counters and address arithmetic out of the
+// per-element work, and each unit's per-row scalar work runs once, on lanes
+// 0 to NR - 1, instead of on the whole warp per row.
 
 // Three-input max (sm_100): max(a, b, c) in one instruction.
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -657,12 +658,12 @@ __device__ __forceinline__ void top2_merge(float& t1, float& t2, float u1, float
   t2 = fmax3(t2, u2, y);
 }
 
-// A full unit of NR rows (NR = 3: K4 = 128; NR = 1: K4 = 384) staged at buf:
-// lane holds groups lane + 32 i, i < 12; row k owns i in [12k / NR, 12(k+1) / NR).
+// A full unit of NR rows staged at buf (NR = 3: rows of 128 groups; NR = 1:
+// one row of 384): lane holds groups lane + 32 i, i < 12; row k owns i in
+// [12k / NR, 12(k + 1) / NR).
 template <int NR>
 __device__ __forceinline__ void export_unit384(const ExportDescDev& d, int64_t row0,
                                                const float4* __restrict__ buf, int lane) {
-  constexpr int K4 = 384 / NR;
   // three chains of four groups: chain c = row c (NR = 3) or a third of the row
   float t1[3], t2[3];
 #pragma unroll
@@ -721,7 +722,6 @@ __device__ __forceinline__ void export_unit384(const ExportDescDev& d, int64_t r
       for (int i = 0; i < 4; ++i) oc[32 * i] = codes4_t<BITS, R>(qc, v[i]);
     }
   });
-  (void)K4;
 }
 
 // ---- clip search (the leaderboard's "GPTQ-lite" clip search, read as: per row,
