@@ -1,6 +1,7 @@
 """Host-side checks of the benchmark's bookkeeping (no GPU): the DRAM traffic
 it reports next to the roofline belongs to the GEMM sources in the tree, and
-the clock record keeps only the samples taken inside the timed window."""
+the clock record keeps only the samples taken inside the timed window, and
+an auxiliary sub-measurement that fails is recorded, not fatal."""
 import bench
 
 
@@ -37,3 +38,12 @@ def test_clock_window_empty_reports_why():
     s = c.summary()
     assert s["samples"] == 0 and s["samples_outside_window"] == 1
     assert s["nvml_error"] == "NVMLError: test"
+
+
+def test_auxiliary_measurement_records_an_exception():
+    """A failing auxiliary sub-measurement leaves its error in the line; a
+    working one returns its object unchanged."""
+    def boom():
+        raise RuntimeError("no such tensor")
+    assert bench.auxiliary(boom) == {"error": "RuntimeError: no such tensor"}
+    assert bench.auxiliary(lambda: {"value": 1.0}) == {"value": 1.0}
